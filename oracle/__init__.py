@@ -1,0 +1,181 @@
+"""Float64 CPU oracle of the DeepSeekMoE layer — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, the package's ``smoke()`` check and ``bench.py``'s CPU-baseline
+leg may import this package.  The product path (the CUDA library and its Python
+binding) never imports, links or calls anything here, and this package imports
+nothing from the product.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, float64, single thread); this
+module builds it with gcc, wraps it with ctypes, and spells out the layer's
+forward exactly as the teaching code of "The Evolving Transformer · 07 —
+DeepSeek V2 & V3" (§ 02 DeepSeekMoE, ``MoE.forward``; § 03 Shared Expert) does:
+
+    shared_out = shared_expert(x)            # every token
+    weights, indices = router(x)             # (tokens, top_k)
+    output = 0
+    for each slot k and expert i:
+        mask = indices[:, k] == i
+        output[mask] += weights[mask, k] * expert_i(x[mask])
+    return shared_out + output
+
+The only liberty taken: the expert loop is the outer loop (so each expert's
+weights are fetched once) and each (token, slot) contribution is stored, then
+summed in slot order k = 0..top_k-1 — the same additions, in the same order per
+token, as the page's k-outer loop.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Callable, Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c with gcc (strict IEEE float64: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC",
+                               "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("hidden_size", ctypes.c_int32), ("n_routed_experts", ctypes.c_int32),
+                ("num_experts_per_tok", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("moe_intermediate_size", ctypes.c_int32),
+                ("n_shared_experts", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_double)]
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        p = ctypes.c_void_p
+        lib.oracle_route.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, p, p, p, p, p, p, p]
+        lib.oracle_route.restype = ctypes.c_int
+        lib.oracle_swiglu.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                      p, p, p, p, p]
+        lib.oracle_swiglu.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected bf16 bits as uint16, got {a.dtype}")
+    return a
+
+
+def _cfg(shape) -> _Cfg:
+    return _Cfg(shape.hidden_size, shape.n_routed_experts, shape.num_experts_per_tok,
+                shape.n_group, shape.topk_group, shape.moe_intermediate_size,
+                shape.n_shared_experts, int(bool(shape.norm_topk_prob)),
+                float(shape.routed_scaling_factor))
+
+
+def route(shape, x_bits, router_w, e_bias, want_scores: bool = False):
+    """Router for every row of ``x_bits`` [n, H] (bf16 bits).
+
+    Returns (idx int32 [n,k], w float64 [n,k], margin float64 [n]) and, when
+    asked, the unbiased sigmoid scores float64 [n,E].
+    """
+    lib = _load()
+    x_bits = _u16(x_bits)
+    n = x_bits.shape[0]
+    k, E = shape.num_experts_per_tok, shape.n_routed_experts
+    rw = np.ascontiguousarray(router_w, dtype=np.float32)
+    eb = np.ascontiguousarray(e_bias, dtype=np.float32)
+    idx = np.zeros((n, k), np.int32)
+    w = np.zeros((n, k), np.float64)
+    margin = np.zeros((n,), np.float64)
+    scores = np.zeros((n, E), np.float64) if want_scores else None
+    rc = lib.oracle_route(ctypes.byref(_cfg(shape)), n, _ptr(x_bits), _ptr(rw), _ptr(eb),
+                          _ptr(idx), _ptr(w), _ptr(margin),
+                          _ptr(scores) if want_scores else None)
+    if rc != 0:
+        raise ValueError(f"oracle_route rejected the configuration {shape}")
+    return (idx, w, margin, scores) if want_scores else (idx, w, margin)
+
+
+def swiglu(x_bits, w_gate, w_up, w_down) -> np.ndarray:
+    """down(silu(gate x) * up x) in float64 for rows x_bits [n,H]; weights (out, in)."""
+    lib = _load()
+    x_bits, w_gate, w_up, w_down = (_u16(a) for a in (x_bits, w_gate, w_up, w_down))
+    n, H = x_bits.shape
+    I = w_gate.shape[0]
+    assert w_gate.shape == (I, H) and w_up.shape == (I, H) and w_down.shape == (H, I)
+    out = np.zeros((n, H), np.float64)
+    if n == 0 or I == 0:
+        return out
+    rc = lib.oracle_swiglu(n, H, I, _ptr(x_bits), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                           _ptr(out))
+    if rc != 0:
+        raise MemoryError("oracle_swiglu failed to allocate")
+    return out
+
+
+ExpertFetch = Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarray]]
+
+
+def moe_layer(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
+              shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]],
+              routing: Optional[Tuple[np.ndarray, np.ndarray]] = None):
+    """The layer's forward for the rows of ``x_bits`` (any subset of tokens).
+
+    ``expert(e)`` returns (w_gate[e], w_up[e], w_down[e]) as bf16 bits; it is
+    called once per expert that some row uses.  ``shared`` is the concatenated
+    shared expert (ws_gate [S*I,H], ws_up [S*I,H], ws_down [H,S*I]) or None.
+    ``routing`` optionally supplies (idx, w) instead of the oracle's own router
+    (used to score an alternative, equally correct near-tie selection).
+
+    Returns (y float64 [n,H], idx, w, margin or None).
+    """
+    x_bits = _u16(x_bits)
+    n, H = x_bits.shape
+    k = shape.num_experts_per_tok
+    margin = None
+    if routing is None:
+        idx, w, margin = route(shape, x_bits, router_w, e_bias)
+    else:
+        idx, w = routing
+        idx = np.asarray(idx, np.int32)
+        w = np.asarray(w, np.float64)
+
+    # shared_expert(x): runs unconditionally for every row.
+    if shared is not None and shape.n_shared_experts > 0:
+        shared_out = swiglu(x_bits, *shared)
+    else:
+        shared_out = np.zeros((n, H), np.float64)
+
+    # routed: contribution of (row, slot) = w[row, slot] * expert_e(x[row]).
+    contrib = np.zeros((n, k, H), np.float64)
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        wg, wu, wd = expert(int(e))
+        out = swiglu(x_bits[rows], wg, wu, wd)
+        contrib[rows, slots] = w[rows, slots][:, None] * out
+    output = np.zeros((n, H), np.float64)
+    for j in range(k):
+        output += contrib[:, j]
+    return shared_out + output, idx, w, margin
+
+
+def in_memory_experts(w_gate, w_up, w_down) -> ExpertFetch:
+    """Expert fetcher over host arrays [E,I,H], [E,I,H], [E,H,I] of bf16 bits."""
+    return lambda e: (w_gate[e], w_up[e], w_down[e])
+

@@ -1,0 +1,197 @@
+/*
+ * Float64 CPU oracle of the DeepSeekMoE feed-forward layer (noaux_tc routing).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file: only the tests, the package's smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header or constant with the CUDA
+ * library, and it is deliberately plain: single-threaded, no BLAS, no blocking,
+ * no fast-math, every sum taken in float64 in index order.
+ *
+ * Inputs are the same stored bits the GPU reads: x and expert weights as bf16
+ * (passed as uint16 bit patterns), router weight and correction bias as fp32.
+ * Each is widened to double exactly.
+ *
+ * Sources for what is computed:
+ *  - "DeepSeekV3.2-Tiered-Implementations" README, § Architecture: sigmoid
+ *    routing with a per-expert correction bias (topk_method "noaux_tc"),
+ *    group-based routing with n_group groups of which topk_group are kept,
+ *    256 routed experts, top-8.
+ *  - "The Evolving Transformer · 07 — DeepSeek V2 & V3", § 02 DeepSeekMoE and
+ *    § 03 Shared Expert: router(x) -> (weights, indices); routed outputs are
+ *    added with their weights; the shared expert runs for every token; the
+ *    layer returns shared + routed.  § 06: the bias only steers selection
+ *    (nudged by load); weights come from the unbiased score.
+ *  - Points the pages leave open (group score = sum of the two largest biased
+ *    scores of the group, contiguous groups, exclusion of dropped groups,
+ *    lower index wins ties, normalisation then routed_scaling_factor) follow
+ *    the DeepSeek-V3 noaux_tc definition; each is listed with its reading in
+ *    the design notes.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t hidden_size;
+    int32_t n_routed_experts;
+    int32_t num_experts_per_tok;
+    int32_t n_group;
+    int32_t topk_group;
+    int32_t moe_intermediate_size;
+    int32_t n_shared_experts;
+    int32_t norm_topk_prob;
+    double routed_scaling_factor;
+} oracle_cfg;
+
+static double widen_bf16(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* sigma(z) = 1 / (1 + e^-z), the router's score function. */
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/* silu(z) = z * sigma(z), the SwiGLU gate activation. */
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* "a beats b": larger value wins; on equal values the lower index wins. */
+static int beats(double va, int ia, double vb, int ib)
+{
+    return va > vb || (va == vb && ia < ib);
+}
+
+/*
+ * Route T tokens (steps 1-7 of the layer definition).
+ *   idx    [T,k]  chosen experts, in descending biased score
+ *   w      [T,k]  routing weights (unbiased sigmoid, normalised, scaled)
+ *   margin [T]    min(group-score gap at the keep boundary,
+ *                     biased-score gap at the top-k boundary); +inf if none
+ *   scores [T,E]  optional: unbiased sigmoid scores
+ * Returns 0, or -1 on an invalid configuration or allocation failure.
+ */
+int oracle_route(const oracle_cfg *c, int64_t T, const uint16_t *x, const float *router_w,
+                 const float *e_bias, int32_t *idx, double *w, double *margin, double *scores)
+{
+    const int H = c->hidden_size, E = c->n_routed_experts, G = c->n_group;
+    const int TG = c->topk_group, K = c->num_experts_per_tok;
+    if (H <= 0 || E <= 0 || G <= 0 || E % G != 0 || TG < 1 || TG > G || K < 1 ||
+        K > TG * (E / G))
+        return -1;
+    const int gsize = E / G;
+
+    double *xs = malloc(sizeof(double) * H);
+    double *s = malloc(sizeof(double) * E);
+    double *b = malloc(sizeof(double) * E);
+    double *gs = malloc(sizeof(double) * G);
+    int *kept = malloc(sizeof(int) * G);
+    int *taken = malloc(sizeof(int) * E);
+    if (!xs || !s || !b || !gs || !kept || !taken) {
+        free(xs); free(s); free(b); free(gs); free(kept); free(taken);
+        return -1;
+    }
+
+    for (int64_t t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) xs[h] = widen_bf16(x[t * H + h]);
+
+        /* 1-3: logits, sigmoid scores, biased scores. */
+        for (int e = 0; e < E; ++e) {
+            double l = 0.0;
+            for (int h = 0; h < H; ++h) l += xs[h] * (double)router_w[(int64_t)e * H + h];
+            s[e] = sigmoid(l);
+            b[e] = s[e] + (double)e_bias[e];
+            if (scores) scores[t * E + e] = s[e];
+        }
+
+        /* 4: group score = largest + second-largest biased score in the group
+         * (a one-expert group scores its only member). */
+        for (int g = 0; g < G; ++g) {
+            int i1 = -1, i2 = -1;
+            for (int e = g * gsize; e < (g + 1) * gsize; ++e) {
+                if (i1 < 0 || beats(b[e], e, b[i1], i1)) { i2 = i1; i1 = e; }
+                else if (i2 < 0 || beats(b[e], e, b[i2], i2)) { i2 = e; }
+            }
+            gs[g] = b[i1] + (i2 >= 0 ? b[i2] : 0.0);
+        }
+
+        /* 5: keep the topk_group best groups (repeated arg-max, lower g on ties). */
+        for (int g = 0; g < G; ++g) kept[g] = 0;
+        double last_kept_gs = 0.0;
+        for (int r = 0; r < TG; ++r) {
+            int best = -1;
+            for (int g = 0; g < G; ++g)
+                if (!kept[g] && (best < 0 || beats(gs[g], g, gs[best], best))) best = g;
+            kept[best] = 1;
+            last_kept_gs = gs[best];
+        }
+        double group_gap = INFINITY;
+        for (int g = 0; g < G; ++g)
+            if (!kept[g] && last_kept_gs - gs[g] < group_gap) group_gap = last_kept_gs - gs[g];
+
+        /* 6: top-k experts among the kept groups only (others are excluded, not
+         * zeroed), by repeated arg-max of the biased score, lower index on ties. */
+        for (int e = 0; e < E; ++e) taken[e] = 0;
+        double last_b = 0.0;
+        for (int j = 0; j < K; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e] || !kept[e / gsize]) continue;
+                if (best < 0 || beats(b[e], e, b[best], best)) best = e;
+            }
+            taken[best] = 1;
+            idx[t * K + j] = best;
+            last_b = b[best];
+        }
+        double expert_gap = INFINITY;
+        for (int e = 0; e < E; ++e)
+            if (!taken[e] && kept[e / gsize] && last_b - b[e] < expert_gap)
+                expert_gap = last_b - b[e];
+        margin[t] = group_gap < expert_gap ? group_gap : expert_gap;
+
+        /* 7: weights from the unbiased scores, normalised, then scaled. */
+        double sum = 0.0;
+        for (int j = 0; j < K; ++j) sum += s[idx[t * K + j]];
+        for (int j = 0; j < K; ++j) {
+            double wj = s[idx[t * K + j]];
+            if (c->norm_topk_prob) wj = wj / sum;
+            w[t * K + j] = wj * c->routed_scaling_factor;
+        }
+    }
+    free(xs); free(s); free(b); free(gs); free(kept); free(taken);
+    return 0;
+}
+
+/*
+ * One SwiGLU expert, down(silu(gate x) * up x), over n rows.
+ *   x  [n,H] bf16 bits; w_gate, w_up [I,H] and w_down [H,I] bf16 bits in the
+ *   nn.Linear (out, in) layout; out [n,H] float64.
+ * Returns 0, or -1 on allocation failure.
+ */
+int oracle_swiglu(int64_t n, int64_t H, int64_t I, const uint16_t *x, const uint16_t *w_gate,
+                  const uint16_t *w_up, const uint16_t *w_down, double *out)
+{
+    double *xs = malloc(sizeof(double) * H);
+    double *hmid = malloc(sizeof(double) * I);
+    if (!xs || !hmid) { free(xs); free(hmid); return -1; }
+    for (int64_t r = 0; r < n; ++r) {
+        for (int64_t h = 0; h < H; ++h) xs[h] = widen_bf16(x[r * H + h]);
+        for (int64_t i = 0; i < I; ++i) {
+            double u = 0.0, v = 0.0;
+            for (int64_t h = 0; h < H; ++h) {
+                u += widen_bf16(w_gate[i * H + h]) * xs[h];
+                v += widen_bf16(w_up[i * H + h]) * xs[h];
+            }
+            hmid[i] = silu(u) * v;
+        }
+        for (int64_t o = 0; o < H; ++o) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < I; ++i) acc += widen_bf16(w_down[o * I + i]) * hmid[i];
+            out[r * H + o] = acc;
+        }
+    }
+    free(xs); free(hmid);
+    return 0;
+}
