@@ -1,0 +1,432 @@
+"""Benchmark of the DeepSeekMoE layer forward (noaux_tc routing) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_prefill]
+    python bench.py --impl reference ...      # the float64 CPU oracle arm
+
+One step = one pass of the whole layer (route, dispatch, gate/up GEMM with
+SwiGLU, down GEMM, combine) over one batch of T synthetic tokens, inputs
+resident in HBM.  Expert weights (22.5 GB at the V3 shape) exceed the 126 MB
+L2 many times over, so every step streams them from HBM.  Under torchrun each
+rank runs its own batch with replicated weights (weak scaling; no collective
+on the data path); the time is the max over ranks.  Rank 0 prints ONE JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_moe_layer_noaux_b200 import MoELayer, abi  # noqa: E402
+from sparse_moe_layer_noaux_b200.workloads import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOP/s at V3 shape (T=128, 16384); % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.rows = []
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- GPU arm
+class StagedStep:
+    """One layer step as its five C-ABI stages, with CUDA events between them
+    on the launching stream (same kernels and order as moe_forward)."""
+
+    NAMES = ("route", "dispatch", "gate_up", "down", "combine")
+
+    def __init__(self, shape, inp):
+        self.shape, self.inp = shape, inp
+        T, k, E, H, I, S = shape.T, shape.k, shape.E, shape.H, shape.I, shape.S
+        d = inp["x"].device
+        self.cfg = abi.MoEConfig.from_shape(shape)
+        self.ws = torch.empty(abi.workspace_size(self.cfg, T), dtype=torch.uint8, device=d)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=d)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=d)
+        self.off = torch.empty(E + 1, dtype=torch.int32, device=d)
+        self.x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=d)
+        self.perm_src = torch.empty(T * k, dtype=torch.int32, device=d)
+        self.row_of = torch.empty((T, k), dtype=torch.int32, device=d)
+        self.h_r = torch.empty((T * k, I), dtype=torch.bfloat16, device=d)
+        self.h_s = torch.empty((T, max(S * I, 8)), dtype=torch.bfloat16, device=d)
+        self.y_perm = torch.empty((T * k + T, H), dtype=torch.bfloat16, device=d)
+        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=d)
+
+    def run(self, events=None):
+        s, i, T = self.shape, self.inp, self.shape.T
+        ev = events or [None] * 6
+
+        def rec(j):
+            if ev[j] is not None:
+                ev[j].record()
+        rec(0)
+        abi.moe_route(self.cfg, i["x"], i["router_w"], i["e_bias"], self.idx, self.w, self.ws)
+        rec(1)
+        abi.moe_dispatch(self.cfg, i["x"], self.idx, self.off, self.x_perm, self.perm_src, self.row_of, self.ws)
+        rec(2)
+        abi.moe_experts_gate_up(self.cfg, T, i["x"], self.x_perm, self.off, i["w_gate"], i["w_up"],
+                                i["ws_gate"], i["ws_up"], self.h_r, self.h_s)
+        rec(3)
+        abi.moe_experts_down(self.cfg, T, self.h_r, self.h_s, self.off, self.perm_src, self.w, i["w_down"],
+                             i["ws_down"], self.y_perm)
+        rec(4)
+        abi.moe_combine(self.cfg, T, self.y_perm, self.row_of, self.y)
+        rec(5)
+
+
+def layer_bytes(shape, idx):
+    """Algorithmic bytes of one step: touched routed experts + shared + router + x and y."""
+    touched = int(torch.unique(idx).numel())
+    b = touched * 3 * shape.H * shape.I * 2 + 3 * shape.H * shape.S * shape.I * 2
+    b += 4 * shape.E * shape.H + 4 * shape.T * shape.H
+    return b, touched
+
+
+def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
+    inp = make_inputs(shape, "cuda", seed=shape.seed * 1000 + rank if rank else shape.seed)
+    if rank:
+        # Replicated weights across ranks; only the tokens differ.
+        w0 = make_inputs(shape.with_(T=1), "cuda")
+        for k in ("router_w", "e_bias", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+            inp[k] = w0[k]
+    st = StagedStep(shape, inp)
+    for _ in range(warmup):
+        st.run()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = abi.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for j in range(steps):
+            st.run(evs[j])
+        torch.cuda.synchronize()
+    launches = abi.launch_count() - n0
+    barrier(world)
+    stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, name in enumerate(StagedStep.NAMES)}
+    total_ms = sum(evs[j][0].elapsed_time(evs[j][5]) for j in range(steps))
+    ms = max_over_ranks(total_ms / steps, world)
+    assert abi.device_status() == 0
+
+    # moe_forward (one call per step) timed alone, for reference.
+    layer = MoELayer.from_inputs(shape, inp)
+    y = torch.empty_like(inp["x"])
+    for _ in range(2):
+        layer(inp["x"], y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        layer(inp["x"], y)
+    e1.record()
+    torch.cuda.synchronize()
+    fwd_ms = e0.elapsed_time(e1) / steps
+
+    flops = shape.flops()
+    lbytes, touched = layer_bytes(shape, st.idx)
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9))
+    res = {
+        "ms": ms, "stage_ms": stage_ms, "forward_ms": fwd_ms, "launches": launches,
+        "tflops": flops / (ms * 1e-3) / 1e12, "layer_bytes": lbytes, "experts_touched": touched,
+        "layer_roofline": {"bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >=
+                           lbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                           "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms,
+                           "hbm_gbs_achieved": lbytes / (ms * 1e-3) / 1e9},
+        "clocks": clk.summary(), "st": st, "inp": inp, "layer": layer,
+    }
+    return res
+
+
+def time_e2e(layer, shape, steps):
+    """The public call with host buffers: pinned x -> HBM, layer, y -> pinned host."""
+    x_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(layer_inputs_host(shape))
+    y_host = torch.empty_like(x_host, pin_memory=True)
+    x_dev = torch.empty_like(x_host, device="cuda")
+    y_dev = torch.empty_like(x_dev)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = x_host.numel() * x_host.element_size()
+    return ms, nbytes, nbytes
+
+
+def layer_inputs_host(shape):
+    g = torch.Generator().manual_seed(shape.seed + 77)
+    return torch.randn((shape.T, shape.H), generator=g).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------- oracle (CPU) arm
+def oracle_sample(shape, inp, n_tokens, seed):
+    """Time the float64 oracle (routing + shared + routed experts) on n_tokens rows.
+    Expert weights are copied from the device one expert at a time; that copy time
+    is excluded.  Returns (seconds of oracle work, rows)."""
+    import oracle
+    oracle.build()
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(shape.T, n_tokens, replace=False))
+    x_bits = bf16_bits(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
+    rw, bias = inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()
+    shared = None
+    if shape.S:
+        shared = tuple(bf16_bits(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
+    fetch_s = [0.0]
+
+    def fetch(e):
+        t0 = time.perf_counter()
+        r = (bf16_bits(inp["w_gate"][e]), bf16_bits(inp["w_up"][e]), bf16_bits(inp["w_down"][e]))
+        fetch_s[0] += time.perf_counter() - t0
+        return r
+    t0 = time.perf_counter()
+    oracle.moe_layer(shape, x_bits, rw, bias, fetch, shared)
+    return time.perf_counter() - t0 - fetch_s[0], rows
+
+
+def oracle_tokens_per_step(shape):
+    per_token_macs = shape.E * shape.H + 3 * shape.H * shape.I * (shape.k + shape.S)
+    return max(1, int(4e8 // per_token_macs))  # about half a second of float64 work
+
+
+def cpu_baseline(shape, inp, budget_tokens=None):
+    n = budget_tokens or max(1, min(shape.T, 24 * oracle_tokens_per_step(shape)))
+    secs, rows = oracle_sample(shape, inp, n, seed=99)
+    return {"value": len(rows) / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(rows)} of the {shape.T} tokens of the {shape.name} batch (seeded): "
+                      f"routing, shared and routed SwiGLU experts in float64, 1 thread; "
+                      f"expert-weight copies from the device excluded"}
+
+
+def run_reference(args, shape, world, rank):
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(shape, dev)
+    per = oracle_tokens_per_step(shape)
+    for j in range(args.warmup):
+        oracle_sample(shape, inp, per, seed=1000 + j)
+    secs = 0.0
+    for j in range(args.steps):
+        s, _ = oracle_sample(shape, inp, per, seed=2000 + j)
+        secs += s
+    value = per * args.steps / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(shape, world),
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": "tokens/s",
+                         "sample": f"{per} seeded tokens of the {shape.T}-token {shape.name} batch per "
+                                   f"step: routing + shared + routed experts in float64, 1 thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(shape, world):
+    return {"workload": f"{shape.name}: DeepSeekMoE layer, T={shape.T} tokens per GPU, hidden {shape.H}, "
+                        f"{shape.E} routed experts (top-{shape.k}, {shape.n_group} groups keep "
+                        f"{shape.topk_group}), intermediate {shape.I}, {shape.S} shared",
+            "T": shape.T, "hidden_size": shape.H, "n_routed_experts": shape.E,
+            "num_experts_per_tok": shape.k, "n_group": shape.n_group, "topk_group": shape.topk_group,
+            "moe_intermediate_size": shape.I, "n_shared_experts": shape.S,
+            "global_batch": shape.T * world, "parallelism": f"replicas x{world} (token-sharded)",
+            "l2": "inputs larger than L2: 22.5 GB of expert weights streamed per step"
+            if shape.H == 7168 else "no L2 flush (weights may stay in L2)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="v3_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    shape = WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args.gpus)
+
+    if args.impl == "reference":
+        run_reference(args, shape, world, rank)
+        finish(world)
+        return
+
+    peaks, peak_src = load_peaks()
+    res = time_gpu(shape, args.steps, args.warmup, world, rank, peaks)
+    ms = res["ms"]
+    value = shape.T * world / (ms * 1e-3)
+
+    # Dominant kernel: the gate/up grouped GEMM with the SwiGLU epilogue.
+    k4_ms = res["stage_ms"]["gate_up"]
+    k4_flops = 4.0 * shape.H * shape.I * shape.T * (shape.k + shape.S)
+    achieved = k4_flops / (k4_ms * 1e-3) / 1e12
+    roofline = {"kernel": "grouped_gemm_kernel<kSwiGLU> (gate/up + SwiGLU)", "bound": "tensor",
+                "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": None,
+                "flops_per_launch": k4_flops, "ms_per_launch": k4_ms}
+
+    e2e_ms, h2d, d2h = time_e2e(res["layer"], shape, max(3, args.steps // 2))
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    extra = {}
+    if not args.no_decode and shape.name == "v3_prefill":
+        dec = WORKLOADS["v3_decode"]
+        del res["st"]
+        torch.cuda.empty_cache()
+        dr = time_gpu(dec, max(args.steps, 20), args.warmup, world, rank, peaks)
+        extra["v3_decode"] = {
+            "tokens_per_s": dec.T * world / (dr["ms"] * 1e-3), "ms_per_step": dr["ms"],
+            "tflops": dr["tflops"], "stage_ms": dr["stage_ms"], "forward_ms": dr["forward_ms"],
+            "layer_roofline": dr["layer_roofline"], "experts_touched": dr["experts_touched"],
+            "layer_bytes": dr["layer_bytes"]}
+        del dr
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
+        "config": workload_config(shape, world),
+        "tflops": res["tflops"] * world, "stage_ms": res["stage_ms"], "forward_ms": res["forward_ms"],
+        "layer_roofline": res["layer_roofline"], "experts_touched": res["experts_touched"],
+        "roofline": roofline,
+        "clocks": res["clocks"],
+        "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": res["launches"],
+    }
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, res["inp"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    finish(world)
+
+
+def finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * moe.h — C ABI of libmoe: the forward pass of the DeepSeekMoE feed-forward
+ * layer with noaux_tc routing, on one NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (per token x, a row of hidden_size values):
+ *   - router: sigmoid scores s_e = sigma(x . router_w[e]) and biased scores
+ *     b_e = s_e + e_bias[e]; experts form n_group contiguous groups; a group's
+ *     score is the sum of its two largest b; the topk_group best groups are
+ *     kept; the num_experts_per_tok best b among the kept groups' experts are
+ *     chosen; their weights are the unbiased s, divided by their sum when
+ *     norm_topk_prob, times routed_scaling_factor.
+ *     ("DeepSeekV3.2-Tiered-Implementations" README, § Architecture: sigmoid
+ *     routing with correction bias, topk_method noaux_tc, n_group / topk_group;
+ *     "The Evolving Transformer · 07 — DeepSeek V2 & V3", § 06: the bias is a
+ *     load-balancing nudge, the weights use the unbiased score.)
+ *   - experts: each chosen expert is a SwiGLU MLP, down(silu(gate x) * up x),
+ *     and the shared expert(s) run on every token; the output is
+ *     shared(x) + sum_j w_j * expert_j(x).
+ *     ("The Evolving Transformer · 07", § 02 DeepSeekMoE, MoE.forward, and
+ *     § 03 Shared Expert.)
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, row-major and contiguous,
+ *     owned by the caller; the library never allocates, frees or keeps them.
+ *     bf16 tensors are passed as void* (IEEE bfloat16 bit patterns).
+ *   - Weights use the nn.Linear (out, in) layout: w_gate, w_up [E, I, H],
+ *     w_down [E, H, I]; the S shared experts are stored concatenated along the
+ *     intermediate axis: ws_gate, ws_up [S*I, H], ws_down [H, S*I] (S separate
+ *     SwiGLU experts sum to exactly this).
+ *   - `stream` is a cudaStream_t (CUstream) handle; NULL means the legacy
+ *     default stream.  Work is enqueued on it and the call returns without
+ *     synchronising; results are valid once the stream reaches that point.
+ *   - Device pointers must be 16-byte aligned; hidden_size and
+ *     moe_intermediate_size must be multiples of 64.
+ *   - T = 0 is a valid no-op.  A call never throws across the ABI; it returns
+ *     one of the moe_status codes below and, on an argument error, enqueues
+ *     nothing.
+ *   - Device-side waits are bounded: a wait that gives up writes a device
+ *     error word (read with moe_device_status) instead of hanging the GPU.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer configuration; field names follow the DeepSeek-V3 config
+ * ("DeepSeekV3.2-Tiered-Implementations" README, § Key Dimensions and
+ * § Architecture). */
+typedef struct moe_config {
+    int32_t hidden_size;            /* H */
+    int32_t n_routed_experts;       /* E, 1..256 */
+    int32_t num_experts_per_tok;    /* k, 1..32 and <= topk_group * E / n_group */
+    int32_t n_group;                /* G, 1..32, divides E */
+    int32_t topk_group;             /* TG, 1..G */
+    int32_t moe_intermediate_size;  /* I */
+    int32_t n_shared_experts;       /* S, >= 0 */
+    int32_t norm_topk_prob;         /* 0 or 1 */
+    float routed_scaling_factor;
+} moe_config;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, T < 0, E % G != 0, TG > G, k out of range, ... */
+    MOE_ERR_UNSUPPORTED = 2,  /* H or I not a multiple of 64, E > 256, G > 32, k > 32,
+                                 a pointer not 16-byte aligned, sizes beyond int32 rows */
+    MOE_ERR_WORKSPACE = 3,    /* workspace null or smaller than moe_workspace_size() */
+    MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    MOE_ERR_TIMEOUT = 5       /* a bounded device wait gave up (from moe_device_status) */
+} moe_status;
+
+/* Bytes of scratch needed by moe_forward (and enough for every other call
+ * that takes a workspace) for T tokens.  Pure host arithmetic. */
+MOE_API int moe_workspace_size(const moe_config *cfg, int64_t T, size_t *bytes);
+
+/*
+ * Router (noaux_tc): for each token t, topk_idx[t, 0..k) are the chosen
+ * experts in descending biased score (lower expert index first on equal
+ * scores) and topk_w[t, 0..k) their routing weights.
+ *   x        bf16  [T, H]
+ *   router_w fp32  [E, H]      e_bias fp32 [E]
+ *   topk_idx int32 [T, k]      topk_w fp32 [T, k]   (outputs)
+ * Logits are accumulated in fp32 (gating is kept in high precision, per the
+ * knlb.dev DeepSeek-V3 notes, § infrastructure / fp8).
+ */
+MOE_API int moe_route(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+              const float *e_bias, int32_t *topk_idx, float *topk_w,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Dispatch: the page's per-expert mask and gather, indices[:, :, k] == i then
+ * x[mask] ("The Evolving Transformer · 07", § 02, MoE.forward), done once for
+ * all experts as a counting sort.  Rows routed to expert e occupy
+ * x_perm[expert_offsets[e] .. expert_offsets[e+1]) in ascending (t, j) order.
+ *   topk_idx        int32 [T, k]            (input, from moe_route)
+ *   expert_offsets  int32 [E + 1]           expert_offsets[E] == T * k
+ *   x_perm          bf16  [T * k, H]        x_perm[r] = x[perm_src[r] / k]
+ *   perm_src        int32 [T * k]           source slot t * k + j of row r
+ *   row_of          int32 [T, k]            row of slot (t, j); inverse of perm_src
+ */
+MOE_API int moe_dispatch(const moe_config *cfg, int64_t T, const void *x, const int32_t *topk_idx,
+                 int32_t *expert_offsets, void *x_perm, int32_t *perm_src, int32_t *row_of,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Experts: every routed row r of expert e gives
+ *   h_routed[r] = silu(x_perm[r] . w_gate[e]^T) * (x_perm[r] . w_up[e]^T)   bf16 [T*k, I]
+ *   y_perm[r]   = topk_w[perm_src[r]] * (h_routed[r] . w_down[e]^T)         bf16 [T*k + T, H]
+ * and every token t runs the shared expert(s) on x itself:
+ *   h_shared[t]        = silu(x[t] . ws_gate^T) * (x[t] . ws_up^T)          bf16 [T, S*I]
+ *   y_perm[T*k + t]    = h_shared[t] . ws_down^T
+ * ("The Evolving Transformer · 07", § 02 and § 03.)  Grouped tensor-core
+ * GEMMs over the variable-length expert segments given by expert_offsets;
+ * fp32 accumulation, bf16 storage.  When S == 0 the shared pointers may be
+ * NULL and y_perm needs only T*k rows.
+ */
+MOE_API int moe_experts(const moe_config *cfg, int64_t T, const void *x, const void *x_perm,
+                const int32_t *expert_offsets, const int32_t *perm_src, const float *topk_w,
+                const void *w_gate, const void *w_up, const void *w_down,
+                const void *ws_gate, const void *ws_up, const void *ws_down,
+                void *h_routed, void *h_shared, void *y_perm, void *stream);
+
+/* The two halves of moe_experts, for callers that schedule them separately:
+ * gate_up writes h_routed / h_shared (gate and up projections with the SwiGLU
+ * epilogue); down writes y_perm from them (down projection with the routing-
+ * weight epilogue).  Arguments as in moe_experts. */
+MOE_API int moe_experts_gate_up(const moe_config *cfg, int64_t T, const void *x, const void *x_perm,
+                                const int32_t *expert_offsets, const void *w_gate, const void *w_up,
+                                const void *ws_gate, const void *ws_up, void *h_routed,
+                                void *h_shared, void *stream);
+MOE_API int moe_experts_down(const moe_config *cfg, int64_t T, const void *h_routed,
+                             const void *h_shared, const int32_t *expert_offsets,
+                             const int32_t *perm_src, const float *topk_w, const void *w_down,
+                             const void *ws_down, void *y_perm, void *stream);
+
+/*
+ * Combine: y[t] = y_perm[T*k + t] (shared, if S > 0) + sum_{j<k} y_perm[row_of[t, j]],
+ * summed in fp32 in that order and stored as bf16 [T, H] — the page's
+ * output[mask] += w * expert_out and `shared_expert_out + output`
+ * ("The Evolving Transformer · 07", § 02), as a deterministic gather.
+ */
+MOE_API int moe_combine(const moe_config *cfg, int64_t T, const void *y_perm, const int32_t *row_of,
+                void *y, void *stream);
+
+/*
+ * The whole layer: route, dispatch, experts, combine, on one stream.
+ *   y bf16 [T, H] (output).  topk_idx_out / topk_w_out: optional [T, k]
+ *   copies of the routing (may be NULL).  workspace: at least
+ *   moe_workspace_size(cfg, T) bytes of device memory, 256-byte aligned.
+ */
+MOE_API int moe_forward(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+                const float *e_bias, const void *w_gate, const void *w_up, const void *w_down,
+                const void *ws_gate, const void *ws_up, const void *ws_down, void *y,
+                int32_t *topk_idx_out, float *topk_w_out, void *workspace,
+                size_t workspace_bytes, void *stream);
+
+/* Static text for a status code. */
+MOE_API const char *moe_status_string(int status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: *device_error = 0 when no bounded wait gave up, else a
+ * nonzero code naming the wait.  Returns MOE_OK, MOE_ERR_TIMEOUT when the
+ * word was set, or MOE_ERR_CUDA. */
+MOE_API int moe_device_status(void *stream, int32_t *device_error);
+
+/* Number of kernels this library has launched in this process. */
+MOE_API uint64_t moe_launch_count(void);
+
+/* Failure-detection self-test: launches one kernel whose thread waits, with the
+ * library's bounded-wait routine, on an mbarrier that nothing ever arrives on.
+ * After limit_ns (1 ns .. 10 s) the wait gives up, records code 0x901 in the
+ * device error word and the kernel returns; the GPU context stays usable.
+ * Read the outcome with moe_device_status.  The layer's design has no
+ * counterpart on the pages: it exists to test the timeout path without a fault. */
+MOE_API int moe_selftest_wait_timeout(uint64_t limit_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,63 @@
+"""B200-native DeepSeekMoE layer forward (noaux_tc routing) behind a C ABI.
+
+The compute path is libmoe.so (hand-written CUDA for sm_100a; see
+include/moe.h).  This package only marshals arguments: `abi` mirrors the C
+entry points one to one, and `MoELayer` is the user-facing call that owns the
+weights and a reusable workspace.  PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import abi
+from .abi import (MoEConfig, MoEError, moe_combine, moe_dispatch, moe_experts, moe_forward,
+                  moe_route, workspace_size)
+from .workloads import MoEShape
+
+__all__ = ["MoELayer", "MoEConfig", "MoEError", "MoEShape", "abi", "moe_route", "moe_dispatch",
+           "moe_experts", "moe_combine", "moe_forward", "workspace_size"]
+
+
+class MoELayer:
+    """One DeepSeekMoE feed-forward layer with caller-provided weights.
+
+    Weights (device tensors, nn.Linear (out, in) layout):
+      router_w fp32 [E,H], e_bias fp32 [E], w_gate/w_up bf16 [E,I,H],
+      w_down bf16 [E,H,I], ws_gate/ws_up bf16 [S*I,H], ws_down bf16 [H,S*I].
+    """
+
+    def __init__(self, shape: MoEShape, router_w, e_bias, w_gate, w_up, w_down,
+                 ws_gate=None, ws_up=None, ws_down=None):
+        self.shape = shape
+        self.cfg = MoEConfig.from_shape(shape)
+        self.router_w, self.e_bias = router_w, e_bias
+        self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
+        self.ws_gate, self.ws_up, self.ws_down = ws_gate, ws_up, ws_down
+        self._ws: Optional[torch.Tensor] = None
+
+    @classmethod
+    def from_inputs(cls, shape: MoEShape, inputs: dict) -> "MoELayer":
+        return cls(shape, inputs["router_w"], inputs["e_bias"], inputs["w_gate"], inputs["w_up"],
+                   inputs["w_down"], inputs.get("ws_gate"), inputs.get("ws_up"), inputs.get("ws_down"))
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = workspace_size(self.cfg, T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.w_gate.device)
+        return self._ws
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+        """y [T,H] bf16 = layer(x [T,H] bf16); optionally also returns the routing."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        moe_forward(self.cfg, x, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
+                    self.ws_gate, self.ws_up, self.ws_down, y, topk_idx, topk_w,
+                    self.workspace(T), stream)
+        return y
+
+    __call__ = forward

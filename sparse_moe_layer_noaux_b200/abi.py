@@ -1,0 +1,172 @@
+"""ctypes binding of libmoe (include/moe.h): argument marshalling only.
+
+Every entry point keeps the C name and order of arguments; tensors are torch
+CUDA tensors (PyTorch provides device memory and the stream), turned into
+device pointers here.  There is no fallback: if libmoe.so is missing or a call
+returns an error status, a MoEError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({status_string(status)})")
+
+
+class MoEConfig(ctypes.Structure):
+    """Mirror of `moe_config` (DeepSeek-V3 config field names)."""
+
+    _fields_ = [("hidden_size", ctypes.c_int32), ("n_routed_experts", ctypes.c_int32),
+                ("num_experts_per_tok", ctypes.c_int32), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("moe_intermediate_size", ctypes.c_int32),
+                ("n_shared_experts", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
+                ("routed_scaling_factor", ctypes.c_float)]
+
+    @classmethod
+    def from_shape(cls, s) -> "MoEConfig":
+        return cls(s.hidden_size, s.n_routed_experts, s.num_experts_per_tok, s.n_group,
+                   s.topk_group, s.moe_intermediate_size, s.n_shared_experts,
+                   int(bool(s.norm_topk_prob)), float(s.routed_scaling_factor))
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib():
+    """The loaded libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not found at {LIB_PATH}; build it with "
+                               "`python -m sparse_moe_layer_noaux_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        cfgp = ctypes.POINTER(MoEConfig)
+        i64, sz = ctypes.c_int64, ctypes.c_size_t
+        L.moe_workspace_size.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
+        L.moe_route.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, sz, _P]
+        L.moe_dispatch.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, _P, sz, _P]
+        L.moe_experts.argtypes = [cfgp, i64] + [_P] * 15
+        L.moe_experts_gate_up.argtypes = [cfgp, i64] + [_P] * 10
+        L.moe_experts_down.argtypes = [cfgp, i64] + [_P] * 9
+        L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, _P]
+        L.moe_forward.argtypes = [cfgp, i64] + [_P] * 12 + [_P, sz, _P]
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
+        L.moe_launch_count.argtypes = []
+        L.moe_launch_count.restype = ctypes.c_uint64
+        L.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
+        for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_experts",
+                   "moe_experts_gate_up", "moe_experts_down",
+                   "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout"):
+            getattr(L, fn).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != MOE_OK:
+        raise MoEError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _cfg(cfg):
+    return cfg if isinstance(cfg, MoEConfig) else MoEConfig.from_shape(cfg)
+
+
+def workspace_size(cfg, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(_cfg(cfg)), T, ctypes.byref(n)))
+    return n.value
+
+
+def moe_route(cfg, x, router_w, e_bias, topk_idx, topk_w, workspace, stream=None):
+    _check("moe_route", lib().moe_route(ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w),
+                                        _ptr(e_bias), _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, workspace, stream=None):
+    _check("moe_dispatch", lib().moe_dispatch(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
+        _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_up, w_down,
+                ws_gate, ws_up, ws_down, h_routed, h_shared, y_perm, stream=None):
+    _check("moe_experts", lib().moe_experts(
+        ctypes.byref(_cfg(cfg)), T, _ptr(x), _ptr(x_perm), _ptr(expert_offsets), _ptr(perm_src),
+        _ptr(topk_w), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up),
+        _ptr(ws_down), _ptr(h_routed), _ptr(h_shared), _ptr(y_perm), _stream(stream)))
+
+
+def moe_experts_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed,
+                        h_shared, stream=None):
+    _check("moe_experts_gate_up", lib().moe_experts_gate_up(
+        ctypes.byref(_cfg(cfg)), T, _ptr(x), _ptr(x_perm), _ptr(expert_offsets), _ptr(w_gate),
+        _ptr(w_up), _ptr(ws_gate), _ptr(ws_up), _ptr(h_routed), _ptr(h_shared), _stream(stream)))
+
+
+def moe_experts_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down,
+                     y_perm, stream=None):
+    _check("moe_experts_down", lib().moe_experts_down(
+        ctypes.byref(_cfg(cfg)), T, _ptr(h_routed), _ptr(h_shared), _ptr(expert_offsets),
+        _ptr(perm_src), _ptr(topk_w), _ptr(w_down), _ptr(ws_down), _ptr(y_perm), _stream(stream)))
+
+
+def moe_combine(cfg, T, y_perm, row_of, y, stream=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(row_of),
+                                            _ptr(y), _stream(stream)))
+
+
+def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
+                topk_idx_out=None, topk_w_out=None, workspace=None, stream=None):
+    _check("moe_forward", lib().moe_forward(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
+        _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y),
+        _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (then clear) the device error word."""
+    word = ctypes.c_int32(0)
+    rc = lib().moe_device_status(_stream(stream), ctypes.byref(word))
+    if rc not in (MOE_OK, MOE_ERR_TIMEOUT):
+        raise MoEError("moe_device_status", rc)
+    return word.value
+
+
+def launch_count() -> int:
+    return int(lib().moe_launch_count())
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(int(limit_ns), _stream(stream)))

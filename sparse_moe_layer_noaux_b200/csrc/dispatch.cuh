@@ -1,0 +1,141 @@
+// Token -> expert dispatch: the per-expert mask and gather of "The Evolving
+// Transformer · 07", § 02 (MoE.forward: mask = indices[:, :, k] == i; x[mask]),
+// done for all experts at once as a stable counting sort:
+//   1. count:  per block of kDispTok tokens, how many slots go to each expert;
+//   2. scan:   expert offsets, and each block's starting row inside every expert;
+//   3. place:  stable rank of every slot (ascending (t, j)) -> row_of / perm_src,
+//              then each token's row is copied once from x and written to its k
+//              rows of x_perm with 16-byte vector stores.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace moe {
+
+constexpr int kDispTok = 32;      // tokens per dispatch block
+constexpr int kDispThreads = 256;
+
+__global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(
+    const int32_t* __restrict__ topk_idx, int T, int K, int E, int32_t* __restrict__ block_counts) {
+    extern __shared__ int cnt[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * kDispTok;
+    const int n = min(kDispTok, T - t0) * K;
+    const int32_t* idx = topk_idx + (int64_t)t0 * K;
+    for (int q = threadIdx.x; q < n; q += blockDim.x) atomicAdd(&cnt[idx[q]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        block_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One block; thread e owns expert e (E <= blockDim.x).
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __restrict__ block_counts,
+                                                            int nb, int E,
+                                                            int32_t* __restrict__ block_base,
+                                                            int32_t* __restrict__ offsets) {
+    __shared__ int warp_sums[8];
+    const int e = threadIdx.x;
+    int total = 0;
+    if (e < E) {
+        int b = 0;
+        for (; b + 4 <= nb; b += 4) {
+            const int c0 = block_counts[(int64_t)(b + 0) * E + e];
+            const int c1 = block_counts[(int64_t)(b + 1) * E + e];
+            const int c2 = block_counts[(int64_t)(b + 2) * E + e];
+            const int c3 = block_counts[(int64_t)(b + 3) * E + e];
+            total += c0 + c1 + c2 + c3;
+        }
+        for (; b < nb; ++b) total += block_counts[(int64_t)b * E + e];
+    }
+    // Exclusive scan of the totals over experts.
+    const int lane = e & 31, warp = e >> 5;
+    int incl = total;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int warp_base = 0;
+    for (int w = 0; w < warp; ++w) warp_base += warp_sums[w];
+    const int excl = warp_base + incl - total;
+    if (e < E) offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + total;
+    if (e < E) {
+        int run = excl;
+        for (int b = 0; b < nb; ++b) {
+            const int c = block_counts[(int64_t)b * E + e];
+            block_base[(int64_t)b * E + e] = run;
+            run += c;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
+    const int32_t* __restrict__ topk_idx, int T, int K, int E, int H,
+    const int32_t* __restrict__ block_base, const __nv_bfloat16* __restrict__ x,
+    __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ perm_src,
+    int32_t* __restrict__ row_of) {
+    extern __shared__ int smem_i[];
+    int* run = smem_i;              // [E] next free row of each expert for this block
+    int* rows = smem_i + E;         // [kDispTok * K] destination rows of this block's slots
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kDispThreads / 32;
+    for (int e = tid; e < E; e += blockDim.x) run[e] = block_base[(int64_t)blockIdx.x * E + e];
+    __syncthreads();
+    const int t0 = blockIdx.x * kDispTok;
+    const int ntok = min(kDispTok, T - t0);
+    const int n = ntok * K;
+    const int64_t q0 = (int64_t)t0 * K;
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    for (int r0 = 0; r0 < n; r0 += kDispThreads) {
+        const int q = r0 + tid;
+        const bool valid = q < n;
+        const int e = valid ? topk_idx[q0 + q] : -1 - lane;  // invalid lanes never match
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int lrank = __popc(peers & lt_mask);
+        const bool leader = lrank == 0;
+        const int wcnt = __popc(peers);
+        int row = 0;
+        // Warps take their turn in order, so ranks follow ascending slot index.
+        for (int w = 0; w < kWarps; ++w) {
+            if (warp == w && valid) {
+                const int base = run[e];
+                __syncwarp(peers);
+                if (leader) run[e] = base + wcnt;
+                row = base + lrank;
+            }
+            __syncthreads();
+        }
+        if (valid) {
+            rows[q] = row;
+            row_of[q0 + q] = row;
+            perm_src[row] = (int32_t)(q0 + q);
+        }
+    }
+    __syncthreads();
+
+    // Copy: each warp moves whole tokens; one 16-byte load feeds K stores, four
+    // loads in flight per lane.
+    const int chunks = H / 8;
+    for (int tl = warp; tl < ntok; tl += kWarps) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + tl) * H);
+        for (int c0 = lane; c0 < chunks; c0 += 128) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c0 + 32 * u < chunks) v[u] = src[c0 + 32 * u];
+            for (int j = 0; j < K; ++j) {
+                uint4* dst = reinterpret_cast<uint4*>(x_perm + (int64_t)rows[tl * K + j] * H);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (c0 + 32 * u < chunks) dst[c0 + 32 * u] = v[u];
+            }
+        }
+    }
+}
+
+}  // namespace moe

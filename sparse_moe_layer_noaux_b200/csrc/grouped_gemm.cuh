@@ -1,0 +1,411 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA.  One persistent CTA per SM walks a static schedule of output
+// tiles over variable-length expert segments read on the device (no host sync):
+//   segment 0        the shared expert over all T tokens (when S > 0);
+//   segment 1 + e    routed expert e, rows expert_offsets[e] .. expert_offsets[e+1].
+// Two instantiations:
+//   kSwiGLU  h = silu(A Wg^T) * (A Wu^T)   — gate and up tiles side by side in one
+//            N = 256 accumulator (128 gate columns | 128 up columns), fused epilogue;
+//   kDown    y = w_row * (h Wd^T)           — N = 256, routing weight in the epilogue.
+// ("The Evolving Transformer · 07", § 02: expert(x[mask]) is a SwiGLU FFN; its
+// output is multiplied by the routing weight.)
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// the MMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Shared memory: kStages x (A 128x64 + B 256x64) bf16 tiles in the 128-byte
+// swizzle layout; TMEM: two 256-column fp32 accumulators so the epilogue of one
+// tile overlaps the main loop of the next.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;           // rows (tokens) per tile
+constexpr int kBN = 256;           // accumulator columns per tile
+constexpr int kBK = 64;            // K per stage (one 128-byte swizzle row of bf16)
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kMaxSeg = 258;       // 256 experts + shared
+constexpr uint32_t kTileABytes = kBM * kBK * 2;   // 16 KB
+constexpr uint32_t kTileBBytes = kBN * kBK * 2;   // 32 KB
+constexpr uint32_t kTmemCols = 512;               // 2 accumulators x 256 columns
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
+
+enum { kSwiGLU = 0, kDown = 1 };
+
+// Device error word (set by a bounded wait that gave up; read by the host).
+__device__ unsigned int g_moe_error;
+
+struct GemmParams {
+    const int32_t* offsets;      // [E+1] routed row offsets
+    int E;
+    int T;                       // rows of the shared segment
+    int has_shared;
+    int n_tiles_routed, n_tiles_shared;   // output column tiles
+    int kb_routed, kb_shared;             // K blocks of 64
+    int n_valid_routed, n_valid_shared;   // valid output columns
+    int b_rows_per_expert;                // rows of one expert in the routed B map
+    __nv_bfloat16* out_routed;            // row r of routed segment -> out_routed + r*ld
+    int64_t ld_routed;
+    __nv_bfloat16* out_shared;            // row t of the shared segment
+    int64_t ld_shared;
+    const int32_t* perm_src;              // kDown: routed row -> slot
+    const float* topk_w;                  // kDown: slot -> routing weight
+};
+
+struct TileInfo {
+    int seg;        // 0 = shared (if present) else routed
+    int routed;     // 1 if routed expert segment
+    int expert;
+    int m, n;       // tile coordinates inside the segment
+    int rows;       // rows of the segment
+    int row0;       // first row of the segment in the A / output row space
+    int kb;         // K blocks
+};
+
+struct GemmSmem {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+    int total_tiles;
+    int nseg;
+    int seg_row0[kMaxSeg];
+    int seg_rows[kMaxSeg];
+    int tile_start[kMaxSeg + 1];
+};
+
+__device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_moe_error, 0u, code); }
+
+// Wait until the phase with parity `parity` of `bar` has completed.  Gives up
+// (returns false) when the CTA is aborting or after kWaitLimitNs.
+__device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned code, uint64_t limit_ns = kWaitLimitNs) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((n & 63u) == 0) {
+            if (abort_flag && *abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > limit_ns) {
+                record_error(code);
+                if (abort_flag) *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ TileInfo decode_tile(const GemmSmem& s, const GemmParams& p, int tile) {
+    int lo = 0, hi = s.nseg - 1;  // largest seg with tile_start[seg] <= tile
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.tile_start[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    TileInfo ti;
+    ti.seg = lo;
+    ti.routed = !(p.has_shared && lo == 0);
+    ti.expert = lo - p.has_shared;
+    ti.rows = s.seg_rows[lo];
+    ti.row0 = s.seg_row0[lo];
+    const int mt = (ti.rows + kBM - 1) / kBM;
+    const int local = tile - s.tile_start[lo];
+    ti.n = local / mt;
+    ti.m = local - ti.n * mt;
+    ti.kb = ti.routed ? p.kb_routed : p.kb_shared;
+    return ti;
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives on; after limit_ns it records `code` in the device error word and the
+// kernel returns normally.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, unsigned code) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(ptx::smem_u32(&bar), 1);
+        ptx::fence_barrier_init();
+        abort_flag = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) bounded_wait(ptx::smem_u32(&bar), 0, &abort_flag, code, limit_ns);
+}
+
+template <int kEpi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
+                        const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB2_r,
+                        const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmB2_s,
+                        const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    // Operand tiles need 1024-byte alignment for the 128-byte swizzle pattern.
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t* smemA = tiles;
+    uint8_t* smemB = tiles + kStages * kTileABytes;
+    GemmSmem& S = *reinterpret_cast<GemmSmem*>(tiles + kStages * (kTileABytes + kTileBBytes));
+    volatile int* abort_flag = &S.abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- set-up: barriers, TMEM, segment table ----
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&S.full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&S.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_u32(&S.tmem_full[i]), 1);
+            ptx::mbar_init(ptx::smem_u32(&S.tmem_empty[i]), 4);
+        }
+        ptx::mbar_init(ptx::smem_u32(&S.mma_done), 1);
+        ptx::fence_barrier_init();
+        S.abort_flag = 0;
+        ptx::prefetch_tensormap(&tmA_r);
+        ptx::prefetch_tensormap(&tmB_r);
+        if (kEpi == kSwiGLU) ptx::prefetch_tensormap(&tmB2_r);
+        if (p.has_shared) {
+            ptx::prefetch_tensormap(&tmA_s);
+            ptx::prefetch_tensormap(&tmB_s);
+            if (kEpi == kSwiGLU) ptx::prefetch_tensormap(&tmB2_s);
+        }
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(&S.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 2) {
+        // Segment table and exclusive prefix of tiles per segment (one warp scan).
+        const int nseg = p.E + p.has_shared;
+        const int per = (nseg + 31) / 32;
+        const int s_begin = lane * per;
+        int local = 0;
+        for (int i = 0; i < per; ++i) {
+            const int sg = s_begin + i;
+            if (sg >= nseg) break;
+            int rows, row0, ntl;
+            if (p.has_shared && sg == 0) {
+                rows = p.T; row0 = 0; ntl = p.n_tiles_shared;
+            } else {
+                const int e = sg - p.has_shared;
+                row0 = p.offsets[e];
+                rows = p.offsets[e + 1] - row0;
+                ntl = p.n_tiles_routed;
+            }
+            S.seg_rows[sg] = rows;
+            S.seg_row0[sg] = row0;
+            local += ((rows + kBM - 1) / kBM) * ntl;
+        }
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        int run = incl - local;
+        for (int i = 0; i < per; ++i) {
+            const int sg = s_begin + i;
+            if (sg >= nseg) break;
+            S.tile_start[sg] = run;
+            const int ntl = (p.has_shared && sg == 0) ? p.n_tiles_shared : p.n_tiles_routed;
+            run += ((S.seg_rows[sg] + kBM - 1) / kBM) * ntl;
+        }
+        if (lane == 31) {
+            S.total_tiles = incl;
+            S.nseg = nseg;
+            S.tile_start[nseg] = incl;
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+
+    const int total = S.total_tiles;
+    const uint32_t tmem_base = S.tmem_base;
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            // Activation tiles are re-read by every column tile of their segment:
+            // keep them in L2 preferentially.  Weight tiles are shared by the CTAs
+            // working on the segment's row tiles at the same time: default policy.
+            const uint64_t pol_a = ptx::policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_parity = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(S, p, tile);
+                const CUtensorMap* mA = ti.routed ? &tmA_r : &tmA_s;
+                const CUtensorMap* mB = ti.routed ? &tmB_r : &tmB_s;
+                const CUtensorMap* mB2 = ti.routed ? &tmB2_r : &tmB2_s;
+                const int a_row = ti.row0 + ti.m * kBM;
+                const int b_base = ti.routed ? ti.expert * p.b_rows_per_expert : 0;
+                for (int kb = 0; kb < ti.kb; ++kb) {
+                    if (!bounded_wait(ptx::smem_u32(&S.empty[stage]), phase ^ 1u, abort_flag, 0x101u)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full = ptx::smem_u32(&S.full[stage]);
+                    ptx::mbar_arrive_expect_tx(full, kTileABytes + kTileBBytes);
+                    const uint32_t a_dst = ptx::smem_u32(smemA + stage * kTileABytes);
+                    const uint32_t b_dst = ptx::smem_u32(smemB + stage * kTileBBytes);
+                    ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
+                    if (kEpi == kSwiGLU) {
+                        const int b_row = b_base + ti.n * (kBN / 2);
+                        ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
+                        ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row);
+                    } else {
+                        const int b_row = b_base + ti.n * kBN;
+                        ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
+                    }
+                    issued_mask |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {
+                // Let this CTA's copies in flight land before the CTA exits.
+                for (int s = 0; s < kStages; ++s)
+                    if (issued_mask & (1u << s))
+                        bounded_wait(ptx::smem_u32(&S.full[s]), (issued_parity >> s) & 1u, nullptr, 0x102u);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(S, p, tile);
+                if (!bounded_wait(ptx::smem_u32(&S.tmem_empty[acc]), acc_phase ^ 1u, abort_flag, 0x201u)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+                for (int kb = 0; kb < ti.kb; ++kb) {
+                    if (!bounded_wait(ptx::smem_u32(&S.full[stage]), phase, abort_flag, 0x202u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_u32(smemA + stage * kTileABytes);
+                    const uint32_t b_addr = ptx::smem_u32(smemB + stage * kTileBBytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint64_t ad = ptx::sw128_kmajor_desc(a_addr + k * 32);
+                        const uint64_t bd = ptx::sw128_kmajor_desc(b_addr + k * 32);
+                        ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(ptx::smem_u32(&S.empty[stage]));
+                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::mma_commit(ptx::smem_u32(&S.tmem_full[acc]));
+                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            }
+            // Every MMA issued by this thread is complete once mma_done flips.
+            ptx::mma_commit(ptx::smem_u32(&S.mma_done));
+            bounded_wait(ptx::smem_u32(&S.mma_done), 0, nullptr, 0x203u);
+        }
+    } else {
+        // ================= epilogue (warps 2..5) =================
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(S, p, tile);
+            const bool got = bounded_wait(ptx::smem_u32(&S.tmem_full[acc]), acc_phase, abort_flag, 0x301u);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, got)) break;
+            ptx::tc_fence_after();
+            const int r_local = ti.m * kBM + quarter * 32 + lane;
+            const bool row_ok = r_local < ti.rows;
+            const int64_t grow = (int64_t)ti.row0 + r_local;
+            const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) +
+                                   (static_cast<uint32_t>(quarter * 32) << 16);
+            if (kEpi == kSwiGLU) {
+                const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
+                __nv_bfloat16* out = ti.routed ? p.out_routed + grow * p.ld_routed
+                                               : p.out_shared + grow * p.ld_shared;
+#pragma unroll 1
+                for (int c = 0; c < (kBN / 2) / 32; ++c) {
+                    __syncwarp();
+                    uint32_t g[32], u[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
+                    ptx::tmem_ld_32x32b_x32(taddr + kBN / 2 + c * 32, u);
+                    ptx::tmem_wait_ld();
+                    const int col = ti.n * (kBN / 2) + c * 32;
+                    if (row_ok && col < n_valid) {
+                        uint4 pk[4];
+                        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(pk);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+                            const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                            h2[q] = __floats2bfloat162_rn(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) dst[q] = pk[q];
+                    }
+                }
+            } else {
+                const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
+                __nv_bfloat16* out = ti.routed ? p.out_routed + grow * p.ld_routed
+                                               : p.out_shared + grow * p.ld_shared;
+                float wrow = 1.0f;
+                if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
+#pragma unroll 1
+                for (int c = 0; c < kBN / 32; ++c) {
+                    __syncwarp();
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    ptx::tmem_wait_ld();
+                    const int col = ti.n * kBN + c * 32;
+                    if (row_ok && col < n_valid) {
+                        uint4 pk[4];
+                        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(pk);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            h2[q] = __floats2bfloat162_rn(__uint_as_float(v[2 * q]) * wrow,
+                                                          __uint_as_float(v[2 * q + 1]) * wrow);
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) dst[q] = pk[q];
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&S.tmem_empty[acc]));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    // ---- teardown ----
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,528 @@
+// libmoe: C ABI of the DeepSeekMoE layer forward on B200 (see include/moe.h).
+// Host side: argument validation, workspace carving, TMA tensor maps, launches.
+// All kernels of the library are in this translation unit.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <initializer_list>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+#include "combine.cuh"
+#include "dispatch.cuh"
+#include "grouped_gemm.cuh"
+#include "router.cuh"
+
+namespace moe {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline void count_launch(int n = 1) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// --------------------------------------------------------------- validation
+int validate_cfg(const moe_config* c, int64_t T) {
+    if (!c || T < 0) return MOE_ERR_INVALID_ARG;
+    const int H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int G = c->n_group, TG = c->topk_group, I = c->moe_intermediate_size;
+    if (H <= 0 || E <= 0 || G <= 0 || I <= 0 || c->n_shared_experts < 0) return MOE_ERR_INVALID_ARG;
+    if (E % G != 0 || TG < 1 || TG > G || K < 1 || K > TG * (E / G)) return MOE_ERR_INVALID_ARG;
+    if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1) return MOE_ERR_INVALID_ARG;
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+    if (H % 64 != 0 || I % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (E > 256 || G > 32 || K > 32) return MOE_ERR_UNSUPPORTED;
+    const int64_t SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    if (SI > (1 << 24) || static_cast<int64_t>(E) * I > (1ll << 31) ||
+        static_cast<int64_t>(E) * H > (1ll << 31))
+        return MOE_ERR_UNSUPPORTED;
+    if (T * K + T >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+// --------------------------------------------------------------- router sizing
+struct RouterPlan {
+    int nsplit, split_len;
+};
+
+// The split count depends only on the shape (not on the device), so the
+// workspace size computed before launch always matches what the launch uses.
+constexpr int kRouterTargetBlocks = 296;  // two waves of blocks on 148 SMs
+
+RouterPlan plan_router(int T, int E, int H) {
+    const int tiles = ((T + kRT - 1) / kRT) * ((E + kRE - 1) / kRE);
+    int want = (kRouterTargetBlocks + tiles - 1) / tiles;
+    const int max_split = H / 256 > 0 ? H / 256 : 1;
+    if (want > max_split) want = max_split;
+    if (want < 1) want = 1;
+    int split_len = (H + want - 1) / want;
+    split_len = (split_len + kRK - 1) / kRK * kRK;
+    RouterPlan r;
+    r.split_len = split_len;
+    r.nsplit = (H + split_len - 1) / split_len;
+    return r;
+}
+
+// --------------------------------------------------------------- device info
+struct DeviceInfo {
+    int num_sms = 0;
+    bool attrs_set = false;
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+int device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.attrs_set) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int smem = static_cast<int>(1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem));
+        static_assert(1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem) <= 227 * 1024,
+                      "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.attrs_set = true;
+    }
+    *out = &d;
+    return MOE_OK;
+}
+
+// --------------------------------------------------------------- workspace
+struct Workspace {
+    float* router_part;       // [nsplit, T, E]
+    int32_t* block_counts;    // [nb, E]
+    int32_t* block_base;      // [nb, E]
+    int32_t* topk_idx;        // [T, k]
+    float* topk_w;            // [T, k]
+    int32_t* offsets;         // [E + 1]
+    int32_t* perm_src;        // [T*k]
+    int32_t* row_of;          // [T, k]
+    __nv_bfloat16* x_perm;    // [T*k, H]
+    __nv_bfloat16* h_routed;  // [T*k, I]
+    __nv_bfloat16* h_shared;  // [T, S*I]
+    __nv_bfloat16* y_perm;    // [T*k + T, H]
+    size_t bytes;
+};
+
+Workspace carve(const moe_config* c, int64_t T, uint8_t* base) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const RouterPlan rp = plan_router(static_cast<int>(T), static_cast<int>(E), static_cast<int>(H));
+    const int64_t nb = (T + kDispTok - 1) / kDispTok;
+    Workspace w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    w.router_part = reinterpret_cast<float*>(take(sizeof(float) * rp.nsplit * T * E));
+    w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.topk_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.topk_w = reinterpret_cast<float*>(take(sizeof(float) * T * K));
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));
+    w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.row_of = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * H));
+    w.h_routed = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * I));
+    w.h_shared = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
+    w.y_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * (T * K + T) * H));
+    w.bytes = off;
+    return w;
+}
+
+size_t workspace_bytes_for(const moe_config* c, int64_t T) { return carve(c, T, nullptr).bytes; }
+
+// --------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [rows, cols]; box = box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    if (rows == 0) rows = 1;  // never addressed: the segment has no tiles
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------- stages
+int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
+                 int32_t* idx, float* w, float* part, cudaStream_t st) {
+    const int H = c->hidden_size, E = c->n_routed_experts;
+    const RouterPlan rp = plan_router(static_cast<int>(T), E, H);
+    dim3 g1((E + kRE - 1) / kRE, static_cast<unsigned>((T + kRT - 1) / kRT), rp.nsplit);
+    router_logits_kernel<<<g1, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, part,
+                                              static_cast<int>(T), E, H, rp.split_len);
+    RouteArgs a;
+    a.part = part;
+    a.nsplit = rp.nsplit;
+    a.T = static_cast<int>(T);
+    a.E = E;
+    a.G = c->n_group;
+    a.TG = c->topk_group;
+    a.K = c->num_experts_per_tok;
+    a.norm = c->norm_topk_prob;
+    a.scale = c->routed_scaling_factor;
+    a.bias = bias;
+    a.topk_idx = idx;
+    a.topk_w = w;
+    const unsigned g2 = static_cast<unsigned>((T + 7) / 8);
+    if (E <= 32) router_select_kernel<1><<<g2, 256, 0, st>>>(a);
+    else if (E <= 64) router_select_kernel<2><<<g2, 256, 0, st>>>(a);
+    else if (E <= 128) router_select_kernel<4><<<g2, 256, 0, st>>>(a);
+    else router_select_kernel<8><<<g2, 256, 0, st>>>(a);
+    count_launch(2);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_dispatch(const moe_config* c, int64_t T, const void* x, const int32_t* idx, int32_t* offsets,
+                    void* x_perm, int32_t* perm_src, int32_t* row_of, int32_t* block_counts,
+                    int32_t* block_base, cudaStream_t st) {
+    const int E = c->n_routed_experts, K = c->num_experts_per_tok, H = c->hidden_size;
+    const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
+                                                                      block_counts);
+    dispatch_scan_kernel<<<1, 256, 0, st>>>(block_counts, nb, E, block_base, offsets);
+    const size_t smem = sizeof(int) * (E + kDispTok * K);
+    dispatch_place_kernel<<<nb, kDispThreads, smem, st>>>(
+        idx, static_cast<int>(T), K, E, H, block_base, static_cast<const __nv_bfloat16*>(x),
+        static_cast<__nv_bfloat16*>(x_perm), perm_src, row_of);
+    count_launch(3);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Persistent grid: one CTA per SM, fewer when there cannot be that many tiles.
+int64_t gemm_grid(int64_t T, int64_t R, int64_t E, int64_t n_cols_max, int has_shared, int num_sms,
+                  int col_tile) {
+    const int64_t m_tiles_bound = (R + kBM - 1) / kBM + E + (has_shared ? (T + kBM - 1) / kBM : 0);
+    const int64_t n_tiles_bound = (n_cols_max + col_tile - 1) / col_tile;
+    int64_t grid = m_tiles_bound * n_tiles_bound;
+    if (grid > num_sms) grid = num_sms;
+    if (grid < 1) grid = 1;
+    return grid;
+}
+
+constexpr size_t kGemmSmemBytes = 1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem);
+
+// K4: h = silu(A Wg^T) * (A Wu^T) for routed rows (A = x_perm) and shared rows (A = x).
+int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_perm, const int32_t* offsets,
+                   const void* w_gate, const void* w_up, const void* ws_gate, const void* ws_up,
+                   void* h_routed, void* h_shared, int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int64_t R = T * K;
+    const int has_shared = SI > 0 ? 1 : 0;
+    CUtensorMap a_r, a_s, b_r, b2_r, b_s, b2_s;
+    bool ok = make_map(&a_r, x_perm, R, H, kBM) && make_map(&b_r, w_gate, E * I, H, kBN / 2) &&
+              make_map(&b2_r, w_up, E * I, H, kBN / 2);
+    if (has_shared)
+        ok = ok && make_map(&a_s, x, T, H, kBM) && make_map(&b_s, ws_gate, SI, H, kBN / 2) &&
+             make_map(&b2_s, ws_up, SI, H, kBN / 2);
+    else {
+        a_s = a_r; b_s = b_r; b2_s = b2_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParams p{};
+    p.offsets = offsets;
+    p.E = static_cast<int>(E);
+    p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = static_cast<int>((I + kBN / 2 - 1) / (kBN / 2));
+    p.n_tiles_shared = static_cast<int>((SI + kBN / 2 - 1) / (kBN / 2));
+    p.kb_routed = static_cast<int>(H / kBK);
+    p.kb_shared = static_cast<int>(H / kBK);
+    p.n_valid_routed = static_cast<int>(I);
+    p.n_valid_shared = static_cast<int>(SI);
+    p.b_rows_per_expert = static_cast<int>(I);
+    p.out_routed = static_cast<__nv_bfloat16*>(h_routed);
+    p.ld_routed = I;
+    p.out_shared = static_cast<__nv_bfloat16*>(h_shared);
+    p.ld_shared = SI;
+    const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
+    grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
+        a_r, a_s, b_r, b2_r, b_s, b2_s, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// K5: y_perm = w * (h Wd^T) for routed rows, h_shared Wsd^T for the shared rows.
+int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void* h_shared,
+                const int32_t* offsets, const int32_t* perm_src, const float* topk_w, const void* w_down,
+                const void* ws_down, void* y_perm, int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int64_t R = T * K;
+    const int has_shared = SI > 0 ? 1 : 0;
+    CUtensorMap a_r, a_s, b_r, b_s;
+    bool ok = make_map(&a_r, h_routed, R, I, kBM) && make_map(&b_r, w_down, E * H, I, kBN);
+    if (has_shared)
+        ok = ok && make_map(&a_s, h_shared, T, SI, kBM) && make_map(&b_s, ws_down, H, SI, kBN);
+    else {
+        a_s = a_r; b_s = b_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParams p{};
+    p.offsets = offsets;
+    p.E = static_cast<int>(E);
+    p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = static_cast<int>((H + kBN - 1) / kBN);
+    p.n_tiles_shared = static_cast<int>((H + kBN - 1) / kBN);
+    p.kb_routed = static_cast<int>(I / kBK);
+    p.kb_shared = static_cast<int>(SI / kBK);
+    p.n_valid_routed = static_cast<int>(H);
+    p.n_valid_shared = static_cast<int>(H);
+    p.b_rows_per_expert = static_cast<int>(H);
+    p.out_routed = static_cast<__nv_bfloat16*>(y_perm);
+    p.ld_routed = H;
+    p.out_shared = static_cast<__nv_bfloat16*>(y_perm) + R * H;
+    p.ld_shared = H;
+    p.perm_src = perm_src;
+    p.topk_w = topk_w;
+    const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
+    grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
+        a_r, a_s, b_r, b_r, b_s, b_s, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
+                   cudaStream_t st) {
+    const unsigned g = static_cast<unsigned>((T + 7) / 8);
+    combine_kernel<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm), row_of,
+                                      static_cast<int>(T), c->num_experts_per_tok, c->hidden_size,
+                                      c->n_shared_experts > 0 ? 1 : 0, static_cast<__nv_bfloat16*>(y));
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_workspace_size(const moe_config* cfg, int64_t T, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    *bytes = workspace_bytes_for(cfg, T);
+    return MOE_OK;
+}
+
+int moe_route(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
+              int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!x || !router_w || !e_bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < workspace_bytes_for(cfg, T)) return MOE_ERR_WORKSPACE;
+    Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
+    return launch_route(cfg, T, x, router_w, e_bias, topk_idx, topk_w, w.router_part,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(const moe_config* cfg, int64_t T, const void* x, const int32_t* topk_idx,
+                 int32_t* expert_offsets, void* x_perm, int32_t* perm_src, int32_t* row_of, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // No rows: every expert segment is empty.
+        if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (cfg->n_routed_experts + 1), st) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!x || !topk_idx || !x_perm || !perm_src || !row_of) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < workspace_bytes_for(cfg, T)) return MOE_ERR_WORKSPACE;
+    Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
+    return launch_dispatch(cfg, T, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, w.block_counts,
+                           w.block_base, st);
+}
+
+namespace {
+int check_ptrs(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!p) return MOE_ERR_INVALID_ARG;
+    for (const void* p : ps)
+        if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+}  // namespace
+
+int moe_experts_gate_up(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
+                        const int32_t* expert_offsets, const void* w_gate, const void* w_up, const void* ws_gate,
+                        const void* ws_up, void* h_routed, void* h_shared, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({x_perm, w_gate, w_up, h_routed})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({x, ws_gate, ws_up, h_shared})) != MOE_OK) return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    return launch_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared,
+                          d->num_sms, static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts_down(const moe_config* cfg, int64_t T, const void* h_routed, const void* h_shared,
+                     const int32_t* expert_offsets, const int32_t* perm_src, const float* topk_w,
+                     const void* w_down, const void* ws_down, void* y_perm, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!expert_offsets || !perm_src || !topk_w) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({h_routed, w_down, y_perm})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({h_shared, ws_down})) != MOE_OK) return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
+                       d->num_sms, static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
+                const int32_t* expert_offsets, const int32_t* perm_src, const float* topk_w, const void* w_gate,
+                const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                const void* ws_down, void* h_routed, void* h_shared, void* y_perm, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!expert_offsets || !perm_src || !topk_w) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({x_perm, w_gate, w_up, w_down, h_routed, y_perm})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({x, ws_gate, ws_up, ws_down, h_shared})) != MOE_OK)
+        return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((v = launch_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared,
+                            d->num_sms, st)) != MOE_OK)
+        return v;
+    return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
+                       d->num_sms, st);
+}
+
+int moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
+                void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !row_of || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
+    return launch_combine(cfg, T, y_perm, row_of, y, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
+                const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                const void* ws_up, const void* ws_down, void* y, int32_t* topk_idx_out, float* topk_w_out,
+                void* workspace, size_t workspace_bytes, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    const bool sh = cfg->n_shared_experts > 0;
+    if (!x || !router_w || !e_bias || !w_gate || !w_up || !w_down || !y) return MOE_ERR_INVALID_ARG;
+    if (sh && (!ws_gate || !ws_up || !ws_down)) return MOE_ERR_INVALID_ARG;
+    const void* al[] = {x, router_w, w_gate, w_up, w_down, y};
+    for (const void* p : al)
+        if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    if (sh) {
+        const void* al2[] = {ws_gate, ws_up, ws_down};
+        for (const void* p : al2)
+            if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+    }
+    if (!workspace || workspace_bytes < workspace_bytes_for(cfg, T) || !aligned16(workspace))
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
+    int32_t* idx = topk_idx_out ? topk_idx_out : w.topk_idx;
+    float* tw = topk_w_out ? topk_w_out : w.topk_w;
+    if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, st)) != MOE_OK)
+        return v;
+    if ((v = launch_dispatch(cfg, T, x, idx, w.offsets, w.x_perm, w.perm_src, w.row_of, w.block_counts,
+                             w.block_base, st)) != MOE_OK)
+        return v;
+    if ((v = launch_gate_up(cfg, T, x, w.x_perm, w.offsets, w_gate, w_up, ws_gate, ws_up, w.h_routed,
+                            w.h_shared, d->num_sms, st)) != MOE_OK)
+        return v;
+    if ((v = launch_down(cfg, T, w.h_routed, w.h_shared, w.offsets, w.perm_src, tw, w_down, ws_down, w.y_perm,
+                         d->num_sms, st)) != MOE_OK)
+        return v;
+    return launch_combine(cfg, T, w.y_perm, w.row_of, y, st);
+}
+
+const char* moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+        default: return "unknown status";
+    }
+}
+
+int moe_device_status(void* stream, int32_t* device_error) {
+    if (!device_error) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int word = 0, zero = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&word, g_moe_error, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(g_moe_error, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+    *device_error = static_cast<int32_t>(word);
+    return word ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+    wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, 0x901u);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,227 @@
+// Router of the DeepSeekMoE layer (noaux_tc): logits, sigmoid scores, biased
+// scores, group top-2 scores, group top-k, expert top-k, weights.
+// "DeepSeekV3.2-Tiered-Implementations" README, § Architecture (sigmoid routing
+// with correction bias, n_group / topk_group); "The Evolving Transformer · 07",
+// § 02 (router(x) -> weights, indices) and § 06 (bias steers selection only).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// K1 (CUDA cores): partial logits P[split][t][e] = sum_{h in split} x[t,h] * Wr[e,h]
+// in fp32.  Block tile 128 tokens x 64 experts, 256 threads, 8x4 outputs each;
+// the hidden axis is cut into `nsplit` slices when T is small so that the grid
+// still covers the GPU.  Partials are summed by the select kernel in split
+// order, so the result is deterministic.
+// ---------------------------------------------------------------------------
+constexpr int kRT = 128, kRE = 64, kRK = 32;
+
+__global__ void __launch_bounds__(256) router_logits_kernel(
+    const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr, float* __restrict__ part,
+    int T, int E, int H, int split_len) {
+    __shared__ float xs[kRK][kRT + 4];
+    __shared__ float ws[kRK][kRE + 4];
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.y * kRT, e0 = blockIdx.x * kRE;
+    const int h_begin = blockIdx.z * split_len;
+    const int h_end = min(H, h_begin + split_len);
+    const int tr = tid / 16;  // 16 row groups of 8 tokens
+    const int tc = tid % 16;  // 16 col groups of 4 experts
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+    for (int h0 = h_begin; h0 < h_end; h0 += kRK) {
+        // x tile: 128 x 32 bf16 = 512 chunks of 8 elements.
+        for (int c = tid; c < kRT * kRK / 8; c += 256) {
+            const int r = c / (kRK / 8), kc = (c % (kRK / 8)) * 8;
+            const int t = t0 + r;
+            float v[8];
+            if (t < T && h0 + kc < h_end) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(x + (int64_t)t * H + h0 + kc);
+                const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(p[q]);
+                    v[2 * q] = f.x;
+                    v[2 * q + 1] = f.y;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xs[kc + q][r] = v[q];
+        }
+        // Wr tile: 64 x 32 fp32 = 512 chunks of 4.
+        for (int c = tid; c < kRE * kRK / 4; c += 256) {
+            const int r = c / (kRK / 4), kc = (c % (kRK / 4)) * 4;
+            const int e = e0 + r;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e < E && h0 + kc < h_end)
+                v = *reinterpret_cast<const float4*>(wr + (int64_t)e * H + h0 + kc);
+            ws[kc + 0][r] = v.x;
+            ws[kc + 1][r] = v.y;
+            ws[kc + 2][r] = v.z;
+            ws[kc + 3][r] = v.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kRK; ++kk) {
+            float a[8], b[4];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] = xs[kk][tr * 8 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = ws[kk][tc * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    float* out = part + (int64_t)blockIdx.z * T * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + tr * 8 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + tc * 4 + j;
+            if (e < E) out[(int64_t)t * E + e] = acc[i][j];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K2: one warp per token.  Expert e lives in lane e % 32, slot e / 32.
+// ---------------------------------------------------------------------------
+struct RouteArgs {
+    const float* part;   // [nsplit][T][E] partial logits
+    int nsplit;
+    int T, E, G, TG, K;
+    int norm;
+    float scale;
+    const float* bias;   // [E]
+    int32_t* topk_idx;   // [T][K]
+    float* topk_w;       // [T][K]
+};
+
+// (value, index) order: larger value first, lower index on equal values.
+__device__ __forceinline__ bool route_beats(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    const int E = a.E, gsize = E / a.G;
+
+    float s[EPL], cand[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        s[i] = 0.f;
+        cand[i] = -CUDART_INF_F;
+        if (e < E) {
+            float l = 0.f;
+            for (int p = 0; p < a.nsplit; ++p) l += a.part[((int64_t)p * a.T + t) * E + e];
+            s[i] = 1.0f / (1.0f + expf(-l));
+            cand[i] = s[i] + a.bias[e];  // biased score b_e
+        }
+    }
+
+    // Group score: sum of the two largest biased scores of the group.
+    float my_gscore = -CUDART_INF_F;  // lane g holds group g's score
+    for (int g = 0; g < a.G; ++g) {
+        float m1 = -CUDART_INF_F, m2 = -CUDART_INF_F;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && e / gsize == g) {
+                const float v = cand[i];
+                if (v > m1) { m2 = m1; m1 = v; }
+                else if (v > m2) { m2 = v; }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float o1 = __shfl_xor_sync(0xffffffffu, m1, off);
+            const float o2 = __shfl_xor_sync(0xffffffffu, m2, off);
+            const float n1 = fmaxf(m1, o1);
+            const float n2 = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
+            m1 = n1;
+            m2 = n2;
+        }
+        const float gs = gsize >= 2 ? m1 + m2 : m1;
+        if (lane == g) my_gscore = gs;
+    }
+
+    // Keep the topk_group best groups (lower group index on equal scores).
+    int rank = 0;
+    for (int g = 0; g < a.G; ++g) {
+        const float v = __shfl_sync(0xffffffffu, my_gscore, g);
+        if (route_beats(v, g, my_gscore, lane)) ++rank;
+    }
+    const unsigned kept = __ballot_sync(0xffffffffu, lane < a.G && rank < a.TG);
+
+    // Experts of dropped groups are excluded from the top-k.
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e >= E || !((kept >> (e / gsize)) & 1u)) cand[i] = -CUDART_INF_F;
+    }
+
+    float my_s = 0.f;
+    int my_idx = 0;
+    for (int j = 0; j < a.K; ++j) {
+        float bv = -CUDART_INF_F, bs = 0.f;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && cand[i] != -CUDART_INF_F && route_beats(cand[i], e, bv, bi)) {
+                bv = cand[i];
+                bi = e;
+                bs = s[i];
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+            if (route_beats(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+                bs = os;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+            if (lane + 32 * i == bi) cand[i] = -CUDART_INF_F;
+        if (lane == j) {
+            my_s = bs;
+            my_idx = bi;
+        }
+    }
+
+    float sum = lane < a.K ? my_s : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < a.K) {
+        float w = a.norm ? my_s / sum : my_s;
+        w *= a.scale;
+        a.topk_idx[(int64_t)t * a.K + lane] = my_idx;
+        a.topk_w[(int64_t)t * a.K + lane] = w;
+    }
+}
+
+}  // namespace moe

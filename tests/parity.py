@@ -1,0 +1,127 @@
+"""Parity helpers shared by the GPU tests, smoke() and bench's CPU baseline.
+
+They compare the CUDA path's results with the float64 oracle on the same bits.
+Tolerances (bf16 storage, fp32 accumulation):
+  max |y - y_ref| <= 2e-2 * RMS(y_ref)
+  sum |y - y_ref| / sum |y_ref| <= 5e-3
+Routing: expert sets must match exactly, except on tokens whose oracle margin
+(the gap at the group-keep or top-k boundary) is below 1e-4; such a token is
+counted, its GPU set must be optimal within that margin, and its output is
+compared with the oracle recomputed on the GPU's set.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List
+
+import numpy as np
+import torch
+
+import oracle
+from sparse_moe_layer_noaux_b200.workloads import MoEShape, bf16_bits
+
+MAX_ABS_REL_RMS = 2e-2
+MEAN_REL = 5e-3
+NEAR_TIE = 1e-4
+
+
+def oracle_route_all(shape: MoEShape, x_bits, rw, bias, workers: int = 0):
+    """Oracle routing of every row (row blocks in spawned processes when large)."""
+    from oracle.pool import route_rows
+    return route_rows(shape, x_bits, rw, bias, workers)
+
+
+@dataclass
+class RoutingReport:
+    tokens: int = 0
+    near_ties: int = 0
+    mismatched_near_ties: int = 0
+    order_mismatches: int = 0
+    mismatched_tokens: List[int] = field(default_factory=list)
+
+
+def compare_routing(shape, gpu_idx, gpu_w, ref_idx, ref_w, margin, scores, bias) -> RoutingReport:
+    """Sets must agree unless the oracle margin is a near tie; weights within 1e-4 relative."""
+    rep = RoutingReport(tokens=len(ref_idx))
+    b = scores + np.asarray(bias, np.float64)[None, :]
+    gsz = shape.E // shape.n_group
+    for t in range(len(ref_idx)):
+        g_set, r_set = set(gpu_idx[t].tolist()), set(ref_idx[t].tolist())
+        near = margin[t] < NEAR_TIE
+        rep.near_ties += int(near)
+        if g_set != r_set:
+            if not near:
+                rep.mismatched_tokens.append(t)
+                continue
+            rep.mismatched_near_ties += 1
+            # The GPU's choice must be valid and optimal within the margin.
+            assert len(g_set) == shape.k
+            assert len({e // gsz for e in g_set}) <= shape.topk_group
+            assert abs(sum(b[t, list(g_set)]) - sum(b[t, list(r_set)])) <= 2 * shape.k * NEAR_TIE
+            continue
+        if gpu_idx[t].tolist() != ref_idx[t].tolist():
+            rep.order_mismatches += 1
+        order = {e: j for j, e in enumerate(ref_idx[t].tolist())}
+        w_ref = np.array([ref_w[t, order[e]] for e in gpu_idx[t].tolist()])
+        np.testing.assert_allclose(gpu_w[t], w_ref, rtol=1e-4, atol=1e-5,
+                                   err_msg=f"routing weights of token {t}")
+    return rep
+
+
+def weights_for_set(shape, scores_row, idx_row):
+    """Routing weights (float64) of a given expert set, from the oracle's unbiased scores."""
+    s = scores_row[np.asarray(idx_row)]
+    w = s / s.sum() if shape.norm_topk_prob else s
+    return w * shape.routed_scaling_factor
+
+
+def output_errors(y, y_ref):
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    max_abs = float(np.max(np.abs(y - y_ref))) if y.size else 0.0
+    rel_l1 = float(np.sum(np.abs(y - y_ref)) / max(np.sum(np.abs(y_ref)), 1e-300))
+    return {"rms": rms, "max_abs": max_abs, "max_abs_over_rms": max_abs / max(rms, 1e-300),
+            "rel_l1": rel_l1}
+
+
+def assert_output_close(y, y_ref, what=""):
+    e = output_errors(y, y_ref)
+    assert e["max_abs_over_rms"] <= MAX_ABS_REL_RMS, (what, e)
+    assert e["rel_l1"] <= MEAN_REL, (what, e)
+    return e
+
+
+def device_expert_fetch(inp):
+    """Oracle expert fetcher copying one expert's bf16 bits from the device at a time."""
+    def fetch(e):
+        return (bf16_bits(inp["w_gate"][e]), bf16_bits(inp["w_up"][e]), bf16_bits(inp["w_down"][e]))
+    return fetch
+
+
+def shared_bits(inp, shape):
+    if shape.n_shared_experts == 0:
+        return None
+    return tuple(bf16_bits(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
+
+
+def oracle_layer_rows(shape, inp, rows, gpu_idx=None, scores=None, ref_idx=None, ref_w=None,
+                      margin=None):
+    """Oracle output for the given token rows.  Where the GPU picked a different
+    (near-tie) expert set, that row is computed on the GPU's set."""
+    x_bits = bf16_bits(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
+    rw = inp["router_w"].cpu().numpy()
+    bias = inp["e_bias"].cpu().numpy()
+    routing = None
+    if gpu_idx is not None and ref_idx is not None:
+        use_idx = ref_idx[rows].copy()
+        use_w = ref_w[rows].copy()
+        for i, t in enumerate(rows):
+            if set(gpu_idx[t].tolist()) != set(ref_idx[t].tolist()):
+                assert margin[t] < NEAR_TIE
+                use_idx[i] = gpu_idx[t]
+                use_w[i] = weights_for_set(shape, scores[t], gpu_idx[t])
+        routing = (use_idx, use_w)
+    y, *_ = oracle.moe_layer(shape, x_bits, rw, bias, device_expert_fetch(inp),
+                             shared_bits(inp, shape), routing=routing)
+    return y

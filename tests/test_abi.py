@@ -1,0 +1,112 @@
+"""The C ABI library on the host (no GPU needed): it builds, loads, exports every
+symbol include/moe.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_layer_noaux_b200 import abi, build
+from sparse_moe_layer_noaux_b200.workloads import MID, TINY, V3_PREFILL
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_header_symbols_exported(lib):
+    names = declared_functions()
+    assert {"moe_route", "moe_dispatch", "moe_forward", "moe_workspace_size",
+            "moe_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert abi.status_string(code)
+    assert abi.status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    c = abi.MoEConfig.from_shape(TINY)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_group=3), abi.MOE_ERR_INVALID_ARG),               # E % G != 0
+    (dict(topk_group=5), abi.MOE_ERR_INVALID_ARG),            # TG > G
+    (dict(num_experts_per_tok=0), abi.MOE_ERR_INVALID_ARG),
+    (dict(num_experts_per_tok=9), abi.MOE_ERR_INVALID_ARG),   # k > TG * E / G = 8
+    (dict(norm_topk_prob=2), abi.MOE_ERR_INVALID_ARG),
+    (dict(hidden_size=0), abi.MOE_ERR_INVALID_ARG),
+    (dict(n_shared_experts=-1), abi.MOE_ERR_INVALID_ARG),
+    (dict(hidden_size=200), abi.MOE_ERR_UNSUPPORTED),          # not a multiple of 64
+    (dict(moe_intermediate_size=96), abi.MOE_ERR_UNSUPPORTED),
+    (dict(n_routed_experts=512, n_group=8), abi.MOE_ERR_UNSUPPORTED),
+])
+def test_bad_config_rejected(lib, kw, code):
+    c = _cfg(**kw)
+    n = ctypes.c_size_t(0)
+    assert lib.moe_workspace_size(ctypes.byref(c), 64, ctypes.byref(n)) == code
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.moe_route(ctypes.byref(c), 64, p, p, p, p, p, p, 1 << 30, None) == code
+    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), p, 1 << 30, None) == code
+
+
+def test_negative_tokens_and_nulls(lib):
+    c = _cfg()
+    p = ctypes.c_void_p(1 << 20)
+    n = ctypes.c_size_t(0)
+    assert lib.moe_workspace_size(ctypes.byref(c), -1, ctypes.byref(n)) == abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_workspace_size(None, 4, ctypes.byref(n)) == abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(ctypes.byref(c), 4, None, p, p, p, p, p, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
+    args = [p] * 12
+    args[9] = None  # y
+    assert lib.moe_forward(ctypes.byref(c), 4, *args, p, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
+
+
+def test_misaligned_pointer_rejected(lib):
+    c = _cfg()
+    p = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.moe_route(ctypes.byref(c), 4, bad, p, p, p, p, p, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+    args = [p] * 12
+    args[3] = bad  # w_gate
+    assert lib.moe_forward(ctypes.byref(c), 4, *args, p, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+
+
+def test_workspace_too_small_rejected(lib):
+    c = _cfg()
+    need = abi.workspace_size(c, 64)
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), p, need - 1, None) == abi.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), None, need, None) == abi.MOE_ERR_WORKSPACE
+    assert lib.moe_route(ctypes.byref(c), 64, p, p, p, p, p, None, need, None) == abi.MOE_ERR_WORKSPACE
+
+
+def test_zero_tokens_needs_nothing(lib):
+    c = _cfg()
+    # T = 0 returns before any pointer or workspace is looked at.
+    assert lib.moe_forward(ctypes.byref(c), 0, *([None] * 12), None, 0, None) == abi.MOE_OK
+    assert lib.moe_route(ctypes.byref(c), 0, None, None, None, None, None, None, 0, None) == abi.MOE_OK
+
+
+def test_workspace_size_scales(lib):
+    small = abi.workspace_size(MID.with_(T=16), 16)
+    big = abi.workspace_size(MID, MID.T)
+    assert 0 < small < big
+    # The prefill workspace holds x_perm, h, y_perm: a few GB, well inside 180 GB.
+    ws = abi.workspace_size(V3_PREFILL, V3_PREFILL.T)
+    assert 4e9 < ws < 6e9

@@ -1,0 +1,236 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle on B200.
+
+Small and ragged shapes are checked on every token; the five workload shapes
+at full size are checked on every token's routing and dispatch, and on a
+seeded sample of tokens for the layer output (rows are independent, so a
+sample is an exact subset check).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_moe_layer_noaux_b200 import abi
+from sparse_moe_layer_noaux_b200.workloads import (MID, TINY, V3_DECODE, V3_PREFILL, V3_SKEWED, MoEShape,
+                                                   bf16_bits, make_inputs)
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from sparse_moe_layer_noaux_b200 import build
+    build.build()
+    oracle.build()
+    yield
+    torch.cuda.empty_cache()
+
+
+def run_forward(shape, inp):
+    T, k = shape.T, shape.k
+    cfg = abi.MoEConfig.from_shape(shape)
+    dev = inp["x"].device
+    y = torch.empty((T, shape.H), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(abi.workspace_size(cfg, T), 256), dtype=torch.uint8, device=dev)
+    abi.moe_forward(cfg, inp["x"], inp["router_w"], inp["e_bias"], inp["w_gate"], inp["w_up"],
+                    inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], y, idx, w, ws)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    return y, idx, w
+
+
+def check_dispatch(shape, x, topk_idx, offsets, x_perm, perm_src, row_of):
+    """Bit-exact: offsets = counts' exclusive scan; rows in stable (t, j) order."""
+    T, k, E = shape.T, shape.k, shape.E
+    flat = topk_idx.cpu().numpy().reshape(-1)
+    counts = np.bincount(flat, minlength=E)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
+    order = np.argsort(flat, kind="stable")
+    np.testing.assert_array_equal(perm_src.cpu().numpy(), order)
+    inv = np.empty(T * k, np.int64)
+    inv[order] = np.arange(T * k)
+    np.testing.assert_array_equal(row_of.cpu().numpy().reshape(-1), inv)
+    src_tok = perm_src.long() // k
+    assert torch.equal(x_perm.view(torch.int16), x[src_tok].view(torch.int16))
+
+
+SMALL = [
+    TINY,
+    TINY.with_(name="tiny_T1", T=1, seed=21),
+    TINY.with_(name="tiny_T3", T=3, seed=22),
+    MoEShape("ragged", T=300, hidden_size=512, n_routed_experts=32, n_group=4, topk_group=2,
+             num_experts_per_tok=4, moe_intermediate_size=256, n_shared_experts=1,
+             routed_scaling_factor=2.5, norm_topk_prob=True, seed=7),
+    # I = 192: the gate/up column tile is cut at 64 of 128; ~500 rows per expert.
+    MoEShape("tiles", T=2000, hidden_size=256, n_routed_experts=8, n_group=2, topk_group=1,
+             num_experts_per_tok=2, moe_intermediate_size=192, n_shared_experts=2,
+             routed_scaling_factor=1.3, norm_topk_prob=False, seed=8),
+    # No shared expert, flat routing, H = 320: the down-projection tile is cut at 64 of 256.
+    MoEShape("noshared", T=500, hidden_size=320, n_routed_experts=16, n_group=1, topk_group=1,
+             num_experts_per_tok=3, moe_intermediate_size=128, n_shared_experts=0,
+             routed_scaling_factor=1.0, norm_topk_prob=True, seed=9),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: s.name)
+def test_small_layer_every_token(shape):
+    inp = make_inputs(shape, "cuda")
+    y, idx, w = run_forward(shape, inp)
+    x_bits = bf16_bits(inp["x"])
+    rw, bias = inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()
+    ref_idx, ref_w, margin, scores = parity.oracle_route_all(shape, x_bits, rw, bias)
+    rep = parity.compare_routing(shape, idx.cpu().numpy(), w.cpu().numpy(), ref_idx, ref_w, margin,
+                                 scores, bias)
+    assert not rep.mismatched_tokens, rep
+    rows = np.arange(shape.T)
+    y_ref = parity.oracle_layer_rows(shape, inp, rows, idx.cpu().numpy(), scores, ref_idx, ref_w, margin)
+    parity.assert_output_close(y.float().cpu().numpy(), y_ref, shape.name)
+
+
+def test_stages_compose_to_forward():
+    """route -> dispatch -> experts -> combine through the C ABI equals moe_forward,
+    and each stage matches its own definition."""
+    shape = SMALL[4]
+    inp = make_inputs(shape, "cuda")
+    T, k, E, H, I, S = shape.T, shape.k, shape.E, shape.H, shape.I, shape.S
+    cfg = abi.MoEConfig.from_shape(shape)
+    dev = "cuda"
+    ws = torch.empty(abi.workspace_size(cfg, T), dtype=torch.uint8, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    abi.moe_route(cfg, inp["x"], inp["router_w"], inp["e_bias"], idx, w, ws)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    perm_src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_of = torch.empty((T, k), dtype=torch.int32, device=dev)
+    abi.moe_dispatch(cfg, inp["x"], idx, offsets, x_perm, perm_src, row_of, ws)
+    torch.cuda.synchronize()
+    check_dispatch(shape, inp["x"], idx, offsets, x_perm, perm_src, row_of)
+
+    h_r = torch.empty((T * k, I), dtype=torch.bfloat16, device=dev)
+    h_s = torch.empty((T, S * I), dtype=torch.bfloat16, device=dev)
+    y_perm = torch.empty((T * k + T, H), dtype=torch.bfloat16, device=dev)
+    abi.moe_experts(cfg, T, inp["x"], x_perm, offsets, perm_src, w, inp["w_gate"], inp["w_up"],
+                    inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], h_r, h_s, y_perm)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    abi.moe_combine(cfg, T, y_perm, row_of, y)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+
+    # Expert stage against float64 matrix products of the same bf16 operands.
+    off = offsets.cpu().tolist()
+    for e in range(E):
+        a, b = off[e], off[e + 1]
+        if a == b:
+            continue
+        xe = x_perm[a:b].double()
+        g = xe @ inp["w_gate"][e].double().T
+        u = xe @ inp["w_up"][e].double().T
+        h_ref = torch.nn.functional.silu(g) * u
+        parity.assert_output_close(h_r[a:b].double().cpu(), h_ref.cpu(), f"h expert {e}")
+        y_ref = (h_r[a:b].double() @ inp["w_down"][e].double().T) * w.view(-1)[perm_src[a:b].long()].double()[:, None]
+        parity.assert_output_close(y_perm[a:b].double().cpu(), y_ref.cpu(), f"y_perm expert {e}")
+    gs = inp["x"].double() @ inp["ws_gate"].double().T
+    us = inp["x"].double() @ inp["ws_up"].double().T
+    parity.assert_output_close(h_s.double().cpu(), (torch.nn.functional.silu(gs) * us).cpu(), "h shared")
+    ys_ref = h_s.double() @ inp["ws_down"].double().T
+    parity.assert_output_close(y_perm[T * k:].double().cpu(), ys_ref.cpu(), "y shared")
+    # Combine is an fp32 gather-sum of bf16 rows: check it exactly in float64 then round.
+    ref = y_perm[T * k:].float() + sum(y_perm[row_of[:, j].long()].float() for j in range(k))
+    assert (y.float() - ref).abs().max().item() <= 2 ** -7 * ref.abs().max().item()
+
+    y_fwd, idx_fwd, w_fwd = run_forward(shape, inp)
+    assert torch.equal(idx_fwd, idx) and torch.equal(w_fwd, w)
+    assert torch.equal(y_fwd.view(torch.int16), y.view(torch.int16))
+
+
+def test_zero_tokens_is_noop():
+    shape = TINY.with_(T=0)
+    cfg = abi.MoEConfig.from_shape(shape)
+    inp = make_inputs(TINY, "cuda")
+    empty = torch.empty((0, shape.H), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(empty)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    n0 = abi.launch_count()
+    abi.moe_forward(cfg, empty, inp["router_w"], inp["e_bias"], inp["w_gate"], inp["w_up"],
+                    inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], y, workspace=ws)
+    assert abi.launch_count() == n0
+
+
+def test_bounded_wait_gives_up_cleanly():
+    """A wait on a barrier nothing arrives on returns an error status; the context survives."""
+    assert abi.device_status() == 0
+    abi.selftest_wait_timeout(20_000_000)  # 20 ms
+    assert abi.device_status() == 0x901
+    assert abi.device_status() == 0
+    run_forward(TINY, make_inputs(TINY, "cuda"))  # the GPU still computes
+
+
+def test_deterministic_and_launch_count():
+    shape = SMALL[3]
+    inp = make_inputs(shape, "cuda")
+    n0 = abi.launch_count()
+    y1, i1, w1 = run_forward(shape, inp)
+    per_call = abi.launch_count() - n0
+    assert per_call == 8  # router 2, dispatch 3, experts 2, combine 1
+    y2, i2, w2 = run_forward(shape, inp)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)) and torch.equal(i1, i2)
+
+
+# ---------------------------------------------------------------------------
+# The five workload shapes at full size.
+# ---------------------------------------------------------------------------
+FULL = [(TINY, None), (MID, 48), (V3_DECODE, 16), (V3_PREFILL, 12), (V3_SKEWED, 12)]
+
+
+@pytest.mark.parametrize("shape,n_sample", FULL, ids=lambda v: getattr(v, "name", str(v)))
+def test_workload_full_size(shape, n_sample):
+    inp = make_inputs(shape, "cuda")
+    T, k, E = shape.T, shape.k, shape.E
+    y, idx, w = run_forward(shape, inp)
+    idx_h, w_h = idx.cpu().numpy(), w.cpu().numpy()
+
+    # Routing of every token.
+    x_bits = bf16_bits(inp["x"])
+    rw, bias = inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()
+    ref_idx, ref_w, margin, scores = parity.oracle_route_all(shape, x_bits, rw, bias)
+    rep = parity.compare_routing(shape, idx_h, w_h, ref_idx, ref_w, margin, scores, bias)
+    assert not rep.mismatched_tokens, rep
+    print(f"{shape.name}: near-ties {rep.near_ties}, differing near-tie sets "
+          f"{rep.mismatched_near_ties}, order differences {rep.order_mismatches}")
+
+    # Dispatch of every slot, in the launch configuration of moe_forward.
+    cfg = abi.MoEConfig.from_shape(shape)
+    ws = torch.empty(abi.workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty((T * k, shape.H), dtype=torch.bfloat16, device="cuda")
+    perm_src = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    abi.moe_dispatch(cfg, inp["x"], idx, offsets, x_perm, perm_src, row_of, ws)
+    torch.cuda.synchronize()
+    check_dispatch(shape, inp["x"], idx, offsets, x_perm, perm_src, row_of)
+    del x_perm, ws
+
+    # Layer output: every token when small, else a seeded sample (incl. first/last token
+    # and, for the skewed load, tokens of the most loaded expert).
+    if n_sample is None:
+        rows = np.arange(T)
+    else:
+        rng = np.random.default_rng(1234 + shape.seed)
+        rows = set(rng.choice(T, n_sample - 2, replace=False).tolist()) | {0, T - 1}
+        hot = int(np.bincount(idx_h.reshape(-1), minlength=E).argmax())
+        rows |= set(np.nonzero((idx_h == hot).any(1))[0][:2].tolist())
+        rows = np.array(sorted(rows))
+    y_ref = parity.oracle_layer_rows(shape, inp, rows, idx_h, scores, ref_idx, ref_w, margin)
+    err = parity.assert_output_close(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(),
+                                     y_ref, shape.name)
+    print(f"{shape.name}: {len(rows)} rows, {err}")
+    # Properties at any size: finite output, every token routed to k distinct experts.
+    assert torch.isfinite(y.float()).all()
+    srt = torch.sort(idx, dim=1).values
+    assert (srt[:, 1:] != srt[:, :-1]).all()
