@@ -115,14 +115,16 @@ MOE_API int moe_dispatch(const moe_config *cfg, int64_t T, const void *x, const 
 /*
  * Experts: every routed row r of expert e gives
  *   h_routed[r] = silu(x_perm[r] . w_gate[e]^T) * (x_perm[r] . w_up[e]^T)   bf16 [T*k, I]
- *   y_perm[r]   = topk_w[perm_src[r]] * (h_routed[r] . w_down[e]^T)         bf16 [T*k + T, H]
+ *   y_perm[r]   = topk_w[perm_src[r]] * (h_routed[r] . w_down[e]^T)         fp32 [T*k + T, H]
  * and every token t runs the shared expert(s) on x itself:
  *   h_shared[t]        = silu(x[t] . ws_gate^T) * (x[t] . ws_up^T)          bf16 [T, S*I]
  *   y_perm[T*k + t]    = h_shared[t] . ws_down^T
  * ("The Evolving Transformer · 07", § 02 and § 03.)  Grouped tensor-core
  * GEMMs over the variable-length expert segments given by expert_offsets;
- * fp32 accumulation, bf16 storage.  When S == 0 the shared pointers may be
- * NULL and y_perm needs only T*k rows.
+ * fp32 accumulation; h is stored as bf16 (it is the next GEMM's operand) and
+ * y_perm as fp32, so the layer output is rounded to bf16 only once, in the
+ * combine.  When S == 0 the shared pointers may be NULL and y_perm needs only
+ * T*k rows.
  */
 MOE_API int moe_experts(const moe_config *cfg, int64_t T, const void *x, const void *x_perm,
                 const int32_t *expert_offsets, const int32_t *perm_src, const float *topk_w,
@@ -145,7 +147,7 @@ MOE_API int moe_experts_down(const moe_config *cfg, int64_t T, const void *h_rou
 
 /*
  * Combine: y[t] = y_perm[T*k + t] (shared, if S > 0) + sum_{j<k} y_perm[row_of[t, j]],
- * summed in fp32 in that order and stored as bf16 [T, H] — the page's
+ * y_perm fp32 rows summed in fp32 in that order and stored as bf16 [T, H] — the page's
  * output[mask] += w * expert_out and `shared_expert_out + output`
  * ("The Evolving Transformer · 07", § 02), as a deterministic gather.
  */

@@ -1,7 +1,7 @@
 // Combine: y[t] = shared_out[t] + sum_j w_j * expert_j(x[t]).  The routing
 // weights are already applied by the down-projection epilogue, so this is a
-// gather of k + 1 rows per token summed in fp32 in a fixed order (shared first,
-// then slots 0..k-1) — the page's `output[mask] += w * expert_out` followed by
+// gather of k + 1 fp32 rows per token summed in fp32 in a fixed order (shared
+// first, then slots 0..k-1) and rounded once to bf16 — the page's `output[mask] += w * expert_out` followed by
 // `shared_expert_out + output` ("The Evolving Transformer · 07", § 02 / § 03),
 // without atomics and therefore deterministic.
 #pragma once
@@ -10,36 +10,30 @@
 
 namespace moe {
 
-__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& v) {
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(p[q]);
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
-    }
-}
-
-// One warp per token; each lane owns 16-byte chunks (8 values) of the row.
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ y_perm,
+// One warp per token; each lane owns 8-value (32-byte) slices of the row.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y_perm,
                                                       const int32_t* __restrict__ row_of, int T,
                                                       int K, int H, int has_shared,
                                                       __nv_bfloat16* __restrict__ y) {
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    __shared__ int rows_s[8][33];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int t = blockIdx.x * (blockDim.x >> 5) + wib;
     if (t >= T) return;
-    int rows[33];
-    int nrows = 0;
-    if (has_shared) rows[nrows++] = (int)((int64_t)T * K + t);
-    for (int j = 0; j < K; ++j) rows[nrows++] = row_of[(int64_t)t * K + j];
-    const int chunks = H / 8;
-    for (int c = lane; c < chunks; c += 32) {
+    int* rows = rows_s[wib];
+    const int nrows = K + has_shared;
+    if (lane == 0 && has_shared) rows[0] = (int)((int64_t)T * K + t);
+    if (lane < K) rows[has_shared + lane] = row_of[(int64_t)t * K + lane];
+    __syncwarp();
+    const int slices = H / 8;
+    for (int c = lane; c < slices; c += 32) {
         float acc[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
         for (int r = 0; r < nrows; ++r) {
-            const uint4 v = reinterpret_cast<const uint4*>(y_perm + (int64_t)rows[r] * H)[c];
-            acc_bf16x8(acc, v);
+            const float4* src = reinterpret_cast<const float4*>(y_perm + (int64_t)rows[r] * H) + 2 * c;
+            const float4 a = src[0], b = src[1];
+            acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+            acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
         }
         uint4 out;
         __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&out);

@@ -6,7 +6,9 @@
 // Two instantiations:
 //   kSwiGLU  h = silu(A Wg^T) * (A Wu^T)   — gate and up tiles side by side in one
 //            N = 256 accumulator (128 gate columns | 128 up columns), fused epilogue;
-//   kDown    y = w_row * (h Wd^T)           — N = 256, routing weight in the epilogue.
+//   kDown    y = w_row * (h Wd^T)           — N = 256, routing weight in the epilogue,
+//            fp32 output (the combine sums k + 1 of these rows before the single
+//            rounding of the layer output to bf16).
 // ("The Evolving Transformer · 07", § 02: expert(x[mask]) is a SwiGLU FFN; its
 // output is multiplied by the routing weight.)
 //
@@ -49,9 +51,9 @@ struct GemmParams {
     int kb_routed, kb_shared;             // K blocks of 64
     int n_valid_routed, n_valid_shared;   // valid output columns
     int b_rows_per_expert;                // rows of one expert in the routed B map
-    __nv_bfloat16* out_routed;            // row r of routed segment -> out_routed + r*ld
-    int64_t ld_routed;
-    __nv_bfloat16* out_shared;            // row t of the shared segment
+    void* out_routed;                     // row r of routed segment -> out_routed + r*ld
+    int64_t ld_routed;                    // (bf16 elements for kSwiGLU, fp32 for kDown)
+    void* out_shared;                     // row t of the shared segment
     int64_t ld_shared;
     const int32_t* perm_src;              // kDown: routed row -> slot
     const float* topk_w;                  // kDown: slot -> routing weight
@@ -339,8 +341,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                    (static_cast<uint32_t>(quarter * 32) << 16);
             if (kEpi == kSwiGLU) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
-                __nv_bfloat16* out = ti.routed ? p.out_routed + grow * p.ld_routed
-                                               : p.out_shared + grow * p.ld_shared;
+                __nv_bfloat16* out = ti.routed
+                                         ? static_cast<__nv_bfloat16*>(p.out_routed) + grow * p.ld_routed
+                                         : static_cast<__nv_bfloat16*>(p.out_shared) + grow * p.ld_shared;
 #pragma unroll 1
                 for (int c = 0; c < (kBN / 2) / 32; ++c) {
                     __syncwarp();
@@ -367,8 +370,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
-                __nv_bfloat16* out = ti.routed ? p.out_routed + grow * p.ld_routed
-                                               : p.out_shared + grow * p.ld_shared;
+                float* out = ti.routed ? static_cast<float*>(p.out_routed) + grow * p.ld_routed
+                                       : static_cast<float*>(p.out_shared) + grow * p.ld_shared;
                 float wrow = 1.0f;
                 if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
 #pragma unroll 1
@@ -379,15 +382,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tmem_wait_ld();
                     const int col = ti.n * kBN + c * 32;
                     if (row_ok && col < n_valid) {
-                        uint4 pk[4];
-                        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(pk);
+                        float4* dst = reinterpret_cast<float4*>(out + col);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            h2[q] = __floats2bfloat162_rn(__uint_as_float(v[2 * q]) * wrow,
-                                                          __uint_as_float(v[2 * q + 1]) * wrow);
-                        uint4* dst = reinterpret_cast<uint4*>(out + col);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = pk[q];
+                        for (int q = 0; q < 8; ++q)
+                            dst[q] = make_float4(__uint_as_float(v[4 * q]) * wrow, __uint_as_float(v[4 * q + 1]) * wrow,
+                                                 __uint_as_float(v[4 * q + 2]) * wrow,
+                                                 __uint_as_float(v[4 * q + 3]) * wrow);
                     }
                 }
             }

@@ -114,7 +114,7 @@ struct Workspace {
     __nv_bfloat16* x_perm;    // [T*k, H]
     __nv_bfloat16* h_routed;  // [T*k, I]
     __nv_bfloat16* h_shared;  // [T, S*I]
-    __nv_bfloat16* y_perm;    // [T*k + T, H]
+    float* y_perm;            // [T*k + T, H] fp32
     size_t bytes;
 };
 
@@ -141,7 +141,7 @@ Workspace carve(const moe_config* c, int64_t T, uint8_t* base) {
     w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * H));
     w.h_routed = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * I));
     w.h_shared = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
-    w.y_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * (T * K + T) * H));
+    w.y_perm = reinterpret_cast<float*>(take(4 * (T * K + T) * H));
     w.bytes = off;
     return w;
 }
@@ -309,9 +309,9 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.n_valid_routed = static_cast<int>(H);
     p.n_valid_shared = static_cast<int>(H);
     p.b_rows_per_expert = static_cast<int>(H);
-    p.out_routed = static_cast<__nv_bfloat16*>(y_perm);
+    p.out_routed = y_perm;
     p.ld_routed = H;
-    p.out_shared = static_cast<__nv_bfloat16*>(y_perm) + R * H;
+    p.out_shared = static_cast<float*>(y_perm) + R * H;
     p.ld_shared = H;
     p.perm_src = perm_src;
     p.topk_w = topk_w;
@@ -325,7 +325,7 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
                    cudaStream_t st) {
     const unsigned g = static_cast<unsigned>((T + 7) / 8);
-    combine_kernel<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm), row_of,
+    combine_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
                                       static_cast<int>(T), c->num_experts_per_tok, c->hidden_size,
                                       c->n_shared_experts > 0 ? 1 : 0, static_cast<__nv_bfloat16*>(y));
     count_launch();

@@ -1,0 +1,47 @@
+"""The multi-rank host logic of bench.py on CPU with the gloo backend (world size 2):
+weights are replicated, tokens differ per rank, the step time is the max over
+ranks and the throughput counts every rank's tokens."""
+import os
+import socket
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from sparse_moe_layer_noaux_b200.workloads import TINY
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    inp = bench.rank_inputs(TINY, rank, "cpu")
+    sums = torch.tensor([inp["w_gate"].float().sum().item(), inp["router_w"].sum().item(),
+                         inp["x"].float().sum().item()], dtype=torch.float64)
+    gathered = [torch.zeros_like(sums) for _ in range(world)]
+    dist.all_gather(gathered, sums)
+    ms = bench.max_over_ranks(10.0 + rank, world)
+    out[rank] = (gathered[0].tolist(), gathered[1].tolist(), ms,
+                 bench.job_throughput(TINY.T, world, ms))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_replicas():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    g0, g1, ms, thr = res[0]
+    assert g0[0] == g1[0] and g0[1] == g1[1]      # same weights on both ranks
+    assert g0[2] != g1[2]                          # different tokens
+    assert ms == 11.0 and res[1][2] == 11.0        # max over ranks, seen by all
+    assert abs(thr - 2 * TINY.T / 11e-3) < 1e-6    # all ranks' tokens / slowest time
