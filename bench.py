@@ -168,7 +168,7 @@ class StagedStep:
         self.h_r = torch.empty((T * k, I), dtype=torch.bfloat16, device=d)
         self.h_s = torch.empty((T, max(S * I, 8)), dtype=torch.bfloat16, device=d)
         self.y_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=d)
-        self.y = torch.empty((T, H), dtype=torch.bfloat16, device=d)
+        self.y = torch.empty((T, H), dtype=torch.float32, device=d)
 
     def run(self, events=None):
         s, i, T = self.shape, self.inp, self.shape.T
@@ -226,7 +226,7 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
 
     # moe_forward (one call per step) timed alone, for reference.
     layer = MoELayer.from_inputs(shape, inp)
-    y = torch.empty_like(inp["x"])
+    y = torch.empty(inp["x"].shape, dtype=torch.float32, device=inp["x"].device)
     for _ in range(2):
         layer(inp["x"], y)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -256,9 +256,9 @@ def time_e2e(layer, shape, steps):
     """The public call with host buffers: pinned x -> HBM, layer, y -> pinned host."""
     x_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(layer_inputs_host(shape))
-    y_host = torch.empty_like(x_host, pin_memory=True)
+    y_host = torch.empty(x_host.shape, dtype=torch.float32, pin_memory=True)
     x_dev = torch.empty_like(x_host, device="cuda")
-    y_dev = torch.empty_like(x_dev)
+    y_dev = torch.empty(x_host.shape, dtype=torch.float32, device="cuda")
     for _ in range(2):
         x_dev.copy_(x_host, non_blocking=True)
         layer(x_dev, y_dev)
@@ -273,8 +273,7 @@ def time_e2e(layer, shape, steps):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    nbytes = x_host.numel() * x_host.element_size()
-    return ms, nbytes, nbytes
+    return ms, x_host.numel() * x_host.element_size(), y_host.numel() * y_host.element_size()
 
 
 def layer_inputs_host(shape):

@@ -79,6 +79,12 @@ typedef enum moe_status {
     MOE_ERR_TIMEOUT = 5       /* a bounded device wait gave up (from moe_device_status) */
 } moe_status;
 
+/* Element type of the layer output y. */
+typedef enum moe_dtype {
+    MOE_DTYPE_F32 = 0,   /* fp32: the fp32 sum of the expert outputs, unrounded */
+    MOE_DTYPE_BF16 = 1   /* bf16: that fp32 sum rounded once, to nearest even */
+} moe_dtype;
+
 /* Bytes of scratch needed by moe_forward (and enough for every other call
  * that takes a workspace) for T tokens.  Pure host arithmetic. */
 MOE_API int moe_workspace_size(const moe_config *cfg, int64_t T, size_t *bytes);
@@ -147,23 +153,25 @@ MOE_API int moe_experts_down(const moe_config *cfg, int64_t T, const void *h_rou
 
 /*
  * Combine: y[t] = y_perm[T*k + t] (shared, if S > 0) + sum_{j<k} y_perm[row_of[t, j]],
- * y_perm fp32 rows summed in fp32 in that order and stored as bf16 [T, H] — the page's
- * output[mask] += w * expert_out and `shared_expert_out + output`
- * ("The Evolving Transformer · 07", § 02), as a deterministic gather.
+ * y_perm fp32 rows summed in fp32 in that order and stored as y_dtype [T, H]
+ * (a moe_dtype) — the page's output[mask] += w * expert_out and
+ * `shared_expert_out + output` ("The Evolving Transformer · 07", § 02), as a
+ * deterministic gather.
  */
 MOE_API int moe_combine(const moe_config *cfg, int64_t T, const void *y_perm, const int32_t *row_of,
-                void *y, void *stream);
+                void *y, int32_t y_dtype, void *stream);
 
 /*
  * The whole layer: route, dispatch, experts, combine, on one stream.
- *   y bf16 [T, H] (output).  topk_idx_out / topk_w_out: optional [T, k]
+ *   y [T, H] (output) of element type y_dtype (a moe_dtype: fp32, or bf16
+ *   rounded once from the fp32 result).  topk_idx_out / topk_w_out: optional [T, k]
  *   copies of the routing (may be NULL).  workspace: at least
  *   moe_workspace_size(cfg, T) bytes of device memory, 256-byte aligned.
  */
 MOE_API int moe_forward(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
                 const float *e_bias, const void *w_gate, const void *w_up, const void *w_down,
                 const void *ws_gate, const void *ws_up, const void *ws_down, void *y,
-                int32_t *topk_idx_out, float *topk_w_out, void *workspace,
+                int32_t y_dtype, int32_t *topk_idx_out, float *topk_w_out, void *workspace,
                 size_t workspace_bytes, void *stream);
 
 /* Static text for a status code. */

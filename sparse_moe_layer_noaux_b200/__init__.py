@@ -50,11 +50,12 @@ class MoELayer:
 
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
                 topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
-                stream=None) -> torch.Tensor:
-        """y [T,H] bf16 = layer(x [T,H] bf16); optionally also returns the routing."""
+                stream=None, out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        """y [T,H] = layer(x [T,H] bf16).  y is fp32 (the unrounded fp32 sum) unless a
+        bf16 `y` or out_dtype is given; topk_idx / topk_w optionally receive the routing."""
         T = x.shape[0]
         if y is None:
-            y = torch.empty_like(x)
+            y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
         moe_forward(self.cfg, x, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
                     self.ws_gate, self.ws_up, self.ws_down, y, topk_idx, topk_w,
                     self.workspace(T), stream)

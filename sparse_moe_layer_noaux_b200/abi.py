@@ -17,6 +17,16 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+
+
+def out_dtype_code(t: torch.Tensor) -> int:
+    """moe_dtype of an output tensor (fp32 or bf16)."""
+    if t.dtype == torch.float32:
+        return MOE_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_DTYPE_BF16
+    raise TypeError(f"layer output must be float32 or bfloat16, got {t.dtype}")
 
 
 class MoEError(RuntimeError):
@@ -61,8 +71,8 @@ def lib():
         L.moe_experts.argtypes = [cfgp, i64] + [_P] * 15
         L.moe_experts_gate_up.argtypes = [cfgp, i64] + [_P] * 10
         L.moe_experts_down.argtypes = [cfgp, i64] + [_P] * 9
-        L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, _P]
-        L.moe_forward.argtypes = [cfgp, i64] + [_P] * 12 + [_P, sz, _P]
+        L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, ctypes.c_int32, _P]
+        L.moe_forward.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, _P, _P, _P, sz, _P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
@@ -143,7 +153,7 @@ def moe_experts_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_
 
 def moe_combine(cfg, T, y_perm, row_of, y, stream=None):
     _check("moe_combine", lib().moe_combine(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(row_of),
-                                            _ptr(y), _stream(stream)))
+                                            _ptr(y), out_dtype_code(y), _stream(stream)))
 
 
 def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
@@ -151,7 +161,7 @@ def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, 
     _check("moe_forward", lib().moe_forward(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
         _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y),
-        _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+        out_dtype_code(y), _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

@@ -323,11 +323,18 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
 }
 
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
-                   cudaStream_t st) {
+                   int y_dtype, cudaStream_t st) {
     const unsigned g = static_cast<unsigned>((T + 7) / 8);
-    combine_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
-                                      static_cast<int>(T), c->num_experts_per_tok, c->hidden_size,
-                                      c->n_shared_experts > 0 ? 1 : 0, static_cast<__nv_bfloat16*>(y));
+    const int has_shared = c->n_shared_experts > 0 ? 1 : 0;
+    if (y_dtype == MOE_DTYPE_BF16)
+        combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
+                                                         static_cast<int>(T), c->num_experts_per_tok,
+                                                         c->hidden_size, has_shared,
+                                                         static_cast<__nv_bfloat16*>(y));
+    else
+        combine_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
+                                                 static_cast<int>(T), c->num_experts_per_tok, c->hidden_size,
+                                                 has_shared, static_cast<float*>(y));
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -444,21 +451,23 @@ int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_p
 }
 
 int moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
-                void* stream) {
+                int32_t y_dtype, void* stream) {
     int v = validate_cfg(cfg, T);
     if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!y_perm || !row_of || !y) return MOE_ERR_INVALID_ARG;
     if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
-    return launch_combine(cfg, T, y_perm, row_of, y, static_cast<cudaStream_t>(stream));
+    return launch_combine(cfg, T, y_perm, row_of, y, y_dtype, static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
                 const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
-                const void* ws_up, const void* ws_down, void* y, int32_t* topk_idx_out, float* topk_w_out,
-                void* workspace, size_t workspace_bytes, void* stream) {
+                const void* ws_up, const void* ws_down, void* y, int32_t y_dtype, int32_t* topk_idx_out,
+                float* topk_w_out, void* workspace, size_t workspace_bytes, void* stream) {
     int v = validate_cfg(cfg, T);
     if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     const bool sh = cfg->n_shared_experts > 0;
     if (!x || !router_w || !e_bias || !w_gate || !w_up || !w_down || !y) return MOE_ERR_INVALID_ARG;
@@ -490,7 +499,7 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
     if ((v = launch_down(cfg, T, w.h_routed, w.h_shared, w.offsets, w.perm_src, tw, w_down, ws_down, w.y_perm,
                          d->num_sms, st)) != MOE_OK)
         return v;
-    return launch_combine(cfg, T, w.y_perm, w.row_of, y, st);
+    return launch_combine(cfg, T, w.y_perm, w.row_of, y, y_dtype, st);
 }
 
 const char* moe_status_string(int status) {

@@ -92,6 +92,16 @@ def assert_output_close(y, y_ref, what=""):
     return e
 
 
+def assert_bf16_rounded(t, ref, what=""):
+    """A bf16-stored intermediate: within one bf16 rounding (2^-8 relative) of the
+    float64 reference, plus a small fp32-accumulation allowance."""
+    t = t.double()
+    ref = ref.double().to(t.device)
+    rms = ref.pow(2).mean().sqrt()
+    bad = (t - ref).abs() > 2.0 ** -8 * ref.abs() + 2e-3 * rms
+    assert not bool(bad.any()), (what, int(bad.sum()), float((t - ref).abs().max()), float(rms))
+
+
 def device_expert_fetch(inp):
     """Oracle expert fetcher copying one expert's bf16 bits from the device at a time."""
     def fetch(e):

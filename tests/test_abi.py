@@ -37,6 +37,11 @@ def test_status_strings(lib):
     assert abi.status_string(99) == "unknown status"
 
 
+def fwd(lib, c, T, ptrs, ws, nbytes, y_dtype=0):
+    """moe_forward with the 12 pointer arguments x .. topk_w_out given as a list."""
+    return lib.moe_forward(ctypes.byref(c), T, *ptrs[:10], y_dtype, ptrs[10], ptrs[11], ws, nbytes, None)
+
+
 def _cfg(**kw):
     c = abi.MoEConfig.from_shape(TINY)
     for k, v in kw.items():
@@ -62,7 +67,7 @@ def test_bad_config_rejected(lib, kw, code):
     assert lib.moe_workspace_size(ctypes.byref(c), 64, ctypes.byref(n)) == code
     p = ctypes.c_void_p(1 << 20)
     assert lib.moe_route(ctypes.byref(c), 64, p, p, p, p, p, p, 1 << 30, None) == code
-    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), p, 1 << 30, None) == code
+    assert fwd(lib, c, 64, [p] * 12, p, 1 << 30) == code
 
 
 def test_negative_tokens_and_nulls(lib):
@@ -74,7 +79,8 @@ def test_negative_tokens_and_nulls(lib):
     assert lib.moe_route(ctypes.byref(c), 4, None, p, p, p, p, p, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
     args = [p] * 12
     args[9] = None  # y
-    assert lib.moe_forward(ctypes.byref(c), 4, *args, p, 1 << 30, None) == abi.MOE_ERR_INVALID_ARG
+    assert fwd(lib, c, 4, args, p, 1 << 30) == abi.MOE_ERR_INVALID_ARG
+    assert fwd(lib, c, 4, [p] * 12, p, 1 << 30, y_dtype=7) == abi.MOE_ERR_INVALID_ARG
 
 
 def test_misaligned_pointer_rejected(lib):
@@ -84,22 +90,22 @@ def test_misaligned_pointer_rejected(lib):
     assert lib.moe_route(ctypes.byref(c), 4, bad, p, p, p, p, p, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
     args = [p] * 12
     args[3] = bad  # w_gate
-    assert lib.moe_forward(ctypes.byref(c), 4, *args, p, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+    assert fwd(lib, c, 4, args, p, 1 << 30) == abi.MOE_ERR_UNSUPPORTED
 
 
 def test_workspace_too_small_rejected(lib):
     c = _cfg()
     need = abi.workspace_size(c, 64)
     p = ctypes.c_void_p(1 << 20)
-    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), p, need - 1, None) == abi.MOE_ERR_WORKSPACE
-    assert lib.moe_forward(ctypes.byref(c), 64, *([p] * 12), None, need, None) == abi.MOE_ERR_WORKSPACE
+    assert fwd(lib, c, 64, [p] * 12, p, need - 1) == abi.MOE_ERR_WORKSPACE
+    assert fwd(lib, c, 64, [p] * 12, None, need) == abi.MOE_ERR_WORKSPACE
     assert lib.moe_route(ctypes.byref(c), 64, p, p, p, p, p, None, need, None) == abi.MOE_ERR_WORKSPACE
 
 
 def test_zero_tokens_needs_nothing(lib):
     c = _cfg()
     # T = 0 returns before any pointer or workspace is looked at.
-    assert lib.moe_forward(ctypes.byref(c), 0, *([None] * 12), None, 0, None) == abi.MOE_OK
+    assert fwd(lib, c, 0, [None] * 12, None, 0) == abi.MOE_OK
     assert lib.moe_route(ctypes.byref(c), 0, None, None, None, None, None, None, 0, None) == abi.MOE_OK
 
 

@@ -29,11 +29,11 @@ def _gpu():
     torch.cuda.empty_cache()
 
 
-def run_forward(shape, inp):
+def run_forward(shape, inp, out_dtype=torch.float32):
     T, k = shape.T, shape.k
     cfg = abi.MoEConfig.from_shape(shape)
     dev = inp["x"].device
-    y = torch.empty((T, shape.H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, shape.H), dtype=out_dtype, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     ws = torch.empty(max(abi.workspace_size(cfg, T), 256), dtype=torch.uint8, device=dev)
@@ -119,8 +119,10 @@ def test_stages_compose_to_forward():
     y_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=dev)
     abi.moe_experts(cfg, T, inp["x"], x_perm, offsets, perm_src, w, inp["w_gate"], inp["w_up"],
                     inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], h_r, h_s, y_perm)
-    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
     abi.moe_combine(cfg, T, y_perm, row_of, y)
+    y16 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    abi.moe_combine(cfg, T, y_perm, row_of, y16)
     torch.cuda.synchronize()
     assert abi.device_status() == 0
 
@@ -134,23 +136,27 @@ def test_stages_compose_to_forward():
         g = xe @ inp["w_gate"][e].double().T
         u = xe @ inp["w_up"][e].double().T
         h_ref = torch.nn.functional.silu(g) * u
-        parity.assert_output_close(h_r[a:b].double().cpu(), h_ref.cpu(), f"h expert {e}")
+        parity.assert_bf16_rounded(h_r[a:b], h_ref, f"h expert {e}")
         y_ref = (h_r[a:b].double() @ inp["w_down"][e].double().T) * w.view(-1)[perm_src[a:b].long()].double()[:, None]
         parity.assert_output_close(y_perm[a:b].double().cpu(), y_ref.cpu(), f"y_perm expert {e}")
     gs = inp["x"].double() @ inp["ws_gate"].double().T
     us = inp["x"].double() @ inp["ws_up"].double().T
-    parity.assert_output_close(h_s.double().cpu(), (torch.nn.functional.silu(gs) * us).cpu(), "h shared")
+    parity.assert_bf16_rounded(h_s, torch.nn.functional.silu(gs) * us, "h shared")
     ys_ref = h_s.double() @ inp["ws_down"].double().T
     parity.assert_output_close(y_perm[T * k:].double().cpu(), ys_ref.cpu(), "y shared")
-    # Combine: fp32 gather-sum in the order shared, slot 0..k-1, rounded once to bf16.
+    # Combine: fp32 gather-sum in the order shared, slot 0..k-1; the bf16 output is
+    # that sum rounded once to nearest.
     ref = y_perm[T * k:].clone()
     for j in range(k):
         ref += y_perm[row_of[:, j].long()]
-    assert torch.equal(y.view(torch.int16), ref.to(torch.bfloat16).view(torch.int16))
+    assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
+    assert torch.equal(y16.view(torch.int16), ref.to(torch.bfloat16).view(torch.int16))
 
     y_fwd, idx_fwd, w_fwd = run_forward(shape, inp)
     assert torch.equal(idx_fwd, idx) and torch.equal(w_fwd, w)
-    assert torch.equal(y_fwd.view(torch.int16), y.view(torch.int16))
+    assert torch.equal(y_fwd.view(torch.int32), y.view(torch.int32))
+    y_fwd16, _, _ = run_forward(shape, inp, torch.bfloat16)
+    assert torch.equal(y_fwd16.view(torch.int16), y16.view(torch.int16))
 
 
 def test_zero_tokens_is_noop():
@@ -183,7 +189,7 @@ def test_deterministic_and_launch_count():
     per_call = abi.launch_count() - n0
     assert per_call == 8  # router 2, dispatch 3, experts 2, combine 1
     y2, i2, w2 = run_forward(shape, inp)
-    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)) and torch.equal(i1, i2)
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32)) and torch.equal(i1, i2)
 
 
 # ---------------------------------------------------------------------------
