@@ -8,7 +8,10 @@
 //            N = 256 accumulator (128 gate columns | 128 up columns), fused epilogue;
 //   kDown    y = w_row * (h Wd^T)           — N = 256, routing weight in the epilogue,
 //            fp32 output (the combine sums k + 1 of these rows before the single
-//            rounding of the layer output to bf16).
+//            rounding of the layer output to bf16);
+//   kLogits  router logits l = x Wr^T in fp32 from an exact three-way bf16 split
+//            Wr = hi + mid + lo (one segment of T rows, K = 3 H concatenated over the
+//            three planes, N = E rounded up to 16), fp32 output.
 // ("The Evolving Transformer · 07", § 02: expert(x[mask]) is a SwiGLU FFN; its
 // output is multiplied by the routing weight.)
 //
@@ -37,7 +40,7 @@ constexpr uint32_t kTileBBytes = kBN * kBK * 2;   // 32 KB
 constexpr uint32_t kTmemCols = 512;               // 2 accumulators x 256 columns
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 
-enum { kSwiGLU = 0, kDown = 1 };
+enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
 
 // Device error word (set by a bounded wait that gave up; read by the host).
 __device__ unsigned int g_moe_error;
@@ -57,6 +60,10 @@ struct GemmParams {
     int64_t ld_shared;
     const int32_t* perm_src;              // kDown: routed row -> slot
     const float* topk_w;                  // kDown: slot -> routing weight
+    uint32_t idesc;                       // MMA instruction descriptor (M = 128, N)
+    uint32_t b_tile_bytes;                // bytes one B tile load brings in
+    int kb_plane;                         // kLogits: K blocks per plane (H / 64)
+    int b_plane_rows;                     // kLogits: rows of one plane in the B map (E)
 };
 
 struct TileInfo {
@@ -257,15 +264,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     const uint32_t full = ptx::smem_u32(&S.full[stage]);
-                    ptx::mbar_arrive_expect_tx(full, kTileABytes + kTileBBytes);
+                    ptx::mbar_arrive_expect_tx(full, kTileABytes + p.b_tile_bytes);
                     const uint32_t a_dst = ptx::smem_u32(smemA + stage * kTileABytes);
                     const uint32_t b_dst = ptx::smem_u32(smemB + stage * kTileBBytes);
-                    ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
-                    if (kEpi == kSwiGLU) {
+                    if (kEpi == kLogits) {
+                        // K runs over the three planes of Wr back to back; x is re-read per plane.
+                        const int plane = kb / p.kb_plane;
+                        const int kcol = (kb - plane * p.kb_plane) * kBK;
+                        ptx::tma_load_2d(a_dst, mA, full, kcol, a_row, pol_a);
+                        ptx::tma_load_2d(b_dst, mB, full, kcol, plane * p.b_plane_rows);
+                    } else if (kEpi == kSwiGLU) {
+                        ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
                         const int b_row = b_base + ti.n * (kBN / 2);
                         ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
                         ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row);
                     } else {
+                        ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
                         const int b_row = b_base + ti.n * kBN;
                         ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
                     }
@@ -284,7 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ================= MMA issuer =================
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, kBN);
+            const uint32_t idesc = p.idesc;
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -368,7 +382,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int q = 0; q < 4; ++q) dst[q] = pk[q];
                     }
                 }
-            } else {
+            } else if (kEpi == kDown) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
                 float* out = ti.routed ? static_cast<float*>(p.out_routed) + grow * p.ld_routed
                                        : static_cast<float*>(p.out_shared) + grow * p.ld_shared;
@@ -388,6 +402,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             dst[q] = make_float4(__uint_as_float(v[4 * q]) * wrow, __uint_as_float(v[4 * q + 1]) * wrow,
                                                  __uint_as_float(v[4 * q + 2]) * wrow,
                                                  __uint_as_float(v[4 * q + 3]) * wrow);
+                    }
+                }
+            } else {
+                const int n_valid = p.n_valid_shared;  // E
+                float* out = static_cast<float*>(p.out_shared) + grow * p.ld_shared;
+#pragma unroll 1
+                for (int c = 0; c * 32 < n_valid; ++c) {
+                    __syncwarp();
+                    uint32_t v[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    ptx::tmem_wait_ld();
+                    if (row_ok) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const int col = c * 32 + 4 * q;
+                            if (col < n_valid)
+                                *reinterpret_cast<float4*>(out + col) =
+                                    make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                        }
                     }
                 }
             }

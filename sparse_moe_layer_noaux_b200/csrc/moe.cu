@@ -57,7 +57,12 @@ struct RouterPlan {
 // workspace size computed before launch always matches what the launch uses.
 constexpr int kRouterTargetBlocks = 296;  // two waves of blocks on 148 SMs
 
+// Token counts from which the logits run on the tensor cores (below it, the
+// CUDA-core kernel with a split hidden axis fills the GPU better).
+constexpr int kRouterTensorCoreMinT = 2048;
+
 RouterPlan plan_router(int T, int E, int H) {
+    if (T >= kRouterTensorCoreMinT) return RouterPlan{1, H};
     const int tiles = ((T + kRT - 1) / kRT) * ((E + kRE - 1) / kRE);
     int want = (kRouterTargetBlocks + tiles - 1) / tiles;
     const int max_split = H / 256 > 0 ? H / 256 : 1;
@@ -93,6 +98,8 @@ int device_info(DeviceInfo** out) {
         if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_kernel<kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.attrs_set = true;
@@ -103,6 +110,7 @@ int device_info(DeviceInfo** out) {
 
 // --------------------------------------------------------------- workspace
 struct Workspace {
+    __nv_bfloat16* router_w3; // [3, E, H] exact bf16 split of router_w
     float* router_part;       // [nsplit, T, E]
     int32_t* block_counts;    // [nb, E]
     int32_t* block_base;      // [nb, E]
@@ -130,6 +138,7 @@ Workspace carve(const moe_config* c, int64_t T, uint8_t* base) {
         off += align_up(bytes);
         return p;
     };
+    w.router_w3 = reinterpret_cast<__nv_bfloat16*>(take(2 * 3 * E * H));
     w.router_part = reinterpret_cast<float*>(take(sizeof(float) * rp.nsplit * T * E));
     w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
     w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
@@ -182,13 +191,44 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // --------------------------------------------------------------- stages
+constexpr size_t kGemmSmemBytes = 1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem);
+
 int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
-                 int32_t* idx, float* w, float* part, cudaStream_t st) {
+                 int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
     const int H = c->hidden_size, E = c->n_routed_experts;
     const RouterPlan rp = plan_router(static_cast<int>(T), E, H);
-    dim3 g1((E + kRE - 1) / kRE, static_cast<unsigned>((T + kRT - 1) / kRT), rp.nsplit);
-    router_logits_kernel<<<g1, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, part,
-                                              static_cast<int>(T), E, H, rp.split_len);
+    if (T >= kRouterTensorCoreMinT) {
+        // Logits on the tensor cores: exact 3-term bf16 split of Wr, one GEMM, K = 3 H.
+        const int64_t n = static_cast<int64_t>(E) * H;
+        router_split_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
+                              st>>>(wr, w3, n);
+        const int npad = (E + 15) / 16 * 16;
+        CUtensorMap a, b;
+        if (!make_map(&a, x, T, H, kBM) || !make_map(&b, w3, 3ull * E, H, npad)) return MOE_ERR_CUDA;
+        GemmParams p{};
+        p.E = 0;
+        p.T = static_cast<int>(T);
+        p.has_shared = 1;
+        p.n_tiles_shared = 1;
+        p.kb_shared = 3 * (H / kBK);
+        p.n_valid_shared = E;
+        p.out_shared = part;
+        p.ld_shared = E;
+        p.idesc = ptx::idesc_bf16_f32(kBM, npad);
+        p.b_tile_bytes = static_cast<uint32_t>(npad) * kBK * 2;
+        p.kb_plane = H / kBK;
+        p.b_plane_rows = E;
+        int64_t grid = (T + kBM - 1) / kBM;
+        if (grid > num_sms) grid = num_sms;
+        grouped_gemm_kernel<kLogits><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
+            a, a, b, b, b, b, p);
+        count_launch(2);
+    } else {
+        dim3 g1((E + kRE - 1) / kRE, static_cast<unsigned>((T + kRT - 1) / kRT), rp.nsplit);
+        router_logits_kernel<<<g1, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, part,
+                                                  static_cast<int>(T), E, H, rp.split_len);
+        count_launch();
+    }
     RouteArgs a;
     a.part = part;
     a.nsplit = rp.nsplit;
@@ -207,7 +247,7 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
     else if (E <= 64) router_select_kernel<2><<<g2, 256, 0, st>>>(a);
     else if (E <= 128) router_select_kernel<4><<<g2, 256, 0, st>>>(a);
     else router_select_kernel<8><<<g2, 256, 0, st>>>(a);
-    count_launch(2);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -237,8 +277,6 @@ int64_t gemm_grid(int64_t T, int64_t R, int64_t E, int64_t n_cols_max, int has_s
     if (grid < 1) grid = 1;
     return grid;
 }
-
-constexpr size_t kGemmSmemBytes = 1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem);
 
 // K4: h = silu(A Wg^T) * (A Wu^T) for routed rows (A = x_perm) and shared rows (A = x).
 int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_perm, const int32_t* offsets,
@@ -274,6 +312,8 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.ld_routed = I;
     p.out_shared = static_cast<__nv_bfloat16*>(h_shared);
     p.ld_shared = SI;
+    p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
+    p.b_tile_bytes = kTileBBytes;
     const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -315,6 +355,8 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.ld_shared = H;
     p.perm_src = perm_src;
     p.topk_w = topk_w;
+    p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
+    p.b_tile_bytes = kTileBBytes;
     const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);
@@ -362,8 +404,10 @@ int moe_route(const moe_config* cfg, int64_t T, const void* x, const float* rout
     if (!x || !router_w || !e_bias || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < workspace_bytes_for(cfg, T)) return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
     Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
-    return launch_route(cfg, T, x, router_w, e_bias, topk_idx, topk_w, w.router_part,
+    return launch_route(cfg, T, x, router_w, e_bias, topk_idx, topk_w, w.router_part, w.router_w3, d->num_sms,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -488,7 +532,7 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
     Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
     int32_t* idx = topk_idx_out ? topk_idx_out : w.topk_idx;
     float* tw = topk_w_out ? topk_w_out : w.topk_w;
-    if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, st)) != MOE_OK)
+    if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, w.router_w3, d->num_sms, st)) != MOE_OK)
         return v;
     if ((v = launch_dispatch(cfg, T, x, idx, w.offsets, w.x_perm, w.perm_src, w.row_of, w.block_counts,
                              w.block_base, st)) != MOE_OK)

@@ -99,6 +99,31 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// K1 (tensor cores), step 1: split each fp32 router weight exactly into three
+// bf16 terms, w = hi + mid + lo (each term rounds the remainder of the previous
+// ones to nearest; 3 x 8 significant bits cover fp32's 24).  A bf16 x times a
+// bf16 term is exact in fp32, so x . Wr^T = x . hi^T + x . mid^T + x . lo^T is
+// computed by one bf16 tensor-core GEMM with K = 3 H and fp32 accumulation.
+// (Splitting a float into bfloat16 terms: Henry, Tang & Heinecke, "Leveraging
+// the bfloat16 Artificial Intelligence Datatype For Higher-Precision
+// Computations", ARITH 2019.)  Output planes: w3[p][e][h], p = 0, 1, 2.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ wr,
+                                                           __nv_bfloat16* __restrict__ w3, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float w = wr[i];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        w3[i] = hi;
+        w3[n + i] = mid;
+        w3[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // K2: one warp per token.  Expert e lives in lane e % 32, slot e / 32.
 // ---------------------------------------------------------------------------
 struct RouteArgs {

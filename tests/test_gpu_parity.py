@@ -66,8 +66,9 @@ SMALL = [
     MoEShape("ragged", T=300, hidden_size=512, n_routed_experts=32, n_group=4, topk_group=2,
              num_experts_per_tok=4, moe_intermediate_size=256, n_shared_experts=1,
              routed_scaling_factor=2.5, norm_topk_prob=True, seed=7),
-    # I = 192: the gate/up column tile is cut at 64 of 128; ~500 rows per expert.
-    MoEShape("tiles", T=2000, hidden_size=256, n_routed_experts=8, n_group=2, topk_group=1,
+    # I = 192: the gate/up column tile is cut at 64 of 128; ~550 rows per expert;
+    # T >= 2048 puts the router logits on the tensor cores.
+    MoEShape("tiles", T=2200, hidden_size=256, n_routed_experts=8, n_group=2, topk_group=1,
              num_experts_per_tok=2, moe_intermediate_size=192, n_shared_experts=2,
              routed_scaling_factor=1.3, norm_topk_prob=False, seed=8),
     # No shared expert, flat routing, H = 320: the down-projection tile is cut at 64 of 256.
