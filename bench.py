@@ -369,10 +369,21 @@ def main():
     ap.add_argument("--workload", default="v3_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--profile-only", action="store_true",
+                    help="run warmup + steps layer passes and exit without timing (for profilers)")
     args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
     shape = WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
+    if args.profile_only:
+        st = StagedStep(shape, rank_inputs(shape, rank, "cuda"))
+        for _ in range(args.warmup + args.steps):
+            st.run()
+        torch.cuda.synchronize()
+        assert abi.device_status() == 0
+        print(f"profile-only: {args.warmup + args.steps} passes of {shape.name}", flush=True)
+        finish(world)
+        return
+    args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
         run_reference(args, shape, world, rank)

@@ -98,8 +98,12 @@ V3_DECODE = MoEShape("v3_decode", T=128, hidden_size=7168, n_routed_experts=256,
 V3_PREFILL = V3_DECODE.with_(name="v3_prefill", T=16384, seed=3)
 V3_SKEWED = V3_DECODE.with_(name="v3_skewed", T=8192, bias_kind="zipf", seed=4)
 
+# V3 dimensions with 32 experts (2.8 GB of weights, still 22x the L2): the case
+# for detailed profiler captures, which must stay a few GB on the device.
+V3_E32 = V3_DECODE.with_(name="v3_e32", T=4096, n_routed_experts=32, seed=5)
+
 WORKLOADS: Dict[str, MoEShape] = {w.name: w for w in
-                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED)}
+                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED, V3_E32)}
 
 
 def _normal(shape, std, gen, device, dtype):

@@ -11,8 +11,8 @@ import torch
 
 import oracle
 from sparse_moe_layer_noaux_b200 import abi
-from sparse_moe_layer_noaux_b200.workloads import (MID, TINY, V3_DECODE, V3_PREFILL, V3_SKEWED, MoEShape,
-                                                   bf16_bits, make_inputs)
+from sparse_moe_layer_noaux_b200.workloads import (MID, TINY, V3_DECODE, V3_E32, V3_PREFILL, V3_SKEWED,
+                                                   MoEShape, bf16_bits, make_inputs)
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -196,7 +196,7 @@ def test_deterministic_and_launch_count():
 # ---------------------------------------------------------------------------
 # The five workload shapes at full size.
 # ---------------------------------------------------------------------------
-FULL = [(TINY, None), (MID, 48), (V3_DECODE, 16), (V3_PREFILL, 12), (V3_SKEWED, 12)]
+FULL = [(TINY, None), (MID, 48), (V3_DECODE, 16), (V3_PREFILL, 12), (V3_SKEWED, 12), (V3_E32, 12)]
 
 
 @pytest.mark.parametrize("shape,n_sample", FULL, ids=lambda v: getattr(v, "name", str(v)))
