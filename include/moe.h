@@ -76,7 +76,8 @@ typedef enum moe_status {
                                  a pointer not 16-byte aligned, sizes beyond int32 rows */
     MOE_ERR_WORKSPACE = 3,    /* workspace null or smaller than moe_workspace_size() */
     MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
-    MOE_ERR_TIMEOUT = 5       /* a bounded device wait gave up (from moe_device_status) */
+    MOE_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (from moe_device_status) */
+    MOE_ERR_STATIC_LIMIT = 6  /* moe_dispatch_noalloc: T * E beyond its fixed scratch */
 } moe_status;
 
 /* Element type of the layer output y. */
@@ -117,6 +118,31 @@ MOE_API int moe_route(const moe_config *cfg, int64_t T, const void *x, const flo
 MOE_API int moe_dispatch(const moe_config *cfg, int64_t T, const void *x, const int32_t *topk_idx,
                  int32_t *expert_offsets, void *x_perm, int32_t *perm_src, int32_t *row_of,
                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * moe_dispatch for callers that cannot allocate device memory.  The paper has
+ * no counterpart to this entry point: it exists for callers that must not
+ * call cudaMalloc or any allocating routine themselves, for example a serving
+ * process that has handed all free device memory to a fixed pool up front, or
+ * an embedding runtime that gives this library only the buffers it already
+ * owns.  It computes exactly what moe_dispatch computes, with the same
+ * arguments minus the workspace.
+ *   Scratch: a file-scope device array of 1 MiB (262144 int32) holding the
+ *   per-block counts and bases, 2 * ceil(T / 32) * n_routed_experts int32
+ *   values; larger sizes return MOE_ERR_STATIC_LIMIT and enqueue nothing (at
+ *   n_routed_experts = 256 the limit is T <= 16384).  The array is part of the
+ *   library image: every GPU that loads the library holds it until the
+ *   process exits, and nothing is allocated or freed by this call.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents.  Calls that overlap on the GPU (on different streams
+ *   without ordering between them) race on it and give undefined results.
+ */
+MOE_API int moe_dispatch_noalloc(const moe_config *cfg, int64_t T, const void *x,
+                                 const int32_t *topk_idx, int32_t *expert_offsets, void *x_perm,
+                                 int32_t *perm_src, int32_t *row_of, void *stream);
 
 /*
  * Experts: every routed row r of expert e gives

@@ -16,7 +16,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+(MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
+ MOE_ERR_STATIC_LIMIT) = range(7)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
 
@@ -69,6 +70,7 @@ def lib():
         L.moe_route.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, sz, _P]
         L.moe_dispatch.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, _P, sz, _P]
         L.moe_experts.argtypes = [cfgp, i64] + [_P] * 15
+        L.moe_dispatch_noalloc.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, _P]
         L.moe_experts_gate_up.argtypes = [cfgp, i64] + [_P] * 10
         L.moe_experts_down.argtypes = [cfgp, i64] + [_P] * 9
         L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, ctypes.c_int32, _P]
@@ -79,7 +81,7 @@ def lib():
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
-        for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_experts",
+        for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout"):
             getattr(L, fn).restype = ctypes.c_int
@@ -127,6 +129,14 @@ def moe_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, wor
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
         _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_dispatch_noalloc(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, stream=None):
+    """moe_dispatch without a workspace: its scratch is a fixed 1 MiB array inside
+    the library (see include/moe.h for the size limit and the sharing rules)."""
+    _check("moe_dispatch_noalloc", lib().moe_dispatch_noalloc(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
+        _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _stream(stream)))
 
 
 def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_up, w_down,

@@ -381,6 +381,32 @@ int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const int
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- no-allocation dispatch
+// Scratch of moe_dispatch_noalloc: per-block expert counts and per-block bases
+// (2 x ceil(T / kDispTok) x E int32), held in this file-scope device array
+// instead of a caller workspace.  Every GPU that loads the library keeps it
+// until the process exits.
+constexpr int64_t kStaticDispatchInts = 1 << 18;  // 1 MiB
+static __device__ __align__(256) int32_t g_dispatch_scratch[kStaticDispatchInts];
+
+int32_t* g_dispatch_scratch_addr[64];
+std::mutex g_dispatch_scratch_mu;
+
+// Device address of g_dispatch_scratch on the current device, looked up once per
+// device (host code cannot use the symbol itself as a device pointer).
+int dispatch_scratch(int32_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dispatch_scratch_mu);
+    if (!g_dispatch_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        g_dispatch_scratch_addr[dev] = static_cast<int32_t*>(p);
+    }
+    *out = g_dispatch_scratch_addr[dev];
+    return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -442,6 +468,29 @@ int check_ptrs(std::initializer_list<const void*> ps) {
     return MOE_OK;
 }
 }  // namespace
+
+int moe_dispatch_noalloc(const moe_config* cfg, int64_t T, const void* x, const int32_t* topk_idx,
+                         int32_t* expert_offsets, void* x_perm, int32_t* perm_src, int32_t* row_of, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t E = cfg->n_routed_experts;
+    const int64_t nb = (T + kDispTok - 1) / kDispTok;
+    if (2 * nb * E > kStaticDispatchInts) return MOE_ERR_STATIC_LIMIT;
+    if (T == 0) {
+        if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), st) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!x || !topk_idx || !x_perm || !perm_src || !row_of) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_UNSUPPORTED;
+    int32_t* scratch = nullptr;
+    if ((v = dispatch_scratch(&scratch)) != MOE_OK) return v;
+    // Both halves are fully written by the count and scan kernels before they
+    // are read, so nothing has to be cleared between calls.
+    return launch_dispatch(cfg, T, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, scratch,
+                           scratch + nb * E, st);
+}
 
 int moe_experts_gate_up(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
                         const int32_t* expert_offsets, const void* w_gate, const void* w_up, const void* ws_gate,
@@ -554,6 +603,9 @@ const char* moe_status_string(int status) {
         case MOE_ERR_WORKSPACE: return "workspace missing or too small";
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case MOE_ERR_STATIC_LIMIT:
+            return "size exceeds the fixed scratch of the no-allocation entry point "
+                   "(2 * ceil(T / 32) * n_routed_experts must be <= 262144)";
         default: return "unknown status";
     }
 }
