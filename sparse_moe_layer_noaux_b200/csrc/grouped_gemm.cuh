@@ -38,6 +38,14 @@ constexpr int kMaxSeg = 258;       // 256 experts + shared
 constexpr uint32_t kTileABytes = kBM * kBK * 2;   // 16 KB
 constexpr uint32_t kTileBBytes = kBN * kBK * 2;   // 32 KB
 constexpr uint32_t kTmemCols = 512;               // 2 accumulators x 256 columns
+// Epilogue staging: each epilogue warp bounces its 32 rows x 32 columns through
+// shared memory so that global stores write whole lines.  Row pitch 36 floats
+// (144 B) keeps both the row-per-lane writes and the line-per-8-lanes reads of
+// 16-byte vectors free of extra bank conflicts.
+constexpr int kStagePitchF = 36;
+constexpr uint32_t kStageBytesPerWarp = 32 * kStagePitchF * 4;   // 4608 B
+constexpr uint32_t kStageBytes = 4 * kStageBytesPerWarp;         // 18 KB
+constexpr int kStagePitchH = 40;                                 // bf16 row pitch (80 B)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 
 enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
@@ -160,7 +168,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t* smemA = tiles;
     uint8_t* smemB = tiles + kStages * kTileABytes;
-    GemmSmem& S = *reinterpret_cast<GemmSmem*>(tiles + kStages * (kTileABytes + kTileBBytes));
+    uint8_t* stage_base = tiles + kStages * (kTileABytes + kTileBBytes);
+    GemmSmem& S = *reinterpret_cast<GemmSmem*>(stage_base + kStageBytes);
     volatile int* abort_flag = &S.abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -353,11 +362,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t grow = (int64_t)ti.row0 + r_local;
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
+            uint8_t* stage = stage_base + (warp - 2) * kStageBytesPerWarp;
+            const int r_warp0 = ti.m * kBM + quarter * 32;  // first row of this warp
             if (kEpi == kSwiGLU) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
-                __nv_bfloat16* out = ti.routed
-                                         ? static_cast<__nv_bfloat16*>(p.out_routed) + grow * p.ld_routed
-                                         : static_cast<__nv_bfloat16*>(p.out_shared) + grow * p.ld_shared;
+                __nv_bfloat16* out_base = ti.routed ? static_cast<__nv_bfloat16*>(p.out_routed)
+                                                    : static_cast<__nv_bfloat16*>(p.out_shared);
+                const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
+                __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(stage);
 #pragma unroll 1
                 for (int c = 0; c < (kBN / 2) / 32; ++c) {
                     __syncwarp();
@@ -366,26 +378,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tmem_ld_32x32b_x32(taddr + kBN / 2 + c * 32, u);
                     ptx::tmem_wait_ld();
                     const int col = ti.n * (kBN / 2) + c * 32;
-                    if (row_ok && col < n_valid) {
-                        uint4 pk[4];
-                        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(pk);
+                    if (col >= n_valid) continue;  // uniform across the warp
+                    // h = silu(g) * u for this lane's row, 32 columns -> staging row `lane`.
+                    uint4 pk[4];
+                    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(pk);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
-                            const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
-                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            h2[q] = __floats2bfloat162_rn(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+                    for (int q = 0; q < 16; ++q) {
+                        const float g0 = __uint_as_float(g[2 * q]), g1 = __uint_as_float(g[2 * q + 1]);
+                        const float u0 = __uint_as_float(u[2 * q]), u1 = __uint_as_float(u[2 * q + 1]);
+                        const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                        const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                        h2[q] = __floats2bfloat162_rn(h0, h1);
+                    }
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) dst[q] = pk[q];
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(hs + lane * kStagePitchH + 8 * q) = pk[q];
+                    __syncwarp();
+                    // 8 rows x 64 B per instruction: lanes 4r..4r+3 write row r's 32 values.
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int rw = it * 8 + (lane >> 2);
+                        const int r_local = r_warp0 + rw;
+                        const uint4 v = *reinterpret_cast<const uint4*>(hs + rw * kStagePitchH + 8 * (lane & 3));
+                        if (r_local < ti.rows)
+                            *reinterpret_cast<uint4*>(out_base + ((int64_t)ti.row0 + r_local) * ld + col +
+                                                      8 * (lane & 3)) = v;
                     }
                 }
             } else if (kEpi == kDown) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
-                float* out = ti.routed ? static_cast<float*>(p.out_routed) + grow * p.ld_routed
-                                       : static_cast<float*>(p.out_shared) + grow * p.ld_shared;
+                float* out_base = ti.routed ? static_cast<float*>(p.out_routed) : static_cast<float*>(p.out_shared);
+                const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
+                float* fs = reinterpret_cast<float*>(stage);
                 float wrow = 1.0f;
                 if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
 #pragma unroll 1
@@ -395,13 +419,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
                     ptx::tmem_wait_ld();
                     const int col = ti.n * kBN + c * 32;
-                    if (row_ok && col < n_valid) {
-                        float4* dst = reinterpret_cast<float4*>(out + col);
+                    if (col >= n_valid) continue;  // uniform across the warp
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            dst[q] = make_float4(__uint_as_float(v[4 * q]) * wrow, __uint_as_float(v[4 * q + 1]) * wrow,
-                                                 __uint_as_float(v[4 * q + 2]) * wrow,
-                                                 __uint_as_float(v[4 * q + 3]) * wrow);
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4*>(fs + lane * kStagePitchF + 4 * q) =
+                            make_float4(__uint_as_float(v[4 * q]) * wrow, __uint_as_float(v[4 * q + 1]) * wrow,
+                                        __uint_as_float(v[4 * q + 2]) * wrow, __uint_as_float(v[4 * q + 3]) * wrow);
+                    __syncwarp();
+                    // 4 rows x 128 B per instruction: lanes 8r..8r+7 write row r's 32 values.
+#pragma unroll
+                    for (int it = 0; it < 8; ++it) {
+                        const int rw = it * 4 + (lane >> 3);
+                        const int r_local = r_warp0 + rw;
+                        const float4 val = *reinterpret_cast<const float4*>(fs + rw * kStagePitchF + 4 * (lane & 7));
+                        if (r_local < ti.rows)
+                            *reinterpret_cast<float4*>(out_base + ((int64_t)ti.row0 + r_local) * ld + col +
+                                                       4 * (lane & 7)) = val;
                     }
                 }
             } else {

@@ -76,6 +76,10 @@ RouterPlan plan_router(int T, int E, int H) {
     return r;
 }
 
+constexpr size_t kGemmSmemBytes =
+    1024 + kStages * (kTileABytes + kTileBBytes) + kStageBytes + sizeof(GemmSmem);
+static_assert(kGemmSmemBytes <= 227 * 1024, "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
+
 // --------------------------------------------------------------- device info
 struct DeviceInfo {
     int num_sms = 0;
@@ -92,9 +96,7 @@ int device_info(DeviceInfo** out) {
     if (!d.attrs_set) {
         if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
-        const int smem = static_cast<int>(1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem));
-        static_assert(1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem) <= 227 * 1024,
-                      "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
+        const int smem = static_cast<int>(kGemmSmemBytes);
         if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -191,7 +193,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // --------------------------------------------------------------- stages
-constexpr size_t kGemmSmemBytes = 1024 + kStages * (kTileABytes + kTileBBytes) + sizeof(GemmSmem);
 
 int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
                  int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
