@@ -167,7 +167,8 @@ class StagedStep:
         self.row_of = torch.empty((T, k), dtype=torch.int32, device=d)
         self.h_r = torch.empty((T * k, I), dtype=torch.bfloat16, device=d)
         self.h_s = torch.empty((T, max(S * I, 8)), dtype=torch.bfloat16, device=d)
-        self.y_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=d)
+        self.y_perm = torch.empty((T * k + T, H), dtype=torch.float16, device=d)
+        self.y_sc = torch.empty((T * k + T, abi.y_perm_scale_cols(H)), dtype=torch.uint8, device=d)
         self.y = torch.empty((T, H), dtype=torch.float32, device=d)
 
     def run(self, events=None):
@@ -186,9 +187,9 @@ class StagedStep:
                                 i["ws_gate"], i["ws_up"], self.h_r, self.h_s)
         rec(3)
         abi.moe_experts_down(self.cfg, T, self.h_r, self.h_s, self.off, self.perm_src, self.w, i["w_down"],
-                             i["ws_down"], self.y_perm)
+                             i["ws_down"], self.y_perm, self.y_sc)
         rec(4)
-        abi.moe_combine(self.cfg, T, self.y_perm, self.row_of, self.y)
+        abi.moe_combine(self.cfg, T, self.y_perm, self.y_sc, self.row_of, self.y)
         rec(5)
 
 

@@ -147,22 +147,25 @@ MOE_API int moe_dispatch_noalloc(const moe_config *cfg, int64_t T, const void *x
 /*
  * Experts: every routed row r of expert e gives
  *   h_routed[r] = silu(x_perm[r] . w_gate[e]^T) * (x_perm[r] . w_up[e]^T)   bf16 [T*k, I]
- *   y_perm[r]   = topk_w[perm_src[r]] * (h_routed[r] . w_down[e]^T)         fp32 [T*k + T, H]
+ *   y_perm[r]   = topk_w[perm_src[r]] * (h_routed[r] . w_down[e]^T)
  * and every token t runs the shared expert(s) on x itself:
  *   h_shared[t]        = silu(x[t] . ws_gate^T) * (x[t] . ws_up^T)          bf16 [T, S*I]
  *   y_perm[T*k + t]    = h_shared[t] . ws_down^T
  * ("The Evolving Transformer · 07", § 02 and § 03.)  Grouped tensor-core
  * GEMMs over the variable-length expert segments given by expert_offsets;
- * fp32 accumulation; h is stored as bf16 (it is the next GEMM's operand) and
- * y_perm as fp32, so the layer output is rounded to bf16 only once, in the
- * combine.  When S == 0 the shared pointers may be NULL and y_perm needs only
- * T*k rows.
+ * fp32 accumulation; h is stored as bf16 (it is the next GEMM's operand).
+ * y_perm [T*k + T, H] is stored block-scaled: fp16 values plus one scale code
+ * per 32 columns in y_perm_scale [T*k + T, ceil(H / 256) * 8] (uint8); a value
+ * is fp16 * 2^(code - 141), the code chosen so that the block's largest
+ * magnitude lies in [2^14, 2^15) before rounding to fp16 (fp16 precision
+ * relative to the block maximum, no overflow).  When S == 0 the shared
+ * pointers may be NULL and y_perm needs only T*k rows.
  */
 MOE_API int moe_experts(const moe_config *cfg, int64_t T, const void *x, const void *x_perm,
                 const int32_t *expert_offsets, const int32_t *perm_src, const float *topk_w,
                 const void *w_gate, const void *w_up, const void *w_down,
                 const void *ws_gate, const void *ws_up, const void *ws_down,
-                void *h_routed, void *h_shared, void *y_perm, void *stream);
+                void *h_routed, void *h_shared, void *y_perm, void *y_perm_scale, void *stream);
 
 /* The two halves of moe_experts, for callers that schedule them separately:
  * gate_up writes h_routed / h_shared (gate and up projections with the SwiGLU
@@ -175,17 +178,19 @@ MOE_API int moe_experts_gate_up(const moe_config *cfg, int64_t T, const void *x,
 MOE_API int moe_experts_down(const moe_config *cfg, int64_t T, const void *h_routed,
                              const void *h_shared, const int32_t *expert_offsets,
                              const int32_t *perm_src, const float *topk_w, const void *w_down,
-                             const void *ws_down, void *y_perm, void *stream);
+                             const void *ws_down, void *y_perm, void *y_perm_scale, void *stream);
 
 /*
  * Combine: y[t] = y_perm[T*k + t] (shared, if S > 0) + sum_{j<k} y_perm[row_of[t, j]],
- * y_perm fp32 rows summed in fp32 in that order and stored as y_dtype [T, H]
+ * block-scaled y_perm rows (see moe_experts) decoded and summed in fp32 in
+ * that order, stored as y_dtype [T, H]
  * (a moe_dtype) — the page's output[mask] += w * expert_out and
  * `shared_expert_out + output` ("The Evolving Transformer · 07", § 02), as a
  * deterministic gather.
  */
-MOE_API int moe_combine(const moe_config *cfg, int64_t T, const void *y_perm, const int32_t *row_of,
-                void *y, int32_t y_dtype, void *stream);
+MOE_API int moe_combine(const moe_config *cfg, int64_t T, const void *y_perm,
+                const void *y_perm_scale, const int32_t *row_of, void *y, int32_t y_dtype,
+                void *stream);
 
 /*
  * The whole layer: route, dispatch, experts, combine, on one stream.

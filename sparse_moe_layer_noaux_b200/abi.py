@@ -69,11 +69,11 @@ def lib():
         L.moe_workspace_size.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
         L.moe_route.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, sz, _P]
         L.moe_dispatch.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, _P, sz, _P]
-        L.moe_experts.argtypes = [cfgp, i64] + [_P] * 15
+        L.moe_experts.argtypes = [cfgp, i64] + [_P] * 16
         L.moe_dispatch_noalloc.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P, _P]
         L.moe_experts_gate_up.argtypes = [cfgp, i64] + [_P] * 10
-        L.moe_experts_down.argtypes = [cfgp, i64] + [_P] * 9
-        L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, ctypes.c_int32, _P]
+        L.moe_experts_down.argtypes = [cfgp, i64] + [_P] * 10
+        L.moe_combine.argtypes = [cfgp, i64, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.moe_forward.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, _P, _P, _P, sz, _P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -139,12 +139,26 @@ def moe_dispatch_noalloc(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row
         _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _stream(stream)))
 
 
+def y_perm_scale_cols(H: int) -> int:
+    """Row pitch (bytes) of the y_perm block-scale codes: one per 32 columns, padded to 8."""
+    return (H // 32 + 7) // 8 * 8
+
+
+def decode_y_perm(y_perm: torch.Tensor, y_perm_scale: torch.Tensor) -> torch.Tensor:
+    """fp32 values of a block-scaled y_perm: fp16 * 2^(code - 141), one code per 32 columns."""
+    rows, H = y_perm.shape
+    codes = y_perm_scale[:, : H // 32].to(torch.int32)
+    f = torch.ldexp(torch.ones_like(codes, dtype=torch.float32), codes - 141)
+    return (y_perm.float().view(rows, H // 32, 32) * f[:, :, None]).view(rows, H)
+
+
 def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_up, w_down,
-                ws_gate, ws_up, ws_down, h_routed, h_shared, y_perm, stream=None):
+                ws_gate, ws_up, ws_down, h_routed, h_shared, y_perm, y_perm_scale, stream=None):
     _check("moe_experts", lib().moe_experts(
         ctypes.byref(_cfg(cfg)), T, _ptr(x), _ptr(x_perm), _ptr(expert_offsets), _ptr(perm_src),
         _ptr(topk_w), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up),
-        _ptr(ws_down), _ptr(h_routed), _ptr(h_shared), _ptr(y_perm), _stream(stream)))
+        _ptr(ws_down), _ptr(h_routed), _ptr(h_shared), _ptr(y_perm), _ptr(y_perm_scale),
+        _stream(stream)))
 
 
 def moe_experts_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed,
@@ -155,15 +169,16 @@ def moe_experts_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate
 
 
 def moe_experts_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down,
-                     y_perm, stream=None):
+                     y_perm, y_perm_scale, stream=None):
     _check("moe_experts_down", lib().moe_experts_down(
         ctypes.byref(_cfg(cfg)), T, _ptr(h_routed), _ptr(h_shared), _ptr(expert_offsets),
-        _ptr(perm_src), _ptr(topk_w), _ptr(w_down), _ptr(ws_down), _ptr(y_perm), _stream(stream)))
+        _ptr(perm_src), _ptr(topk_w), _ptr(w_down), _ptr(ws_down), _ptr(y_perm), _ptr(y_perm_scale),
+        _stream(stream)))
 
 
-def moe_combine(cfg, T, y_perm, row_of, y, stream=None):
-    _check("moe_combine", lib().moe_combine(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(row_of),
-                                            _ptr(y), out_dtype_code(y), _stream(stream)))
+def moe_combine(cfg, T, y_perm, y_perm_scale, row_of, y, stream=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(y_perm_scale),
+                                            _ptr(row_of), _ptr(y), out_dtype_code(y), _stream(stream)))
 
 
 def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,

@@ -3,9 +3,9 @@
 // done for all experts at once as a stable counting sort:
 //   1. count:  per block of kDispTok tokens, how many slots go to each expert;
 //   2. scan:   expert offsets, and each block's starting row inside every expert;
-//   3. place:  stable rank of every slot (ascending (t, j)) -> row_of / perm_src,
-//              then each token's row is copied once from x and written to its k
-//              rows of x_perm with 16-byte vector stores.
+//   3. place:  stable rank of every slot (ascending (t, j)) -> row_of / perm_src;
+//   4. scatter: each token's row is read once from x and written to its k rows
+//              of x_perm with 16-byte vector stores.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -74,13 +74,10 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __res
 }
 
 __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
-    const int32_t* __restrict__ topk_idx, int T, int K, int E, int H,
-    const int32_t* __restrict__ block_base, const __nv_bfloat16* __restrict__ x,
-    __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ perm_src,
-    int32_t* __restrict__ row_of) {
+    const int32_t* __restrict__ topk_idx, int T, int K, int E, const int32_t* __restrict__ block_base,
+    int32_t* __restrict__ perm_src, int32_t* __restrict__ row_of) {
     extern __shared__ int smem_i[];
     int* run = smem_i;              // [E] next free row of each expert for this block
-    int* rows = smem_i + E;         // [kDispTok * K] destination rows of this block's slots
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int kWarps = kDispThreads / 32;
     for (int e = tid; e < E; e += blockDim.x) run[e] = block_base[(int64_t)blockIdx.x * E + e];
@@ -111,31 +108,27 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
             __syncthreads();
         }
         if (valid) {
-            rows[q] = row;
             row_of[q0 + q] = row;
             perm_src[row] = (int32_t)(q0 + q);
         }
     }
-    __syncthreads();
+}
 
-    // Copy: each warp moves whole tokens; one 16-byte load feeds K stores, four
-    // loads in flight per lane.
-    const int chunks = H / 8;
-    for (int tl = warp; tl < ntok; tl += kWarps) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t0 + tl) * H);
-        for (int c0 = lane; c0 < chunks; c0 += 128) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (c0 + 32 * u < chunks) v[u] = src[c0 + 32 * u];
-            for (int j = 0; j < K; ++j) {
-                uint4* dst = reinterpret_cast<uint4*>(x_perm + (int64_t)rows[tl * K + j] * H);
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (c0 + 32 * u < chunks) dst[c0 + 32 * u] = v[u];
-            }
-        }
-    }
+// Row copy: block (t, c) moves 16-byte slices [256 c, 256 c + 256) of token t's
+// row; each slice is loaded once and stored to the token's k rows of x_perm.
+// The grid is T x ceil(H / 2048) blocks, so small batches still spread over
+// every SM.
+__global__ void __launch_bounds__(256) dispatch_scatter_kernel(const __nv_bfloat16* __restrict__ x,
+                                                               const int32_t* __restrict__ row_of, int K,
+                                                               int H, __nv_bfloat16* __restrict__ x_perm) {
+    __shared__ int rows[32];
+    const int t = blockIdx.x;
+    if (threadIdx.x < K) rows[threadIdx.x] = row_of[(int64_t)t * K + threadIdx.x];
+    __syncthreads();
+    const int c = blockIdx.y * 256 + threadIdx.x;
+    if (c >= H / 8) return;
+    const uint4 v = reinterpret_cast<const uint4*>(x + (int64_t)t * H)[c];
+    for (int j = 0; j < K; ++j) reinterpret_cast<uint4*>(x_perm + (int64_t)rows[j] * H)[c] = v;
 }
 
 }  // namespace moe

@@ -7,8 +7,10 @@
 //   kSwiGLU  h = silu(A Wg^T) * (A Wu^T)   — gate and up tiles side by side in one
 //            N = 256 accumulator (128 gate columns | 128 up columns), fused epilogue;
 //   kDown    y = w_row * (h Wd^T)           — N = 256, routing weight in the epilogue,
-//            fp32 output (the combine sums k + 1 of these rows before the single
-//            rounding of the layer output to bf16);
+//            output in block-scaled fp16 (fp16 values, one power-of-two scale per
+//            32 consecutive columns of a row, chosen from the block's largest
+//            magnitude): fp16's 11-bit precision relative to the block maximum, no
+//            overflow, half the bytes of fp32;
 //   kLogits  router logits l = x Wr^T in fp32 from an exact three-way bf16 split
 //            Wr = hi + mid + lo (one segment of T rows, K = 3 H concatenated over the
 //            three planes, N = E rounded up to 16), fp32 output.
@@ -24,6 +26,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "sm100_ptx.cuh"
 
@@ -47,6 +50,11 @@ constexpr uint32_t kStageBytesPerWarp = 32 * kStagePitchF * 4;   // 4608 B
 constexpr uint32_t kStageBytes = 4 * kStageBytesPerWarp;         // 18 KB
 constexpr int kStagePitchH = 40;                                 // bf16 row pitch (80 B)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
+// Partial row tiles with at most this many valid rows are computed transposed.
+#ifndef MOE_SWAP_MAX_ROWS
+#define MOE_SWAP_MAX_ROWS 112
+#endif
+constexpr int kSwapMaxRows = MOE_SWAP_MAX_ROWS;
 
 enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
 
@@ -63,15 +71,19 @@ struct GemmParams {
     int n_valid_routed, n_valid_shared;   // valid output columns
     int b_rows_per_expert;                // rows of one expert in the routed B map
     void* out_routed;                     // row r of routed segment -> out_routed + r*ld
-    int64_t ld_routed;                    // (bf16 elements for kSwiGLU, fp32 for kDown)
+    int64_t ld_routed;                    // (bf16 elements for kSwiGLU, fp16 for kDown)
     void* out_shared;                     // row t of the shared segment
     int64_t ld_shared;
+    uint8_t* scale_routed;                // kDown: block scale codes, [rows][scale_ld]
+    uint8_t* scale_shared;
+    int64_t scale_ld;
     const int32_t* perm_src;              // kDown: routed row -> slot
     const float* topk_w;                  // kDown: slot -> routing weight
     uint32_t idesc;                       // MMA instruction descriptor (M = 128, N)
     uint32_t b_tile_bytes;                // bytes one B tile load brings in
     int kb_plane;                         // kLogits: K blocks per plane (H / 64)
     int b_plane_rows;                     // kLogits: rows of one plane in the B map (E)
+    int allow_swap;                       // compute partial row tiles transposed
 };
 
 struct TileInfo {
@@ -82,6 +94,9 @@ struct TileInfo {
     int rows;       // rows of the segment
     int row0;       // first row of the segment in the A / output row space
     int kb;         // K blocks
+    int r;          // valid rows in this tile (1..128)
+    int swap;       // 1: computed transposed (weights as the M operand, see below)
+    int rpad;       // swap: token columns of the MMA, r rounded up to 16
 };
 
 struct GemmSmem {
@@ -100,6 +115,16 @@ struct GemmSmem {
 };
 
 __device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_moe_error, 0u, code); }
+
+// Block-scaled fp16: a block of 32 values whose largest magnitude has biased
+// fp32 exponent E gets the code c = clamp(E, 15, 254); values are stored as
+// fp16(v * 2^(141 - c)), which puts the block maximum in [2^14, 2^15), and read
+// back as fp16 * 2^(c - 141).  Both factors are normal fp32 powers of two, so
+// scaling is exact; NaN and Inf keep their class.
+__device__ __forceinline__ uint32_t block_scale_code(uint32_t max_abs_bits) {
+    return min(max(max_abs_bits >> 23, 15u), 254u);
+}
+__device__ __forceinline__ float block_encode_factor(uint32_t code) { return __uint_as_float((268u - code) << 23); }
 
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up
 // (returns false) when the CTA is aborting or after kWaitLimitNs.
@@ -138,6 +163,16 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem& s, const GemmPar
     ti.n = local / mt;
     ti.m = local - ti.n * mt;
     ti.kb = ti.routed ? p.kb_routed : p.kb_shared;
+    ti.r = min(kBM, ti.rows - ti.m * kBM);
+    // A segment that fits in one partial row tile (decode-sized: a few tokens per
+    // expert) is computed transposed: the two 128-row halves of the weight tile
+    // become the M = 128 operand and the r token rows the N operand (N = r rounded
+    // up to 16); the operand tiles in shared memory are the same as for a normal
+    // tile.  The last partial tile of a larger segment stays a normal 128-row tile:
+    // measured on B200, narrow-N MMAs are not proportionally cheaper, and while
+    // the gate/up GEMM is tensor-bound transposing those tails made it slower.
+    ti.swap = (p.allow_swap && ti.rows <= kSwapMaxRows) ? 1 : 0;
+    ti.rpad = (ti.r + 15) & ~15;
     return ti;
 }
 
@@ -329,11 +364,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ptx::smem_u32(smemA + stage * kTileABytes);
                     const uint32_t b_addr = ptx::smem_u32(smemB + stage * kTileBBytes);
+                    if (!ti.swap) {
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        const uint64_t ad = ptx::sw128_kmajor_desc(a_addr + k * 32);
-                        const uint64_t bd = ptx::sw128_kmajor_desc(b_addr + k * 32);
-                        ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            const uint64_t ad = ptx::sw128_kmajor_desc(a_addr + k * 32);
+                            const uint64_t bd = ptx::sw128_kmajor_desc(b_addr + k * 32);
+                            ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+                        }
+                    } else {
+                        // D0[i][j] = W[i] . A[j] for weight rows i of the first B half,
+                        // D1 (128 columns further) for the second half.
+                        const uint32_t idesc_t = ptx::idesc_bf16_f32(kBM, ti.rpad);
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            const uint64_t xd = ptx::sw128_kmajor_desc(a_addr + k * 32);
+                            const uint64_t w0 = ptx::sw128_kmajor_desc(b_addr + k * 32);
+                            const uint64_t w1 = ptx::sw128_kmajor_desc(b_addr + kTileBBytes / 2 + k * 32);
+                            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+                            ptx::mma_bf16(d_tmem, w0, xd, idesc_t, accum);
+                            ptx::mma_bf16(d_tmem + kBN / 2, w1, xd, idesc_t, accum);
+                        }
                     }
                     ptx::mma_commit(ptx::smem_u32(&S.empty[stage]));
                     if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -364,7 +414,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                    (static_cast<uint32_t>(quarter * 32) << 16);
             uint8_t* stage = stage_base + (warp - 2) * kStageBytesPerWarp;
             const int r_warp0 = ti.m * kBM + quarter * 32;  // first row of this warp
-            if (kEpi == kSwiGLU) {
+            const int64_t tile_row0 = (int64_t)ti.row0 + ti.m * kBM;
+            if (ti.swap && kEpi == kSwiGLU) {
+                // Transposed tile: TMEM lane = output column i of this 128-column tile,
+                // TMEM column j = token row j (gate at 0.., up at 128..).
+                const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
+                __nv_bfloat16* out_base = ti.routed ? static_cast<__nv_bfloat16*>(p.out_routed)
+                                                    : static_cast<__nv_bfloat16*>(p.out_shared);
+                const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
+                const int col = ti.n * (kBN / 2) + quarter * 32 + lane;
+                const bool col_ok = col < n_valid;
+#pragma unroll 1
+                for (int c = 0; c * 32 < ti.r; ++c) {
+                    __syncwarp();
+                    uint32_t g[32], u[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, g);
+                    ptx::tmem_ld_32x32b_x32(taddr + kBN / 2 + c * 32, u);
+                    ptx::tmem_wait_ld();
+                    const int jmax = min(32, ti.r - c * 32);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        if (jj < jmax && col_ok) {
+                            const float gv = __uint_as_float(g[jj]), uv = __uint_as_float(u[jj]);
+                            out_base[(tile_row0 + c * 32 + jj) * ld + col] =
+                                __float2bfloat16_rn(gv / (1.0f + __expf(-gv)) * uv);
+                        }
+                    }
+                }
+            } else if (ti.swap && kEpi == kDown) {
+                // Transposed tile: TMEM lane = output column, column j = token row j;
+                // the second 128 output columns sit 128 TMEM columns further.  The 32
+                // lanes of a warp hold exactly one 32-column scale block of a row.
+                const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
+                __half* out_base = ti.routed ? static_cast<__half*>(p.out_routed) : static_cast<__half*>(p.out_shared);
+                uint8_t* sc_base = ti.routed ? p.scale_routed : p.scale_shared;
+                const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
+#pragma unroll 1
+                for (int c = 0; c * 32 < ti.r; ++c) {
+                    // Routing weight of token row c*32 + lane, shared across the warp below.
+                    float wl = 1.0f;
+                    if (ti.routed && c * 32 + lane < ti.r) wl = p.topk_w[p.perm_src[tile_row0 + c * 32 + lane]];
+                    const int jmax = min(32, ti.r - c * 32);
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int col0 = ti.n * kBN + hh * (kBN / 2) + quarter * 32;  // block start
+                        const bool blk_ok = col0 < n_valid;                            // warp-uniform
+                        __syncwarp();
+                        uint32_t v[32];
+                        ptx::tmem_ld_32x32b_x32(taddr + hh * (kBN / 2) + c * 32, v);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const float val = __uint_as_float(v[jj]) * __shfl_sync(0xffffffffu, wl, jj);
+                            const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(val)));
+                            if (jj < jmax && blk_ok) {
+                                const uint32_t code = block_scale_code(mx);
+                                const int64_t row = tile_row0 + c * 32 + jj;
+                                out_base[row * ld + col0 + lane] = __float2half_rn(val * block_encode_factor(code));
+                                if (lane == 0) sc_base[row * p.scale_ld + col0 / 32] = static_cast<uint8_t>(code);
+                            }
+                        }
+                    }
+                }
+            } else if (kEpi == kSwiGLU) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
                 __nv_bfloat16* out_base = ti.routed ? static_cast<__nv_bfloat16*>(p.out_routed)
                                                     : static_cast<__nv_bfloat16*>(p.out_shared);
@@ -407,34 +519,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else if (kEpi == kDown) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
-                float* out_base = ti.routed ? static_cast<float*>(p.out_routed) : static_cast<float*>(p.out_shared);
+                __half* out_base = ti.routed ? static_cast<__half*>(p.out_routed) : static_cast<__half*>(p.out_shared);
+                uint8_t* sc_base = ti.routed ? p.scale_routed : p.scale_shared;
                 const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
-                float* fs = reinterpret_cast<float*>(stage);
+                __half* hs = reinterpret_cast<__half*>(stage);
                 float wrow = 1.0f;
                 if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
-#pragma unroll 1
+                uint32_t codes[kBN / 32];
+#pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) {
                     __syncwarp();
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
                     ptx::tmem_wait_ld();
                     const int col = ti.n * kBN + c * 32;
+                    codes[c] = 0;
                     if (col >= n_valid) continue;  // uniform across the warp
+                    // This lane's row, one 32-column block: scale from the block maximum.
+                    uint32_t mx = 0;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<float4*>(fs + lane * kStagePitchF + 4 * q) =
-                            make_float4(__uint_as_float(v[4 * q]) * wrow, __uint_as_float(v[4 * q + 1]) * wrow,
-                                        __uint_as_float(v[4 * q + 2]) * wrow, __uint_as_float(v[4 * q + 3]) * wrow);
+                    for (int q = 0; q < 32; ++q) mx = max(mx, __float_as_uint(fabsf(__uint_as_float(v[q]) * wrow)));
+                    const uint32_t code = block_scale_code(mx);
+                    const float f = block_encode_factor(code);
+                    codes[c] = code;
+                    uint4 pk[4];
+                    __half2* h2 = reinterpret_cast<__half2*>(pk);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        h2[q] = __floats2half2_rn(__uint_as_float(v[2 * q]) * wrow * f,
+                                                  __uint_as_float(v[2 * q + 1]) * wrow * f);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(hs + lane * kStagePitchH + 8 * q) = pk[q];
                     __syncwarp();
-                    // 4 rows x 128 B per instruction: lanes 8r..8r+7 write row r's 32 values.
+                    // 8 rows x 64 B per instruction: lanes 4r..4r+3 write row r's 32 values.
 #pragma unroll
-                    for (int it = 0; it < 8; ++it) {
-                        const int rw = it * 4 + (lane >> 3);
+                    for (int it = 0; it < 4; ++it) {
+                        const int rw = it * 8 + (lane >> 2);
                         const int r_local = r_warp0 + rw;
-                        const float4 val = *reinterpret_cast<const float4*>(fs + rw * kStagePitchF + 4 * (lane & 7));
+                        const uint4 val = *reinterpret_cast<const uint4*>(hs + rw * kStagePitchH + 8 * (lane & 3));
                         if (r_local < ti.rows)
-                            *reinterpret_cast<float4*>(out_base + ((int64_t)ti.row0 + r_local) * ld + col +
-                                                       4 * (lane & 7)) = val;
+                            *reinterpret_cast<uint4*>(out_base + ((int64_t)ti.row0 + r_local) * ld + col +
+                                                      8 * (lane & 3)) = val;
+                    }
+                }
+                // The row's scale codes of this 256-column tile: one 8-byte store when whole.
+                if (row_ok) {
+                    uint8_t* dst = sc_base + grow * p.scale_ld + ti.n * (kBN / 32);
+                    const int nblk = min(kBN / 32, (n_valid - ti.n * kBN) / 32);
+                    if (nblk == kBN / 32) {
+                        uint2 pk;
+                        pk.x = codes[0] | (codes[1] << 8) | (codes[2] << 16) | (codes[3] << 24);
+                        pk.y = codes[4] | (codes[5] << 8) | (codes[6] << 16) | (codes[7] << 24);
+                        *reinterpret_cast<uint2*>(dst) = pk;
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < kBN / 32; ++c)
+                            if (c < nblk) dst[c] = static_cast<uint8_t>(codes[c]);
                     }
                 }
             } else {

@@ -29,6 +29,9 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Row pitch in bytes of the y_perm scale codes: one per 32 columns, padded to 8.
+inline int64_t scale_ld(int64_t H) { return (H / 32 + 7) / 8 * 8; }
+
 // --------------------------------------------------------------- validation
 int validate_cfg(const moe_config* c, int64_t T) {
     if (!c || T < 0) return MOE_ERR_INVALID_ARG;
@@ -124,7 +127,8 @@ struct Workspace {
     __nv_bfloat16* x_perm;    // [T*k, H]
     __nv_bfloat16* h_routed;  // [T*k, I]
     __nv_bfloat16* h_shared;  // [T, S*I]
-    float* y_perm;            // [T*k + T, H] fp32
+    __half* y_perm;           // [T*k + T, H] block-scaled fp16 values
+    uint8_t* y_scale;         // [T*k + T, scale_ld] block scale codes
     size_t bytes;
 };
 
@@ -152,7 +156,8 @@ Workspace carve(const moe_config* c, int64_t T, uint8_t* base) {
     w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * H));
     w.h_routed = reinterpret_cast<__nv_bfloat16*>(take(2 * T * K * I));
     w.h_shared = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
-    w.y_perm = reinterpret_cast<float*>(take(4 * (T * K + T) * H));
+    w.y_perm = reinterpret_cast<__half*>(take(2 * (T * K + T) * H));
+    w.y_scale = reinterpret_cast<uint8_t*>(take((T * K + T) * scale_ld(H)));
     w.bytes = off;
     return w;
 }
@@ -260,11 +265,12 @@ int launch_dispatch(const moe_config* c, int64_t T, const void* x, const int32_t
     dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
                                                                       block_counts);
     dispatch_scan_kernel<<<1, 256, 0, st>>>(block_counts, nb, E, block_base, offsets);
-    const size_t smem = sizeof(int) * (E + kDispTok * K);
-    dispatch_place_kernel<<<nb, kDispThreads, smem, st>>>(
-        idx, static_cast<int>(T), K, E, H, block_base, static_cast<const __nv_bfloat16*>(x),
-        static_cast<__nv_bfloat16*>(x_perm), perm_src, row_of);
-    count_launch(3);
+    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
+                                                                     perm_src, row_of);
+    const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
+    dispatch_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H,
+                                                static_cast<__nv_bfloat16*>(x_perm));
+    count_launch(4);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -315,6 +321,7 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.ld_shared = SI;
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
+    p.allow_swap = 1;
     const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -325,7 +332,7 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
 // K5: y_perm = w * (h Wd^T) for routed rows, h_shared Wsd^T for the shared rows.
 int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void* h_shared,
                 const int32_t* offsets, const int32_t* perm_src, const float* topk_w, const void* w_down,
-                const void* ws_down, void* y_perm, int num_sms, cudaStream_t st) {
+                const void* ws_down, void* y_perm, void* y_scale, int num_sms, cudaStream_t st) {
     const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
     const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
     const int64_t R = T * K;
@@ -352,12 +359,16 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.b_rows_per_expert = static_cast<int>(H);
     p.out_routed = y_perm;
     p.ld_routed = H;
-    p.out_shared = static_cast<float*>(y_perm) + R * H;
+    p.out_shared = static_cast<__half*>(y_perm) + R * H;
     p.ld_shared = H;
+    p.scale_ld = scale_ld(H);
+    p.scale_routed = static_cast<uint8_t*>(y_scale);
+    p.scale_shared = static_cast<uint8_t*>(y_scale) + R * p.scale_ld;
     p.perm_src = perm_src;
     p.topk_w = topk_w;
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
+    p.allow_swap = 1;
     const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);
@@ -365,19 +376,20 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
-                   int y_dtype, cudaStream_t st) {
-    const unsigned g = static_cast<unsigned>((T + 7) / 8);
+int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const void* y_scale,
+                   const int32_t* row_of, void* y, int y_dtype, cudaStream_t st) {
+    const dim3 g(static_cast<unsigned>(T), static_cast<unsigned>((c->hidden_size / 8 + 255) / 256));
     const int has_shared = c->n_shared_experts > 0 ? 1 : 0;
     if (y_dtype == MOE_DTYPE_BF16)
-        combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
-                                                         static_cast<int>(T), c->num_experts_per_tok,
-                                                         c->hidden_size, has_shared,
-                                                         static_cast<__nv_bfloat16*>(y));
+        combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+            static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
+            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared,
+            static_cast<__nv_bfloat16*>(y));
     else
-        combine_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(y_perm), row_of,
-                                                 static_cast<int>(T), c->num_experts_per_tok, c->hidden_size,
-                                                 has_shared, static_cast<float*>(y));
+        combine_kernel<float><<<g, 256, 0, st>>>(
+            static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
+            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared,
+            static_cast<float*>(y));
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -510,28 +522,29 @@ int moe_experts_gate_up(const moe_config* cfg, int64_t T, const void* x, const v
 
 int moe_experts_down(const moe_config* cfg, int64_t T, const void* h_routed, const void* h_shared,
                      const int32_t* expert_offsets, const int32_t* perm_src, const float* topk_w,
-                     const void* w_down, const void* ws_down, void* y_perm, void* stream) {
+                     const void* w_down, const void* ws_down, void* y_perm, void* y_perm_scale, void* stream) {
     int v = validate_cfg(cfg, T);
     if (v != MOE_OK) return v;
     if (T == 0) return MOE_OK;
     if (!expert_offsets || !perm_src || !topk_w) return MOE_ERR_INVALID_ARG;
-    if ((v = check_ptrs({h_routed, w_down, y_perm})) != MOE_OK) return v;
+    if ((v = check_ptrs({h_routed, w_down, y_perm, y_perm_scale})) != MOE_OK) return v;
     if (cfg->n_shared_experts > 0 && (v = check_ptrs({h_shared, ws_down})) != MOE_OK) return v;
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
     return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
-                       d->num_sms, static_cast<cudaStream_t>(stream));
+                       y_perm_scale, d->num_sms, static_cast<cudaStream_t>(stream));
 }
 
 int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
                 const int32_t* expert_offsets, const int32_t* perm_src, const float* topk_w, const void* w_gate,
                 const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
-                const void* ws_down, void* h_routed, void* h_shared, void* y_perm, void* stream) {
+                const void* ws_down, void* h_routed, void* h_shared, void* y_perm, void* y_perm_scale,
+                void* stream) {
     int v = validate_cfg(cfg, T);
     if (v != MOE_OK) return v;
     if (T == 0) return MOE_OK;
     if (!expert_offsets || !perm_src || !topk_w) return MOE_ERR_INVALID_ARG;
-    if ((v = check_ptrs({x_perm, w_gate, w_up, w_down, h_routed, y_perm})) != MOE_OK) return v;
+    if ((v = check_ptrs({x_perm, w_gate, w_up, w_down, h_routed, y_perm, y_perm_scale})) != MOE_OK) return v;
     if (cfg->n_shared_experts > 0 && (v = check_ptrs({x, ws_gate, ws_up, ws_down, h_shared})) != MOE_OK)
         return v;
     DeviceInfo* d = nullptr;
@@ -541,18 +554,18 @@ int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_p
                             d->num_sms, st)) != MOE_OK)
         return v;
     return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
-                       d->num_sms, st);
+                       y_perm_scale, d->num_sms, st);
 }
 
-int moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const int32_t* row_of, void* y,
-                int32_t y_dtype, void* stream) {
+int moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const void* y_perm_scale,
+                const int32_t* row_of, void* y, int32_t y_dtype, void* stream) {
     int v = validate_cfg(cfg, T);
     if (v != MOE_OK) return v;
     if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!y_perm || !row_of || !y) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
-    return launch_combine(cfg, T, y_perm, row_of, y, y_dtype, static_cast<cudaStream_t>(stream));
+    if (!y_perm || !y_perm_scale || !row_of || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(y) || !aligned16(y_perm_scale)) return MOE_ERR_UNSUPPORTED;
+    return launch_combine(cfg, T, y_perm, y_perm_scale, row_of, y, y_dtype, static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
@@ -591,9 +604,9 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
                             w.h_shared, d->num_sms, st)) != MOE_OK)
         return v;
     if ((v = launch_down(cfg, T, w.h_routed, w.h_shared, w.offsets, w.perm_src, tw, w_down, ws_down, w.y_perm,
-                         d->num_sms, st)) != MOE_OK)
+                         w.y_scale, d->num_sms, st)) != MOE_OK)
         return v;
-    return launch_combine(cfg, T, w.y_perm, w.row_of, y, y_dtype, st);
+    return launch_combine(cfg, T, w.y_perm, w.y_scale, w.row_of, y, y_dtype, st);
 }
 
 const char* moe_status_string(int status) {

@@ -117,17 +117,23 @@ def test_stages_compose_to_forward():
 
     h_r = torch.empty((T * k, I), dtype=torch.bfloat16, device=dev)
     h_s = torch.empty((T, S * I), dtype=torch.bfloat16, device=dev)
-    y_perm = torch.empty((T * k + T, H), dtype=torch.float32, device=dev)
+    y_perm = torch.empty((T * k + T, H), dtype=torch.float16, device=dev)
+    y_sc = torch.empty((T * k + T, abi.y_perm_scale_cols(H)), dtype=torch.uint8, device=dev)
     abi.moe_experts(cfg, T, inp["x"], x_perm, offsets, perm_src, w, inp["w_gate"], inp["w_up"],
-                    inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], h_r, h_s, y_perm)
+                    inp["w_down"], inp["ws_gate"], inp["ws_up"], inp["ws_down"], h_r, h_s, y_perm, y_sc)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
-    abi.moe_combine(cfg, T, y_perm, row_of, y)
+    abi.moe_combine(cfg, T, y_perm, y_sc, row_of, y)
     y16 = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    abi.moe_combine(cfg, T, y_perm, row_of, y16)
+    abi.moe_combine(cfg, T, y_perm, y_sc, row_of, y16)
     torch.cuda.synchronize()
     assert abi.device_status() == 0
 
     # Expert stage against float64 matrix products of the same bf16 operands.
+    yp = abi.decode_y_perm(y_perm, y_sc)
+    # Block scaling: every 32-column block's largest magnitude sits in [2^14, 2^15] as fp16.
+    blk = y_perm.float().abs().view(y_perm.shape[0], -1, 32).amax(-1)
+    nz = blk > 0
+    assert bool(((blk[nz] >= 2.0 ** 14) & (blk[nz] <= 2.0 ** 15)).all())
     off = offsets.cpu().tolist()
     for e in range(E):
         a, b = off[e], off[e + 1]
@@ -139,17 +145,17 @@ def test_stages_compose_to_forward():
         h_ref = torch.nn.functional.silu(g) * u
         parity.assert_bf16_rounded(h_r[a:b], h_ref, f"h expert {e}")
         y_ref = (h_r[a:b].double() @ inp["w_down"][e].double().T) * w.view(-1)[perm_src[a:b].long()].double()[:, None]
-        parity.assert_output_close(y_perm[a:b].double().cpu(), y_ref.cpu(), f"y_perm expert {e}")
+        parity.assert_output_close(yp[a:b].double().cpu(), y_ref.cpu(), f"y_perm expert {e}")
     gs = inp["x"].double() @ inp["ws_gate"].double().T
     us = inp["x"].double() @ inp["ws_up"].double().T
     parity.assert_bf16_rounded(h_s, torch.nn.functional.silu(gs) * us, "h shared")
     ys_ref = h_s.double() @ inp["ws_down"].double().T
-    parity.assert_output_close(y_perm[T * k:].double().cpu(), ys_ref.cpu(), "y shared")
-    # Combine: fp32 gather-sum in the order shared, slot 0..k-1; the bf16 output is
-    # that sum rounded once to nearest.
-    ref = y_perm[T * k:].clone()
+    parity.assert_output_close(yp[T * k:].double().cpu(), ys_ref.cpu(), "y shared")
+    # Combine: fp32 gather-sum of the decoded rows in the order shared, slot 0..k-1;
+    # the bf16 output is that sum rounded once to nearest.
+    ref = yp[T * k:].clone()
     for j in range(k):
-        ref += y_perm[row_of[:, j].long()]
+        ref += yp[row_of[:, j].long()]
     assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
     assert torch.equal(y16.view(torch.int16), ref.to(torch.bfloat16).view(torch.int16))
 
@@ -188,7 +194,7 @@ def test_deterministic_and_launch_count():
     n0 = abi.launch_count()
     y1, i1, w1 = run_forward(shape, inp)
     per_call = abi.launch_count() - n0
-    assert per_call == 8  # router 2, dispatch 3, experts 2, combine 1
+    assert per_call == 9  # router 2, dispatch 4, experts 2, combine 1
     y2, i2, w2 = run_forward(shape, inp)
     assert torch.equal(y1.view(torch.int32), y2.view(torch.int32)) and torch.equal(i1, i2)
 
