@@ -205,6 +205,22 @@ MOE_API int moe_forward(const moe_config *cfg, int64_t T, const void *x, const f
                 int32_t y_dtype, int32_t *topk_idx_out, float *topk_w_out, void *workspace,
                 size_t workspace_bytes, void *stream);
 
+/*
+ * Auxiliary-loss-free load balancing step, run after a batch has been routed
+ * ("The Evolving Transformer · 07", § 06: the per-expert bias is nudged down
+ * when the expert is overloaded and up when it is underloaded, with no
+ * auxiliary loss).  With load_e = number of entries of topk_idx [T, k] equal to
+ * e and the mean load T*k/E:
+ *   e_bias[e] -= gamma if load_e > T*k/E;  e_bias[e] += gamma if load_e < T*k/E;
+ *   unchanged if equal (the comparison is exact, load_e * E against T * k).
+ * e_bias fp32 [E] is updated in place (one fp32 add per expert); expert_load
+ * int32 [E] optionally receives the loads (may be NULL).  gamma (the update
+ * speed) is not given by the pages; it is the caller's, >= 0.  With T = 0
+ * every load equals the mean (0), so no bias moves.
+ */
+MOE_API int moe_bias_update(const moe_config *cfg, int64_t T, const int32_t *topk_idx, float *e_bias,
+                            float gamma, int32_t *expert_load, void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

@@ -66,6 +66,9 @@ def _load():
         lib.oracle_swiglu.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                       p, p, p, p, p]
         lib.oracle_swiglu.restype = ctypes.c_int
+        lib.oracle_bias_update.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p,
+                                           ctypes.c_float, p]
+        lib.oracle_bias_update.restype = None
         _lib = lib
     return _lib
 
@@ -179,3 +182,14 @@ def in_memory_experts(w_gate, w_up, w_down) -> ExpertFetch:
     """Expert fetcher over host arrays [E,I,H], [E,I,H], [E,H,I] of bf16 bits."""
     return lambda e: (w_gate[e], w_up[e], w_down[e])
 
+
+
+def bias_update(idx, n_experts: int, bias, gamma: float):
+    """Aux-loss-free bias step: returns (new bias fp32 [E], load int64 [E])."""
+    lib = _load()
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    b = np.array(bias, dtype=np.float32, copy=True)
+    load = np.zeros(n_experts, np.int64)
+    lib.oracle_bias_update(T, k, n_experts, _ptr(idx), _ptr(b), ctypes.c_float(gamma), _ptr(load))
+    return b, load

@@ -195,3 +195,28 @@ int oracle_swiglu(int64_t n, int64_t H, int64_t I, const uint16_t *x, const uint
     free(xs); free(hmid);
     return 0;
 }
+
+/*
+ * Auxiliary-loss-free bias update ("The Evolving Transformer · 07", § 06: the
+ * per-expert bias is nudged down when the expert is overloaded and up when it
+ * is underloaded; knlb.dev DeepSeek-V3 notes, § architecture).  Load of expert
+ * e = number of the batch's (token, slot) pairs routed to e; the reference load
+ * is the mean T*k/E.  The step is gamma: bias_e <- bias_e - gamma if load_e is
+ * above the mean, + gamma if below, unchanged if equal.  The bias is fp32 state,
+ * so the sum is rounded to fp32 (the float64 sum of two floats, rounded once).
+ *   idx [T,k] chosen experts; bias [E] updated in place; load [E] (output).
+ */
+void oracle_bias_update(int64_t T, int32_t K, int32_t E, const int32_t *idx, float *bias, float gamma,
+                        int64_t *load)
+{
+    for (int e = 0; e < E; ++e) load[e] = 0;
+    for (int64_t q = 0; q < T * K; ++q) load[idx[q]] += 1;
+    for (int e = 0; e < E; ++e) {
+        /* load_e vs T*K/E compared exactly as load_e * E vs T * K */
+        const int64_t lhs = load[e] * (int64_t)E, rhs = T * (int64_t)K;
+        double step = 0.0;
+        if (lhs > rhs) step = -(double)gamma;
+        else if (lhs < rhs) step = (double)gamma;
+        bias[e] = (float)((double)bias[e] + step);
+    }
+}

@@ -81,9 +81,11 @@ def lib():
         L.moe_launch_count.argtypes = []
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
+        L.moe_bias_update.argtypes = [cfgp, i64, _P, _P, ctypes.c_float, _P, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
-                   "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout"):
+                   "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
+                   "moe_bias_update"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -205,3 +207,11 @@ def launch_count() -> int:
 
 def selftest_wait_timeout(limit_ns: int, stream=None):
     _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def moe_bias_update(cfg, topk_idx, e_bias, gamma: float, expert_load=None, stream=None):
+    """Aux-loss-free balancing step: e_bias -= gamma where the expert was overloaded,
+    += gamma where underloaded (in place); expert_load [E] int32 optionally receives the loads."""
+    _check("moe_bias_update", lib().moe_bias_update(ctypes.byref(_cfg(cfg)), topk_idx.shape[0],
+                                                    _ptr(topk_idx), _ptr(e_bias), float(gamma),
+                                                    _ptr(expert_load), _stream(stream)))

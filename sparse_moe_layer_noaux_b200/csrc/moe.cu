@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/moe.h"
+#include "balance.cuh"
 #include "combine.cuh"
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
@@ -636,6 +637,17 @@ int moe_device_status(void* stream, int32_t* device_error) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_bias_update(const moe_config* cfg, int64_t T, const int32_t* topk_idx, float* e_bias, float gamma,
+                    int32_t* expert_load, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (!topk_idx || !e_bias || !(gamma == gamma) || gamma < 0.0f || gamma > 3.0e38f) return MOE_ERR_INVALID_ARG;
+    bias_update_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+        topk_idx, T * cfg->num_experts_per_tok, cfg->n_routed_experts, gamma, e_bias, expert_load);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 int moe_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
     if (limit_ns == 0 || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
