@@ -37,6 +37,10 @@
  *     nothing.
  *   - Device-side waits are bounded: a wait that gives up writes a device
  *     error word (read with moe_device_status) instead of hanging the GPU.
+ *   - The expert GEMMs normally run one CTA per tile.  Setting the environment
+ *     variable MOE_PAIR_GEMM=1 (read at each call) runs prefill-sized batches on
+ *     CTA pairs (256-row tiles, tcgen05 cta_group::2) instead; results are the
+ *     same, only the schedule differs.
  */
 #ifndef MOE_H_
 #define MOE_H_

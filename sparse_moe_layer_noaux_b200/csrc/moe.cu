@@ -3,6 +3,7 @@
 // All kernels of the library are in this translation unit.
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <initializer_list>
 #include <mutex>
@@ -16,6 +17,7 @@
 #include "combine.cuh"
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_2sm.cuh"
 #include "router.cuh"
 
 namespace moe {
@@ -83,6 +85,18 @@ RouterPlan plan_router(int T, int E, int H) {
 constexpr size_t kGemmSmemBytes =
     1024 + kStages * (kTileABytes + kTileBBytes) + kStageBytes + sizeof(GemmSmem);
 static_assert(kGemmSmemBytes <= 227 * 1024, "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
+static_assert(kGemm2SmemBytes <= 227 * 1024, "pair GEMM shared memory exceeds the 227 KB per-CTA limit");
+
+// The CTA-pair GEMMs (256-row tiles) can take prefill-sized batches (expert
+// segments averaging at least 128 rows).  They are built but off by default:
+// measured on B200 under the 1000 W cap they do ~3% more work per clock than the
+// single-CTA kernel yet run at ~15% lower SM clocks, so they are slower end to
+// end.  The environment variable MOE_PAIR_GEMM=1 (read at each call) selects them.
+inline bool use_pair_kernel(int64_t R, int64_t E, int num_sms) {
+    const char* v = std::getenv("MOE_PAIR_GEMM");
+    const bool on = v != nullptr && v[0] == '1';
+    return on && num_sms >= 2 && R >= 128 * E;
+}
 
 // --------------------------------------------------------------- device info
 struct DeviceInfo {
@@ -106,7 +120,11 @@ int device_info(DeviceInfo** out) {
             cudaFuncSetAttribute(grouped_gemm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_kernel<kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
+                                 smem) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -323,6 +341,18 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
+    if (use_pair_kernel(R, E, num_sms)) {
+        // Pair tiles: each CTA loads 64 gate rows and 64 up rows of the 128-column tile.
+        if (!make_map(&b_r, w_gate, E * I, H, 64) || !make_map(&b2_r, w_up, E * I, H, 64)) return MOE_ERR_CUDA;
+        if (has_shared && (!make_map(&b_s, ws_gate, SI, H, 64) || !make_map(&b2_s, ws_up, SI, H, 64)))
+            return MOE_ERR_CUDA;
+        if (!has_shared) { b_s = b_r; b2_s = b2_r; }
+        const int64_t grid = 2 * (num_sms / 2);
+        grouped_gemm_2sm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemm2SmemBytes, st>>>(
+            a_r, a_s, b_r, b2_r, b_s, b2_s, p);
+        count_launch();
+        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
     const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -370,6 +400,17 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
+    if (use_pair_kernel(R, E, num_sms)) {
+        // Pair tiles: each CTA loads its 128 of the 256 output columns' weight rows.
+        if (!make_map(&b_r, w_down, E * H, I, 128)) return MOE_ERR_CUDA;
+        if (has_shared && !make_map(&b_s, ws_down, H, SI, 128)) return MOE_ERR_CUDA;
+        if (!has_shared) b_s = b_r;
+        const int64_t grid = 2 * (num_sms / 2);
+        grouped_gemm_2sm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemm2SmemBytes, st>>>(
+            a_r, a_s, b_r, b_r, b_s, b_s, p);
+        count_launch();
+        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
     const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);

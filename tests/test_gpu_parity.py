@@ -251,3 +251,15 @@ def test_workload_full_size(shape, n_sample):
     assert torch.isfinite(y.float()).all()
     srt = torch.sort(idx, dim=1).values
     assert (srt[:, 1:] != srt[:, :-1]).all()
+
+
+@pytest.mark.parametrize("shape", [SMALL[4], V3_E32], ids=lambda s: s.name)
+def test_pair_gemm_gives_the_same_bits(shape, monkeypatch):
+    """MOE_PAIR_GEMM=1 runs the expert GEMMs on CTA pairs (tcgen05 cta_group::2,
+    256-row tiles, 128-row pair tiles for segment tails); same MMA order, same bits."""
+    inp = make_inputs(shape, "cuda")
+    y1, i1, w1 = run_forward(shape, inp)
+    monkeypatch.setenv("MOE_PAIR_GEMM", "1")
+    y2, i2, w2 = run_forward(shape, inp)
+    assert torch.equal(i1, i2)
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
