@@ -131,9 +131,10 @@ MOE_API int moe_dispatch(const moe_config *cfg, int64_t T, const void *x, const 
  * an embedding runtime that gives this library only the buffers it already
  * owns.  It computes exactly what moe_dispatch computes, with the same
  * arguments minus the workspace.
- *   Scratch: a file-scope device array of 1 MiB (262144 int32) holding the
- *   per-block counts and bases, 2 * ceil(T / 32) * n_routed_experts int32
- *   values; larger sizes return MOE_ERR_STATIC_LIMIT and enqueue nothing (at
+ *   Scratch: a file-scope device array of 1 MiB + 4 KiB (263168 int32) holding
+ *   the per-block counts and bases and the per-expert totals,
+ *   2 * ceil(T / 32) * n_routed_experts + n_routed_experts int32 values;
+ *   larger sizes return MOE_ERR_STATIC_LIMIT and enqueue nothing (at
  *   n_routed_experts = 256 the limit is T <= 16384).  The array is part of the
  *   library image: every GPU that loads the library holds it until the
  *   process exits, and nothing is allocated or freed by this call.

@@ -2,8 +2,10 @@
 // Transformer · 07", § 02 (MoE.forward: mask = indices[:, :, k] == i; x[mask]),
 // done for all experts at once as a stable counting sort:
 //   1. count:  per block of kDispTok tokens, how many slots go to each expert;
-//   2. scan:   expert offsets, and each block's starting row inside every expert;
-//   3. place:  stable rank of every slot (ascending (t, j)) -> row_of / perm_src;
+//   2. scan:   per expert, each block's starting row inside the expert's segment
+//              and the expert's total (one warp per expert);
+//   3. place:  expert offsets from the totals, then the stable rank of every
+//              slot (ascending (t, j)) -> row_of / perm_src;
 //   4. scatter: each token's row is read once from x and written to its k rows
 //              of x_perm with 16-byte vector stores.
 #pragma once
@@ -15,6 +17,7 @@ namespace moe {
 constexpr int kDispTok = 32;      // tokens per dispatch block
 constexpr int kDispThreads = 256;
 
+// Per-block expert counts, stored expert-major: block_counts[e * nb + b].
 __global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(
     const int32_t* __restrict__ topk_idx, int T, int K, int E, int32_t* __restrict__ block_counts) {
     extern __shared__ int cnt[];
@@ -26,61 +29,63 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(
     for (int q = threadIdx.x; q < n; q += blockDim.x) atomicAdd(&cnt[idx[q]], 1);
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
-        block_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
+        block_counts[(int64_t)e * gridDim.x + blockIdx.x] = cnt[e];
 }
 
-// One block; thread e owns expert e (E <= blockDim.x).
-__global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __restrict__ block_counts,
-                                                            int nb, int E,
-                                                            int32_t* __restrict__ block_base,
-                                                            int32_t* __restrict__ offsets) {
-    __shared__ int warp_sums[8];
-    const int e = threadIdx.x;
-    int total = 0;
-    if (e < E) {
-        int b = 0;
-        for (; b + 4 <= nb; b += 4) {
-            const int c0 = block_counts[(int64_t)(b + 0) * E + e];
-            const int c1 = block_counts[(int64_t)(b + 1) * E + e];
-            const int c2 = block_counts[(int64_t)(b + 2) * E + e];
-            const int c3 = block_counts[(int64_t)(b + 3) * E + e];
-            total += c0 + c1 + c2 + c3;
-        }
-        for (; b < nb; ++b) total += block_counts[(int64_t)b * E + e];
-    }
-    // Exclusive scan of the totals over experts.
-    const int lane = e & 31, warp = e >> 5;
-    int incl = total;
+// One warp per expert: exclusive prefix of its counts over the blocks (the row
+// each block starts at inside the expert's segment) and the expert's total.
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __restrict__ block_counts, int nb,
+                                                            int E, int32_t* __restrict__ block_base,
+                                                            int32_t* __restrict__ totals) {
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (e >= E) return;
+    const int32_t* c = block_counts + (int64_t)e * nb;
+    int32_t* out = block_base + (int64_t)e * nb;
+    int carry = 0;
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+        const int v = b0 + lane < nb ? c[b0 + lane] : 0;
+        int incl = v;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    int warp_base = 0;
-    for (int w = 0; w < warp; ++w) warp_base += warp_sums[w];
-    const int excl = warp_base + incl - total;
-    if (e < E) offsets[e] = excl;
-    if (e == E - 1) offsets[E] = excl + total;
-    if (e < E) {
-        int run = excl;
-        for (int b = 0; b < nb; ++b) {
-            const int c = block_counts[(int64_t)b * E + e];
-            block_base[(int64_t)b * E + e] = run;
-            run += c;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
         }
+        if (b0 + lane < nb) out[b0 + lane] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (lane == 0) totals[e] = carry;
 }
 
 __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
     const int32_t* __restrict__ topk_idx, int T, int K, int E, const int32_t* __restrict__ block_base,
-    int32_t* __restrict__ perm_src, int32_t* __restrict__ row_of) {
+    const int32_t* __restrict__ totals, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
+    int32_t* __restrict__ row_of) {
     extern __shared__ int smem_i[];
     int* run = smem_i;              // [E] next free row of each expert for this block
+    __shared__ int warp_sums[kDispThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int kWarps = kDispThreads / 32;
-    for (int e = tid; e < E; e += blockDim.x) run[e] = block_base[(int64_t)blockIdx.x * E + e];
+    // Expert offsets: exclusive scan of the totals (E <= 256 = one value per thread).
+    const int tot = tid < E ? totals[tid] : 0;
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_sums[w];
+    const int excl = base + incl - tot;
+    if (tid < E) {
+        run[tid] = excl + block_base[(int64_t)tid * gridDim.x + blockIdx.x];
+        if (blockIdx.x == 0) {
+            offsets[tid] = excl;
+            if (tid == E - 1) offsets[E] = excl + tot;
+        }
+    }
     __syncthreads();
     const int t0 = blockIdx.x * kDispTok;
     const int ntok = min(kDispTok, T - t0);

@@ -136,8 +136,9 @@ int device_info(DeviceInfo** out) {
 struct Workspace {
     __nv_bfloat16* router_w3; // [3, E, H] exact bf16 split of router_w
     float* router_part;       // [nsplit, T, E]
-    int32_t* block_counts;    // [nb, E]
-    int32_t* block_base;      // [nb, E]
+    int32_t* block_counts;    // [E, nb]
+    int32_t* block_base;      // [E, nb]
+    int32_t* totals;          // [E]
     int32_t* topk_idx;        // [T, k]
     float* topk_w;            // [T, k]
     int32_t* offsets;         // [E + 1]
@@ -167,6 +168,7 @@ Workspace carve(const moe_config* c, int64_t T, uint8_t* base) {
     w.router_part = reinterpret_cast<float*>(take(sizeof(float) * rp.nsplit * T * E));
     w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
     w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.totals = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * E));
     w.topk_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
     w.topk_w = reinterpret_cast<float*>(take(sizeof(float) * T * K));
     w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));
@@ -278,14 +280,14 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
 
 int launch_dispatch(const moe_config* c, int64_t T, const void* x, const int32_t* idx, int32_t* offsets,
                     void* x_perm, int32_t* perm_src, int32_t* row_of, int32_t* block_counts,
-                    int32_t* block_base, cudaStream_t st) {
+                    int32_t* block_base, int32_t* totals, cudaStream_t st) {
     const int E = c->n_routed_experts, K = c->num_experts_per_tok, H = c->hidden_size;
     const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
     dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
                                                                       block_counts);
-    dispatch_scan_kernel<<<1, 256, 0, st>>>(block_counts, nb, E, block_base, offsets);
+    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(block_counts, nb, E, block_base, totals);
     dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
-                                                                     perm_src, row_of);
+                                                                     totals, offsets, perm_src, row_of);
     const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
     dispatch_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H,
                                                 static_cast<__nv_bfloat16*>(x_perm));
@@ -437,11 +439,11 @@ int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const voi
 }
 
 // ---------------------------------------------------------------- no-allocation dispatch
-// Scratch of moe_dispatch_noalloc: per-block expert counts and per-block bases
-// (2 x ceil(T / kDispTok) x E int32), held in this file-scope device array
-// instead of a caller workspace.  Every GPU that loads the library keeps it
-// until the process exits.
-constexpr int64_t kStaticDispatchInts = 1 << 18;  // 1 MiB
+// Scratch of moe_dispatch_noalloc: per-block expert counts, per-block bases and
+// per-expert totals (2 x ceil(T / kDispTok) x E + E int32), held in this
+// file-scope device array instead of a caller workspace.  Every GPU that loads
+// the library keeps it until the process exits.
+constexpr int64_t kStaticDispatchInts = (1 << 18) + 1024;  // 1 MiB + 4 KiB
 static __device__ __align__(256) int32_t g_dispatch_scratch[kStaticDispatchInts];
 
 int32_t* g_dispatch_scratch_addr[64];
@@ -511,7 +513,7 @@ int moe_dispatch(const moe_config* cfg, int64_t T, const void* x, const int32_t*
     if (!workspace || workspace_bytes < workspace_bytes_for(cfg, T)) return MOE_ERR_WORKSPACE;
     Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
     return launch_dispatch(cfg, T, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, w.block_counts,
-                           w.block_base, st);
+                           w.block_base, w.totals, st);
 }
 
 namespace {
@@ -532,7 +534,7 @@ int moe_dispatch_noalloc(const moe_config* cfg, int64_t T, const void* x, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t E = cfg->n_routed_experts;
     const int64_t nb = (T + kDispTok - 1) / kDispTok;
-    if (2 * nb * E > kStaticDispatchInts) return MOE_ERR_STATIC_LIMIT;
+    if (2 * nb * E + E > kStaticDispatchInts) return MOE_ERR_STATIC_LIMIT;
     if (T == 0) {
         if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), st) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
@@ -541,10 +543,10 @@ int moe_dispatch_noalloc(const moe_config* cfg, int64_t T, const void* x, const 
     if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_UNSUPPORTED;
     int32_t* scratch = nullptr;
     if ((v = dispatch_scratch(&scratch)) != MOE_OK) return v;
-    // Both halves are fully written by the count and scan kernels before they
-    // are read, so nothing has to be cleared between calls.
+    // Every part is fully written by the count and scan kernels before it is
+    // read, so nothing has to be cleared between calls.
     return launch_dispatch(cfg, T, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, scratch,
-                           scratch + nb * E, st);
+                           scratch + nb * E, scratch + 2 * nb * E, st);
 }
 
 int moe_experts_gate_up(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
@@ -640,7 +642,7 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
     if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, w.router_w3, d->num_sms, st)) != MOE_OK)
         return v;
     if ((v = launch_dispatch(cfg, T, x, idx, w.offsets, w.x_perm, w.perm_src, w.row_of, w.block_counts,
-                             w.block_base, st)) != MOE_OK)
+                             w.block_base, w.totals, st)) != MOE_OK)
         return v;
     if ((v = launch_gate_up(cfg, T, x, w.x_perm, w.offsets, w_gate, w_up, ws_gate, ws_up, w.h_routed,
                             w.h_shared, d->num_sms, st)) != MOE_OK)
@@ -661,7 +663,7 @@ const char* moe_status_string(int status) {
         case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
         case MOE_ERR_STATIC_LIMIT:
             return "size exceeds the fixed scratch of the no-allocation entry point "
-                   "(2 * ceil(T / 32) * n_routed_experts must be <= 262144)";
+                   "(2 * ceil(T / 32) * n_routed_experts + n_routed_experts must be <= 263168)";
         default: return "unknown status";
     }
 }

@@ -59,7 +59,7 @@ def test_noalloc_dispatch_matches_workspace_dispatch(shapes):
 def test_noalloc_dispatch_rejects_sizes_beyond_its_scratch():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    shape = V3_DECODE.with_(T=16384 + 32)  # 2 * 513 * 256 int32 > 262144
+    shape = V3_DECODE.with_(T=16384 + 64)  # 2 * 514 * 256 + 256 int32 > 263168
     cfg = abi.MoEConfig.from_shape(shape)
     p = torch.empty(16, dtype=torch.int32, device="cuda")
     x = torch.empty((1, 1), dtype=torch.bfloat16, device="cuda")
