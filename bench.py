@@ -35,6 +35,43 @@ METRIC = "MoE-layer tokens/s and TFLOP/s at V3 shape (T=128, 16384); % of roofli
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the gate/up
+# GEMM, from one single-pass ncu capture of `bench.py --profile-only` at the full
+# workload (the capture and its command are summarised under profiles/).  A figure is
+# reported only while the kernel sources hash to the value it was taken on.
+GEMM_SOURCES = ("grouped_gemm.cuh", "sm100_ptx.cuh")
+MEASURED_TRAFFIC = {
+    "v3_prefill": {"sources_sha1": "e7d5607b536d216d743ee1e1d7c7295424a80916",
+                   "dram_read": 20528930560, "dram_write": 604112640},
+}
+
+
+def gemm_sources_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "sparse_moe_layer_noaux_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    m = MEASURED_TRAFFIC.get(workload)
+    if m is None or m["sources_sha1"] != gemm_sources_sha1():
+        return None
+    return m["dram_read"] + m["dram_write"]
+
+
+def gate_up_algorithmic_bytes(shape, touched):
+    """Compulsory HBM bytes of one gate/up launch: gate and up weights of the touched
+    routed experts and of the shared experts, the T*k gathered rows and the T token
+    rows they read, and the bf16 h rows written (T*(k+S) x I)."""
+    w = (touched + shape.S) * 2 * shape.I * shape.H * 2
+    a = (shape.T * shape.k + (shape.T if shape.S else 0)) * shape.H * 2
+    h = shape.T * (shape.k + shape.S) * shape.I * 2
+    return w + a + h
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -404,7 +441,9 @@ def main():
                 "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
-                "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": None,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "traffic": measured_traffic(shape.name),
+                "algorithmic_bytes": gate_up_algorithmic_bytes(shape, res["experts_touched"]),
                 "flops_per_launch": k4_flops, "ms_per_launch": k4_ms}
 
     e2e_ms, h2d, d2h = time_e2e(res["layer"], shape, max(3, args.steps // 2))
