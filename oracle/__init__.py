@@ -69,6 +69,16 @@ def _load():
         lib.oracle_bias_update.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p,
                                            ctypes.c_float, p]
         lib.oracle_bias_update.restype = None
+        lib.oracle_e4m3_round.argtypes = [ctypes.c_double]
+        lib.oracle_e4m3_round.restype = ctypes.c_double
+        lib.oracle_mx_scale_code.argtypes = [ctypes.c_double]
+        lib.oracle_mx_scale_code.restype = ctypes.c_int
+        lib.oracle_mx_quantize.argtypes = [ctypes.c_int64, ctypes.c_int64, p, p, p, p]
+        lib.oracle_mx_quantize.restype = None
+        lib.oracle_e4m3_round_n.argtypes = [ctypes.c_int64, p, p]
+        lib.oracle_e4m3_round_n.restype = None
+        lib.oracle_e4m3_bits_n.argtypes = [ctypes.c_int64, p, p]
+        lib.oracle_e4m3_bits_n.restype = None
         _lib = lib
     return _lib
 
@@ -182,6 +192,113 @@ def in_memory_experts(w_gate, w_up, w_down) -> ExpertFetch:
     """Expert fetcher over host arrays [E,I,H], [E,I,H], [E,H,I] of bf16 bits."""
     return lambda e: (w_gate[e], w_up[e], w_down[e])
 
+
+
+# ----------------------------------------------------------------------------
+# MXFP8 variant of the expert FFNs ("DeepSeek-V3 notes" (knlb.dev), § fp8:
+# fine-grained block-wise E4M3 quantisation with scales taken online from each
+# block's maximum; gating kept in high precision).  Quantised operands: the token
+# rows entering the experts (blocks of 32 along H), the gate/up weights (blocks of
+# 32 along H, the contraction axis), the SwiGLU output h (blocks of 32 along I)
+# and the down weights (blocks of 32 along I).  Everything else — routing, the
+# products and their sums, SwiGLU itself, the weighted combine — stays float64.
+# ----------------------------------------------------------------------------
+
+def e4m3_round(v) -> np.ndarray:
+    """Nearest E4M3 value of each element (ties to even), float64."""
+    lib = _load()
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty_like(v)
+    lib.oracle_e4m3_round_n(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def e4m3_bits(q) -> np.ndarray:
+    """E4M3 bit patterns (uint8) of values already on the E4M3 grid."""
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    out = np.empty(q.shape, np.uint8)
+    lib.oracle_e4m3_bits_n(q.size, _ptr(q), _ptr(out))
+    return out
+
+
+def mx_scale_code(amax: float) -> int:
+    return int(_load().oracle_mx_scale_code(float(amax)))
+
+
+def mx_quantize(a):
+    """Blocks of 32 along the last axis of a [rows, K] array (float64 or bf16 bits).
+
+    Returns (q, codes, deq): E4M3 element values (float64, unscaled), uint8 scale
+    codes [rows, K/32] and the dequantised values q * 2^(code - 127)."""
+    lib = _load()
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        a = widen_bf16(a)
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    rows, K = a.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q = np.empty_like(a)
+    deq = np.empty_like(a)
+    codes = np.empty((rows, K // 32), np.uint8)
+    lib.oracle_mx_quantize(rows, K, _ptr(a), _ptr(q), _ptr(codes), _ptr(deq))
+    return q, codes, deq
+
+
+def widen_bf16(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def swiglu_mx(x_deq, w_gate, w_up, w_down, h_out=None) -> np.ndarray:
+    """One expert with MXFP8 operands, float64 arithmetic: rows x_deq [n,H] are the
+    already-quantised tokens; the weights (bf16 bits, (out, in) layout) are
+    quantised here; h = silu(gate x) * up x is quantised before the down
+    projection.  Returns [n,H]; ``h_out`` (optional list) receives the float64 h."""
+    wg = mx_quantize(w_gate)[2]
+    wu = mx_quantize(w_up)[2]
+    wd = mx_quantize(w_down)[2]
+    g = x_deq @ wg.T
+    u = x_deq @ wu.T
+    h = g / (1.0 + np.exp(-g)) * u
+    if h_out is not None:
+        h_out.append(h)
+    return mx_quantize(h)[2] @ wd.T
+
+
+def moe_layer_mx(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
+                 shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]],
+                 routing: Optional[Tuple[np.ndarray, np.ndarray]] = None):
+    """The layer's forward with MXFP8 expert FFNs, for the rows of ``x_bits``.
+
+    Same structure as ``moe_layer`` (shared expert on every row; routed outputs
+    weighted and summed in slot order); the router is the float64 one on the
+    unquantised bf16 rows.  Returns (y float64 [n,H], idx, w, margin or None)."""
+    x_bits = _u16(x_bits)
+    n, H = x_bits.shape
+    k = shape.num_experts_per_tok
+    margin = None
+    if routing is None:
+        idx, w, margin = route(shape, x_bits, router_w, e_bias)
+    else:
+        idx = np.asarray(routing[0], np.int32)
+        w = np.asarray(routing[1], np.float64)
+    xq = mx_quantize(x_bits)[2]
+    if shared is not None and shape.n_shared_experts > 0:
+        shared_out = swiglu_mx(xq, *shared)
+    else:
+        shared_out = np.zeros((n, H), np.float64)
+    contrib = np.zeros((n, k, H), np.float64)
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        out = swiglu_mx(xq[rows], *expert(int(e)))
+        contrib[rows, slots] = w[rows, slots][:, None] * out
+    output = np.zeros((n, H), np.float64)
+    for j in range(k):
+        output += contrib[:, j]
+    return shared_out + output, idx, w, margin
 
 
 def bias_update(idx, n_experts: int, bias, gamma: float):

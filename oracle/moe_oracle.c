@@ -220,3 +220,104 @@ void oracle_bias_update(int64_t T, int32_t K, int32_t E, const int32_t *idx, flo
         bias[e] = (float)((double)bias[e] + step);
     }
 }
+
+/*
+ * MXFP8 quantisation ("DeepSeek-V3 notes" (knlb.dev), § fp8: fine-grained
+ * block-wise quantisation, E4M3 throughout, scales derived online from the
+ * block's maximum; "DeepSeekV3.2-Tiered-Implementations", § DeepGEMM: FP8 grouped
+ * GEMM for the MoE experts).  Written from the format definitions:
+ *
+ *  - E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no infinities;
+ *    normal values (1 + m/8) 2^(e-7) for e = 1..15 (e = 15, m = 7 is NaN), so the
+ *    largest finite value is 448; subnormals (m/8) 2^-6, i.e. multiples of 2^-9.
+ *  - One scale per block of 32 consecutive elements along the contraction axis,
+ *    a power of two stored as an 8-bit biased exponent (scale = 2^(code - 127)).
+ *
+ * The scale of a block is the smallest power of two that brings its largest
+ * magnitude within the E4M3 range, so no element saturates.
+ */
+
+/* Nearest E4M3 value to v, ties to the even significand.  |v| > 448 saturates to
+ * 448 (the quantiser never produces such inputs).  NaN passes through. */
+double oracle_e4m3_round(double v)
+{
+    if (v != v) return v;
+    const double a = fabs(v);
+    if (a == 0.0) return v;
+    double step;
+    if (a < ldexp(1.0, -6)) {
+        step = ldexp(1.0, -9);                 /* subnormal spacing */
+    } else {
+        int p;
+        frexp(a, &p);                          /* a in [2^(p-1), 2^p) */
+        step = ldexp(1.0, (p - 1) - 3);        /* 3 mantissa bits */
+    }
+    double q = nearbyint(a / step) * step;     /* a / step is exact; default mode: ties to even */
+    if (q > 448.0) q = 448.0;
+    return v < 0 ? -q : q;
+}
+
+/* E4M3 bit pattern of a value already on the E4M3 grid (|q| <= 448). */
+uint8_t oracle_e4m3_bits(double q)
+{
+    uint8_t sign = (q < 0 || (q == 0 && signbit(q))) ? 0x80 : 0x00;
+    double a = fabs(q);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -6)) return sign | (uint8_t)(a / ldexp(1.0, -9));      /* exponent field 0 */
+    int p;
+    frexp(a, &p);
+    const int e = (p - 1) + 7;                                                /* biased exponent */
+    const int m = (int)(a / ldexp(1.0, p - 1) * 8.0) - 8;                      /* 0..7 */
+    return sign | (uint8_t)(e << 3) | (uint8_t)m;
+}
+
+/* Scale code of a block whose largest magnitude is amax: 127 + e for the smallest
+ * integer e with amax <= 448 * 2^e, clamped to [0, 254]; an all-zero block gets 0. */
+int oracle_mx_scale_code(double amax)
+{
+    if (!(amax > 0.0)) return 0;
+    int p;
+    const double m = frexp(amax, &p);          /* amax = m 2^p, m in [0.5, 1); 448 = 0.875 * 2^9 */
+    const int e = (m <= 0.875) ? p - 9 : p - 8;
+    const int code = 127 + e;
+    return code < 0 ? 0 : (code > 254 ? 254 : code);
+}
+
+/*
+ * Quantise rows [rows, K] (K a multiple of 32) in blocks of 32 along K.
+ *   q     [rows, K]    the E4M3 element values (on the E4M3 grid, unscaled)
+ *   codes [rows, K/32] the blocks' scale codes
+ *   deq   [rows, K]    q * 2^(code - 127), the value the GEMM multiplies with
+ * Any output pointer may be NULL.
+ */
+void oracle_mx_quantize(int64_t rows, int64_t K, const double *src, double *q, uint8_t *codes,
+                        double *deq)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const double *v = src + r * K + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i)
+                if (fabs(v[i]) > amax) amax = fabs(v[i]);
+            const int code = oracle_mx_scale_code(amax);
+            const double scale = ldexp(1.0, code - 127);
+            if (codes) codes[r * (K / 32) + b] = (uint8_t)code;
+            for (int i = 0; i < 32; ++i) {
+                const double e = oracle_e4m3_round(v[i] / scale);   /* division by 2^k is exact */
+                if (q) q[r * K + b * 32 + i] = e;
+                if (deq) deq[r * K + b * 32 + i] = e * scale;
+            }
+        }
+    }
+}
+
+/* Element-wise forms of the two E4M3 helpers above, over n values. */
+void oracle_e4m3_round_n(int64_t n, const double *v, double *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_round(v[i]);
+}
+
+void oracle_e4m3_bits_n(int64_t n, const double *q, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_bits(q[i]);
+}
