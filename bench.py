@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from sparse_moe_layer_noaux_b200 import MoELayer, abi  # noqa: E402
+from sparse_moe_layer_noaux_b200 import MoELayer, MoELayerMX, abi  # noqa: E402
 from sparse_moe_layer_noaux_b200.workloads import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s at V3 shape (T=128, 16384); % of roofline"
@@ -230,6 +230,123 @@ class StagedStep:
         rec(5)
 
 
+class StagedStepMX:
+    """The MXFP8 layer step as its C-ABI stages (route, dispatch with quantisation,
+    gate/up, down, combine), events between them; the weights are quantised once
+    at construction, outside any timed region."""
+
+    NAMES = StagedStep.NAMES
+
+    def __init__(self, shape, inp):
+        self.shape, self.inp = shape, inp
+        T, k, E, H, I, S = shape.T, shape.k, shape.E, shape.H, shape.I, shape.S
+        d = inp["x"].device
+        self.cfg = abi.MoEConfig.from_shape(shape)
+        self.layer = MoELayerMX.from_inputs(shape, inp)
+        rp, tp = abi.mx_routed_rows(self.cfg, T), (T + 127) // 128 * 128
+        self.rp = rp
+        n_ws = max(abi.workspace_size_mx(self.cfg, T), abi.workspace_size(self.cfg, T))
+        self.ws = torch.empty(n_ws, dtype=torch.uint8, device=d)
+        u8 = lambda *sh: torch.empty(sh, dtype=torch.uint8, device=d)
+        i32 = lambda *sh: torch.empty(sh, dtype=torch.int32, device=d)
+        self.idx, self.w = i32(T, k), torch.empty((T, k), dtype=torch.float32, device=d)
+        self.off, self.cnt, self.perm_src, self.row_of = i32(E + 1), i32(E), i32(rp), i32(T, k)
+        self.xq, self.xsf = u8(rp, H), u8(abi.mx_scale_bytes(rp, H))
+        self.xqs, self.xssf = u8(tp, H), u8(max(abi.mx_scale_bytes(tp, H), 16))
+        self.hq, self.hsf = u8(rp, I), u8(abi.mx_scale_bytes(rp, I))
+        self.hqs, self.hssf = u8(tp, max(S * I, 128)), u8(max(abi.mx_scale_bytes(tp, max(S * I, 128)), 16))
+        self.y_perm = torch.empty((rp + T, H), dtype=torch.float16, device=d)
+        self.y_sc = u8(rp + T, abi.y_perm_scale_cols(H))
+        self.y = torch.empty((T, H), dtype=torch.float32, device=d)
+
+    def run(self, events=None):
+        i, T, L = self.inp, self.shape.T, self.layer
+        ev = events or [None] * 6
+
+        def rec(j):
+            if ev[j] is not None:
+                ev[j].record()
+        rec(0)
+        abi.moe_route(self.cfg, i["x"], i["router_w"], i["e_bias"], self.idx, self.w, self.ws)
+        rec(1)
+        abi.moe_dispatch_mx(self.cfg, i["x"], self.idx, self.off, self.cnt, self.xq, self.xsf, self.xqs, self.xssf,
+                            self.perm_src, self.row_of, self.ws)
+        rec(2)
+        abi.moe_experts_gate_up_mx(self.cfg, T, self.xq, self.xsf, self.xqs, self.xssf, self.off, self.cnt,
+                                   L.weights, self.hq, self.hsf, self.hqs, self.hssf)
+        rec(3)
+        abi.moe_experts_down_mx(self.cfg, T, self.hq, self.hsf, self.hqs, self.hssf, self.off, self.cnt,
+                                self.perm_src, self.w, L.weights, self.y_perm, self.y_sc)
+        rec(4)
+        abi.moe_combine_mx(self.cfg, T, self.y_perm, self.y_sc, self.row_of, self.y)
+        rec(5)
+
+
+def layer_bytes_mx(shape, idx):
+    """Algorithmic bytes of one MXFP8 step: E4M3 weights of the touched routed experts
+    and the shared experts (1 byte per element + one scale byte per 32), the fp32
+    router, and x (bf16) in and y (fp32) out."""
+    touched = int(torch.unique(idx).numel())
+    b = (touched + shape.S) * 3 * shape.H * shape.I * (1 + 1 / 32)
+    b += 4 * shape.E * shape.H + 2 * shape.T * shape.H + 4 * shape.T * shape.H
+    return int(b), touched
+
+
+def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
+    """The MXFP8 layer: staged step timed like the bf16 one, and moe_forward_mx alone."""
+    inp = inp if inp is not None else rank_inputs(shape, rank, "cuda")
+    st = StagedStepMX(shape, inp)
+    for _ in range(warmup):
+        st.run()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = abi.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for j in range(steps):
+            st.run(evs[j])
+        torch.cuda.synchronize()
+    launches = abi.launch_count() - n0
+    barrier(world)
+    stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, name in enumerate(StagedStepMX.NAMES)}
+    ms = max_over_ranks(sum(evs[j][0].elapsed_time(evs[j][5]) for j in range(steps)) / steps, world)
+    assert abi.device_status() == 0
+    y = torch.empty(inp["x"].shape, dtype=torch.float32, device=inp["x"].device)
+    for _ in range(2):
+        st.layer(inp["x"], y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        st.layer(inp["x"], y)
+    e1.record()
+    torch.cuda.synchronize()
+    fwd_ms = e0.elapsed_time(e1) / steps
+    fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio (4.5 / 2.25) x measured bf16
+    flops = shape.flops()
+    lbytes, touched = layer_bytes_mx(shape, st.idx)
+    t_roof = max(flops / (fp8_peak * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9))
+    gu_ms = stage_ms["gate_up"]
+    gu_flops = 4.0 * shape.H * shape.I * shape.T * (shape.k + shape.S)
+    out = {
+        "ms_per_step": ms, "tokens_per_s": job_throughput(shape.T, world, ms), "stage_ms": stage_ms,
+        "forward_ms": fwd_ms, "tflops": flops / (ms * 1e-3) / 1e12 * world, "gpu_launches": launches,
+        "experts_touched": touched, "layer_bytes": lbytes,
+        "layer_roofline": {"bound": "tensor" if flops / (fp8_peak * 1e12) >= lbytes / (peaks["hbm_gbs"] * 1e9)
+                           else "hbm", "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms},
+        "roofline": {"kernel": "grouped_gemm_mx_kernel<kSwiGLU> (MXFP8 gate/up + SwiGLU + h quantisation)",
+                     "bound": "tensor", "achieved": gu_flops / (gu_ms * 1e-3) / 1e12, "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": gu_flops / (gu_ms * 1e-3) / 1e12 / fp8_peak,
+                     "peak_source": "measured bf16 burst x 2 (nominal dense fp8/bf16 ratio)",
+                     "traffic": None, "ms_per_launch": gu_ms},
+        "clocks": clk.summary(),
+    }
+    del st
+    return out
+
+
 def layer_bytes(shape, idx):
     """Algorithmic bytes of one step: touched routed experts + shared + router + x and y."""
     touched = int(torch.unique(idx).numel())
@@ -406,6 +523,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="v3_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mx", action="store_true", help="skip the MXFP8 variant of the layer")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--profile-only", action="store_true",
                     help="run warmup + steps layer passes and exit without timing (for profilers)")
@@ -461,6 +579,14 @@ def main():
             "layer_roofline": dr["layer_roofline"], "experts_touched": dr["experts_touched"],
             "layer_bytes": dr["layer_bytes"]}
         del dr
+    if not args.no_mx and shape.name == "v3_prefill":
+        # The MXFP8 expert FFNs on the same workload (fine-grained FP8 of the pages'
+        # FP8 notes): a second precision of the same layer, reported beside it.
+        torch.cuda.empty_cache()
+        extra["mxfp8"] = time_gpu_mx(shape, args.steps, args.warmup, world, rank, peaks, inp=res["inp"])
+        dec = WORKLOADS["v3_decode"]
+        extra["mxfp8_decode"] = time_gpu_mx(dec, max(args.steps, 20), args.warmup, world, rank, peaks)
+        torch.cuda.empty_cache()
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

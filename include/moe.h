@@ -226,6 +226,109 @@ MOE_API int moe_forward(const moe_config *cfg, int64_t T, const void *x, const f
 MOE_API int moe_bias_update(const moe_config *cfg, int64_t T, const int32_t *topk_idx, float *e_bias,
                             float gamma, int32_t *expert_load, void *stream);
 
+/* ------------------------------------------------------------------------
+ * MXFP8 expert FFNs ("DeepSeek-V3 notes" (knlb.dev), § fp8: fine-grained
+ * block-wise quantisation, E4M3 throughout, scales derived online from each
+ * block's maximum, activations cached and dispatched in FP8, gating kept in
+ * high precision; "DeepSeekV3.2-Tiered-Implementations", § DeepGEMM: FP8 grouped
+ * GEMM for the MoE experts).
+ *
+ * Format of an MXFP8 matrix [rows, K] (K the contraction axis, a multiple of 128):
+ *   q   uint8 [rows, K]   E4M3 bytes (1 sign, 4 exponent bits with bias 7, 3
+ *                         mantissa bits; largest finite value 448), row-major;
+ *   sf  uint8 scale codes, one per 32 consecutive elements of a row, the scale
+ *       being 2^(code - 127); code = 127 + e for the smallest e with
+ *       max|block| <= 448 * 2^e (0 for an all-zero block), so nothing saturates.
+ *       Stored in 512-byte atoms of 128 rows x 128 K: atom (rb, kb) at byte
+ *       (rb * K/128 + kb) * 512, and within it the code of row r (0..127) and
+ *       32-block j (0..3) at byte 16 * (r % 32) + 4 * (r / 32) + j.  Rows are
+ *       padded to a multiple of 128 (moe_mx_scale_bytes gives the size).
+ * Quantised here: the token rows entering the experts (blocks along H), gate and
+ * up weights (along H), the SwiGLU output h (along I) and down weights (along I).
+ * Routing, products and sums (fp32 accumulation in the tensor core), SwiGLU and
+ * the weighted combine are as in the bf16 path.
+ * ------------------------------------------------------------------------ */
+typedef struct moe_mx_matrix {
+    const void *q;   /* E4M3 bytes, [rows, K] */
+    const void *sf;  /* scale atoms (layout above) */
+} moe_mx_matrix;
+
+/* The layer's expert weights in MXFP8, each in the (out, in) layout of the bf16
+ * weights: gate, up [E*I, H]; down [E*H, I]; shared_gate, shared_up [S*I, H];
+ * shared_down [H, S*I] (the shared members unused when S = 0). */
+typedef struct moe_mx_weights {
+    moe_mx_matrix gate, up, down, shared_gate, shared_up, shared_down;
+} moe_mx_weights;
+
+/* Bytes of the scale atoms of an MXFP8 matrix [rows, K]; -1 if K is not a
+ * positive multiple of 128. */
+MOE_API int64_t moe_mx_scale_bytes(int64_t rows, int64_t K);
+
+/* Quantise a bf16 matrix src [rows, K] into q [rows, K] and sf
+ * (moe_mx_scale_bytes(rows, K) bytes).  MOE_ERR_UNSUPPORTED unless K % 128 == 0.
+ * Used once per weight set (the scheme keeps master weights in higher precision
+ * and multiplies FP8 copies). */
+MOE_API int moe_mx_quantize(int64_t rows, int64_t K, const void *src, void *q, void *sf, void *stream);
+
+/* Workspace of moe_forward_mx / moe_dispatch_mx.  Shapes: hidden_size a multiple
+ * of 256, moe_intermediate_size a multiple of 128 (else MOE_ERR_UNSUPPORTED). */
+MOE_API int moe_workspace_size_mx(const moe_config *cfg, int64_t T, size_t *bytes);
+
+/* Rows of the padded routed row space: every expert's segment starts on a
+ * multiple of 128 rows, so T*k rows take at most
+ * round_up(T*k + 127*n_routed_experts, 128) rows. */
+MOE_API int moe_mx_routed_rows(const moe_config *cfg, int64_t T, int64_t *rows);
+
+/* Dispatch with quantisation.  Same counting sort as moe_dispatch (slots in
+ * ascending (t, j) order inside each segment) with each expert's segment
+ * starting on a multiple of 128 rows:
+ *   expert_offsets [E+1] first row of each segment (expert_offsets[E] = end);
+ *   expert_counts  [E]   rows routed to each expert;
+ *   xq_perm [Rp, H] / xq_perm_sf: the MXFP8 quantisation of x[t] (blocks of 32
+ *       along H) in row row_of[t, j]; rows between segments are left unwritten;
+ *   xq_shared [round_up(T,128), H] / xq_shared_sf: the same rows in token order
+ *       (for the shared experts; unused and may be NULL when S = 0);
+ *   perm_src [Rp] flat slot t*k + j of each occupied row; row_of [T, k].
+ * Rp = moe_mx_routed_rows. */
+MOE_API int moe_dispatch_mx(const moe_config *cfg, int64_t T, const void *x, const int32_t *topk_idx,
+                            int32_t *expert_offsets, int32_t *expert_counts, void *xq_perm, void *xq_perm_sf,
+                            void *xq_shared, void *xq_shared_sf, int32_t *perm_src, int32_t *row_of,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* The gate/up GEMM of the MXFP8 path: for routed expert e, rows
+ * expert_offsets[e] .. + expert_counts[e] of xq_perm (as written by
+ * moe_dispatch_mx), h = silu(x Wg_e^T) * (x Wu_e^T) with fp32 accumulation,
+ * quantised to MXFP8 (blocks of 32 along I) into hq_routed [Rp, I] and its scale
+ * atoms hq_routed_sf (moe_mx_scale_bytes(Rp, I)); the shared experts likewise
+ * from xq_shared into hq_shared [round_up(T,128), S*I].  Rows of a segment past
+ * its count (up to the next multiple of 128) are written as zeros. */
+MOE_API int moe_experts_gate_up_mx(const moe_config *cfg, int64_t T, const void *xq_perm, const void *xq_perm_sf,
+                                   const void *xq_shared, const void *xq_shared_sf, const int32_t *expert_offsets,
+                                   const int32_t *expert_counts, const moe_mx_weights *weights, void *hq_routed,
+                                   void *hq_routed_sf, void *hq_shared, void *hq_shared_sf, void *stream);
+
+/* The down GEMM of the MXFP8 path: y_perm row r = topk_w[perm_src[r]] *
+ * (h_r Wd_e^T) for the occupied rows of each routed segment, and row Rp + t =
+ * h_shared[t] Ws_down^T, in the block-scaled fp16 format of moe_experts
+ * (y_perm [Rp + T, H], y_perm_scale [Rp + T, round_up(H/32, 8)]). */
+MOE_API int moe_experts_down_mx(const moe_config *cfg, int64_t T, const void *hq_routed, const void *hq_routed_sf,
+                                const void *hq_shared, const void *hq_shared_sf, const int32_t *expert_offsets,
+                                const int32_t *expert_counts, const int32_t *perm_src, const float *topk_w,
+                                const moe_mx_weights *weights, void *y_perm, void *y_perm_scale, void *stream);
+
+/* moe_combine for the MXFP8 path's y_perm, whose shared rows start at row Rp. */
+MOE_API int moe_combine_mx(const moe_config *cfg, int64_t T, const void *y_perm, const void *y_perm_scale,
+                           const int32_t *row_of, void *y, int32_t y_dtype, void *stream);
+
+/* The layer forward with MXFP8 expert FFNs: route (as moe_route, on the bf16 x),
+ * dispatch with quantisation, gate/up GEMM with SwiGLU and h quantised to MXFP8,
+ * down GEMM with the routing weights, combine.  Arguments as moe_forward, with
+ * the expert weights given as MXFP8 matrices (moe_mx_quantize). */
+MOE_API int moe_forward_mx(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+                           const float *e_bias, const moe_mx_weights *weights, void *y, int32_t y_dtype,
+                           int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

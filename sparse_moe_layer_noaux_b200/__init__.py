@@ -16,7 +16,7 @@ from .abi import (MoEConfig, MoEError, moe_combine, moe_dispatch, moe_experts, m
                   moe_route, workspace_size)
 from .workloads import MoEShape
 
-__all__ = ["MoELayer", "MoEConfig", "MoEError", "MoEShape", "abi", "moe_route", "moe_dispatch",
+__all__ = ["MoELayer", "MoELayerMX", "MoEConfig", "MoEError", "MoEShape", "abi", "moe_route", "moe_dispatch",
            "moe_experts", "moe_combine", "moe_forward", "workspace_size"]
 
 
@@ -59,6 +59,47 @@ class MoELayer:
         moe_forward(self.cfg, x, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
                     self.ws_gate, self.ws_up, self.ws_down, y, topk_idx, topk_w,
                     self.workspace(T), stream)
+        return y
+
+    __call__ = forward
+
+
+class MoELayerMX:
+    """The layer with MXFP8 expert FFNs (E4M3 with power-of-two scales per 32
+    elements, include/moe.h).  The bf16 weights are quantised once, here, through
+    the library (moe_mx_quantize); the router keeps its fp32 weights."""
+
+    def __init__(self, shape: MoEShape, router_w, e_bias, w_gate, w_up, w_down,
+                 ws_gate=None, ws_up=None, ws_down=None, stream=None):
+        self.shape = shape
+        self.cfg = MoEConfig.from_shape(shape)
+        self.router_w, self.e_bias = router_w, e_bias
+        q = lambda w: None if w is None else abi.mx_quantize(w.reshape(-1, w.shape[-1]), stream)
+        self.gate, self.up, self.down = q(w_gate), q(w_up), q(w_down)
+        self.shared = tuple(q(w) for w in (ws_gate, ws_up, ws_down)) if shape.n_shared_experts > 0 \
+            else (None, None, None)
+        self.weights = abi.mx_weights(self.gate, self.up, self.down, *self.shared)
+        self._ws: Optional[torch.Tensor] = None
+
+    @classmethod
+    def from_inputs(cls, shape: MoEShape, inputs: dict) -> "MoELayerMX":
+        return cls(shape, inputs["router_w"], inputs["e_bias"], inputs["w_gate"], inputs["w_up"],
+                   inputs["w_down"], inputs.get("ws_gate"), inputs.get("ws_up"), inputs.get("ws_down"))
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = abi.workspace_size_mx(self.cfg, T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.router_w.device)
+        return self._ws
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                stream=None, out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+        abi.moe_forward_mx(self.cfg, x, self.router_w, self.e_bias, self.weights, y, topk_idx, topk_w,
+                           self.workspace(T), stream)
         return y
 
     __call__ = forward

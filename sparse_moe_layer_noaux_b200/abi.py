@@ -56,6 +56,19 @@ _lib = None
 _P = ctypes.c_void_p
 
 
+class MXMatrix(ctypes.Structure):
+    """Mirror of `moe_mx_matrix`: E4M3 bytes and their scale atoms (device pointers)."""
+
+    _fields_ = [("q", ctypes.c_void_p), ("sf", ctypes.c_void_p)]
+
+
+class MXWeights(ctypes.Structure):
+    """Mirror of `moe_mx_weights`."""
+
+    _fields_ = [("gate", MXMatrix), ("up", MXMatrix), ("down", MXMatrix), ("shared_gate", MXMatrix),
+                ("shared_up", MXMatrix), ("shared_down", MXMatrix)]
+
+
 def lib():
     """The loaded libmoe.so (raises if it has not been built)."""
     global _lib
@@ -82,10 +95,24 @@ def lib():
         L.moe_launch_count.restype = ctypes.c_uint64
         L.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _P]
         L.moe_bias_update.argtypes = [cfgp, i64, _P, _P, ctypes.c_float, _P, _P]
+        L.moe_mx_scale_bytes.argtypes = [i64, i64]
+        L.moe_mx_scale_bytes.restype = ctypes.c_int64
+        L.moe_mx_quantize.argtypes = [i64, i64, _P, _P, _P, _P]
+        L.moe_workspace_size_mx.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
+        L.moe_mx_routed_rows.argtypes = [cfgp, i64, ctypes.POINTER(i64)]
+        L.moe_dispatch_mx.argtypes = [cfgp, i64] + [_P] * 11 + [sz, _P]
+        L.moe_forward_mx.argtypes = [cfgp, i64, _P, _P, _P, ctypes.POINTER(MXWeights), _P, ctypes.c_int32,
+                                     _P, _P, _P, sz, _P]
+        wp = ctypes.POINTER(MXWeights)
+        L.moe_experts_gate_up_mx.argtypes = [cfgp, i64] + [_P] * 6 + [wp] + [_P] * 5
+        L.moe_experts_down_mx.argtypes = [cfgp, i64] + [_P] * 8 + [wp] + [_P] * 3
+        L.moe_combine_mx.argtypes = [cfgp, i64, _P, _P, _P, _P, ctypes.c_int32, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
-                   "moe_bias_update"):
+                   "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
+                   "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
+                   "moe_combine_mx"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -215,3 +242,84 @@ def moe_bias_update(cfg, topk_idx, e_bias, gamma: float, expert_load=None, strea
     _check("moe_bias_update", lib().moe_bias_update(ctypes.byref(_cfg(cfg)), topk_idx.shape[0],
                                                     _ptr(topk_idx), _ptr(e_bias), float(gamma),
                                                     _ptr(expert_load), _stream(stream)))
+
+
+# ---------------------------------------------------------------- MXFP8 path
+
+def mx_scale_bytes(rows: int, K: int) -> int:
+    n = int(lib().moe_mx_scale_bytes(rows, K))
+    if n < 0:
+        raise MoEError("moe_mx_scale_bytes", MOE_ERR_UNSUPPORTED)
+    return n
+
+
+def moe_mx_quantize(src: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, stream=None):
+    """E4M3 bytes q [rows, K] and scale atoms sf of the bf16 matrix src [rows, K]."""
+    rows, K = src.shape
+    _check("moe_mx_quantize", lib().moe_mx_quantize(rows, K, _ptr(src), _ptr(q), _ptr(sf), _stream(stream)))
+
+
+def mx_quantize(src: torch.Tensor, stream=None):
+    """Allocate and fill (q uint8 [rows, K], sf uint8 [moe_mx_scale_bytes]) for a 2-D bf16 tensor."""
+    src = src.reshape(-1, src.shape[-1])
+    q = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    sf = torch.empty(mx_scale_bytes(*src.shape), dtype=torch.uint8, device=src.device)
+    moe_mx_quantize(src, q, sf, stream)
+    return q, sf
+
+
+def workspace_size_mx(cfg, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_workspace_size_mx", lib().moe_workspace_size_mx(ctypes.byref(_cfg(cfg)), T, ctypes.byref(n)))
+    return n.value
+
+
+def mx_routed_rows(cfg, T: int) -> int:
+    n = ctypes.c_int64(0)
+    _check("moe_mx_routed_rows", lib().moe_mx_routed_rows(ctypes.byref(_cfg(cfg)), T, ctypes.byref(n)))
+    return n.value
+
+
+def moe_dispatch_mx(cfg, x, topk_idx, expert_offsets, expert_counts, xq_perm, xq_perm_sf, xq_shared,
+                    xq_shared_sf, perm_src, row_of, workspace, stream=None):
+    _check("moe_dispatch_mx", lib().moe_dispatch_mx(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
+        _ptr(expert_counts), _ptr(xq_perm), _ptr(xq_perm_sf), _ptr(xq_shared), _ptr(xq_shared_sf),
+        _ptr(perm_src), _ptr(row_of), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def mx_weights(gate, up, down, shared_gate=None, shared_up=None, shared_down=None) -> MXWeights:
+    """MXWeights from (q, sf) tensor pairs (the shared ones may be None)."""
+    def m(pair):
+        return MXMatrix(None, None) if pair is None else MXMatrix(pair[0].data_ptr(), pair[1].data_ptr())
+    return MXWeights(m(gate), m(up), m(down), m(shared_gate), m(shared_up), m(shared_down))
+
+
+def moe_forward_mx(cfg, x, router_w, e_bias, weights: MXWeights, y, topk_idx_out=None, topk_w_out=None,
+                   workspace=None, stream=None):
+    _check("moe_forward_mx", lib().moe_forward_mx(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), ctypes.byref(weights),
+        _ptr(y), out_dtype_code(y), _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_experts_gate_up_mx(cfg, T, xq_perm, xq_perm_sf, xq_shared, xq_shared_sf, expert_offsets, expert_counts,
+                           weights: MXWeights, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf, stream=None):
+    _check("moe_experts_gate_up_mx", lib().moe_experts_gate_up_mx(
+        ctypes.byref(_cfg(cfg)), T, _ptr(xq_perm), _ptr(xq_perm_sf), _ptr(xq_shared), _ptr(xq_shared_sf),
+        _ptr(expert_offsets), _ptr(expert_counts), ctypes.byref(weights), _ptr(hq_routed), _ptr(hq_routed_sf),
+        _ptr(hq_shared), _ptr(hq_shared_sf), _stream(stream)))
+
+
+def moe_experts_down_mx(cfg, T, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf, expert_offsets, expert_counts,
+                        perm_src, topk_w, weights: MXWeights, y_perm, y_perm_scale, stream=None):
+    _check("moe_experts_down_mx", lib().moe_experts_down_mx(
+        ctypes.byref(_cfg(cfg)), T, _ptr(hq_routed), _ptr(hq_routed_sf), _ptr(hq_shared), _ptr(hq_shared_sf),
+        _ptr(expert_offsets), _ptr(expert_counts), _ptr(perm_src), _ptr(topk_w), ctypes.byref(weights),
+        _ptr(y_perm), _ptr(y_perm_scale), _stream(stream)))
+
+
+def moe_combine_mx(cfg, T, y_perm, y_perm_scale, row_of, y, stream=None):
+    _check("moe_combine_mx", lib().moe_combine_mx(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(y_perm_scale),
+                                                  _ptr(row_of), _ptr(y), out_dtype_code(y), _stream(stream)))

@@ -28,17 +28,17 @@ __device__ __forceinline__ void store8(__nv_bfloat16* dst, const float (&a)[8]) 
 // Block (t, c) combines 8-value (16-byte) slices [256 c, 256 c + 256) of token
 // t's row, one slice per thread, so small batches still spread over every SM.
 // Each y_perm row is block-scaled fp16: value = fp16 * 2^(code - 141), one code
-// per 32 columns.  OutT = float (the layer output unrounded) or __nv_bfloat16
+// per 32 columns; the shared expert's output for token t is row shared_row0 + t.  OutT = float (the layer output unrounded) or __nv_bfloat16
 // (rounded once, to nearest).
 template <typename OutT>
 __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ y_perm,
                                                       const uint8_t* __restrict__ y_scale, int64_t scale_ld,
                                                       const int32_t* __restrict__ row_of, int T, int K, int H,
-                                                      int has_shared, OutT* __restrict__ y) {
+                                                      int has_shared, int64_t shared_row0, OutT* __restrict__ y) {
     __shared__ int rows[33];
     const int t = blockIdx.x;
     const int nrows = K + has_shared;
-    if (threadIdx.x == 0 && has_shared) rows[0] = (int)((int64_t)T * K + t);
+    if (threadIdx.x == 0 && has_shared) rows[0] = (int)(shared_row0 + t);
     if (threadIdx.x < K) rows[has_shared + threadIdx.x] = row_of[(int64_t)t * K + threadIdx.x];
     __syncthreads();
     const int c = blockIdx.y * 256 + threadIdx.x;

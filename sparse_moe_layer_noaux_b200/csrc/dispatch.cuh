@@ -4,8 +4,9 @@
 //   1. count:  per block of kDispTok tokens, how many slots go to each expert;
 //   2. scan:   per expert, each block's starting row inside the expert's segment
 //              and the expert's total (one warp per expert);
-//   3. place:  expert offsets from the totals, then the stable rank of every
-//              slot (ascending (t, j)) -> row_of / perm_src;
+//   3. place:  expert offsets from the totals (optionally each segment padded to
+//              a multiple of 128 rows), then the stable rank of every slot
+//              (ascending (t, j)) -> row_of / perm_src;
 //   4. scatter: each token's row is read once from x and written to its k rows
 //              of x_perm with 16-byte vector stores.
 #pragma once
@@ -59,15 +60,17 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __res
 
 __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
     const int32_t* __restrict__ topk_idx, int T, int K, int E, const int32_t* __restrict__ block_base,
-    const int32_t* __restrict__ totals, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
+    const int32_t* __restrict__ totals, int pad, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
     int32_t* __restrict__ row_of) {
     extern __shared__ int smem_i[];
     int* run = smem_i;              // [E] next free row of each expert for this block
     __shared__ int warp_sums[kDispThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int kWarps = kDispThreads / 32;
-    // Expert offsets: exclusive scan of the totals (E <= 256 = one value per thread).
-    const int tot = tid < E ? totals[tid] : 0;
+    // Expert offsets: exclusive scan of the totals (E <= 256 = one value per thread),
+    // each segment rounded up to a multiple of `pad` rows (1, or 128 for MXFP8
+    // operands whose scale atoms cover 128 rows).
+    const int tot = tid < E ? (totals[tid] + pad - 1) / pad * pad : 0;
     int incl = tot;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {

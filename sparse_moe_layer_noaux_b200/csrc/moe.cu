@@ -18,6 +18,8 @@
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_2sm.cuh"
+#include "grouped_gemm_mx.cuh"
+#include "mx.cuh"
 #include "router.cuh"
 
 namespace moe {
@@ -68,7 +70,7 @@ constexpr int kRouterTargetBlocks = 296;  // two waves of blocks on 148 SMs
 constexpr int kRouterTensorCoreMinT = 2048;
 
 RouterPlan plan_router(int T, int E, int H) {
-    if (T >= kRouterTensorCoreMinT) return RouterPlan{1, H};
+    if (T >= kRouterTensorCoreMinT || T <= 0) return RouterPlan{1, H};
     const int tiles = ((T + kRT - 1) / kRT) * ((E + kRE - 1) / kRE);
     int want = (kRouterTargetBlocks + tiles - 1) / tiles;
     const int max_split = H / 256 > 0 ? H / 256 : 1;
@@ -86,6 +88,7 @@ constexpr size_t kGemmSmemBytes =
     1024 + kStages * (kTileABytes + kTileBBytes) + kStageBytes + sizeof(GemmSmem);
 static_assert(kGemmSmemBytes <= 227 * 1024, "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
 static_assert(kGemm2SmemBytes <= 227 * 1024, "pair GEMM shared memory exceeds the 227 KB per-CTA limit");
+static_assert(kGemmMxSmemBytes <= 227 * 1024, "MXFP8 GEMM shared memory exceeds the 227 KB per-CTA limit");
 
 // The CTA-pair GEMMs (256-row tiles) can take prefill-sized batches (expert
 // segments averaging at least 128 rows).  They are built but off by default:
@@ -124,7 +127,11 @@ int device_info(DeviceInfo** out) {
             cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGemm2SmemBytes)) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess)
+                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_mx_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_mx_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -287,7 +294,7 @@ int launch_dispatch(const moe_config* c, int64_t T, const void* x, const int32_t
                                                                       block_counts);
     dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(block_counts, nb, E, block_base, totals);
     dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
-                                                                     totals, offsets, perm_src, row_of);
+                                                                     totals, 1, offsets, perm_src, row_of);
     const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
     dispatch_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H,
                                                 static_cast<__nv_bfloat16*>(x_perm));
@@ -421,19 +428,280 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
 }
 
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const void* y_scale,
-                   const int32_t* row_of, void* y, int y_dtype, cudaStream_t st) {
+                   const int32_t* row_of, void* y, int y_dtype, cudaStream_t st, int64_t shared_row0 = -1) {
+    if (shared_row0 < 0) shared_row0 = T * c->num_experts_per_tok;
     const dim3 g(static_cast<unsigned>(T), static_cast<unsigned>((c->hidden_size / 8 + 255) / 256));
     const int has_shared = c->n_shared_experts > 0 ? 1 : 0;
     if (y_dtype == MOE_DTYPE_BF16)
         combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
             static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
-            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared,
+            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
             static_cast<__nv_bfloat16*>(y));
     else
         combine_kernel<float><<<g, 256, 0, st>>>(
             static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
-            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared,
+            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
             static_cast<float*>(y));
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+
+// ---------------------------------------------------------------- MXFP8 path
+// Shapes the MXFP8 expert GEMMs take: scale atoms cover 128 K-elements, and the
+// down GEMM's 256-column tiles must not straddle two experts' weight rows.
+int validate_mx(const moe_config* c, int64_t T) {
+    const int v = validate_cfg(c, T);
+    if (v != MOE_OK) return v;
+    if (c->hidden_size % 256 != 0 || c->moe_intermediate_size % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+inline int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
+inline int64_t mx_scale_bytes(int64_t rows, int64_t K) { return round128(rows) / 128 * (K / 128) * kMxAtomBytes; }
+
+// Rows of the padded routed row space: every expert segment starts on a multiple
+// of 128, so the segments of T*k rows take at most T*k + 127*E rows.
+inline int64_t mx_routed_rows(const moe_config* c, int64_t T) {
+    return round128(T * c->num_experts_per_tok + 127ll * c->n_routed_experts);
+}
+
+struct WorkspaceMx {
+    __nv_bfloat16* router_w3;
+    float* router_part;
+    int32_t* block_counts;
+    int32_t* block_base;
+    int32_t* totals;          // [E] rows routed to each expert
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* offsets;         // [E + 1] padded segment starts
+    int32_t* perm_src;        // [Rp]
+    int32_t* row_of;          // [T, k]
+    uint8_t* xq_perm;         // [Rp, H] E4M3
+    uint8_t* xq_perm_sf;      // scale atoms of xq_perm
+    uint8_t* xq_shared;       // [Tp, H]
+    uint8_t* xq_shared_sf;
+    uint8_t* hq_routed;       // [Rp, I]
+    uint8_t* hq_routed_sf;
+    uint8_t* hq_shared;       // [Tp, S*I]
+    uint8_t* hq_shared_sf;
+    __half* y_perm;           // [Rp + T, H] block-scaled fp16
+    uint8_t* y_scale;
+    int64_t rp;
+    size_t bytes;
+};
+
+WorkspaceMx carve_mx(const moe_config* c, int64_t T, uint8_t* base) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const RouterPlan rp = plan_router(static_cast<int>(T), static_cast<int>(E), static_cast<int>(H));
+    const int64_t nb = (T + kDispTok - 1) / kDispTok;
+    const int64_t Rp = mx_routed_rows(c, T), Tp = round128(T);
+    WorkspaceMx w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    w.router_w3 = reinterpret_cast<__nv_bfloat16*>(take(2 * 3 * E * H));
+    w.router_part = reinterpret_cast<float*>(take(sizeof(float) * rp.nsplit * T * E));
+    w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.totals = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * E));
+    w.topk_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.topk_w = reinterpret_cast<float*>(take(sizeof(float) * T * K));
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));
+    w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * Rp));
+    w.row_of = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.xq_perm = take(Rp * H);
+    w.xq_perm_sf = take(mx_scale_bytes(Rp, H));
+    w.xq_shared = take(SI > 0 ? Tp * H : 0);
+    w.xq_shared_sf = take(SI > 0 ? mx_scale_bytes(Tp, H) : 0);
+    w.hq_routed = take(Rp * I);
+    w.hq_routed_sf = take(mx_scale_bytes(Rp, I));
+    w.hq_shared = take(Tp * SI);
+    w.hq_shared_sf = take(SI > 0 ? mx_scale_bytes(Tp, SI) : 0);
+    w.y_perm = reinterpret_cast<__half*>(take(2 * (Rp + T) * H));
+    w.y_scale = take((Rp + T) * scale_ld(H));
+    w.rp = Rp;
+    w.bytes = off;
+    return w;
+}
+
+// Row-major E4M3 matrix [rows, cols] (cols a multiple of 128); box = box_rows x 128
+// bytes, 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    if (rows == 0) rows = 1;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKq), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_mx_quantize(int64_t rows, int64_t K, const void* src, void* q, void* sf, cudaStream_t st) {
+    const dim3 g(static_cast<unsigned>(rows), static_cast<unsigned>((K / 8 + 255) / 256));
+    mx_quantize_rows_kernel<<<g, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), static_cast<int>(K),
+                                               static_cast<uint8_t*>(q), static_cast<uint8_t*>(sf));
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Dispatch with quantisation: counting sort with 128-row aligned segments, then
+// each token row quantised once and written to its k rows (and the shared rows).
+int launch_dispatch_mx(const moe_config* c, int64_t T, const void* x, const int32_t* idx, int32_t* offsets,
+                       uint8_t* xq_perm, uint8_t* xq_perm_sf, uint8_t* xq_shared, uint8_t* xq_shared_sf,
+                       int32_t* perm_src, int32_t* row_of, int32_t* block_counts, int32_t* block_base,
+                       int32_t* totals, cudaStream_t st) {
+    const int E = c->n_routed_experts, K = c->num_experts_per_tok, H = c->hidden_size;
+    const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
+                                                                      block_counts);
+    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(block_counts, nb, E, block_base, totals);
+    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
+                                                                     totals, kMxAtomRows, offsets, perm_src, row_of);
+    const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
+    dispatch_scatter_mx_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H, xq_perm,
+                                                   xq_perm_sf, c->n_shared_experts > 0 ? xq_shared : nullptr,
+                                                   xq_shared_sf);
+    count_launch(4);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int64_t gemm_grid_mx(int64_t T, int64_t Rp, int64_t n_tiles_max, int has_shared, int num_sms) {
+    int64_t grid = (Rp / kBM + (has_shared ? (T + kBM - 1) / kBM : 0)) * n_tiles_max;
+    if (grid > num_sms) grid = num_sms;
+    if (grid < 1) grid = 1;
+    return grid;
+}
+
+// Device buffers of the MXFP8 expert stage (from the workspace, or the caller's).
+struct MxBuffers {
+    const int32_t* offsets;
+    const int32_t* counts;
+    const uint8_t* xq_perm;
+    const uint8_t* xq_perm_sf;
+    const uint8_t* xq_shared;
+    const uint8_t* xq_shared_sf;
+    uint8_t* hq_routed;
+    uint8_t* hq_routed_sf;
+    uint8_t* hq_shared;
+    uint8_t* hq_shared_sf;
+    const int32_t* perm_src;
+    __half* y_perm;
+    uint8_t* y_scale;
+    int64_t rp;
+};
+
+MxBuffers buffers_of(const WorkspaceMx& w) {
+    return MxBuffers{w.offsets,   w.totals,       w.xq_perm,   w.xq_perm_sf,   w.xq_shared, w.xq_shared_sf,
+                     w.hq_routed, w.hq_routed_sf, w.hq_shared, w.hq_shared_sf, w.perm_src,  w.y_perm,
+                     w.y_scale,   w.rp};
+}
+
+int launch_gate_up_mx(const moe_config* c, int64_t T, const MxBuffers& w, const moe_mx_weights* wt,
+                      int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    CUtensorMap a_r, a_s, b_r, b2_r, b_s, b2_s;
+    bool ok = make_map_u8(&a_r, w.xq_perm, w.rp, H, kBM) && make_map_u8(&b_r, wt->gate.q, E * I, H, kBN / 2) &&
+              make_map_u8(&b2_r, wt->up.q, E * I, H, kBN / 2);
+    if (has_shared)
+        ok = ok && make_map_u8(&a_s, w.xq_shared, round128(T), H, kBM) &&
+             make_map_u8(&b_s, wt->shared_gate.q, SI, H, kBN / 2) && make_map_u8(&b2_s, wt->shared_up.q, SI, H, kBN / 2);
+    else {
+        a_s = a_r; b_s = b_r; b2_s = b2_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParamsMx p{};
+    p.offsets = w.offsets;
+    p.counts = w.counts;
+    p.E = static_cast<int>(E);
+    p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = static_cast<int>(I / (kBN / 2));
+    p.n_tiles_shared = static_cast<int>(SI / (kBN / 2));
+    p.kb_routed = static_cast<int>(H / kBKq);
+    p.kb_shared = static_cast<int>(H / kBKq);
+    p.n_valid_routed = static_cast<int>(I);
+    p.n_valid_shared = static_cast<int>(SI);
+    p.b_rows_per_expert = static_cast<int>(I);
+    p.sfa_routed = w.xq_perm_sf;
+    p.sfa_shared = w.xq_shared_sf;
+    p.sfb_routed = static_cast<const uint8_t*>(wt->gate.sf);
+    p.sfb2_routed = static_cast<const uint8_t*>(wt->up.sf);
+    p.sfb_shared = has_shared ? static_cast<const uint8_t*>(wt->shared_gate.sf) : p.sfb_routed;
+    p.sfb2_shared = has_shared ? static_cast<const uint8_t*>(wt->shared_up.sf) : p.sfb2_routed;
+    p.b_rows_routed = E * I;
+    p.b_rows_shared = SI;
+    p.out_routed = w.hq_routed;
+    p.ld_routed = I;
+    p.out_shared = w.hq_shared;
+    p.ld_shared = SI;
+    p.hsf_routed = w.hq_routed_sf;
+    p.hsf_shared = w.hq_shared_sf;
+    p.hsf_katoms_routed = static_cast<int>(I / kMxAtomK);
+    p.hsf_katoms_shared = static_cast<int>(SI / kMxAtomK);
+    const int64_t grid = gemm_grid_mx(T, w.rp, I > SI ? I / (kBN / 2) : SI / (kBN / 2), has_shared, num_sms);
+    grouped_gemm_mx_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
+        a_r, a_s, b_r, b2_r, b_s, b2_s, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_down_mx(const moe_config* c, int64_t T, const MxBuffers& w, const moe_mx_weights* wt,
+                   const float* topk_w, int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    CUtensorMap a_r, a_s, b_r, b_s;
+    bool ok = make_map_u8(&a_r, w.hq_routed, w.rp, I, kBM) && make_map_u8(&b_r, wt->down.q, E * H, I, kBN);
+    if (has_shared)
+        ok = ok && make_map_u8(&a_s, w.hq_shared, round128(T), SI, kBM) &&
+             make_map_u8(&b_s, wt->shared_down.q, H, SI, kBN);
+    else {
+        a_s = a_r; b_s = b_r;
+    }
+    if (!ok) return MOE_ERR_CUDA;
+    GemmParamsMx p{};
+    p.offsets = w.offsets;
+    p.counts = w.counts;
+    p.E = static_cast<int>(E);
+    p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = static_cast<int>(H / kBN);
+    p.n_tiles_shared = static_cast<int>(H / kBN);
+    p.kb_routed = static_cast<int>(I / kBKq);
+    p.kb_shared = static_cast<int>(SI / kBKq);
+    p.n_valid_routed = static_cast<int>(H);
+    p.n_valid_shared = static_cast<int>(H);
+    p.b_rows_per_expert = static_cast<int>(H);
+    p.sfa_routed = w.hq_routed_sf;
+    p.sfa_shared = w.hq_shared_sf;
+    p.sfb_routed = static_cast<const uint8_t*>(wt->down.sf);
+    p.sfb2_routed = p.sfb_routed;
+    p.sfb_shared = has_shared ? static_cast<const uint8_t*>(wt->shared_down.sf) : p.sfb_routed;
+    p.sfb2_shared = p.sfb_shared;
+    p.b_rows_routed = E * H;
+    p.b_rows_shared = H;
+    p.out_routed = w.y_perm;
+    p.ld_routed = H;
+    p.out_shared = w.y_perm + w.rp * H;
+    p.ld_shared = H;
+    p.scale_ld = scale_ld(H);
+    p.scale_routed = w.y_scale;
+    p.scale_shared = w.y_scale + w.rp * p.scale_ld;
+    p.perm_src = w.perm_src;
+    p.topk_w = topk_w;
+    const int64_t grid = gemm_grid_mx(T, w.rp, H / kBN, has_shared, num_sms);
+    grouped_gemm_mx_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
+        a_r, a_s, b_r, b_r, b_s, b_s, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -651,6 +919,190 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
                          w.y_scale, d->num_sms, st)) != MOE_OK)
         return v;
     return launch_combine(cfg, T, w.y_perm, w.y_scale, w.row_of, y, y_dtype, st);
+}
+
+int64_t moe_mx_scale_bytes(int64_t rows, int64_t K) {
+    if (rows < 0 || K <= 0 || K % 128 != 0) return -1;
+    return mx_scale_bytes(rows, K);
+}
+
+int moe_mx_quantize(int64_t rows, int64_t K, const void* src, void* q, void* sf, void* stream) {
+    if (rows < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+    if (K % 128 != 0 || rows >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    int v;
+    if ((v = check_ptrs({src, q, sf})) != MOE_OK) return v;
+    return launch_mx_quantize(rows, K, src, q, sf, static_cast<cudaStream_t>(stream));
+}
+
+int moe_workspace_size_mx(const moe_config* cfg, int64_t T, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    *bytes = carve_mx(cfg, T, nullptr).bytes;
+    return MOE_OK;
+}
+
+int moe_mx_routed_rows(const moe_config* cfg, int64_t T, int64_t* rows) {
+    if (!rows) return MOE_ERR_INVALID_ARG;
+    const int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    *rows = mx_routed_rows(cfg, T);
+    return MOE_OK;
+}
+
+int moe_dispatch_mx(const moe_config* cfg, int64_t T, const void* x, const int32_t* topk_idx,
+                    int32_t* expert_offsets, int32_t* expert_counts, void* xq_perm, void* xq_perm_sf,
+                    void* xq_shared, void* xq_shared_sf, int32_t* perm_src, int32_t* row_of, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t E = cfg->n_routed_experts;
+    if (T == 0) {
+        if (cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), st) != cudaSuccess ||
+            cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!topk_idx || !perm_src || !row_of) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({x, xq_perm, xq_perm_sf})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({xq_shared, xq_shared_sf})) != MOE_OK) return v;
+    if (!workspace || workspace_bytes < carve_mx(cfg, T, nullptr).bytes) return MOE_ERR_WORKSPACE;
+    WorkspaceMx w = carve_mx(cfg, T, static_cast<uint8_t*>(workspace));
+    if ((v = launch_dispatch_mx(cfg, T, x, topk_idx, expert_offsets, static_cast<uint8_t*>(xq_perm),
+                                static_cast<uint8_t*>(xq_perm_sf), static_cast<uint8_t*>(xq_shared),
+                                static_cast<uint8_t*>(xq_shared_sf), perm_src, row_of, w.block_counts,
+                                w.block_base, w.totals, st)) != MOE_OK)
+        return v;
+    if (cudaMemcpyAsync(expert_counts, w.totals, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int moe_forward_mx(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
+                   const moe_mx_weights* weights, void* y, int32_t y_dtype, int32_t* topk_idx_out,
+                   float* topk_w_out, void* workspace, size_t workspace_bytes, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!weights || !e_bias) return MOE_ERR_INVALID_ARG;
+    const moe_mx_weights* wt = weights;
+    if ((v = check_ptrs({x, router_w, y, wt->gate.q, wt->gate.sf, wt->up.q, wt->up.sf, wt->down.q, wt->down.sf})) !=
+        MOE_OK)
+        return v;
+    if (cfg->n_shared_experts > 0 &&
+        (v = check_ptrs({wt->shared_gate.q, wt->shared_gate.sf, wt->shared_up.q, wt->shared_up.sf,
+                         wt->shared_down.q, wt->shared_down.sf})) != MOE_OK)
+        return v;
+    if (!workspace || workspace_bytes < carve_mx(cfg, T, nullptr).bytes || !aligned16(workspace))
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    WorkspaceMx w = carve_mx(cfg, T, static_cast<uint8_t*>(workspace));
+    int32_t* idx = topk_idx_out ? topk_idx_out : w.topk_idx;
+    float* tw = topk_w_out ? topk_w_out : w.topk_w;
+    if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, w.router_w3, d->num_sms, st)) != MOE_OK)
+        return v;
+    if ((v = launch_dispatch_mx(cfg, T, x, idx, w.offsets, w.xq_perm, w.xq_perm_sf, w.xq_shared, w.xq_shared_sf,
+                                w.perm_src, w.row_of, w.block_counts, w.block_base, w.totals, st)) != MOE_OK)
+        return v;
+    const MxBuffers b = buffers_of(w);
+    if ((v = launch_gate_up_mx(cfg, T, b, wt, d->num_sms, st)) != MOE_OK) return v;
+    if ((v = launch_down_mx(cfg, T, b, wt, tw, d->num_sms, st)) != MOE_OK) return v;
+    return launch_combine(cfg, T, w.y_perm, w.y_scale, w.row_of, y, y_dtype, st, w.rp);
+}
+
+namespace {
+int check_mx_weights(const moe_config* cfg, const moe_mx_weights* wt, bool gate_up, bool down) {
+    if (!wt) return MOE_ERR_INVALID_ARG;
+    int v;
+    if (gate_up && (v = check_ptrs({wt->gate.q, wt->gate.sf, wt->up.q, wt->up.sf})) != MOE_OK) return v;
+    if (down && (v = check_ptrs({wt->down.q, wt->down.sf})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0) {
+        if (gate_up && (v = check_ptrs({wt->shared_gate.q, wt->shared_gate.sf, wt->shared_up.q,
+                                        wt->shared_up.sf})) != MOE_OK)
+            return v;
+        if (down && (v = check_ptrs({wt->shared_down.q, wt->shared_down.sf})) != MOE_OK) return v;
+    }
+    return MOE_OK;
+}
+}  // namespace
+
+int moe_experts_gate_up_mx(const moe_config* cfg, int64_t T, const void* xq_perm, const void* xq_perm_sf,
+                           const void* xq_shared, const void* xq_shared_sf, const int32_t* expert_offsets,
+                           const int32_t* expert_counts, const moe_mx_weights* weights, void* hq_routed,
+                           void* hq_routed_sf, void* hq_shared, void* hq_shared_sf, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({xq_perm, xq_perm_sf, hq_routed, hq_routed_sf})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({xq_shared, xq_shared_sf, hq_shared, hq_shared_sf})) != MOE_OK)
+        return v;
+    if ((v = check_mx_weights(cfg, weights, true, false)) != MOE_OK) return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    MxBuffers b{expert_offsets,
+                expert_counts,
+                static_cast<const uint8_t*>(xq_perm),
+                static_cast<const uint8_t*>(xq_perm_sf),
+                static_cast<const uint8_t*>(xq_shared),
+                static_cast<const uint8_t*>(xq_shared_sf),
+                static_cast<uint8_t*>(hq_routed),
+                static_cast<uint8_t*>(hq_routed_sf),
+                static_cast<uint8_t*>(hq_shared),
+                static_cast<uint8_t*>(hq_shared_sf),
+                nullptr,
+                nullptr,
+                nullptr,
+                mx_routed_rows(cfg, T)};
+    return launch_gate_up_mx(cfg, T, b, weights, d->num_sms, static_cast<cudaStream_t>(stream));
+}
+
+int moe_experts_down_mx(const moe_config* cfg, int64_t T, const void* hq_routed, const void* hq_routed_sf,
+                        const void* hq_shared, const void* hq_shared_sf, const int32_t* expert_offsets,
+                        const int32_t* expert_counts, const int32_t* perm_src, const float* topk_w,
+                        const moe_mx_weights* weights, void* y_perm, void* y_perm_scale, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (T == 0) return MOE_OK;
+    if (!expert_offsets || !expert_counts || !perm_src || !topk_w) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({hq_routed, hq_routed_sf, y_perm, y_perm_scale})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({hq_shared, hq_shared_sf})) != MOE_OK) return v;
+    if ((v = check_mx_weights(cfg, weights, false, true)) != MOE_OK) return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    MxBuffers b{expert_offsets,
+                expert_counts,
+                nullptr,
+                nullptr,
+                nullptr,
+                nullptr,
+                const_cast<uint8_t*>(static_cast<const uint8_t*>(hq_routed)),
+                const_cast<uint8_t*>(static_cast<const uint8_t*>(hq_routed_sf)),
+                const_cast<uint8_t*>(static_cast<const uint8_t*>(hq_shared)),
+                const_cast<uint8_t*>(static_cast<const uint8_t*>(hq_shared_sf)),
+                perm_src,
+                static_cast<__half*>(y_perm),
+                static_cast<uint8_t*>(y_perm_scale),
+                mx_routed_rows(cfg, T)};
+    return launch_down_mx(cfg, T, b, weights, topk_w, d->num_sms, static_cast<cudaStream_t>(stream));
+}
+
+int moe_combine_mx(const moe_config* cfg, int64_t T, const void* y_perm, const void* y_perm_scale,
+                   const int32_t* row_of, void* y, int32_t y_dtype, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !y_perm_scale || !row_of || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(y) || !aligned16(y_perm_scale)) return MOE_ERR_UNSUPPORTED;
+    return launch_combine(cfg, T, y_perm, y_perm_scale, row_of, y, y_dtype, static_cast<cudaStream_t>(stream),
+                          mx_routed_rows(cfg, T));
 }
 
 const char* moe_status_string(int status) {

@@ -171,6 +171,55 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- MXFP8 (block-scaled) operands
+// Contiguous bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completion counted on `bar` like a tensor load.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand without swizzling: 8-row core
+// matrices of 16-byte rows, `sbo` bytes between consecutive 8-row groups.
+__device__ __forceinline__ uint64_t plain_kmajor_desc(uint32_t smem_addr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(sbo >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;  // layout field (bits 61-63) 0: no swizzle
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM lanes 0..31 and the same
+// data into lanes 32..63, 64..95 and 96..127 (four columns of 32 bits per lane).
+// Used for the 512-byte scale atoms of the block-scaled MMA.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T, kind::mxf8f6f4 with one 8-bit power-of-two
+// scale per 32 K-elements of each row of A and B, read from TMEM.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor, block-scaled kind::mxf8f6f4: E4M3 A and B (format 0),
+// both K-major, dense, 8-bit exponent scales (bit 23), K = 32 per instruction.
+// sf_a / sf_b select which byte of the 32-bit TMEM scale word this instruction
+// uses (bits 29-30 and 4-5): byte j holds the scale of the j-th 32-element block
+// of the current 128-element K slice.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_a, uint32_t sf_b) {
+    return (sf_b << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24) | (sf_a << 29);
+}
+
 }  // namespace ptx
 }  // namespace moe
 

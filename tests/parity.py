@@ -116,9 +116,10 @@ def shared_bits(inp, shape):
 
 
 def oracle_layer_rows(shape, inp, rows, gpu_idx=None, scores=None, ref_idx=None, ref_w=None,
-                      margin=None):
+                      margin=None, layer=None):
     """Oracle output for the given token rows.  Where the GPU picked a different
-    (near-tie) expert set, that row is computed on the GPU's set."""
+    (near-tie) expert set, that row is computed on the GPU's set.  ``layer`` is the
+    oracle layer function (default: the bf16 one; oracle.moe_layer_mx for MXFP8)."""
     x_bits = bf16_bits(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
     rw = inp["router_w"].cpu().numpy()
     bias = inp["e_bias"].cpu().numpy()
@@ -132,6 +133,6 @@ def oracle_layer_rows(shape, inp, rows, gpu_idx=None, scores=None, ref_idx=None,
                 use_idx[i] = gpu_idx[t]
                 use_w[i] = weights_for_set(shape, scores[t], gpu_idx[t])
         routing = (use_idx, use_w)
-    y, *_ = oracle.moe_layer(shape, x_bits, rw, bias, device_expert_fetch(inp),
-                             shared_bits(inp, shape), routing=routing)
+    y, *_ = (layer or oracle.moe_layer)(shape, x_bits, rw, bias, device_expert_fetch(inp),
+                                        shared_bits(inp, shape), routing=routing)
     return y

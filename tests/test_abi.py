@@ -116,3 +116,30 @@ def test_workspace_size_scales(lib):
     # The prefill workspace holds x_perm, h, y_perm: a few GB, well inside 180 GB.
     ws = abi.workspace_size(V3_PREFILL, V3_PREFILL.T)
     assert 4.5e9 < ws < 5.5e9  # x_perm 1.9 GB + h 0.6 GB + block-scaled fp16 y_perm 2.2 GB
+
+
+def test_workspace_size_of_an_empty_batch(lib):
+    # Sizing a workspace for T = 0 is a valid query (no router tiles at all).
+    assert 0 < abi.workspace_size(TINY, 0) < abi.workspace_size(TINY, 64)
+    assert 0 < abi.workspace_size_mx(TINY, 0) < abi.workspace_size_mx(TINY, 64)
+
+
+def test_mx_host_queries(lib):
+    # Scale atoms: 512 bytes per 128 rows x 128 K, rows rounded up to 128.
+    assert abi.mx_scale_bytes(1, 128) == 512
+    assert abi.mx_scale_bytes(129, 256) == 2 * 2 * 512
+    assert lib.moe_mx_scale_bytes(128, 100) == -1
+    # Padded routed rows: T*k + 127*E rounded up to 128.
+    assert abi.mx_routed_rows(V3_PREFILL, V3_PREFILL.T) == (16384 * 8 + 127 * 256 + 127) // 128 * 128
+    # Shapes the MXFP8 GEMMs do not take.
+    with pytest.raises(abi.MoEError) as ei:
+        abi.workspace_size_mx(TINY.with_(hidden_size=320), 4)
+    assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+    with pytest.raises(abi.MoEError):
+        abi.workspace_size_mx(TINY.with_(moe_intermediate_size=192), 4)
+    # The MXFP8 prefill workspace: E4M3 x_perm 1.17 GB + h 0.34 GB + y_perm 2.6 GB.
+    ws = abi.workspace_size_mx(V3_PREFILL, V3_PREFILL.T)
+    assert 4.0e9 < ws < 4.8e9
+    # Quantising nothing is a no-op; a K that is not a multiple of 128 is refused.
+    assert lib.moe_mx_quantize(0, 256, None, None, None, None) == abi.MOE_OK
+    assert lib.moe_mx_quantize(4, 96, None, None, None, None) == abi.MOE_ERR_UNSUPPORTED
