@@ -301,29 +301,17 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
     torch.cuda.synchronize()
     assert abi.device_status() == 0
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
-    barrier(world)
     torch.cuda.synchronize()
-    n0 = abi.launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for j in range(steps):
-            st.run(evs[j])
-        torch.cuda.synchronize()
-    launches = abi.launch_count() - n0
-    barrier(world)
+    for j in range(steps):
+        st.run(evs[j])
+    torch.cuda.synchronize()
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
                 for i, name in enumerate(StagedStepMX.NAMES)}
-    ms = max_over_ranks(sum(evs[j][0].elapsed_time(evs[j][5]) for j in range(steps)) / steps, world)
+    staged_ms = statistics.mean(e[0].elapsed_time(e[5]) for e in evs)
     assert abi.device_status() == 0
     y = torch.empty(inp["x"].shape, dtype=torch.float32, device=inp["x"].device)
-    for _ in range(2):
-        st.layer(inp["x"], y)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        st.layer(inp["x"], y)
-    e1.record()
-    torch.cuda.synchronize()
-    fwd_ms = e0.elapsed_time(e1) / steps
+    ms, launches, clk = time_steps(lambda: st.layer(inp["x"], y), steps, warmup, world)
+    fwd_ms = ms
     fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 / bf16 ratio (4.5 / 2.25) x measured bf16
     flops = shape.flops()
     lbytes, touched = layer_bytes_mx(shape, st.idx)
@@ -332,7 +320,7 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
     gu_flops = 4.0 * shape.H * shape.I * shape.T * (shape.k + shape.S)
     out = {
         "ms_per_step": ms, "tokens_per_s": job_throughput(shape.T, world, ms), "stage_ms": stage_ms,
-        "forward_ms": fwd_ms, "tflops": flops / (ms * 1e-3) / 1e12 * world, "gpu_launches": launches,
+        "staged_ms": staged_ms, "forward_ms": fwd_ms, "tflops": flops / (ms * 1e-3) / 1e12 * world, "gpu_launches": launches,
         "experts_touched": touched, "layer_bytes": lbytes,
         "layer_roofline": {"bound": "tensor" if flops / (fp8_peak * 1e12) >= lbytes / (peaks["hbm_gbs"] * 1e9)
                            else "hbm", "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms},
@@ -341,7 +329,7 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
                      "unit": "TFLOP/s", "frac": gu_flops / (gu_ms * 1e-3) / 1e12 / fp8_peak,
                      "peak_source": "measured bf16 burst x 2 (nominal dense fp8/bf16 ratio)",
                      "traffic": None, "ms_per_launch": gu_ms},
-        "clocks": clk.summary(),
+        "clocks": clk,
     }
     del st
     return out
@@ -363,48 +351,59 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
     torch.cuda.synchronize()
     assert abi.device_status() == 0
 
+    # Stage breakdown: the five C-ABI stages in sequence, events between them.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
-    barrier(world)
     torch.cuda.synchronize()
-    n0 = abi.launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for j in range(steps):
-            st.run(evs[j])
-        torch.cuda.synchronize()
-    launches = abi.launch_count() - n0
-    barrier(world)
+    for j in range(steps):
+        st.run(evs[j])
+    torch.cuda.synchronize()
     stage_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
                 for i, name in enumerate(StagedStep.NAMES)}
-    total_ms = sum(evs[j][0].elapsed_time(evs[j][5]) for j in range(steps))
-    ms = max_over_ranks(total_ms / steps, world)
+    staged_ms = statistics.mean(e[0].elapsed_time(e[5]) for e in evs)
     assert abi.device_status() == 0
 
-    # moe_forward (one call per step) timed alone, for reference.
+    # The step: one moe_forward call (the public entry point).
     layer = MoELayer.from_inputs(shape, inp)
     y = torch.empty(inp["x"].shape, dtype=torch.float32, device=inp["x"].device)
-    for _ in range(2):
-        layer(inp["x"], y)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        layer(inp["x"], y)
-    e1.record()
-    torch.cuda.synchronize()
-    fwd_ms = e0.elapsed_time(e1) / steps
+    ms, launches, clk = time_steps(lambda: layer(inp["x"], y), steps, warmup, world)
+    fwd_ms = ms
 
     flops = shape.flops()
     lbytes, touched = layer_bytes(shape, st.idx)
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9))
     res = {
-        "ms": ms, "stage_ms": stage_ms, "forward_ms": fwd_ms, "launches": launches,
+        "ms": ms, "stage_ms": stage_ms, "staged_ms": staged_ms, "forward_ms": fwd_ms, "launches": launches,
         "tflops": flops / (ms * 1e-3) / 1e12, "layer_bytes": lbytes, "experts_touched": touched,
         "layer_roofline": {"bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >=
                            lbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
                            "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms,
                            "hbm_gbs_achieved": lbytes / (ms * 1e-3) / 1e9},
-        "clocks": clk.summary(), "st": st, "inp": inp, "layer": layer,
+        "clocks": clk, "st": st, "inp": inp, "layer": layer,
     }
     return res
+
+
+def time_steps(step, steps, warmup, world):
+    """Exactly `steps` calls of step() between a barrier + synchronize on both sides,
+    CUDA events on the current stream, clocks sampled meanwhile; max over ranks."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = abi.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record()
+        for _ in range(steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    launches = abi.launch_count() - n0
+    barrier(world)
+    assert abi.device_status() == 0
+    return max_over_ranks(e0.elapsed_time(e1) / steps, world), launches, clk.summary()
 
 
 def time_e2e(layer, shape, steps):
@@ -525,13 +524,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mx", action="store_true", help="skip the MXFP8 variant of the layer")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "mxfp8"],
+                    help="expert FFN precision of --profile-only passes")
     ap.add_argument("--profile-only", action="store_true",
                     help="run warmup + steps layer passes and exit without timing (for profilers)")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
     if args.profile_only:
-        st = StagedStep(shape, rank_inputs(shape, rank, "cuda"))
+        stepper = StagedStepMX if args.precision == "mxfp8" else StagedStep
+        st = stepper(shape, rank_inputs(shape, rank, "cuda"))
         for _ in range(args.warmup + args.steps):
             st.run()
         torch.cuda.synchronize()
@@ -593,7 +595,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights)",
         "config": workload_config(shape, world),
-        "tflops": res["tflops"] * world, "stage_ms": res["stage_ms"], "forward_ms": res["forward_ms"],
+        "tflops": res["tflops"] * world, "stage_ms": res["stage_ms"], "staged_ms": res["staged_ms"],
+        "forward_ms": res["forward_ms"],
         "layer_roofline": res["layer_roofline"], "experts_touched": res["experts_touched"],
         "roofline": roofline,
         "clocks": res["clocks"],

@@ -265,3 +265,27 @@ def test_mx_stages_compose_to_forward():
     # rows past the segment's count, up to the next multiple of 128, are zeros
     pad_end = a + (n + 127) // 128 * 128
     assert int(hq[a + n:pad_end].sum().item()) == 0
+
+
+def test_mx_forward_replays_from_a_cuda_graph():
+    shape = SMALL_MX[3]
+    inp = make_inputs(shape, "cuda")
+    layer = MoELayerMX.from_inputs(shape, inp)
+    y_eager = layer(inp["x"])
+    y = torch.empty_like(y_eager)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer(inp["x"], y)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    y.zero_()
+    with torch.cuda.graph(g):
+        layer(inp["x"], y)
+    g.replay()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    assert torch.equal(y, y_eager)
+    del g

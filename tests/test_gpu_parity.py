@@ -263,3 +263,29 @@ def test_pair_gemm_gives_the_same_bits(shape, monkeypatch):
     y2, i2, w2 = run_forward(shape, inp)
     assert torch.equal(i1, i2)
     assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """moe_forward captured into a CUDA graph and replayed gives the eager bits."""
+    shape = SMALL[3]
+    inp = make_inputs(shape, "cuda")
+    from sparse_moe_layer_noaux_b200 import MoELayer
+    layer = MoELayer.from_inputs(shape, inp)
+    y_eager = layer(inp["x"])
+    y = torch.empty_like(y_eager)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer(inp["x"], y)  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    y.zero_()
+    with torch.cuda.graph(g):
+        layer(inp["x"], y)
+    g.replay()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    assert torch.equal(y, y_eager)
+    del g
