@@ -329,6 +329,28 @@ MOE_API int moe_forward_mx(const moe_config *cfg, int64_t T, const void *x, cons
                            int32_t *topk_idx_out, float *topk_w_out, void *workspace, size_t workspace_bytes,
                            void *stream);
 
+/* ------------------------------------------------------------------------
+ * Backward pass of the layer: gradients of L = sum(y * dy) for an upstream
+ * gradient dy, with the expert selection held fixed (the group keep and top-k
+ * choice is piecewise constant; the correction bias gets no gradient) — the
+ * chain rule of the forward above, checked in float64 by finite differences as
+ * the "dsv3-native-reference" page, § NumPy Oracle, does.  Shapes as
+ * moe_forward_mx (hidden_size % 256 == 0, moe_intermediate_size % 128 == 0).
+ *   dy [T, H] bf16; dx [T, H] fp32; d_router_w [E, H] fp32;
+ *   d_w_gate, d_w_up [E, I, H], d_w_down [E, H, I], d_ws_gate, d_ws_up [S*I, H],
+ *   d_ws_down [H, S*I], all bf16 (fp32 sums, rounded once).
+ * The routing is recomputed (same kernels and inputs as the forward, hence the
+ * same selection) and the experts' g = x Wg^T and u = x Wu^T are recomputed
+ * rather than kept.  T = 0 writes zero weight gradients.
+ * ------------------------------------------------------------------------ */
+MOE_API int moe_workspace_size_bwd(const moe_config *cfg, int64_t T, size_t *bytes);
+
+MOE_API int moe_backward(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+                         const float *e_bias, const void *w_gate, const void *w_up, const void *w_down,
+                         const void *ws_gate, const void *ws_up, const void *ws_down, const void *dy, float *dx,
+                         float *d_router_w, void *d_w_gate, void *d_w_up, void *d_w_down, void *d_ws_gate,
+                         void *d_ws_up, void *d_ws_down, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

@@ -102,7 +102,7 @@ def moe_layer_backward(shape, x_bits, router_w, e_bias, expert: Callable, shared
     concatenated shared expert or None; ``routing`` optionally the expert
     selection idx [n, k] to hold fixed (default: the oracle router's)."""
     x = _f64(x_bits)
-    dy = np.asarray(dy, np.float64)
+    dy = _f64(dy)
     n, H = x.shape
     E, k = shape.n_routed_experts, shape.num_experts_per_tok
     rw = np.asarray(router_w, np.float64)

@@ -63,6 +63,27 @@ class MoELayer:
 
     __call__ = forward
 
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
+        """Gradients of sum(layer(x) * dy) (dy bf16 [T,H]), expert selection held fixed:
+        dx fp32, router_w fp32, expert / shared weights bf16 (same shapes as the weights)."""
+        T = x.shape[0]
+        dev = x.device
+        g = {"x": torch.empty(x.shape, dtype=torch.float32, device=dev),
+             "router_w": torch.empty_like(self.router_w, dtype=torch.float32),
+             "w_gate": torch.empty_like(self.w_gate), "w_up": torch.empty_like(self.w_up),
+             "w_down": torch.empty_like(self.w_down)}
+        if self.shape.n_shared_experts > 0:
+            g.update(ws_gate=torch.empty_like(self.ws_gate), ws_up=torch.empty_like(self.ws_up),
+                     ws_down=torch.empty_like(self.ws_down))
+        need = abi.workspace_size_bwd(self.cfg, T)
+        if getattr(self, "_ws_bwd", None) is None or self._ws_bwd.numel() < need:
+            self._ws_bwd = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        abi.moe_backward(self.cfg, x, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
+                         self.ws_gate, self.ws_up, self.ws_down, dy, g["x"], g["router_w"], g["w_gate"],
+                         g["w_up"], g["w_down"], g.get("ws_gate"), g.get("ws_up"), g.get("ws_down"),
+                         self._ws_bwd, stream)
+        return g
+
 
 class MoELayerMX:
     """The layer with MXFP8 expert FFNs (E4M3 with power-of-two scales per 32

@@ -107,12 +107,14 @@ def lib():
         L.moe_experts_gate_up_mx.argtypes = [cfgp, i64] + [_P] * 6 + [wp] + [_P] * 5
         L.moe_experts_down_mx.argtypes = [cfgp, i64] + [_P] * 8 + [wp] + [_P] * 3
         L.moe_combine_mx.argtypes = [cfgp, i64, _P, _P, _P, _P, ctypes.c_int32, _P]
+        L.moe_workspace_size_bwd.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
+        L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
                    "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
-                   "moe_combine_mx"):
+                   "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -323,3 +325,22 @@ def moe_experts_down_mx(cfg, T, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf
 def moe_combine_mx(cfg, T, y_perm, y_perm_scale, row_of, y, stream=None):
     _check("moe_combine_mx", lib().moe_combine_mx(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(y_perm_scale),
                                                   _ptr(row_of), _ptr(y), out_dtype_code(y), _stream(stream)))
+
+
+# ---------------------------------------------------------------- backward pass
+
+def workspace_size_bwd(cfg, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_workspace_size_bwd", lib().moe_workspace_size_bwd(ctypes.byref(_cfg(cfg)), T, ctypes.byref(n)))
+    return n.value
+
+
+def moe_backward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dy, dx, d_router_w,
+                 d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down, workspace, stream=None):
+    """Gradients of sum(y * dy): dx fp32 [T,H], d_router_w fp32 [E,H], expert and shared
+    weight gradients bf16 in the weights' layouts (include/moe.h)."""
+    _check("moe_backward", lib().moe_backward(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w),
+        _ptr(d_w_gate), _ptr(d_w_up), _ptr(d_w_down), _ptr(d_ws_gate), _ptr(d_ws_up), _ptr(d_ws_down),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -19,6 +19,8 @@
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_2sm.cuh"
 #include "grouped_gemm_mx.cuh"
+#include "grouped_gemm_bwd.cuh"
+#include "bwd_small.cuh"
 #include "mx.cuh"
 #include "router.cuh"
 
@@ -89,6 +91,7 @@ constexpr size_t kGemmSmemBytes =
 static_assert(kGemmSmemBytes <= 227 * 1024, "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
 static_assert(kGemm2SmemBytes <= 227 * 1024, "pair GEMM shared memory exceeds the 227 KB per-CTA limit");
 static_assert(kGemmMxSmemBytes <= 227 * 1024, "MXFP8 GEMM shared memory exceeds the 227 KB per-CTA limit");
+static_assert(kGemmBwdSmemBytes <= 227 * 1024, "backward GEMM shared memory exceeds the 227 KB per-CTA limit");
 
 // The CTA-pair GEMMs (256-row tiles) can take prefill-sized batches (expert
 // segments averaging at least 128 rows).  They are built but off by default:
@@ -131,7 +134,15 @@ int device_info(DeviceInfo** out) {
             cudaFuncSetAttribute(grouped_gemm_mx_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_mx_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess)
+                                 static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kRecompute>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kDh>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kWgrad>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -706,6 +717,251 @@ int launch_down_mx(const moe_config* c, int64_t T, const MxBuffers& w, const moe
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+
+// ---------------------------------------------------------------- backward pass
+struct WorkspaceBwd {
+    __nv_bfloat16* router_w3;
+    float* router_part;
+    int32_t* block_counts;
+    int32_t* block_base;
+    int32_t* totals;          // [E] rows per expert
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* offsets;         // [E+1] 128-aligned segment starts
+    int32_t* perm_src;        // [Rp]
+    int32_t* row_of;          // [T, k]
+    __nv_bfloat16* x_perm;    // [Rp, H]
+    __nv_bfloat16* do_perm;   // [Rp, H]  w * dy
+    __nv_bfloat16* gu_r;      // [Rp, 2I]
+    __nv_bfloat16* gu_s;      // [T, 2SI]
+    __nv_bfloat16* dgu_r;     // [Rp, 2I]
+    __nv_bfloat16* dgu_s;     // [T, 2SI]
+    __nv_bfloat16* h_r;       // [Rp, I]
+    __nv_bfloat16* h_s;       // [T, SI]
+    float* dw_part;           // [Rp, ceil(I/256)]
+    float* dlogit;            // [T, k]
+    __half* dxq;              // [Rp + T, H] block-scaled fp16
+    uint8_t* dxs;             // [Rp + T, scale_ld]
+    int64_t rp;
+    size_t bytes;
+};
+
+WorkspaceBwd carve_bwd(const moe_config* c, int64_t T, uint8_t* base) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const RouterPlan rp = plan_router(static_cast<int>(T), static_cast<int>(E), static_cast<int>(H));
+    const int64_t nb = (T + kDispTok - 1) / kDispTok;
+    const int64_t Rp = mx_routed_rows(c, T);
+    WorkspaceBwd w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    w.router_w3 = reinterpret_cast<__nv_bfloat16*>(take(2 * 3 * E * H));
+    w.router_part = reinterpret_cast<float*>(take(sizeof(float) * rp.nsplit * T * E));
+    w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * E));
+    w.totals = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * E));
+    w.topk_idx = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.topk_w = reinterpret_cast<float*>(take(sizeof(float) * T * K));
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (E + 1)));
+    w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * Rp));
+    w.row_of = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * H));
+    w.do_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * H));
+    w.gu_r = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * 2 * I));
+    w.gu_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * 2 * SI));
+    w.dgu_r = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * 2 * I));
+    w.dgu_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * 2 * SI));
+    w.h_r = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * I));
+    w.h_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
+    w.dw_part = reinterpret_cast<float*>(take(sizeof(float) * Rp * ((I + kBN - 1) / kBN)));
+    w.dlogit = reinterpret_cast<float*>(take(sizeof(float) * T * K));
+    w.dxq = reinterpret_cast<__half*>(take(2 * (Rp + T) * H));
+    w.dxs = take((Rp + T) * scale_ld(H));
+    w.rp = Rp;
+    w.bytes = off;
+    return w;
+}
+
+struct BwdArgs {
+    const void *x, *dy, *w_gate, *w_up, *w_down, *ws_gate, *ws_up, *ws_down;
+    void *d_w_gate, *d_w_up, *d_w_down, *d_ws_gate, *d_ws_up, *d_ws_down;
+};
+
+template <int kMode>
+int launch_bwd_gemm(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b2_r,
+                    const CUtensorMap& b_s, const CUtensorMap& b2_s, const BwdParams& p, int64_t tiles_bound,
+                    int num_sms, cudaStream_t st) {
+    int64_t grid = tiles_bound < num_sms ? tiles_bound : num_sms;
+    if (grid < 1) grid = 1;
+    grouped_gemm_bwd_kernel<kMode><<<static_cast<unsigned>(grid), kGemmThreads, kGemmBwdSmemBytes, st>>>(
+        a_r, a_s, b_r, b2_r, b_s, b2_s, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_backward(const moe_config* c, int64_t T, const float* router_w, const float* e_bias, const BwdArgs& a,
+                    float* dx, float* d_router_w, const WorkspaceBwd& w, int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    const int64_t Rp = w.rp;
+    const int nti = static_cast<int>((I + kBN - 1) / kBN), nts = static_cast<int>((SI + kBN - 1) / kBN);
+    int v;
+    // 1. routing, recomputed (same kernels and inputs as the forward: the same selection)
+    if ((v = launch_route(c, T, a.x, router_w, e_bias, w.topk_idx, w.topk_w, w.router_part, w.router_w3, num_sms,
+                          st)) != MOE_OK)
+        return v;
+    // 2. dispatch of x and w * dy into 128-row aligned segments, padding rows zeroed
+    const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(w.topk_idx, static_cast<int>(T),
+                                                                      static_cast<int>(K), static_cast<int>(E),
+                                                                      w.block_counts);
+    dispatch_scan_kernel<<<static_cast<unsigned>((E + 7) / 8), 256, 0, st>>>(w.block_counts, nb, static_cast<int>(E),
+                                                                            w.block_base, w.totals);
+    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(
+        w.topk_idx, static_cast<int>(T), static_cast<int>(K), static_cast<int>(E), w.block_base, w.totals,
+        kMxAtomRows, w.offsets, w.perm_src, w.row_of);
+    const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
+    bwd_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x),
+                                            static_cast<const __nv_bfloat16*>(a.dy), w.row_of, w.topk_w,
+                                            static_cast<int>(K), static_cast<int>(H), w.x_perm, w.do_perm);
+    bwd_zero_pad_kernel<<<dim3(static_cast<unsigned>(E), 8), 256, 0, st>>>(w.offsets, w.totals, static_cast<int>(H),
+                                                                          w.x_perm, w.do_perm);
+    count_launch(5);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+    const int64_t m_bound = Rp / kBM + (has_shared ? (T + kBM - 1) / kBM : 0);
+    // 3. g, u recomputed
+    {
+        CUtensorMap ar, as, br, b2r, bs, b2s;
+        bool ok = make_map(&ar, w.x_perm, Rp, H, kBM) && make_map(&br, a.w_gate, E * I, H, kBN / 2) &&
+                  make_map(&b2r, a.w_up, E * I, H, kBN / 2);
+        if (has_shared)
+            ok = ok && make_map(&as, a.x, T, H, kBM) && make_map(&bs, a.ws_gate, SI, H, kBN / 2) &&
+                 make_map(&b2s, a.ws_up, SI, H, kBN / 2);
+        else { as = ar; bs = br; b2s = b2r; }
+        if (!ok) return MOE_ERR_CUDA;
+        BwdParams p{};
+        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+        p.has_shared = has_shared;
+        p.n_tiles_routed = static_cast<int>(I / (kBN / 2)); p.n_tiles_shared = static_cast<int>(SI / (kBN / 2));
+        p.kb_routed = p.kb_shared = static_cast<int>(H / kBK);
+        p.b_rows_per_expert = static_cast<int>(I);
+        p.out_routed = w.gu_r; p.ld_routed = 2 * I; p.out_shared = w.gu_s; p.ld_shared = 2 * SI;
+        p.half_routed = static_cast<int>(I); p.half_shared = static_cast<int>(SI);
+        p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 0);
+        if ((v = launch_bwd_gemm<kRecompute>(ar, as, br, b2r, bs, b2s, p, m_bound * (I / (kBN / 2)), num_sms, st)) !=
+            MOE_OK)
+            return v;
+    }
+    // 4. dh = dO Wd with the SwiGLU backward
+    {
+        CUtensorMap ar, as, br, bs;
+        bool ok = make_map(&ar, w.do_perm, Rp, H, kBM) && make_map(&br, a.w_down, E * H, I, 64);
+        if (has_shared) ok = ok && make_map(&as, a.dy, T, H, kBM) && make_map(&bs, a.ws_down, H, SI, 64);
+        else { as = ar; bs = br; }
+        if (!ok) return MOE_ERR_CUDA;
+        BwdParams p{};
+        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+        p.has_shared = has_shared;
+        p.n_tiles_routed = nti; p.n_tiles_shared = nts;
+        p.kb_routed = p.kb_shared = static_cast<int>(H / kBK);
+        p.b_rows_per_expert = static_cast<int>(H);
+        p.out_routed = w.dgu_r; p.ld_routed = 2 * I; p.out_shared = w.dgu_s; p.ld_shared = 2 * SI;
+        p.out2_routed = w.h_r; p.ld2_routed = I; p.out2_shared = w.h_s; p.ld2_shared = SI;
+        p.gu_routed = w.gu_r; p.gu_ld_routed = 2 * I; p.gu_shared = w.gu_s; p.gu_ld_shared = 2 * SI;
+        p.half_routed = static_cast<int>(I); p.half_shared = static_cast<int>(SI);
+        p.n_valid_routed = static_cast<int>(I); p.n_valid_shared = static_cast<int>(SI);
+        p.dw_part = w.dw_part;
+        p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 1);
+        if ((v = launch_bwd_gemm<kDh>(ar, as, br, br, bs, bs, p, m_bound * (nti > nts ? nti : nts), num_sms, st)) !=
+            MOE_OK)
+            return v;
+    }
+    // 5. dx_perm = dg Wg + du Wu (block-scaled fp16)
+    {
+        CUtensorMap ar, as, br, b2r, bs, b2s;
+        bool ok = make_map(&ar, w.dgu_r, Rp, 2 * I, kBM) && make_map(&br, a.w_gate, E * I, H, 64) &&
+                  make_map(&b2r, a.w_up, E * I, H, 64);
+        if (has_shared)
+            ok = ok && make_map(&as, w.dgu_s, T, 2 * SI, kBM) && make_map(&bs, a.ws_gate, SI, H, 64) &&
+                 make_map(&b2s, a.ws_up, SI, H, 64);
+        else { as = ar; bs = br; b2s = b2r; }
+        if (!ok) return MOE_ERR_CUDA;
+        BwdParams p{};
+        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+        p.has_shared = has_shared;
+        p.n_tiles_routed = p.n_tiles_shared = static_cast<int>(H / kBN);
+        p.kb_routed = static_cast<int>(2 * I / kBK); p.kb_shared = static_cast<int>(2 * SI / kBK);
+        p.i_blocks_routed = static_cast<int>(I / kBK); p.i_blocks_shared = static_cast<int>(SI / kBK);
+        p.b_rows_per_expert = static_cast<int>(I);
+        p.n_valid_routed = p.n_valid_shared = static_cast<int>(H);
+        p.yq_routed = w.dxq; p.yq_shared = w.dxq + Rp * H; p.yq_ld = H;
+        p.ysc_routed = w.dxs; p.ysc_shared = w.dxs + Rp * scale_ld(H); p.ysc_ld = scale_ld(H);
+        p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 1);
+        if ((v = launch_bwd_gemm<kDx>(ar, as, br, b2r, bs, b2s, p, m_bound * (H / kBN), num_sms, st)) != MOE_OK)
+            return v;
+    }
+    // 6. weight gradients: dWd = dO^T h, [dWg; dWu] = [dg du]^T x
+    {
+        CUtensorMap ar, as, br, bs;
+        bool ok = make_map(&ar, w.do_perm, Rp, H, 64) && make_map(&br, w.h_r, Rp, I, 64);
+        if (has_shared) ok = ok && make_map(&as, a.dy, T, H, 64) && make_map(&bs, w.h_s, T, SI, 64);
+        else { as = ar; bs = br; }
+        if (!ok) return MOE_ERR_CUDA;
+        BwdParams p{};
+        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+        p.has_shared = has_shared;
+        p.m_tiles_wgrad_routed = p.m_tiles_wgrad_shared = static_cast<int>(H / kBM);
+        p.n_tiles_routed = nti; p.n_tiles_shared = nts;
+        p.n_valid_routed = static_cast<int>(I); p.n_valid_shared = static_cast<int>(SI);
+        p.out_routed = static_cast<__nv_bfloat16*>(a.d_w_down); p.ld_routed = I; p.out_expert_stride = H * I;
+        p.out_shared = static_cast<__nv_bfloat16*>(a.d_ws_down); p.ld_shared = SI;
+        p.split_rows_routed = p.split_rows_shared = static_cast<int>(H);
+        p.idesc = idesc_bf16_f32_major(kBM, kBN, 1, 1);
+        const int64_t tiles = (E + has_shared) * (H / kBM) * (nti > nts ? nti : nts);
+        if ((v = launch_bwd_gemm<kWgrad>(ar, as, br, br, bs, bs, p, tiles, num_sms, st)) != MOE_OK) return v;
+    }
+    {
+        CUtensorMap ar, as, br, bs;
+        bool ok = make_map(&ar, w.dgu_r, Rp, 2 * I, 64) && make_map(&br, w.x_perm, Rp, H, 64);
+        if (has_shared) ok = ok && make_map(&as, w.dgu_s, T, 2 * SI, 64) && make_map(&bs, a.x, T, H, 64);
+        else { as = ar; bs = br; }
+        if (!ok) return MOE_ERR_CUDA;
+        BwdParams p{};
+        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+        p.has_shared = has_shared;
+        p.m_tiles_wgrad_routed = static_cast<int>(2 * I / kBM);
+        p.m_tiles_wgrad_shared = static_cast<int>(2 * SI / kBM);
+        p.n_tiles_routed = p.n_tiles_shared = static_cast<int>(H / kBN);
+        p.n_valid_routed = p.n_valid_shared = static_cast<int>(H);
+        p.out_routed = static_cast<__nv_bfloat16*>(a.d_w_gate); p.ld_routed = H; p.out_expert_stride = I * H;
+        p.out2_routed = static_cast<__nv_bfloat16*>(a.d_w_up); p.ld2_routed = H; p.out2_expert_stride = I * H;
+        p.out_shared = static_cast<__nv_bfloat16*>(a.d_ws_gate); p.ld_shared = H;
+        p.out2_shared = static_cast<__nv_bfloat16*>(a.d_ws_up); p.ld2_shared = H;
+        p.split_rows_routed = static_cast<int>(I); p.split_rows_shared = static_cast<int>(SI);
+        p.idesc = idesc_bf16_f32_major(kBM, kBN, 1, 1);
+        const int64_t tiles = (E + has_shared) * (2 * (I > SI ? I : SI) / kBM) * (H / kBN);
+        if ((v = launch_bwd_gemm<kWgrad>(ar, as, br, br, bs, bs, p, tiles, num_sms, st)) != MOE_OK) return v;
+    }
+    // 7. router backward, router weight gradient, dx
+    const RouterPlan rp = plan_router(static_cast<int>(T), static_cast<int>(E), static_cast<int>(H));
+    bwd_router_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(
+        w.router_part, rp.nsplit, static_cast<int>(T), static_cast<int>(E), static_cast<int>(K), c->norm_topk_prob,
+        c->routed_scaling_factor, w.topk_idx, w.topk_w, w.row_of, w.dw_part, nti, w.dlogit);
+    bwd_router_wgrad_kernel<<<dim3(static_cast<unsigned>(E), static_cast<unsigned>((H / 8 + 255) / 256)), 256, 0,
+                              st>>>(w.offsets, w.totals, w.perm_src, w.dlogit, w.x_perm, static_cast<int>(H),
+                                    d_router_w);
+    bwd_dx_kernel<<<gs, 256, 0, st>>>(w.dxq, w.dxs, scale_ld(H), w.row_of, w.topk_idx, w.dlogit, router_w,
+                                      static_cast<int>(K), static_cast<int>(H), has_shared, Rp, dx);
+    count_launch(3);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- no-allocation dispatch
 // Scratch of moe_dispatch_noalloc: per-block expert counts, per-block bases and
 // per-expert totals (2 x ceil(T / kDispTok) x E + E int32), held in this
@@ -1103,6 +1359,51 @@ int moe_combine_mx(const moe_config* cfg, int64_t T, const void* y_perm, const v
     if (!aligned16(y_perm) || !aligned16(y) || !aligned16(y_perm_scale)) return MOE_ERR_UNSUPPORTED;
     return launch_combine(cfg, T, y_perm, y_perm_scale, row_of, y, y_dtype, static_cast<cudaStream_t>(stream),
                           mx_routed_rows(cfg, T));
+}
+
+int moe_workspace_size_bwd(const moe_config* cfg, int64_t T, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    *bytes = carve_bwd(cfg, T, nullptr).bytes;
+    return MOE_OK;
+}
+
+int moe_backward(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
+                 const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                 const void* ws_down, const void* dy, float* dx, float* d_router_w, void* d_w_gate, void* d_w_up,
+                 void* d_w_down, void* d_ws_gate, void* d_ws_up, void* d_ws_down, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    const bool sh = cfg->n_shared_experts > 0;
+    if ((v = check_ptrs({router_w, w_gate, w_up, w_down, d_router_w, d_w_gate, d_w_up, d_w_down})) != MOE_OK) return v;
+    if (sh && (v = check_ptrs({ws_gate, ws_up, ws_down, d_ws_gate, d_ws_up, d_ws_down})) != MOE_OK) return v;
+    if (!e_bias) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t H = cfg->hidden_size, E = cfg->n_routed_experts, I = cfg->moe_intermediate_size;
+    const int64_t SI = static_cast<int64_t>(cfg->n_shared_experts) * I;
+    if (T == 0) {
+        // No tokens: every gradient is zero.
+        const size_t wb = sizeof(uint16_t) * E * I * H, sb = sizeof(uint16_t) * SI * H;
+        if (cudaMemsetAsync(d_router_w, 0, sizeof(float) * E * H, st) != cudaSuccess ||
+            cudaMemsetAsync(d_w_gate, 0, wb, st) != cudaSuccess || cudaMemsetAsync(d_w_up, 0, wb, st) != cudaSuccess ||
+            cudaMemsetAsync(d_w_down, 0, wb, st) != cudaSuccess ||
+            (sh && (cudaMemsetAsync(d_ws_gate, 0, sb, st) != cudaSuccess ||
+                    cudaMemsetAsync(d_ws_up, 0, sb, st) != cudaSuccess ||
+                    cudaMemsetAsync(d_ws_down, 0, sb, st) != cudaSuccess)))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if ((v = check_ptrs({x, dy, dx})) != MOE_OK) return v;
+    if (!workspace || workspace_bytes < carve_bwd(cfg, T, nullptr).bytes || !aligned16(workspace))
+        return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    const WorkspaceBwd w = carve_bwd(cfg, T, static_cast<uint8_t*>(workspace));
+    const BwdArgs a{x, dy, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                    d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down};
+    return launch_backward(cfg, T, router_w, e_bias, a, dx, d_router_w, w, d->num_sms, st);
 }
 
 const char* moe_status_string(int status) {

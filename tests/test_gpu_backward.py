@@ -1,0 +1,146 @@
+"""Backward pass on B200 against the float64 backward oracle (oracle/backward.py,
+pinned by finite differences).  Every gradient — dx, the router weight, each
+expert's gate / up / down weights and the shared expert's — is compared with
+the oracle on the same bits, with the expert selection the GPU's router made
+(the backward holds it fixed).  Full-size shapes: sampled token rows of dx and
+the weight gradients of a sampled expert."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import backward as B
+from sparse_moe_layer_noaux_b200 import MoELayer, abi
+from sparse_moe_layer_noaux_b200.workloads import MID, TINY, V3_PREFILL, MoEShape, bf16_bits, make_inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+# Tolerance, from the arithmetic: every gradient element is an fp32 sum of products
+# of three bf16-rounded factors (dO = w dy, g / u or h, x or the weights), each
+# rounded once to bf16 (2^-9 relative), so an element can be off by ~3 * 2^-9 of
+# its own size and, with few rows per expert, that does not average out.  Bar:
+# max |err| <= 2e-2 * max |ref| (per tensor) and relative L1 <= 1e-2.
+MAX_ABS_REL_MAX = 2e-2
+REL_L1 = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from sparse_moe_layer_noaux_b200 import build
+    build.build()
+    oracle.build()
+    yield
+    torch.cuda.empty_cache()
+
+
+def close(got, ref, what):
+    e = parity.output_errors(np.asarray(got, np.float64), ref)
+    e["max_abs_over_max"] = e["max_abs"] / max(float(np.abs(ref).max()), 1e-300)
+    print(what, e)
+    assert e["max_abs_over_max"] <= MAX_ABS_REL_MAX and e["rel_l1"] <= REL_L1, (what, e)
+    return e
+
+
+def gpu_backward(shape, inp, seed=0):
+    g = torch.Generator(device="cuda").manual_seed(1000 + seed)
+    dy = torch.randn((shape.T, shape.H), device="cuda", generator=g).bfloat16()
+    layer = MoELayer.from_inputs(shape, inp)
+    grads = layer.backward(inp["x"], dy)
+    cfg = abi.MoEConfig.from_shape(shape)
+    ws = torch.empty(max(abi.workspace_size(cfg, shape.T), 256), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, inp["x"], inp["router_w"], inp["e_bias"], idx, w, ws)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    return grads, dy, idx.cpu().numpy()
+
+
+SMALL = [
+    TINY,
+    MoEShape("ragged", T=300, hidden_size=512, n_routed_experts=32, n_group=4, topk_group=2,
+             num_experts_per_tok=4, moe_intermediate_size=256, n_shared_experts=1,
+             routed_scaling_factor=2.5, norm_topk_prob=True, seed=7),
+    MoEShape("tiles", T=2200, hidden_size=512, n_routed_experts=8, n_group=2, topk_group=1,
+             num_experts_per_tok=4, moe_intermediate_size=384, n_shared_experts=2,
+             routed_scaling_factor=1.3, norm_topk_prob=False, seed=8),
+    MoEShape("noshared", T=500, hidden_size=256, n_routed_experts=16, n_group=1, topk_group=1,
+             num_experts_per_tok=3, moe_intermediate_size=128, n_shared_experts=0,
+             routed_scaling_factor=1.0, norm_topk_prob=True, seed=9),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: s.name)
+def test_backward_small_every_gradient(shape):
+    inp = make_inputs(shape, "cuda")
+    grads, dy, idx = gpu_backward(shape, inp)
+    fetch = parity.device_expert_fetch(inp)
+    shared = parity.shared_bits(inp, shape)
+    ref = B.moe_layer_backward(shape, bf16_bits(inp["x"]), inp["router_w"].cpu().numpy(),
+                               inp["e_bias"].cpu().numpy(), fetch, shared, bf16_bits(dy), routing=idx)
+    close(grads["x"].cpu().numpy(), ref.dx, f"{shape.name} dx")
+    close(grads["router_w"].cpu().numpy(), ref.d_router_w, f"{shape.name} d_router_w")
+    for j, name in enumerate(("w_gate", "w_up", "w_down")):
+        got = grads[name].float().cpu().numpy()
+        want = np.zeros_like(got, dtype=np.float64)
+        for e, gr in ref.d_experts.items():
+            want[e] = gr[j]
+        close(got, want, f"{shape.name} d_{name}")
+        unused = sorted(set(range(shape.E)) - set(ref.d_experts))
+        assert all((got[e] == 0).all() for e in unused)
+    if shape.S > 0:
+        for j, name in enumerate(("ws_gate", "ws_up", "ws_down")):
+            close(grads[name].float().cpu().numpy(), ref.d_shared[j], f"{shape.name} d_{name}")
+
+
+def test_backward_deterministic():
+    shape = SMALL[1]
+    inp = make_inputs(shape, "cuda")
+    g1, *_ = gpu_backward(shape, inp)
+    g2, *_ = gpu_backward(shape, inp)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+@pytest.mark.parametrize("shape,n_rows", [(MID, 16), (V3_PREFILL, 8)], ids=lambda v: getattr(v, "name", str(v)))
+def test_backward_full_size_sampled(shape, n_rows):
+    """dx of sampled rows, and the weight gradients of one sampled expert (all of its
+    rows) against the oracle's expert backward on the same operands."""
+    inp = make_inputs(shape, "cuda")
+    grads, dy, idx = gpu_backward(shape, inp)
+    rng = np.random.default_rng(shape.seed)
+    rows = np.sort(rng.choice(shape.T, n_rows, replace=False))
+    x_rows = bf16_bits(inp["x"][torch.as_tensor(rows, device="cuda")])
+    ref = B.moe_layer_backward(shape, x_rows, inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy(),
+                               parity.device_expert_fetch(inp), parity.shared_bits(inp, shape),
+                               bf16_bits(dy[torch.as_tensor(rows, device="cuda")]), routing=idx[rows])
+    close(grads["x"].cpu().numpy()[rows], ref.dx, f"{shape.name} dx rows")
+    # One expert's weight gradients over all of its rows.
+    e = int(rng.choice(np.unique(idx)))
+    toks, slots = np.nonzero(idx == e)
+    xt = oracle.widen_bf16(bf16_bits(inp["x"]))[toks]
+    rw = inp["router_w"].cpu().numpy().astype(np.float64)
+    s = 1.0 / (1.0 + np.exp(-(xt @ rw.T)))
+    s_sel = np.take_along_axis(s, idx[toks].astype(np.int64), axis=1)
+    w = s_sel / s_sel.sum(1, keepdims=True) if shape.norm_topk_prob else s_sel
+    w = shape.routed_scaling_factor * w[np.arange(len(toks)), slots]
+    do = w[:, None] * oracle.widen_bf16(bf16_bits(dy))[toks]
+    wg, wu, wd = (oracle.widen_bf16(a) for a in parity.device_expert_fetch(inp)(e))
+    _, dwg, dwu, dwd, _ = B._swiglu_backward(xt, wg, wu, wd, do)
+    close(grads["w_gate"][e].float().cpu().numpy(), dwg, f"{shape.name} d_w_gate[{e}]")
+    close(grads["w_up"][e].float().cpu().numpy(), dwu, f"{shape.name} d_w_up[{e}]")
+    close(grads["w_down"][e].float().cpu().numpy(), dwd, f"{shape.name} d_w_down[{e}]")
+
+
+def test_backward_empty_batch_gives_zero_weight_gradients():
+    shape = TINY.with_(T=0)
+    inp = make_inputs(shape, "cuda")
+    dy = torch.empty((0, shape.H), dtype=torch.bfloat16, device="cuda")
+    layer = MoELayer.from_inputs(shape, inp)
+    grads = layer.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    for k in ("router_w", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+        assert not grads[k].float().abs().sum().item(), k
