@@ -335,6 +335,47 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
     return out
 
 
+def time_backward(shape, steps, warmup, world, rank, peaks, inp):
+    """moe_backward (gradients of sum(y * dy) for x, the router weight and every
+    expert weight) on the same workload, K calls timed like the forward."""
+    layer = MoELayer.from_inputs(shape, inp)
+    g = torch.Generator(device="cuda").manual_seed(shape.seed + 99)
+    dy = torch.randn((shape.T, shape.H), device="cuda", generator=g).bfloat16()
+    grads = layer.backward(inp["x"], dy)  # allocates the gradients and the workspace once
+    cfg = layer.cfg
+    ws = layer._ws_bwd
+
+    def step():
+        abi.moe_backward(cfg, inp["x"], layer.router_w, layer.e_bias, layer.w_gate, layer.w_up, layer.w_down,
+                         layer.ws_gate, layer.ws_up, layer.ws_down, dy, grads["x"], grads["router_w"],
+                         grads["w_gate"], grads["w_up"], grads["w_down"], grads.get("ws_gate"), grads.get("ws_up"),
+                         grads.get("ws_down"), ws)
+    ms, launches, clk = time_steps(step, steps, warmup, world)
+    # recompute g,u (4), dh (2), dx (4), dWd (2), dWg + dWu (4): 16 H I per (token, expert) pair
+    flops = 16.0 * shape.H * shape.I * shape.T * (shape.k + shape.S) + 4.0 * shape.T * shape.E * shape.H
+    # weights read (gate/up twice, down twice), weight gradients written (bf16)
+    touched = int(torch.unique(layer_route_idx(shape, inp)).numel())
+    wbytes = (touched + shape.S) * 3 * shape.H * shape.I * 2
+    bytes_ = 2 * wbytes + wbytes + 2 * 2 * shape.T * shape.H + 4 * shape.T * shape.H
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    out = {"ms_per_step": ms, "tokens_per_s": job_throughput(shape.T, world, ms),
+           "tflops": flops / (ms * 1e-3) / 1e12 * world, "flops": flops, "gpu_launches": launches,
+           "layer_roofline": {"bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= bytes_ / (peaks["hbm_gbs"] * 1e9)
+                              else "hbm", "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms},
+           "clocks": clk}
+    del grads, layer
+    return out
+
+
+def layer_route_idx(shape, inp):
+    cfg = abi.MoEConfig.from_shape(shape)
+    ws = torch.empty(abi.workspace_size(cfg, shape.T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, inp["x"], inp["router_w"], inp["e_bias"], idx, w, ws)
+    return idx
+
+
 def layer_bytes(shape, idx):
     """Algorithmic bytes of one step: touched routed experts + shared + router + x and y."""
     touched = int(torch.unique(idx).numel())
@@ -523,17 +564,28 @@ def main():
     ap.add_argument("--workload", default="v3_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mx", action="store_true", help="skip the MXFP8 variant of the layer")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--precision", default="bf16", choices=["bf16", "mxfp8"],
-                    help="expert FFN precision of --profile-only passes")
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "mxfp8", "backward"],
+                    help="what --profile-only runs: the bf16 or MXFP8 forward stages, or the backward")
     ap.add_argument("--profile-only", action="store_true",
                     help="run warmup + steps layer passes and exit without timing (for profilers)")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
     if args.profile_only:
-        stepper = StagedStepMX if args.precision == "mxfp8" else StagedStep
-        st = stepper(shape, rank_inputs(shape, rank, "cuda"))
+        inp0 = rank_inputs(shape, rank, "cuda")
+        if args.precision == "backward":
+            layer = MoELayer.from_inputs(shape, inp0)
+            dy = torch.randn((shape.T, shape.H), device="cuda").bfloat16()
+
+            class _B:
+                def run(self):
+                    layer.backward(inp0["x"], dy)
+            st = _B()
+        else:
+            stepper = StagedStepMX if args.precision == "mxfp8" else StagedStep
+            st = stepper(shape, inp0)
         for _ in range(args.warmup + args.steps):
             st.run()
         torch.cuda.synchronize()
@@ -588,6 +640,10 @@ def main():
         extra["mxfp8"] = time_gpu_mx(shape, args.steps, args.warmup, world, rank, peaks, inp=res["inp"])
         dec = WORKLOADS["v3_decode"]
         extra["mxfp8_decode"] = time_gpu_mx(dec, max(args.steps, 20), args.warmup, world, rank, peaks)
+        torch.cuda.empty_cache()
+    if not args.no_bwd and shape.name == "v3_prefill":
+        extra["backward"] = time_backward(shape, max(3, args.steps // 4), args.warmup, world, rank, peaks,
+                                          res["inp"])
         torch.cuda.empty_cache()
 
     line = {

@@ -8,7 +8,8 @@
 //   bwd_router_kernel      per token: dL/dw_j = sum(dh h)_j / w_j (from the dh
 //                          GEMM's per-tile partial sums), then through the weight
 //                          normalisation and the sigmoid to dL/dlogit;
-//   bwd_router_wgrad_kernel  dWr[e] = sum over expert e's rows of dlogit * x;
+//   bwd_router_wgrad_kernel  dWr[e] = sum over expert e's rows of dlogit * x
+//                          (row chunks in parallel, then an ordered reduction);
 //   bwd_dx_kernel          dx[t] = shared row + sum_j expert rows (block-scaled
 //                          fp16, the kDx GEMM's output) + sum_j dlogit_j Wr[e_j].
 #pragma once
@@ -103,33 +104,61 @@ __global__ void __launch_bounds__(256) bwd_router_kernel(const float* __restrict
     }
 }
 
-// Block (e, c): 256 threads x 8 columns = 2048 columns c*2048.. of dWr[e], summed
-// over expert e's rows in row order (deterministic).
+// Block (e, c, q): 256 threads x 8 columns = 2048 columns c*2048.. of expert e,
+// summed over the q-th of kRouterSplit row chunks of the expert's segment, eight
+// rows per step with independent loads; partial sums go to
+// part[q][e][H] and bwd_router_wgrad_reduce_kernel adds them in order
+// (deterministic).
+constexpr int kRouterSplit = 4;
+
 __global__ void __launch_bounds__(256) bwd_router_wgrad_kernel(const int32_t* __restrict__ offsets,
                                                                const int32_t* __restrict__ counts,
                                                                const int32_t* __restrict__ perm_src,
                                                                const float* __restrict__ dlogit,
-                                                               const __nv_bfloat16* __restrict__ x_perm, int H,
-                                                               float* __restrict__ d_router_w) {
-    const int e = blockIdx.x;
+                                                               const __nv_bfloat16* __restrict__ x_perm, int H, int E,
+                                                               float* __restrict__ part) {
+    const int e = blockIdx.x, q = blockIdx.z;
     const int c = blockIdx.y * 256 + threadIdx.x;
-    if (c >= H / 8) return;
-    const int64_t r0 = offsets[e], n = counts[e];
+    const int64_t n = counts[e];
+    const int64_t chunk = (n + kRouterSplit - 1) / kRouterSplit;
+    const int64_t i0 = q * chunk, i1 = min(n, i0 + chunk);
+    const int64_t r0 = offsets[e];
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int64_t i = 0; i < n; ++i) {
-        const float d = dlogit[perm_src[r0 + i]];
-        const uint4 v = reinterpret_cast<const uint4*>(x_perm + (r0 + i) * H)[c];
-        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+    if (c < H / 8) {
+        for (int64_t i = i0; i < i1; i += 8) {
+            float d[8];
+            uint4 v[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float2 f = __bfloat1622float2(v2[q]);
-            acc[2 * q] += d * f.x;
-            acc[2 * q + 1] += d * f.y;
+            for (int u = 0; u < 8; ++u) {
+                const bool in = i + u < i1;
+                d[u] = in ? dlogit[perm_src[r0 + i + u]] : 0.0f;
+                v[u] = in ? reinterpret_cast<const uint4*>(x_perm + (r0 + i + u) * H)[c] : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float2 f = __bfloat1622float2(v2[w]);
+                    acc[2 * w] += d[u] * f.x;
+                    acc[2 * w + 1] += d[u] * f.y;
+                }
+            }
         }
+        float4* out = reinterpret_cast<float4*>(part + ((int64_t)q * E + e) * H + 8 * c);
+        out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-    float4* out = reinterpret_cast<float4*>(d_router_w + (int64_t)e * H + 8 * c);
-    out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+__global__ void __launch_bounds__(256) bwd_router_wgrad_reduce_kernel(const float* __restrict__ part, int64_t n,
+                                                                      float* __restrict__ d_router_w) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float s = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kRouterSplit; ++q) s += part[q * n + i];
+    d_router_w[i] = s;
 }
 
 // Block (t, c): dx of token t, columns 8*(c*256 + thread) ..; expert rows are

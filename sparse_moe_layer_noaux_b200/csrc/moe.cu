@@ -740,6 +740,7 @@ struct WorkspaceBwd {
     __nv_bfloat16* h_s;       // [T, SI]
     float* dw_part;           // [Rp, ceil(I/256)]
     float* dlogit;            // [T, k]
+    float* dwr_part;          // [kRouterSplit, E, H]
     __half* dxq;              // [Rp + T, H] block-scaled fp16
     uint8_t* dxs;             // [Rp + T, scale_ld]
     int64_t rp;
@@ -779,6 +780,7 @@ WorkspaceBwd carve_bwd(const moe_config* c, int64_t T, uint8_t* base) {
     w.h_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
     w.dw_part = reinterpret_cast<float*>(take(sizeof(float) * Rp * ((I + kBN - 1) / kBN)));
     w.dlogit = reinterpret_cast<float*>(take(sizeof(float) * T * K));
+    w.dwr_part = reinterpret_cast<float*>(take(sizeof(float) * kRouterSplit * E * H));
     w.dxq = reinterpret_cast<__half*>(take(2 * (Rp + T) * H));
     w.dxs = take((Rp + T) * scale_ld(H));
     w.rp = Rp;
@@ -953,12 +955,15 @@ int launch_backward(const moe_config* c, int64_t T, const float* router_w, const
     bwd_router_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(
         w.router_part, rp.nsplit, static_cast<int>(T), static_cast<int>(E), static_cast<int>(K), c->norm_topk_prob,
         c->routed_scaling_factor, w.topk_idx, w.topk_w, w.row_of, w.dw_part, nti, w.dlogit);
-    bwd_router_wgrad_kernel<<<dim3(static_cast<unsigned>(E), static_cast<unsigned>((H / 8 + 255) / 256)), 256, 0,
-                              st>>>(w.offsets, w.totals, w.perm_src, w.dlogit, w.x_perm, static_cast<int>(H),
-                                    d_router_w);
+    bwd_router_wgrad_kernel<<<dim3(static_cast<unsigned>(E), static_cast<unsigned>((H / 8 + 255) / 256),
+                                   kRouterSplit),
+                              256, 0, st>>>(w.offsets, w.totals, w.perm_src, w.dlogit, w.x_perm, static_cast<int>(H),
+                                            static_cast<int>(E), w.dwr_part);
+    bwd_router_wgrad_reduce_kernel<<<static_cast<unsigned>((E * H + 255) / 256), 256, 0, st>>>(w.dwr_part, E * H,
+                                                                                             d_router_w);
     bwd_dx_kernel<<<gs, 256, 0, st>>>(w.dxq, w.dxs, scale_ld(H), w.row_of, w.topk_idx, w.dlogit, router_w,
                                       static_cast<int>(K), static_cast<int>(H), has_shared, Rp, dx);
-    count_launch(3);
+    count_launch(4);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
