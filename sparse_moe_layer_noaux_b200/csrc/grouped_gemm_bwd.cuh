@@ -7,8 +7,8 @@
 //               as bf16 (the forward is recomputed instead of kept);
 //   kDh         dh = dO Wd (dO = w dy for routed rows, dy for shared rows), with
 //               the SwiGLU backward in the epilogue: dg = dh u silu'(g),
-//               du = dh silu(g), h = silu(g) u, and per row the partial dot
-//               sum(dh h) that gives the routing-weight gradient;
+//               du = dh silu(g), h = silu(g) u, and per row and half tile the
+//               partial dot sum(dh h) that gives the routing-weight gradient;
 //   kDx         dx_perm = dg Wg + du Wu (K = 2 I over the two weight maps),
 //               block-scaled fp16 like the forward's y_perm;
 //   kWgrad      dW = P^T Q for each expert over its rows (K = the segment's
@@ -51,7 +51,7 @@ struct BwdParams {
     const __nv_bfloat16* gu_shared;
     int64_t gu_ld_routed, gu_ld_shared;
     int half_routed, half_shared;    // kDh: I (where u starts inside a gu row)
-    float* dw_part;                  // kDh: [rows, n_tiles_routed] partial sum(dh h) of routed rows
+    float* dw_part;                  // kDh: [rows, 2 n_tiles_routed] partial sum(dh h) of routed rows
     __half* yq_routed;               // kDx: block-scaled fp16 rows
     __half* yq_shared;
     uint8_t* ysc_routed;
@@ -84,8 +84,14 @@ struct BwdSmem {
     int tile_start[kMaxSeg + 1];
 };
 
+// Eight epilogue warps (two per TMEM lane quarter, each draining half of the 256
+// accumulator columns): the weight-gradient tiles have only ~8 K blocks at the
+// V3 prefill shape, so a four-warp epilogue was as long as the main loop.
+constexpr int kBwdEpiWarps = 8;
+constexpr int kBwdThreads = 64 + 32 * kBwdEpiWarps;
+constexpr uint32_t kBwdStagePerWarp = 32 * kStagePitchH * 2;  // 32 rows x 80 B of 16-bit values
 constexpr size_t kGemmBwdSmemBytes =
-    1024 + kStages * (kTileABytes + kTileBBytes) + kStageBytes + sizeof(BwdSmem);
+    1024 + kStages * (kTileABytes + kTileBBytes) + kBwdEpiWarps * kBwdStagePerWarp + sizeof(BwdSmem);
 
 // Descriptor of an MN-major operand in the 128-byte swizzle layout: atoms of 64
 // contiguous elements (128 B) by 8 K rows (1024 B); consecutive K groups of 8
@@ -143,7 +149,7 @@ __device__ __forceinline__ BwdTile decode_bwd(const BwdSmem& s, const BwdParams&
 }
 
 template <int kMode>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     grouped_gemm_bwd_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                             const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB2_r,
                             const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmB2_s,
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* smemA = tiles;
     uint8_t* smemB = tiles + kStages * kTileABytes;
     uint8_t* stage_base = tiles + kStages * (kTileABytes + kTileBBytes);
-    BwdSmem& S = *reinterpret_cast<BwdSmem*>(stage_base + kStageBytes);
+    BwdSmem& S = *reinterpret_cast<BwdSmem*>(stage_base + kBwdEpiWarps * kBwdStagePerWarp);
     volatile int* abort_flag = &S.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(ptx::smem_u32(&S.tmem_full[i]), 1);
-            ptx::mbar_init(ptx::smem_u32(&S.tmem_empty[i]), 4);
+            ptx::mbar_init(ptx::smem_u32(&S.tmem_empty[i]), kBwdEpiWarps);
         }
         ptx::mbar_init(ptx::smem_u32(&S.mma_done), 1);
         ptx::fence_barrier_init();
@@ -328,7 +334,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // ================= epilogue (warps 2..5) =================
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
+        const int half = (warp - 2) >> 2;    // accumulator columns 128*half .. +127
+        const int c0 = half * (kBN / 64);    // first 32-column chunk of this warp
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * kBN) +
                                    (static_cast<uint32_t>(quarter * 32) << 16);
-            uint8_t* stage = stage_base + (warp - 2) * kStageBytesPerWarp;
+            uint8_t* stage = stage_base + (warp - 2) * kBwdStagePerWarp;
             __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(stage);
             const int r_warp0 = ti.m * kBM + quarter * 32;
             // Stage 32 bf16 values of this lane's row, then write 8 rows x 64 B per instruction.
@@ -367,17 +375,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // Accumulator columns: g at 0..127, u at 128..255 for intermediate columns n*128...
                 __nv_bfloat16* out = ti.routed ? p.out_routed : p.out_shared;
                 const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
-                const int half = ti.routed ? p.half_routed : p.half_shared;
+                const int ioff = ti.routed ? p.half_routed : p.half_shared;  // where u starts in a gu row
                 const int limit = ti.rows;
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int c = c0; c < c0 + kBN / 64; ++c) {
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
                     ptx::tmem_wait_ld();
                     float f[32];
 #pragma unroll
                     for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
-                    const int col = c < 4 ? ti.n * (kBN / 2) + c * 32 : half + ti.n * (kBN / 2) + (c - 4) * 32;
+                    const int col = c < 4 ? ti.n * (kBN / 2) + c * 32 : ioff + ti.n * (kBN / 2) + (c - 4) * 32;
                     store_rows(f, out, ld, col, limit, ti.row0);
                 }
             } else if (kMode == kDh) {
@@ -385,7 +393,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const bool routed = ti.routed;
                 const __nv_bfloat16* gu = routed ? p.gu_routed : p.gu_shared;
                 const int64_t gld = routed ? p.gu_ld_routed : p.gu_ld_shared;
-                const int half = routed ? p.half_routed : p.half_shared;
+                const int ioff = routed ? p.half_routed : p.half_shared;  // where u (du) starts in a row
                 __nv_bfloat16* dgu = routed ? p.out_routed : p.out_shared;
                 const int64_t ld = routed ? p.ld_routed : p.ld_shared;
                 __nv_bfloat16* hout = routed ? p.out2_routed : p.out2_shared;
@@ -397,47 +405,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int64_t grow = (int64_t)ti.row0 + r_local;
                 float dot = 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int c = c0; c < c0 + kBN / 64; ++c) {
                     const int col = ti.n * kBN + c * 32;
                     if (col >= n_valid) break;  // uniform across the warp
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
                     ptx::tmem_wait_ld();
-                    float dg[32], du[32], h[32];
-                    if (row_ok) {
-                        const uint4* gp = reinterpret_cast<const uint4*>(gu + grow * gld + col);
-                        const uint4* up = reinterpret_cast<const uint4*>(gu + grow * gld + half + col);
+                    // g and u of these 32 columns (packed bf16); zeros for rows past the segment.
+                    uint4 gp[4], up[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 ga = gp[q], ua = up[q];
-                            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&ga);
-                            const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&ua);
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 gf = __bfloat1622float2(g2[e2]), uf = __bfloat1622float2(u2[e2]);
-                                const int i0 = q * 8 + e2 * 2;
-                                const float gg[2] = {gf.x, gf.y}, uu[2] = {uf.x, uf.y};
-#pragma unroll
-                                for (int t = 0; t < 2; ++t) {
-                                    const float d = __uint_as_float(v[i0 + t]);
-                                    const float sg = 1.0f / (1.0f + __expf(-gg[t]));
-                                    const float a = gg[t] * sg;
-                                    h[i0 + t] = a * uu[t];
-                                    du[i0 + t] = d * a;
-                                    dg[i0 + t] = d * uu[t] * (sg * (1.0f + gg[t] * (1.0f - sg)));
-                                    dot += d * h[i0 + t];
-                                }
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) dg[q] = du[q] = h[q] = 0.0f;
+                    for (int q = 0; q < 4; ++q) {
+                        gp[q] = row_ok ? reinterpret_cast<const uint4*>(gu + grow * gld + col)[q] : make_uint4(0, 0, 0, 0);
+                        up[q] = row_ok ? reinterpret_cast<const uint4*>(gu + grow * gld + ioff + col)[q]
+                                       : make_uint4(0, 0, 0, 0);
                     }
-                    store_rows(dg, dgu, ld, col, limit, ti.row0);
-                    store_rows(du, dgu, ld, half + col, limit, ti.row0);
-                    store_rows(h, hout, ld2, col, limit, ti.row0);
+                    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gp);
+                    const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(up);
+                    float out[32];
+                    // h = silu(g) u (and the routing-weight partial sum(dh h)), then du, then dg:
+                    // one 32-value output live at a time.
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float2 gf = __bfloat1622float2(g2[q]), uf = __bfloat1622float2(u2[q]);
+                        const float s0 = 1.0f / (1.0f + __expf(-gf.x)), s1 = 1.0f / (1.0f + __expf(-gf.y));
+                        out[2 * q] = gf.x * s0 * uf.x;
+                        out[2 * q + 1] = gf.y * s1 * uf.y;
+                        dot += __uint_as_float(v[2 * q]) * out[2 * q] + __uint_as_float(v[2 * q + 1]) * out[2 * q + 1];
+                    }
+                    store_rows(out, hout, ld2, col, limit, ti.row0);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float2 gf = __bfloat1622float2(g2[q]);
+                        const float s0 = 1.0f / (1.0f + __expf(-gf.x)), s1 = 1.0f / (1.0f + __expf(-gf.y));
+                        out[2 * q] = __uint_as_float(v[2 * q]) * gf.x * s0;
+                        out[2 * q + 1] = __uint_as_float(v[2 * q + 1]) * gf.y * s1;
+                    }
+                    store_rows(out, dgu, ld, ioff + col, limit, ti.row0);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float2 gf = __bfloat1622float2(g2[q]), uf = __bfloat1622float2(u2[q]);
+                        const float s0 = 1.0f / (1.0f + __expf(-gf.x)), s1 = 1.0f / (1.0f + __expf(-gf.y));
+                        out[2 * q] = __uint_as_float(v[2 * q]) * uf.x * (s0 * (1.0f + gf.x * (1.0f - s0)));
+                        out[2 * q + 1] = __uint_as_float(v[2 * q + 1]) * uf.y * (s1 * (1.0f + gf.y * (1.0f - s1)));
+                    }
+                    store_rows(out, dgu, ld, col, limit, ti.row0);
                 }
-                if (routed && row_ok) p.dw_part[grow * p.n_tiles_routed + ti.n] = dot;
+                if (routed && row_ok) p.dw_part[grow * (2 * p.n_tiles_routed) + 2 * ti.n + half] = dot;
             } else if (kMode == kDx) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
                 __half* out_base = ti.routed ? p.yq_routed : p.yq_shared;
@@ -445,22 +458,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 __half* hq = reinterpret_cast<__half*>(stage);
                 const bool row_ok = r_local < ti.rows;
                 const int64_t grow = (int64_t)ti.row0 + r_local;
-                uint32_t codes[kBN / 32];
+                uint32_t codes[kBN / 64];
 #pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int i = 0; i < kBN / 64; ++i) {
+                    const int c = c0 + i;
                     __syncwarp();
                     uint32_t v[32];
                     ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
                     ptx::tmem_wait_ld();
                     const int col = ti.n * kBN + c * 32;
-                    codes[c] = 0;
+                    codes[i] = 0;
                     if (col >= n_valid) continue;
                     uint32_t mx = 0;
 #pragma unroll
                     for (int q = 0; q < 32; ++q) mx = max(mx, __float_as_uint(fabsf(__uint_as_float(v[q]))));
                     const uint32_t code = block_scale_code(mx);
                     const float f = block_encode_factor(code);
-                    codes[c] = code;
+                    codes[i] = code;
                     uint4 pk[4];
                     __half2* h2 = reinterpret_cast<__half2*>(pk);
 #pragma unroll
@@ -482,7 +496,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (row_ok) {
                     uint8_t* dst = sc_base + grow * p.ysc_ld + ti.n * (kBN / 32);
                     const int nblk = min(kBN / 32, (n_valid - ti.n * kBN) / 32);
-                    for (int c = 0; c < nblk; ++c) dst[c] = static_cast<uint8_t>(codes[c]);
+#pragma unroll
+                    for (int i = 0; i < kBN / 64; ++i)
+                        if (c0 + i < nblk) dst[c0 + i] = static_cast<uint8_t>(codes[i]);
                 }
             } else {
                 // kWgrad: output rows m*128 + r of this expert's dW (stacked outputs split at
@@ -502,7 +518,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     origin = -split;
                 }
 #pragma unroll 1
-                for (int c = 0; c < kBN / 32; ++c) {
+                for (int c = c0; c < c0 + kBN / 64; ++c) {
                     float f[32];
                     if (ti.kb > 0) {
                         uint32_t v[32];

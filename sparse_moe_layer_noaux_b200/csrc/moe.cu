@@ -738,7 +738,7 @@ struct WorkspaceBwd {
     __nv_bfloat16* dgu_s;     // [T, 2SI]
     __nv_bfloat16* h_r;       // [Rp, I]
     __nv_bfloat16* h_s;       // [T, SI]
-    float* dw_part;           // [Rp, ceil(I/256)]
+    float* dw_part;           // [Rp, 2 ceil(I/256)]
     float* dlogit;            // [T, k]
     float* dwr_part;          // [kRouterSplit, E, H]
     __half* dxq;              // [Rp + T, H] block-scaled fp16
@@ -778,7 +778,7 @@ WorkspaceBwd carve_bwd(const moe_config* c, int64_t T, uint8_t* base) {
     w.dgu_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * 2 * SI));
     w.h_r = reinterpret_cast<__nv_bfloat16*>(take(2 * Rp * I));
     w.h_s = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
-    w.dw_part = reinterpret_cast<float*>(take(sizeof(float) * Rp * ((I + kBN - 1) / kBN)));
+    w.dw_part = reinterpret_cast<float*>(take(sizeof(float) * Rp * 2 * ((I + kBN - 1) / kBN)));
     w.dlogit = reinterpret_cast<float*>(take(sizeof(float) * T * K));
     w.dwr_part = reinterpret_cast<float*>(take(sizeof(float) * kRouterSplit * E * H));
     w.dxq = reinterpret_cast<__half*>(take(2 * (Rp + T) * H));
@@ -799,7 +799,7 @@ int launch_bwd_gemm(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtens
                     int num_sms, cudaStream_t st) {
     int64_t grid = tiles_bound < num_sms ? tiles_bound : num_sms;
     if (grid < 1) grid = 1;
-    grouped_gemm_bwd_kernel<kMode><<<static_cast<unsigned>(grid), kGemmThreads, kGemmBwdSmemBytes, st>>>(
+    grouped_gemm_bwd_kernel<kMode><<<static_cast<unsigned>(grid), kBwdThreads, kGemmBwdSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -954,7 +954,7 @@ int launch_backward(const moe_config* c, int64_t T, const float* router_w, const
     const RouterPlan rp = plan_router(static_cast<int>(T), static_cast<int>(E), static_cast<int>(H));
     bwd_router_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(
         w.router_part, rp.nsplit, static_cast<int>(T), static_cast<int>(E), static_cast<int>(K), c->norm_topk_prob,
-        c->routed_scaling_factor, w.topk_idx, w.topk_w, w.row_of, w.dw_part, nti, w.dlogit);
+        c->routed_scaling_factor, w.topk_idx, w.topk_w, w.row_of, w.dw_part, 2 * nti, w.dlogit);
     bwd_router_wgrad_kernel<<<dim3(static_cast<unsigned>(E), static_cast<unsigned>((H / 8 + 255) / 256),
                                    kRouterSplit),
                               256, 0, st>>>(w.offsets, w.totals, w.perm_src, w.dlogit, w.x_perm, static_cast<int>(H),
