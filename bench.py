@@ -39,25 +39,28 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # GEMM, from one single-pass ncu capture of `bench.py --profile-only` at the full
 # workload (the capture and its command are summarised under profiles/).  A figure is
 # reported only while the kernel sources hash to the value it was taken on.
-GEMM_SOURCES = ("grouped_gemm.cuh", "sm100_ptx.cuh")
+GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh"),
+                "mxfp8": ("grouped_gemm_mx.cuh", "mx.cuh", "grouped_gemm.cuh", "sm100_ptx.cuh")}
 MEASURED_TRAFFIC = {
-    "v3_prefill": {"sources_sha1": "e7d5607b536d216d743ee1e1d7c7295424a80916",
-                   "dram_read": 20528930560, "dram_write": 604112640},
+    ("bf16", "v3_prefill"): {"sources_sha1": "5f2c875790ce3d534905bd0ce7df0f4d932e5d7f",
+                             "dram_read": 20974602752, "dram_write": 603917312},
+    ("mxfp8", "v3_prefill"): {"sources_sha1": "fabbc337128d5267ef152f93d415734ffde82dc8",
+                              "dram_read": 9616069632, "dram_write": 345936896},
 }
 
 
-def gemm_sources_sha1():
+def gemm_sources_sha1(precision="bf16"):
     import hashlib
     h = hashlib.sha1()
-    for f in GEMM_SOURCES:
+    for f in GEMM_SOURCES[precision]:
         with open(os.path.join(ROOT, "sparse_moe_layer_noaux_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
 
-def measured_traffic(workload):
-    m = MEASURED_TRAFFIC.get(workload)
-    if m is None or m["sources_sha1"] != gemm_sources_sha1():
+def measured_traffic(workload, precision="bf16"):
+    m = MEASURED_TRAFFIC.get((precision, workload))
+    if m is None or m["sources_sha1"] != gemm_sources_sha1(precision):
         return None
     return m["dram_read"] + m["dram_write"]
 
@@ -328,7 +331,7 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
                      "bound": "tensor", "achieved": gu_flops / (gu_ms * 1e-3) / 1e12, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": gu_flops / (gu_ms * 1e-3) / 1e12 / fp8_peak,
                      "peak_source": "measured bf16 burst x 2 (nominal dense fp8/bf16 ratio)",
-                     "traffic": None, "ms_per_launch": gu_ms},
+                     "traffic": measured_traffic(shape.name, "mxfp8"), "ms_per_launch": gu_ms},
         "clocks": clk,
     }
     del st
