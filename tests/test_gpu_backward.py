@@ -11,7 +11,7 @@ import torch
 import oracle
 from oracle import backward as B
 from sparse_moe_layer_noaux_b200 import MoELayer, abi
-from sparse_moe_layer_noaux_b200.workloads import MID, TINY, V3_PREFILL, MoEShape, bf16_bits, make_inputs
+from sparse_moe_layer_noaux_b200.workloads import MID, TINY, V3_PREFILL, V3_SKEWED, MoEShape, bf16_bits, make_inputs
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -105,7 +105,8 @@ def test_backward_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
-@pytest.mark.parametrize("shape,n_rows", [(MID, 16), (V3_PREFILL, 8)], ids=lambda v: getattr(v, "name", str(v)))
+@pytest.mark.parametrize("shape,n_rows", [(MID, 16), (V3_PREFILL, 8), (V3_SKEWED, 8)],
+                         ids=lambda v: getattr(v, "name", str(v)))
 def test_backward_full_size_sampled(shape, n_rows):
     """dx of sampled rows, and the weight gradients of one sampled expert (all of its
     rows) against the oracle's expert backward on the same operands."""
@@ -118,8 +119,13 @@ def test_backward_full_size_sampled(shape, n_rows):
                                parity.device_expert_fetch(inp), parity.shared_bits(inp, shape),
                                bf16_bits(dy[torch.as_tensor(rows, device="cuda")]), routing=idx[rows])
     close(grads["x"].cpu().numpy()[rows], ref.dx, f"{shape.name} dx rows")
-    # One expert's weight gradients over all of its rows.
-    e = int(rng.choice(np.unique(idx)))
+    # One expert's weight gradients over all of its rows (for the skewed workload, where
+    # a few experts take most rows and many take none: the one closest to 1024 rows).
+    used, n_used = np.unique(idx, return_counts=True)
+    e = int(used[np.argmin(np.abs(n_used - 1024))]) if shape.name == "v3_skewed" else int(rng.choice(used))
+    if shape.name == "v3_skewed":
+        unused = sorted(set(range(shape.E)) - set(used.tolist()))
+        assert unused and all(not grads["w_down"][u].float().abs().sum().item() for u in unused[:8])
     toks, slots = np.nonzero(idx == e)
     xt = oracle.widen_bf16(bf16_bits(inp["x"]))[toks]
     rw = inp["router_w"].cpu().numpy().astype(np.float64)
@@ -144,3 +150,33 @@ def test_backward_empty_batch_gives_zero_weight_gradients():
     torch.cuda.synchronize()
     for k in ("router_w", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
         assert not grads[k].float().abs().sum().item(), k
+
+
+def test_backward_replays_from_a_cuda_graph():
+    shape = SMALL[1]
+    inp = make_inputs(shape, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dy = torch.randn((shape.T, shape.H), device="cuda", generator=g).bfloat16()
+    layer = MoELayer.from_inputs(shape, inp)
+    eager = {k: v.clone() for k, v in layer.backward(inp["x"], dy).items()}
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        out = layer.backward(inp["x"], dy)  # allocates the outputs and workspace before capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for v in out.values():
+        v.zero_()
+    cfg = layer.cfg
+    with torch.cuda.graph(graph):
+        abi.moe_backward(cfg, inp["x"], layer.router_w, layer.e_bias, layer.w_gate, layer.w_up, layer.w_down,
+                         layer.ws_gate, layer.ws_up, layer.ws_down, dy, out["x"], out["router_w"], out["w_gate"],
+                         out["w_up"], out["w_down"], out["ws_gate"], out["ws_up"], out["ws_down"], layer._ws_bwd)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    for k in eager:
+        assert torch.equal(out[k], eager[k]), k
+    del graph

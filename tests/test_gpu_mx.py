@@ -12,8 +12,8 @@ import torch
 
 import oracle
 from sparse_moe_layer_noaux_b200 import MoELayerMX, abi
-from sparse_moe_layer_noaux_b200.workloads import (MID, TINY, V3_DECODE, V3_PREFILL, MoEShape, bf16_bits,
-                                                   make_inputs)
+from sparse_moe_layer_noaux_b200.workloads import (MID, TINY, V3_DECODE, V3_PREFILL, V3_SKEWED, MoEShape,
+                                                   bf16_bits, make_inputs)
 from tests import parity
 from tests.test_oracle_mx import decode_e4m3
 
@@ -179,7 +179,8 @@ def test_small_layer_mx_every_token(shape):
     check_layer(shape, inp, y, idx, w, np.arange(shape.T))
 
 
-@pytest.mark.parametrize("shape,n_rows", [(MID, 48), (V3_DECODE, 24), (V3_PREFILL, 12)], ids=lambda v: getattr(v, "name", str(v)))
+@pytest.mark.parametrize("shape,n_rows", [(MID, 48), (V3_DECODE, 24), (V3_PREFILL, 12), (V3_SKEWED, 12)],
+                         ids=lambda v: getattr(v, "name", str(v)))
 def test_full_size_layer_mx_sampled(shape, n_rows):
     inp = make_inputs(shape, "cuda")
     y, idx, w, layer = run_forward_mx(shape, inp)
