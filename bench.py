@@ -450,24 +450,24 @@ def time_steps(step, steps, warmup, world):
     return max_over_ranks(e0.elapsed_time(e1) / steps, world), launches, clk.summary()
 
 
-def time_e2e(layer, shape, steps):
-    """The public call with host buffers: pinned x -> HBM, layer, y -> pinned host."""
+E2E_CHUNKS = 2  # chunks of the batch in the host-buffer forward (copies overlap the layer)
+
+
+def time_e2e(layer, shape, steps, chunks=E2E_CHUNKS):
+    """The public host-buffer call: pinned x on the host -> moe_forward_host (the batch
+    in `chunks` chunks, each chunk's copy in and the previous chunk's copy out
+    overlapping its computation) -> y back in pinned host memory, every step."""
     x_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(layer_inputs_host(shape))
     y_host = torch.empty(x_host.shape, dtype=torch.float32, pin_memory=True)
-    x_dev = torch.empty_like(x_host, device="cuda")
-    y_dev = torch.empty(x_host.shape, dtype=torch.float32, device="cuda")
+    chunk = (shape.T + chunks - 1) // chunks if chunks > 1 else 0
     for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, y_dev)
-        y_host.copy_(y_dev, non_blocking=True)
+        layer.forward_host(x_host, y_host, chunk)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, y_dev)
-        y_host.copy_(y_dev, non_blocking=True)
+        layer.forward_host(x_host, y_host, chunk)
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps

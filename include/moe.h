@@ -351,6 +351,27 @@ MOE_API int moe_backward(const moe_config *cfg, int64_t T, const void *x, const 
                          float *d_router_w, void *d_w_gate, void *d_w_up, void *d_w_down, void *d_ws_gate,
                          void *d_ws_up, void *d_ws_down, void *workspace, size_t workspace_bytes, void *stream);
 
+/* The forward from HOST buffers: x_host [T, H] bf16 and y_host [T, H] (y_dtype)
+ * in host memory (pinned, for the copies to run asynchronously), weights on the
+ * device.  The batch is cut into chunks of chunk_tokens rows (0 or >= T: one
+ * chunk); chunk i's input copy and chunk i-1's output copy run on two internal
+ * copy streams while chunk i is computed on `stream`, so transfers overlap the
+ * layer.  Rows are independent, so y is moe_forward's on the whole batch: bit for
+ * bit when the chunks and the batch take the same router-logit path (at least 2048
+ * rows: tensor cores; fewer: CUDA cores), else up to the fp32 summation order of
+ * the logits.  The workspace (moe_workspace_size_host) holds two staging slots each
+ * for x and y plus the forward's workspace for one chunk.  The call returns
+ * after enqueueing; y_host is complete once `stream` reaches that point.
+ * Calls from several host threads on one device are serialised. */
+MOE_API int moe_workspace_size_host(const moe_config *cfg, int64_t T, int64_t chunk_tokens, int32_t y_dtype,
+                                    size_t *bytes);
+
+MOE_API int moe_forward_host(const moe_config *cfg, int64_t T, const void *x_host, const float *router_w,
+                             const float *e_bias, const void *w_gate, const void *w_up, const void *w_down,
+                             const void *ws_gate, const void *ws_up, const void *ws_down, void *y_host,
+                             int32_t y_dtype, int64_t chunk_tokens, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

@@ -63,6 +63,22 @@ class MoELayer:
 
     __call__ = forward
 
+    def forward_host(self, x_host: torch.Tensor, y_host: Optional[torch.Tensor] = None, chunk_tokens: int = 0,
+                     stream=None, out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        """y_host = layer(x_host) for host tensors (pinned for overlap): the batch goes
+        through in chunks of chunk_tokens rows (0: one chunk) with the copies to and
+        from the GPU overlapping the layer.  Returns once the work is enqueued on
+        `stream`; synchronise it before reading y_host."""
+        T = x_host.shape[0]
+        if y_host is None:
+            y_host = torch.empty(x_host.shape, dtype=out_dtype, pin_memory=True)
+        need = abi.workspace_size_host(self.cfg, T, chunk_tokens, abi.out_dtype_code(y_host))
+        if getattr(self, "_ws_host", None) is None or self._ws_host.numel() < need:
+            self._ws_host = torch.empty(max(need, 256), dtype=torch.uint8, device=self.w_gate.device)
+        abi.moe_forward_host(self.cfg, x_host, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
+                             self.ws_gate, self.ws_up, self.ws_down, y_host, chunk_tokens, self._ws_host, stream)
+        return y_host
+
     def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
         """Gradients of sum(layer(x) * dy) (dy bf16 [T,H]), expert selection held fixed:
         dx fp32, router_w fp32, expert / shared weights bf16 (same shapes as the weights)."""

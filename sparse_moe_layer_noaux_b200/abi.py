@@ -108,13 +108,16 @@ def lib():
         L.moe_experts_down_mx.argtypes = [cfgp, i64] + [_P] * 8 + [wp] + [_P] * 3
         L.moe_combine_mx.argtypes = [cfgp, i64, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.moe_workspace_size_bwd.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
+        L.moe_workspace_size_host.argtypes = [cfgp, i64, i64, ctypes.c_int32, ctypes.POINTER(sz)]
+        L.moe_forward_host.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, i64, _P, sz, _P]
         L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
                    "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
-                   "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward"):
+                   "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward", "moe_workspace_size_host",
+                   "moe_forward_host"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -344,3 +347,22 @@ def moe_backward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up,
         _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w),
         _ptr(d_w_gate), _ptr(d_w_up), _ptr(d_w_down), _ptr(d_ws_gate), _ptr(d_ws_up), _ptr(d_ws_down),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- host buffers
+
+def workspace_size_host(cfg, T: int, chunk_tokens: int, y_dtype: int = MOE_DTYPE_F32) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_workspace_size_host", lib().moe_workspace_size_host(ctypes.byref(_cfg(cfg)), T, chunk_tokens,
+                                                                    y_dtype, ctypes.byref(n)))
+    return n.value
+
+
+def moe_forward_host(cfg, x_host, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y_host,
+                     chunk_tokens, workspace, stream=None):
+    """The forward from pinned host x [T,H] bf16 to host y [T,H] (fp32 or bf16), copies
+    overlapped with the layer chunk by chunk (include/moe.h)."""
+    _check("moe_forward_host", lib().moe_forward_host(
+        ctypes.byref(_cfg(cfg)), x_host.shape[0], _ptr(x_host), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
+        _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_host), out_dtype_code(y_host),
+        int(chunk_tokens), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

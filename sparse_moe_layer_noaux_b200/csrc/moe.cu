@@ -967,6 +967,61 @@ int launch_backward(const moe_config* c, int64_t T, const float* router_w, const
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+
+// ---------------------------------------------------------------- host buffers
+// moe_forward_host: the forward from pinned host x to host y, the batch cut into
+// chunks of rows (rows are independent, so the result is the same as one call):
+// chunk i's input copy and chunk i-1's output copy run on two internal copy
+// streams while chunk i is computed on the caller's stream.  Two staging slots
+// each for x and y in the workspace; an event per slot orders reuse.
+struct HostStreams {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t x_ready[2], computed[2], y_copied[2], start, done;
+    std::mutex mu;
+    bool ready = false;
+};
+HostStreams g_hs[64];
+
+int host_streams(HostStreams** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+    HostStreams& h = g_hs[dev];
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!h.ready) {
+        if (cudaStreamCreateWithFlags(&h.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&h.d2h, cudaStreamNonBlocking) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        cudaEvent_t* evs[] = {&h.x_ready[0], &h.x_ready[1], &h.computed[0], &h.computed[1],
+                              &h.y_copied[0], &h.y_copied[1], &h.start, &h.done};
+        for (cudaEvent_t* e : evs)
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return MOE_ERR_CUDA;
+        h.ready = true;
+    }
+    *out = &h;
+    return MOE_OK;
+}
+
+struct HostPlan {
+    int64_t chunk;       // rows per chunk
+    size_t x_slot, y_slot, fwd_bytes, bytes;
+};
+
+HostPlan plan_host(const moe_config* c, int64_t T, int64_t chunk_tokens, int y_dtype) {
+    HostPlan hp{};
+    hp.chunk = chunk_tokens > 0 && chunk_tokens < T ? chunk_tokens : T;
+    if (hp.chunk < 1) hp.chunk = 1;
+    const int64_t H = c->hidden_size;
+    hp.x_slot = align_up(static_cast<size_t>(hp.chunk * H * 2));
+    hp.y_slot = align_up(static_cast<size_t>(hp.chunk * H * (y_dtype == MOE_DTYPE_BF16 ? 2 : 4)));
+    // The last chunk may be shorter, and a short batch can split the router's
+    // hidden axis further: size for the larger of the two.
+    const int64_t last = T - ((T + hp.chunk - 1) / hp.chunk - 1) * hp.chunk;
+    const size_t a = workspace_bytes_for(c, hp.chunk), b = workspace_bytes_for(c, last > 0 ? last : hp.chunk);
+    hp.fwd_bytes = align_up(a > b ? a : b);
+    hp.bytes = 2 * hp.x_slot + 2 * hp.y_slot + hp.fwd_bytes;
+    return hp;
+}
+
 // ---------------------------------------------------------------- no-allocation dispatch
 // Scratch of moe_dispatch_noalloc: per-block expert counts, per-block bases and
 // per-expert totals (2 x ceil(T / kDispTok) x E + E int32), held in this
@@ -1409,6 +1464,72 @@ int moe_backward(const moe_config* cfg, int64_t T, const void* x, const float* r
     const BwdArgs a{x, dy, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
                     d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down};
     return launch_backward(cfg, T, router_w, e_bias, a, dx, d_router_w, w, d->num_sms, st);
+}
+
+int moe_workspace_size_host(const moe_config* cfg, int64_t T, int64_t chunk_tokens, int32_t y_dtype, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    *bytes = plan_host(cfg, T, chunk_tokens, y_dtype).bytes;
+    return MOE_OK;
+}
+
+int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const float* router_w, const float* e_bias,
+                     const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                     const void* ws_down, void* y_host, int32_t y_dtype, int64_t chunk_tokens, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !y_host || !e_bias) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({router_w, w_gate, w_up, w_down})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({ws_gate, ws_up, ws_down})) != MOE_OK) return v;
+    const HostPlan hp = plan_host(cfg, T, chunk_tokens, y_dtype);
+    if (!workspace || workspace_bytes < hp.bytes || !aligned16(workspace)) return MOE_ERR_WORKSPACE;
+    HostStreams* hs = nullptr;
+    if ((v = host_streams(&hs)) != MOE_OK) return v;
+    std::lock_guard<std::mutex> lk(hs->mu);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    uint8_t* xs[2] = {base, base + hp.x_slot};
+    uint8_t* ys[2] = {base + 2 * hp.x_slot, base + 2 * hp.x_slot + hp.y_slot};
+    void* fwd_ws = base + 2 * hp.x_slot + 2 * hp.y_slot;
+    const int64_t H = cfg->hidden_size;
+    const size_t ysz = y_dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    // The copy streams start after whatever the caller queued before this call.
+    if (cudaEventRecord(hs->start, st) != cudaSuccess || cudaStreamWaitEvent(hs->h2d, hs->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hs->d2h, hs->start, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int64_t n = (T + hp.chunk - 1) / hp.chunk;
+    for (int64_t i = 0; i < n; ++i) {
+        const int s = static_cast<int>(i & 1);
+        const int64_t r0 = i * hp.chunk, rows = (r0 + hp.chunk <= T) ? hp.chunk : T - r0;
+        // Input slot s was last read by chunk i-2's compute.
+        if (i >= 2 && cudaStreamWaitEvent(hs->h2d, hs->computed[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemcpyAsync(xs[s], static_cast<const uint8_t*>(x_host) + r0 * H * 2, rows * H * 2,
+                            cudaMemcpyHostToDevice, hs->h2d) != cudaSuccess ||
+            cudaEventRecord(hs->x_ready[s], hs->h2d) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        // Output slot s was last read by chunk i-2's copy back.
+        if (cudaStreamWaitEvent(st, hs->x_ready[s], 0) != cudaSuccess ||
+            (i >= 2 && cudaStreamWaitEvent(st, hs->y_copied[s], 0) != cudaSuccess))
+            return MOE_ERR_CUDA;
+        if ((v = moe_forward(cfg, rows, xs[s], router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, ys[s],
+                             y_dtype, nullptr, nullptr, fwd_ws, hp.fwd_bytes, stream)) != MOE_OK)
+            return v;
+        if (cudaEventRecord(hs->computed[s], st) != cudaSuccess ||
+            cudaStreamWaitEvent(hs->d2h, hs->computed[s], 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + r0 * H * ysz, ys[s], rows * H * ysz,
+                            cudaMemcpyDeviceToHost, hs->d2h) != cudaSuccess ||
+            cudaEventRecord(hs->y_copied[s], hs->d2h) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    // The caller's stream reaches the end of this call once the last output copy is done.
+    if (cudaEventRecord(hs->done, hs->d2h) != cudaSuccess || cudaStreamWaitEvent(st, hs->done, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
 }
 
 const char* moe_status_string(int status) {

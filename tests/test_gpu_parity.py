@@ -289,3 +289,33 @@ def test_forward_replays_from_a_cuda_graph():
     assert abi.device_status() == 0
     assert torch.equal(y, y_eager)
     del g
+
+
+@pytest.mark.parametrize("shape,chunk", [(SMALL[3], 128), (SMALL[3], 0), (SMALL[4], 1000), (SMALL[0], 7)],
+                         ids=["ragged-3chunks", "ragged-1chunk", "tiles-3chunks", "tiny-10chunks"])
+def test_host_buffer_forward_matches_device_forward(shape, chunk):
+    """moe_forward_host (pinned host x and y, the batch in chunks with copies overlapping
+    the layer) gives moe_forward's output: rows are independent.  Bit for bit when the
+    chunks and the whole batch take the same router-logit path (both >= 2048 rows, on
+    the tensor cores, or both fewer); across that switch the logits' fp32 summation
+    order differs, and the outputs agree to the fp16 rounding of the expert outputs."""
+    inp = make_inputs(shape, "cuda")
+    from sparse_moe_layer_noaux_b200 import MoELayer
+    layer = MoELayer.from_inputs(shape, inp)
+    y_dev = layer(inp["x"])
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = layer.forward_host(x_host, chunk_tokens=chunk)
+    y16 = layer.forward_host(x_host, chunk_tokens=chunk, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    c = chunk if 0 < chunk < shape.T else shape.T
+    last = shape.T - ((shape.T + c - 1) // c - 1) * c
+    same_path = all((n >= 2048) == (shape.T >= 2048) for n in (c, last))
+    if same_path:
+        assert torch.equal(y_host, y_dev.cpu())
+        assert torch.equal(y16, y_dev.cpu().bfloat16())
+    else:
+        # a last-bit change of a routing weight can move an expert output's block-scaled
+        # fp16 storage by one step (2^-11 of its block maximum)
+        ref = y_dev.cpu()
+        assert float((y_host - ref).abs().max()) <= 2.0 ** -9 * float(ref.abs().max())
