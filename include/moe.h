@@ -372,6 +372,27 @@ MOE_API int moe_forward_host(const moe_config *cfg, int64_t T, const void *x_hos
                              int32_t y_dtype, int64_t chunk_tokens, void *workspace, size_t workspace_bytes,
                              void *stream);
 
+/* Training pair: moe_forward_train computes the forward (same arguments as
+ * moe_forward) and keeps what the backward needs — routing, router logits, the
+ * expert-ordered rows and the experts' g = x Wg^T and u = x Wu^T (bf16) — in
+ * `context` (moe_workspace_size_bwd bytes); moe_backward_train then gives the
+ * gradients of moe_backward without recomputing routing, rows, g or u.  The
+ * context must come from moe_forward_train on the same x and weights, unchanged
+ * in between.  moe_forward_train's y is moe_forward's (h is formed from the same
+ * fp32 accumulators with the same expression): bit for bit when every expert
+ * segment has more than 112 rows; moe_forward computes smaller segments
+ * transposed, which can round differently in the last place. */
+MOE_API int moe_forward_train(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+                              const float *e_bias, const void *w_gate, const void *w_up, const void *w_down,
+                              const void *ws_gate, const void *ws_up, const void *ws_down, void *y, int32_t y_dtype,
+                              void *context, size_t context_bytes, void *stream);
+
+MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
+                               const void *w_gate, const void *w_up, const void *w_down, const void *ws_gate,
+                               const void *ws_up, const void *ws_down, const void *dy, float *dx, float *d_router_w,
+                               void *d_w_gate, void *d_w_up, void *d_w_down, void *d_ws_gate, void *d_ws_up,
+                               void *d_ws_down, void *context, size_t context_bytes, void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

@@ -79,6 +79,38 @@ class MoELayer:
                              self.ws_gate, self.ws_up, self.ws_down, y_host, chunk_tokens, self._ws_host, stream)
         return y_host
 
+    def _grads_like(self, x):
+        dev = x.device
+        g = {"x": torch.empty(x.shape, dtype=torch.float32, device=dev),
+             "router_w": torch.empty_like(self.router_w, dtype=torch.float32),
+             "w_gate": torch.empty_like(self.w_gate), "w_up": torch.empty_like(self.w_up),
+             "w_down": torch.empty_like(self.w_down)}
+        if self.shape.n_shared_experts > 0:
+            g.update(ws_gate=torch.empty_like(self.ws_gate), ws_up=torch.empty_like(self.ws_up),
+                     ws_down=torch.empty_like(self.ws_down))
+        return g
+
+    def forward_train(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None,
+                      out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        """The forward, keeping routing, rows and g / u for backward_train (on this layer)."""
+        T = x.shape[0]
+        if y is None:
+            y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+        need = abi.workspace_size_bwd(self.cfg, T)
+        if getattr(self, "_ctx", None) is None or self._ctx.numel() < need:
+            self._ctx = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+        abi.moe_forward_train(self.cfg, x, self.router_w, self.e_bias, self.w_gate, self.w_up, self.w_down,
+                              self.ws_gate, self.ws_up, self.ws_down, y, self._ctx, stream)
+        return y
+
+    def backward_train(self, x: torch.Tensor, dy: torch.Tensor, grads: Optional[dict] = None, stream=None) -> dict:
+        """Gradients as backward(), from the context of the last forward_train(x)."""
+        g = grads if grads is not None else self._grads_like(x)
+        abi.moe_backward_train(self.cfg, x, self.router_w, self.w_gate, self.w_up, self.w_down, self.ws_gate,
+                               self.ws_up, self.ws_down, dy, g["x"], g["router_w"], g["w_gate"], g["w_up"],
+                               g["w_down"], g.get("ws_gate"), g.get("ws_up"), g.get("ws_down"), self._ctx, stream)
+        return g
+
     def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
         """Gradients of sum(layer(x) * dy) (dy bf16 [T,H]), expert selection held fixed:
         dx fp32, router_w fp32, expert / shared weights bf16 (same shapes as the weights)."""

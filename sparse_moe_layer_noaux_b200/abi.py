@@ -109,6 +109,8 @@ def lib():
         L.moe_combine_mx.argtypes = [cfgp, i64, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.moe_workspace_size_bwd.argtypes = [cfgp, i64, ctypes.POINTER(sz)]
         L.moe_workspace_size_host.argtypes = [cfgp, i64, i64, ctypes.c_int32, ctypes.POINTER(sz)]
+        L.moe_forward_train.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, _P, sz, _P]
+        L.moe_backward_train.argtypes = [cfgp, i64] + [_P] * 18 + [sz, _P]
         L.moe_forward_host.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, i64, _P, sz, _P]
         L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
@@ -117,7 +119,7 @@ def lib():
                    "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
                    "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward", "moe_workspace_size_host",
-                   "moe_forward_host"):
+                   "moe_forward_host", "moe_forward_train", "moe_backward_train"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -366,3 +368,21 @@ def moe_forward_host(cfg, x_host, router_w, e_bias, w_gate, w_up, w_down, ws_gat
         ctypes.byref(_cfg(cfg)), x_host.shape[0], _ptr(x_host), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
         _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_host), out_dtype_code(y_host),
         int(chunk_tokens), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_forward_train(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, context,
+                      stream=None):
+    """The forward, keeping in `context` (workspace_size_bwd bytes) what moe_backward_train needs."""
+    _check("moe_forward_train", lib().moe_forward_train(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y), out_dtype_code(y), _ptr(context),
+        context.numel() * context.element_size(), _stream(stream)))
+
+
+def moe_backward_train(cfg, x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dy, dx, d_router_w,
+                       d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down, context, stream=None):
+    _check("moe_backward_train", lib().moe_backward_train(
+        ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w), _ptr(d_w_gate),
+        _ptr(d_w_up), _ptr(d_w_down), _ptr(d_ws_gate), _ptr(d_ws_up), _ptr(d_ws_down), _ptr(context),
+        context.numel() * context.element_size(), _stream(stream)))

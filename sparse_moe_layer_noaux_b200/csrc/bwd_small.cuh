@@ -1,7 +1,7 @@
 // The memory-bound steps of the layer's backward pass (chain rule of the
 // forward of "The Evolving Transformer · 07", § 02 / § 03, with the expert
 // selection held fixed):
-//   bwd_scatter_kernel     x and dO = w * dy of every (token, slot) into the
+//   bwd_scatter_kernel     x and / or dO = w * dy of every (token, slot) into the
 //                          expert-ordered rows (128-row aligned segments);
 //   bwd_zero_pad_kernel    the padding rows of both to zero (the weight-gradient
 //                          GEMMs sum over them);
@@ -35,8 +35,8 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const __nv_bfloat16* _
     __syncthreads();
     const int c = blockIdx.y * 256 + threadIdx.x;  // 8-element slice
     if (c >= H / 8) return;
-    const uint4 xv = reinterpret_cast<const uint4*>(x + t * H)[c];
-    const uint4 dv = reinterpret_cast<const uint4*>(dy + t * H)[c];
+    const uint4 xv = x_perm != nullptr ? reinterpret_cast<const uint4*>(x + t * H)[c] : make_uint4(0, 0, 0, 0);
+    const uint4 dv = do_perm != nullptr ? reinterpret_cast<const uint4*>(dy + t * H)[c] : make_uint4(0, 0, 0, 0);
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
     float d[8];
 #pragma unroll
@@ -47,7 +47,8 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const __nv_bfloat16* _
     }
     for (int j = 0; j < K; ++j) {
         const int64_t r = rows[j];
-        reinterpret_cast<uint4*>(x_perm + r * H)[c] = xv;
+        if (x_perm != nullptr) reinterpret_cast<uint4*>(x_perm + r * H)[c] = xv;
+        if (do_perm == nullptr) continue;
         uint4 o;
         __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll

@@ -4,7 +4,7 @@
 // differences as the "dsv3-native-reference" page's § NumPy Oracle does) needs
 // four products per expert segment, all run by one persistent kernel template:
 //   kRecompute  g = A Wg^T, u = A Wu^T (A = the segment's token rows), stored
-//               as bf16 (the forward is recomputed instead of kept);
+//               as bf16, and optionally h = silu(g) u (the training forward);
 //   kDh         dh = dO Wd (dO = w dy for routed rows, dy for shared rows), with
 //               the SwiGLU backward in the epilogue: dg = dh u silu'(g),
 //               du = dh silu(g), h = silu(g) u, and per row and half tile the
@@ -12,7 +12,10 @@
 //   kDx         dx_perm = dg Wg + du Wu (K = 2 I over the two weight maps),
 //               block-scaled fp16 like the forward's y_perm;
 //   kWgrad      dW = P^T Q for each expert over its rows (K = the segment's
-//               rows): dWd = dO^T h and [dWg; dWu] = [dg du]^T x.
+//               rows): dWd = dO^T h and [dWg; dWu] = [dg du]^T x;
+//   kFwdDown    the forward's down projection y = w (h Wd^T) on the same
+//               128-row aligned segments (the training forward, which keeps g
+//               and u for the backward), block-scaled fp16 like kDx.
 // Weights are read in their stored (out, in) layout: where the product needs
 // them transposed (kDh, kDx) the B operand is loaded MN-major (TMA boxes of 64
 // contiguous elements by 64 K rows, 128-byte swizzle) and the instruction
@@ -24,7 +27,7 @@
 
 namespace moe {
 
-enum { kRecompute = 0, kDh = 1, kDx = 2, kWgrad = 3 };
+enum { kRecompute = 0, kDh = 1, kDx = 2, kWgrad = 3, kFwdDown = 4 };
 
 struct BwdParams {
     const int32_t* offsets;      // [E+1] 128-aligned segment starts
@@ -58,6 +61,8 @@ struct BwdParams {
     uint8_t* ysc_shared;
     int64_t yq_ld, ysc_ld;
     int n_valid_routed, n_valid_shared;
+    const int32_t* perm_src;         // kFwdDown: routed row -> slot
+    const float* topk_w;             // kFwdDown: slot -> routing weight
     uint32_t idesc;
 };
 
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmB2_s,
                             const BwdParams p) {
     constexpr bool kAmn = kMode == kWgrad;                   // A loaded MN-major
-    constexpr bool kBmn = kMode != kRecompute;               // B loaded MN-major
+    constexpr bool kBmn = kMode != kRecompute && kMode != kFwdDown;   // B loaded MN-major
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -267,6 +272,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             const int b_row = b_base + ti.n * (kBN / 2);
                             ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
                             ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row);
+                        } else if (kMode == kFwdDown) {
+                            ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_base + ti.n * kBN);
                         } else {
                             // B MN-major: 4 boxes of 64 output columns x 64 K rows of the weight.
                             const bool second = kMode == kDx && kb >= i_blocks;
@@ -372,21 +379,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             };
             const int r_local = r_warp0 + lane;
             if (kMode == kRecompute) {
-                // Accumulator columns: g at 0..127, u at 128..255 for intermediate columns n*128...
+                // Accumulator columns: g at 0..127, u at 128..255 for intermediate columns
+                // n*128..; each warp takes two gate chunks and the matching up chunks, so it
+                // can also form h = silu(g) u from the fp32 values (the training forward's h,
+                // the same expression as the forward's SwiGLU epilogue).
                 __nv_bfloat16* out = ti.routed ? p.out_routed : p.out_shared;
                 const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
+                __nv_bfloat16* hout = ti.routed ? p.out2_routed : p.out2_shared;
+                const int64_t ld2 = ti.routed ? p.ld2_routed : p.ld2_shared;
                 const int ioff = ti.routed ? p.half_routed : p.half_shared;  // where u starts in a gu row
                 const int limit = ti.rows;
 #pragma unroll 1
-                for (int c = c0; c < c0 + kBN / 64; ++c) {
-                    uint32_t v[32];
-                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
+                for (int i = 0; i < 2; ++i) {
+                    const int c = 2 * half + i;
+                    uint32_t gv[32], uv[32];
+                    ptx::tmem_ld_32x32b_x32(taddr + c * 32, gv);
+                    ptx::tmem_ld_32x32b_x32(taddr + (c + 4) * 32, uv);
                     ptx::tmem_wait_ld();
+                    const int col = ti.n * (kBN / 2) + c * 32;
                     float f[32];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
-                    const int col = c < 4 ? ti.n * (kBN / 2) + c * 32 : ioff + ti.n * (kBN / 2) + (c - 4) * 32;
+                    for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(gv[q]);
                     store_rows(f, out, ld, col, limit, ti.row0);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(uv[q]);
+                    store_rows(f, out, ld, ioff + col, limit, ti.row0);
+                    if (hout != nullptr) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) {
+                            const float g = __uint_as_float(gv[q]);
+                            f[q] = g / (1.0f + __expf(-g)) * __uint_as_float(uv[q]);
+                        }
+                        store_rows(f, hout, ld2, col, limit, ti.row0);
+                    }
                 }
             } else if (kMode == kDh) {
                 // dh for 256 intermediate columns n*256..; g and u of the same columns from gu.
@@ -451,13 +476,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     store_rows(out, dgu, ld, col, limit, ti.row0);
                 }
                 if (routed && row_ok) p.dw_part[grow * (2 * p.n_tiles_routed) + 2 * ti.n + half] = dot;
-            } else if (kMode == kDx) {
+            } else if (kMode == kDx || kMode == kFwdDown) {
                 const int n_valid = ti.routed ? p.n_valid_routed : p.n_valid_shared;
                 __half* out_base = ti.routed ? p.yq_routed : p.yq_shared;
                 uint8_t* sc_base = ti.routed ? p.ysc_routed : p.ysc_shared;
                 __half* hq = reinterpret_cast<__half*>(stage);
                 const bool row_ok = r_local < ti.rows;
                 const int64_t grow = (int64_t)ti.row0 + r_local;
+                float wrow = 1.0f;
+                if (kMode == kFwdDown && ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
                 uint32_t codes[kBN / 64];
 #pragma unroll
                 for (int i = 0; i < kBN / 64; ++i) {
@@ -471,7 +498,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (col >= n_valid) continue;
                     uint32_t mx = 0;
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) mx = max(mx, __float_as_uint(fabsf(__uint_as_float(v[q]))));
+                    for (int q = 0; q < 32; ++q) mx = max(mx, __float_as_uint(fabsf(__uint_as_float(v[q]) * wrow)));
                     const uint32_t code = block_scale_code(mx);
                     const float f = block_encode_factor(code);
                     codes[i] = code;
@@ -479,7 +506,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     __half2* h2 = reinterpret_cast<__half2*>(pk);
 #pragma unroll
                     for (int q = 0; q < 16; ++q)
-                        h2[q] = __floats2half2_rn(__uint_as_float(v[2 * q]) * f, __uint_as_float(v[2 * q + 1]) * f);
+                        h2[q] = __floats2half2_rn(__uint_as_float(v[2 * q]) * wrow * f,
+                                                  __uint_as_float(v[2 * q + 1]) * wrow * f);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(hq + lane * kStagePitchH + 8 * q) = pk[q];
                     __syncwarp();

@@ -142,6 +142,8 @@ int device_info(DeviceInfo** out) {
             cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kWgrad>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_bwd_kernel<kFwdDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGemmBwdSmemBytes)) != cudaSuccess)
             return MOE_ERR_CUDA;
         d.attrs_set = true;
@@ -805,19 +807,15 @@ int launch_bwd_gemm(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtens
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int launch_backward(const moe_config* c, int64_t T, const float* router_w, const float* e_bias, const BwdArgs& a,
-                    float* dx, float* d_router_w, const WorkspaceBwd& w, int num_sms, cudaStream_t st) {
+// Route, dispatch into 128-row aligned segments, x into the expert rows (and dO =
+// w dy when dy is given), padding rows zeroed.
+int bwd_front(const moe_config* c, int64_t T, const float* router_w, const float* e_bias, const void* x,
+              const void* dy, const WorkspaceBwd& w, int num_sms, cudaStream_t st) {
     const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
-    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
-    const int has_shared = SI > 0 ? 1 : 0;
-    const int64_t Rp = w.rp;
-    const int nti = static_cast<int>((I + kBN - 1) / kBN), nts = static_cast<int>((SI + kBN - 1) / kBN);
     int v;
-    // 1. routing, recomputed (same kernels and inputs as the forward: the same selection)
-    if ((v = launch_route(c, T, a.x, router_w, e_bias, w.topk_idx, w.topk_w, w.router_part, w.router_w3, num_sms,
+    if ((v = launch_route(c, T, x, router_w, e_bias, w.topk_idx, w.topk_w, w.router_part, w.router_w3, num_sms,
                           st)) != MOE_OK)
         return v;
-    // 2. dispatch of x and w * dy into 128-row aligned segments, padding rows zeroed
     const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
     dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(w.topk_idx, static_cast<int>(T),
                                                                       static_cast<int>(K), static_cast<int>(E),
@@ -828,37 +826,73 @@ int launch_backward(const moe_config* c, int64_t T, const float* router_w, const
         w.topk_idx, static_cast<int>(T), static_cast<int>(K), static_cast<int>(E), w.block_base, w.totals,
         kMxAtomRows, w.offsets, w.perm_src, w.row_of);
     const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
-    bwd_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x),
-                                            static_cast<const __nv_bfloat16*>(a.dy), w.row_of, w.topk_w,
-                                            static_cast<int>(K), static_cast<int>(H), w.x_perm, w.do_perm);
+    bwd_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy),
+                                            w.row_of, w.topk_w, static_cast<int>(K), static_cast<int>(H), w.x_perm,
+                                            dy ? w.do_perm : nullptr);
     bwd_zero_pad_kernel<<<dim3(static_cast<unsigned>(E), 8), 256, 0, st>>>(w.offsets, w.totals, static_cast<int>(H),
-                                                                          w.x_perm, w.do_perm);
+                                                                          w.x_perm, dy ? w.do_perm : w.x_perm);
     count_launch(5);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
+// g, u of every routed and shared row (the gate/up GEMM keeping both products),
+// and h = silu(g) u as well when `with_h` (the training forward).
+int bwd_recompute(const moe_config* c, int64_t T, const BwdArgs& a, const WorkspaceBwd& w, int num_sms,
+                  cudaStream_t st, bool with_h = false) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    const int64_t Rp = w.rp;
+    CUtensorMap ar, as, br, b2r, bs, b2s;
+    bool ok = make_map(&ar, w.x_perm, Rp, H, kBM) && make_map(&br, a.w_gate, E * I, H, kBN / 2) &&
+              make_map(&b2r, a.w_up, E * I, H, kBN / 2);
+    if (has_shared)
+        ok = ok && make_map(&as, a.x, T, H, kBM) && make_map(&bs, a.ws_gate, SI, H, kBN / 2) &&
+             make_map(&b2s, a.ws_up, SI, H, kBN / 2);
+    else { as = ar; bs = br; b2s = b2r; }
+    if (!ok) return MOE_ERR_CUDA;
+    BwdParams p{};
+    p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = static_cast<int>(I / (kBN / 2)); p.n_tiles_shared = static_cast<int>(SI / (kBN / 2));
+    p.kb_routed = p.kb_shared = static_cast<int>(H / kBK);
+    p.b_rows_per_expert = static_cast<int>(I);
+    p.out_routed = w.gu_r; p.ld_routed = 2 * I; p.out_shared = w.gu_s; p.ld_shared = 2 * SI;
+    if (with_h) {
+        p.out2_routed = w.h_r; p.ld2_routed = I; p.out2_shared = w.h_s; p.ld2_shared = SI;
+    }
+    p.half_routed = static_cast<int>(I); p.half_shared = static_cast<int>(SI);
+    p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 0);
     const int64_t m_bound = Rp / kBM + (has_shared ? (T + kBM - 1) / kBM : 0);
-    // 3. g, u recomputed
-    {
-        CUtensorMap ar, as, br, b2r, bs, b2s;
-        bool ok = make_map(&ar, w.x_perm, Rp, H, kBM) && make_map(&br, a.w_gate, E * I, H, kBN / 2) &&
-                  make_map(&b2r, a.w_up, E * I, H, kBN / 2);
-        if (has_shared)
-            ok = ok && make_map(&as, a.x, T, H, kBM) && make_map(&bs, a.ws_gate, SI, H, kBN / 2) &&
-                 make_map(&b2s, a.ws_up, SI, H, kBN / 2);
-        else { as = ar; bs = br; b2s = b2r; }
-        if (!ok) return MOE_ERR_CUDA;
-        BwdParams p{};
-        p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
-        p.has_shared = has_shared;
-        p.n_tiles_routed = static_cast<int>(I / (kBN / 2)); p.n_tiles_shared = static_cast<int>(SI / (kBN / 2));
-        p.kb_routed = p.kb_shared = static_cast<int>(H / kBK);
-        p.b_rows_per_expert = static_cast<int>(I);
-        p.out_routed = w.gu_r; p.ld_routed = 2 * I; p.out_shared = w.gu_s; p.ld_shared = 2 * SI;
-        p.half_routed = static_cast<int>(I); p.half_shared = static_cast<int>(SI);
-        p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 0);
-        if ((v = launch_bwd_gemm<kRecompute>(ar, as, br, b2r, bs, b2s, p, m_bound * (I / (kBN / 2)), num_sms, st)) !=
-            MOE_OK)
-            return v;
+    return launch_bwd_gemm<kRecompute>(ar, as, br, b2r, bs, b2s, p, m_bound * (I / (kBN / 2)), num_sms, st);
+}
+
+int launch_backward(const moe_config* c, int64_t T, const float* router_w, const float* e_bias, const BwdArgs& a,
+                    float* dx, float* d_router_w, const WorkspaceBwd& w, int num_sms, cudaStream_t st,
+                    bool front_done = false) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    const int64_t Rp = w.rp;
+    const int nti = static_cast<int>((I + kBN - 1) / kBN), nts = static_cast<int>((SI + kBN - 1) / kBN);
+    int v;
+    const int64_t m_bound = Rp / kBM + (has_shared ? (T + kBM - 1) / kBM : 0);
+    const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
+    if (!front_done) {
+        // 1-3. routing and dispatch recomputed (the same kernels and inputs as the
+        // forward: the same selection), g and u recomputed
+        if ((v = bwd_front(c, T, router_w, e_bias, a.x, a.dy, w, num_sms, st)) != MOE_OK) return v;
+        if ((v = bwd_recompute(c, T, a, w, num_sms, st)) != MOE_OK) return v;
+    } else {
+        // Routing, rows and g | u kept by the training forward: only dO = w dy.
+        bwd_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x),
+                                                static_cast<const __nv_bfloat16*>(a.dy), w.row_of, w.topk_w,
+                                                static_cast<int>(K), static_cast<int>(H), nullptr, w.do_perm);
+        bwd_zero_pad_kernel<<<dim3(static_cast<unsigned>(E), 8), 256, 0, st>>>(w.offsets, w.totals,
+                                                                              static_cast<int>(H), w.do_perm,
+                                                                              w.do_perm);
+        count_launch(2);
+        if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     }
     // 4. dh = dO Wd with the SwiGLU backward
     {
@@ -967,6 +1001,43 @@ int launch_backward(const moe_config* c, int64_t T, const float* router_w, const
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+
+// The training forward: the layer's forward computed so that the backward can
+// reuse its routing, expert rows and g | u (kept in a backward workspace, the
+// "context"): route, dispatch into 128-row aligned segments, g and u (bf16) with
+// h = silu(g) u from the same fp32 accumulators, the down projection with the
+// routing weights, combine.
+int launch_forward_train(const moe_config* c, int64_t T, const float* router_w, const float* e_bias,
+                         const BwdArgs& a, void* y, int y_dtype, const WorkspaceBwd& w, int num_sms,
+                         cudaStream_t st) {
+    const int64_t H = c->hidden_size, E = c->n_routed_experts;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int has_shared = SI > 0 ? 1 : 0;
+    const int64_t Rp = w.rp;
+    int v;
+    if ((v = bwd_front(c, T, router_w, e_bias, a.x, nullptr, w, num_sms, st)) != MOE_OK) return v;
+    if ((v = bwd_recompute(c, T, a, w, num_sms, st, true)) != MOE_OK) return v;
+    CUtensorMap ar, as, br, bs;
+    bool ok = make_map(&ar, w.h_r, Rp, I, kBM) && make_map(&br, a.w_down, E * H, I, kBN);
+    if (has_shared) ok = ok && make_map(&as, w.h_s, T, SI, kBM) && make_map(&bs, a.ws_down, H, SI, kBN);
+    else { as = ar; bs = br; }
+    if (!ok) return MOE_ERR_CUDA;
+    BwdParams p{};
+    p.offsets = w.offsets; p.counts = w.totals; p.E = static_cast<int>(E); p.T = static_cast<int>(T);
+    p.has_shared = has_shared;
+    p.n_tiles_routed = p.n_tiles_shared = static_cast<int>(H / kBN);
+    p.kb_routed = static_cast<int>(I / kBK); p.kb_shared = static_cast<int>(SI / kBK);
+    p.b_rows_per_expert = static_cast<int>(H);
+    p.n_valid_routed = p.n_valid_shared = static_cast<int>(H);
+    p.yq_routed = w.dxq; p.yq_shared = w.dxq + Rp * H; p.yq_ld = H;
+    p.ysc_routed = w.dxs; p.ysc_shared = w.dxs + Rp * scale_ld(H); p.ysc_ld = scale_ld(H);
+    p.perm_src = w.perm_src; p.topk_w = w.topk_w;
+    p.idesc = idesc_bf16_f32_major(kBM, kBN, 0, 0);
+    const int64_t m_bound = Rp / kBM + (has_shared ? (T + kBM - 1) / kBM : 0);
+    if ((v = launch_bwd_gemm<kFwdDown>(ar, as, br, br, bs, bs, p, m_bound * (H / kBN), num_sms, st)) != MOE_OK)
+        return v;
+    return launch_combine(c, T, w.dxq, w.dxs, w.row_of, y, y_dtype, st, Rp);
+}
 
 // ---------------------------------------------------------------- host buffers
 // moe_forward_host: the forward from pinned host x to host y, the batch cut into
@@ -1530,6 +1601,61 @@ int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const
     if (cudaEventRecord(hs->done, hs->d2h) != cudaSuccess || cudaStreamWaitEvent(st, hs->done, 0) != cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+int moe_forward_train(const moe_config* cfg, int64_t T, const void* x, const float* router_w, const float* e_bias,
+                      const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                      const void* ws_up, const void* ws_down, void* y, int32_t y_dtype, void* context,
+                      size_t context_bytes, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!e_bias) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({x, router_w, w_gate, w_up, w_down, y})) != MOE_OK) return v;
+    if (cfg->n_shared_experts > 0 && (v = check_ptrs({ws_gate, ws_up, ws_down})) != MOE_OK) return v;
+    if (!context || context_bytes < carve_bwd(cfg, T, nullptr).bytes || !aligned16(context)) return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    const WorkspaceBwd w = carve_bwd(cfg, T, static_cast<uint8_t*>(context));
+    const BwdArgs a{x, nullptr, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                    nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    return launch_forward_train(cfg, T, router_w, e_bias, a, y, y_dtype, w, d->num_sms,
+                                static_cast<cudaStream_t>(stream));
+}
+
+int moe_backward_train(const moe_config* cfg, int64_t T, const void* x, const float* router_w,
+                       const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                       const void* ws_up, const void* ws_down, const void* dy, float* dx, float* d_router_w,
+                       void* d_w_gate, void* d_w_up, void* d_w_down, void* d_ws_gate, void* d_ws_up,
+                       void* d_ws_down, void* context, size_t context_bytes, void* stream) {
+    int v = validate_mx(cfg, T);
+    if (v != MOE_OK) return v;
+    const bool sh = cfg->n_shared_experts > 0;
+    if ((v = check_ptrs({router_w, w_gate, w_up, w_down, d_router_w, d_w_gate, d_w_up, d_w_down})) != MOE_OK) return v;
+    if (sh && (v = check_ptrs({ws_gate, ws_up, ws_down, d_ws_gate, d_ws_up, d_ws_down})) != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        const int64_t H = cfg->hidden_size, E = cfg->n_routed_experts, I = cfg->moe_intermediate_size;
+        const int64_t SI = static_cast<int64_t>(cfg->n_shared_experts) * I;
+        const size_t wb = sizeof(uint16_t) * E * I * H, sb = sizeof(uint16_t) * SI * H;
+        if (cudaMemsetAsync(d_router_w, 0, sizeof(float) * E * H, st) != cudaSuccess ||
+            cudaMemsetAsync(d_w_gate, 0, wb, st) != cudaSuccess || cudaMemsetAsync(d_w_up, 0, wb, st) != cudaSuccess ||
+            cudaMemsetAsync(d_w_down, 0, wb, st) != cudaSuccess ||
+            (sh && (cudaMemsetAsync(d_ws_gate, 0, sb, st) != cudaSuccess ||
+                    cudaMemsetAsync(d_ws_up, 0, sb, st) != cudaSuccess ||
+                    cudaMemsetAsync(d_ws_down, 0, sb, st) != cudaSuccess)))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if ((v = check_ptrs({x, dy, dx})) != MOE_OK) return v;
+    if (!context || context_bytes < carve_bwd(cfg, T, nullptr).bytes || !aligned16(context)) return MOE_ERR_WORKSPACE;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    const WorkspaceBwd w = carve_bwd(cfg, T, static_cast<uint8_t*>(context));
+    const BwdArgs a{x, dy, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                    d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down};
+    return launch_backward(cfg, T, router_w, nullptr, a, dx, d_router_w, w, d->num_sms, st, true);
 }
 
 const char* moe_status_string(int status) {

@@ -180,3 +180,40 @@ def test_backward_replays_from_a_cuda_graph():
     for k in eager:
         assert torch.equal(out[k], eager[k]), k
     del graph
+
+
+@pytest.mark.parametrize("shape", [SMALL[0], SMALL[1], SMALL[2], SMALL[3]], ids=lambda s: s.name)
+def test_training_pair(shape):
+    """moe_forward_train gives moe_forward's output — bit for bit when every expert
+    segment has more than 112 rows (moe_forward computes smaller segments transposed),
+    else to within fp16 rounding of the expert outputs — and the oracle's at the
+    forward's tolerances; moe_backward_train, from its context, gives exactly
+    moe_backward's gradients."""
+    inp = make_inputs(shape, "cuda")
+    layer = MoELayer.from_inputs(shape, inp)
+    g = torch.Generator(device="cuda").manual_seed(1000)
+    dy = torch.randn((shape.T, shape.H), device="cuda", generator=g).bfloat16()
+    y = layer.forward_train(inp["x"])
+    y_fwd = layer(inp["x"])
+    grads_t = layer.backward_train(inp["x"], dy)
+    grads = layer.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    for k in grads:
+        assert torch.equal(grads_t[k], grads[k]), k
+    x_bits = bf16_bits(inp["x"])
+    rw, bias = inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()
+    ref_idx, ref_w, margin, scores = parity.oracle_route_all(shape, x_bits, rw, bias)
+    cfg = abi.MoEConfig.from_shape(shape)
+    ws = torch.empty(max(abi.workspace_size(cfg, shape.T), 256), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    abi.moe_route(cfg, inp["x"], inp["router_w"], inp["e_bias"], idx, w, ws)
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=shape.E)
+    if counts[counts > 0].min() > 112:
+        assert torch.equal(y, y_fwd)
+    else:
+        assert float((y - y_fwd).abs().max()) <= 2.0 ** -9 * float(y_fwd.abs().max())
+    y_ref = parity.oracle_layer_rows(shape, inp, np.arange(shape.T), idx.cpu().numpy(), scores, ref_idx, ref_w,
+                                     margin)
+    parity.assert_output_close(y.cpu().numpy(), y_ref, f"{shape.name} forward_train")
