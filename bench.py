@@ -354,6 +354,15 @@ def time_backward(shape, steps, warmup, world, rank, peaks, inp):
                          grads["w_gate"], grads["w_up"], grads["w_down"], grads.get("ws_gate"), grads.get("ws_up"),
                          grads.get("ws_down"), ws)
     ms, launches, clk = time_steps(step, steps, warmup, world)
+
+    # Training step: moe_forward_train (keeps routing, rows, g | u) + moe_backward_train.
+    y = torch.empty(inp["x"].shape, dtype=torch.float32, device="cuda")
+    layer.forward_train(inp["x"], y)
+
+    def train_step():
+        layer.forward_train(inp["x"], y)
+        layer.backward_train(inp["x"], dy, grads)
+    train_ms, train_launches, train_clk = time_steps(train_step, steps, warmup, world)
     # recompute g,u (4), dh (2), dx (4), dWd (2), dWg + dWu (4): 16 H I per (token, expert) pair
     flops = 16.0 * shape.H * shape.I * shape.T * (shape.k + shape.S) + 4.0 * shape.T * shape.E * shape.H
     # weights read (gate/up twice, down twice), weight gradients written (bf16)
@@ -365,7 +374,13 @@ def time_backward(shape, steps, warmup, world, rank, peaks, inp):
            "tflops": flops / (ms * 1e-3) / 1e12 * world, "flops": flops, "gpu_launches": launches,
            "layer_roofline": {"bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= bytes_ / (peaks["hbm_gbs"] * 1e9)
                               else "hbm", "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms},
-           "clocks": clk}
+           "clocks": clk,
+           "training_step": {"ms_per_step": train_ms, "tokens_per_s": job_throughput(shape.T, world, train_ms),
+                             "what": "moe_forward_train + moe_backward_train (g, u kept, not recomputed)",
+                             "tflops": (6.0 * shape.H * shape.I * shape.T * (shape.k + shape.S) + flops
+                                        - 4.0 * shape.H * shape.I * shape.T * (shape.k + shape.S))
+                             / (train_ms * 1e-3) / 1e12 * world,
+                             "gpu_launches": train_launches, "clocks": train_clk}}
     del grads, layer
     return out
 
