@@ -54,7 +54,9 @@ int validate_cfg(const moe_config* c, int64_t T) {
     if (SI > (1 << 24) || static_cast<int64_t>(E) * I > (1ll << 31) ||
         static_cast<int64_t>(E) * H > (1ll << 31))
         return MOE_ERR_UNSUPPORTED;
-    if (T * K + T >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+    // Every row index (routed rows with up to 127 padding rows per expert
+    // segment, then the shared rows) must fit an int32 and a TMA coordinate.
+    if (T * K + T + 128ll * E >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 

@@ -143,3 +143,18 @@ def test_mx_host_queries(lib):
     # Quantising nothing is a no-op; a K that is not a multiple of 128 is refused.
     assert lib.moe_mx_quantize(0, 256, None, None, None, None) == abi.MOE_OK
     assert lib.moe_mx_quantize(4, 96, None, None, None, None) == abi.MOE_ERR_UNSUPPORTED
+
+
+def test_row_space_beyond_int32_rejected(lib):
+    # Row indices are int32: the routed rows, their per-expert padding to 128
+    # and the shared rows must all fit.  A batch whose unpadded rows fit but
+    # whose padded ones do not is refused before any size is computed.
+    c = abi.MoEConfig.from_shape(V3_PREFILL)
+    n = ctypes.c_size_t(0)
+    k, E = V3_PREFILL.k, V3_PREFILL.E
+    limit = (1 << 31) - 256
+    T_pad_overflow = (limit - 128 * E) // (k + 1) + 1
+    assert T_pad_overflow * (k + 1) < limit
+    assert lib.moe_workspace_size(ctypes.byref(c), T_pad_overflow, ctypes.byref(n)) == abi.MOE_ERR_UNSUPPORTED
+    T_fits = (limit - 128 * E) // (k + 1) - 1
+    assert lib.moe_workspace_size(ctypes.byref(c), T_fits, ctypes.byref(n)) == abi.MOE_OK
