@@ -92,6 +92,43 @@ def assert_output_close(y, y_ref, what=""):
     return e
 
 
+# Gradients (backward pass): every element is an fp32 sum of products of three
+# bf16-rounded factors (dO = w dy, g / u or h, x or the weights), each rounded
+# once to bf16 (2^-9 relative), so an element can be off by ~3 * 2^-9 of its own
+# size and, with few rows per expert, that does not average out.  Bar:
+# max |err| <= 2e-2 * max |ref| (per tensor) and relative L1 <= 1e-2.
+GRAD_MAX_ABS_REL_MAX = 2e-2
+GRAD_REL_L1 = 1e-2
+
+
+def assert_gradient_close(got, ref, what=""):
+    e = output_errors(np.asarray(got, np.float64), ref)
+    e["max_abs_over_max"] = e["max_abs"] / max(float(np.abs(ref).max()), 1e-300)
+    assert e["max_abs_over_max"] <= GRAD_MAX_ABS_REL_MAX and e["rel_l1"] <= GRAD_REL_L1, (what, e)
+    return e
+
+
+def compare_gradients(shape, grads, ref, tag=""):
+    """Every gradient of the layer (dict from MoELayer.backward) against the
+    float64 backward oracle's Grads; experts no token chose must get zero."""
+    out = {"dx": assert_gradient_close(grads["x"].cpu().numpy(), ref.dx, f"{tag} dx"),
+           "router_w": assert_gradient_close(grads["router_w"].cpu().numpy(), ref.d_router_w,
+                                             f"{tag} d_router_w")}
+    for j, name in enumerate(("w_gate", "w_up", "w_down")):
+        got = grads[name].float().cpu().numpy()
+        want = np.zeros_like(got, dtype=np.float64)
+        for e, gr in ref.d_experts.items():
+            want[e] = gr[j]
+        out[name] = assert_gradient_close(got, want, f"{tag} d_{name}")
+        unused = sorted(set(range(shape.E)) - set(ref.d_experts))
+        assert all((got[e] == 0).all() for e in unused), (tag, name, "unused experts")
+    if shape.S > 0:
+        for j, name in enumerate(("ws_gate", "ws_up", "ws_down")):
+            out[name] = assert_gradient_close(grads[name].float().cpu().numpy(), ref.d_shared[j],
+                                              f"{tag} d_{name}")
+    return out
+
+
 def assert_bf16_rounded(t, ref, what=""):
     """A bf16-stored intermediate: within one bf16 rounding (2^-8 relative) of the
     float64 reference, plus a small fp32-accumulation allowance."""

@@ -16,13 +16,8 @@ from tests import parity
 
 pytestmark = pytest.mark.gpu
 
-# Tolerance, from the arithmetic: every gradient element is an fp32 sum of products
-# of three bf16-rounded factors (dO = w dy, g / u or h, x or the weights), each
-# rounded once to bf16 (2^-9 relative), so an element can be off by ~3 * 2^-9 of
-# its own size and, with few rows per expert, that does not average out.  Bar:
-# max |err| <= 2e-2 * max |ref| (per tensor) and relative L1 <= 1e-2.
-MAX_ABS_REL_MAX = 2e-2
-REL_L1 = 1e-2
+# Tolerance (derived beside parity.assert_gradient_close): max |err| <= 2e-2 *
+# max |ref| per tensor and relative L1 <= 1e-2.
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -37,10 +32,8 @@ def _gpu():
 
 
 def close(got, ref, what):
-    e = parity.output_errors(np.asarray(got, np.float64), ref)
-    e["max_abs_over_max"] = e["max_abs"] / max(float(np.abs(ref).max()), 1e-300)
+    e = parity.assert_gradient_close(got, ref, what)
     print(what, e)
-    assert e["max_abs_over_max"] <= MAX_ABS_REL_MAX and e["rel_l1"] <= REL_L1, (what, e)
     return e
 
 
@@ -81,19 +74,7 @@ def test_backward_small_every_gradient(shape):
     shared = parity.shared_bits(inp, shape)
     ref = B.moe_layer_backward(shape, bf16_bits(inp["x"]), inp["router_w"].cpu().numpy(),
                                inp["e_bias"].cpu().numpy(), fetch, shared, bf16_bits(dy), routing=idx)
-    close(grads["x"].cpu().numpy(), ref.dx, f"{shape.name} dx")
-    close(grads["router_w"].cpu().numpy(), ref.d_router_w, f"{shape.name} d_router_w")
-    for j, name in enumerate(("w_gate", "w_up", "w_down")):
-        got = grads[name].float().cpu().numpy()
-        want = np.zeros_like(got, dtype=np.float64)
-        for e, gr in ref.d_experts.items():
-            want[e] = gr[j]
-        close(got, want, f"{shape.name} d_{name}")
-        unused = sorted(set(range(shape.E)) - set(ref.d_experts))
-        assert all((got[e] == 0).all() for e in unused)
-    if shape.S > 0:
-        for j, name in enumerate(("ws_gate", "ws_up", "ws_down")):
-            close(grads[name].float().cpu().numpy(), ref.d_shared[j], f"{shape.name} d_{name}")
+    print(parity.compare_gradients(shape, grads, ref, shape.name))
 
 
 def test_backward_deterministic():
