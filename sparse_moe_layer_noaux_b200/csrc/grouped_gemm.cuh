@@ -12,8 +12,10 @@
 //            magnitude): fp16's 11-bit precision relative to the block maximum, no
 //            overflow, half the bytes of fp32;
 //   kLogits  router logits l = x Wr^T in fp32 from an exact three-way bf16 split
-//            Wr = hi + mid + lo (one segment of T rows, K = 3 H concatenated over the
-//            three planes, N = E rounded up to 16), fp32 output.
+//            Wr = hi + mid + lo (one segment of T rows, K = 3 H: each 64-column
+//            block of x meets the three planes back to back, so its second and
+//            third loads come from L2 and x streams from HBM once; N = E rounded
+//            up to 16), fp32 output.
 // ("The Evolving Transformer · 07", § 02: expert(x[mask]) is a SwiGLU FFN; its
 // output is multiplied by the routing weight.)
 //
@@ -81,7 +83,6 @@ struct GemmParams {
     const float* topk_w;                  // kDown: slot -> routing weight
     uint32_t idesc;                       // MMA instruction descriptor (M = 128, N)
     uint32_t b_tile_bytes;                // bytes one B tile load brings in
-    int kb_plane;                         // kLogits: K blocks per plane (H / 64)
     int b_plane_rows;                     // kLogits: rows of one plane in the B map (E)
     int allow_swap;                       // compute partial row tiles transposed
 };
@@ -312,9 +313,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t a_dst = ptx::smem_u32(smemA + stage * kTileABytes);
                     const uint32_t b_dst = ptx::smem_u32(smemB + stage * kTileBBytes);
                     if (kEpi == kLogits) {
-                        // K runs over the three planes of Wr back to back; x is re-read per plane.
-                        const int plane = kb / p.kb_plane;
-                        const int kcol = (kb - plane * p.kb_plane) * kBK;
+                        // K block kb = 3 * (x column block) + plane: the same x tile is
+                        // loaded for the three planes in a row (L2 hits after the first).
+                        const int plane = kb % 3;
+                        const int kcol = (kb / 3) * kBK;
                         ptx::tma_load_2d(a_dst, mA, full, kcol, a_row, pol_a);
                         ptx::tma_load_2d(b_dst, mB, full, kcol, plane * p.b_plane_rows);
                     } else if (kEpi == kSwiGLU) {

@@ -265,7 +265,6 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
         p.ld_shared = E;
         p.idesc = ptx::idesc_bf16_f32(kBM, npad);
         p.b_tile_bytes = static_cast<uint32_t>(npad) * kBK * 2;
-        p.kb_plane = H / kBK;
         p.b_plane_rows = E;
         int64_t grid = (T + kBM - 1) / kBM;
         if (grid > num_sms) grid = num_sms;
