@@ -42,10 +42,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh"),
                 "mxfp8": ("grouped_gemm_mx.cuh", "mx.cuh", "grouped_gemm.cuh", "sm100_ptx.cuh")}
 MEASURED_TRAFFIC = {
-    ("bf16", "v3_prefill"): {"sources_sha1": "5f2c875790ce3d534905bd0ce7df0f4d932e5d7f",
-                             "dram_read": 20974602752, "dram_write": 603917312},
-    ("mxfp8", "v3_prefill"): {"sources_sha1": "fabbc337128d5267ef152f93d415734ffde82dc8",
-                              "dram_read": 9616069632, "dram_write": 345936896},
+    ("bf16", "v3_prefill"): {"sources_sha1": "4610e681b1a9cc385e096efd6138d0e0a863a661",
+                             "dram_read": 20471961088, "dram_write": 600841984},
+    ("mxfp8", "v3_prefill"): {"sources_sha1": "afe2547cabcad37df852530993b0e83f7373f66d",
+                              "dram_read": 9408662784, "dram_write": 341510400},
 }
 
 
