@@ -150,11 +150,13 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
     const int E = a.E, gsize = E / a.G;
 
     float s[EPL], cand[EPL];
+    int grp[EPL];  // group of this lane's expert in slot i (-1: no expert)
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
         s[i] = 0.f;
         cand[i] = -CUDART_INF_F;
+        grp[i] = e < E ? e / gsize : -1;
         if (e < E) {
             float l = 0.f;
             for (int p = 0; p < a.nsplit; ++p) l += a.part[((int64_t)p * a.T + t) * E + e];
@@ -169,8 +171,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         float m1 = -CUDART_INF_F, m2 = -CUDART_INF_F;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && e / gsize == g) {
+            if (grp[i] == g) {
                 const float v = cand[i];
                 if (v > m1) { m2 = m1; m1 = v; }
                 else if (v > m2) { m2 = v; }
@@ -199,10 +200,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
 
     // Experts of dropped groups are excluded from the top-k.
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e >= E || !((kept >> (e / gsize)) & 1u)) cand[i] = -CUDART_INF_F;
-    }
+    for (int i = 0; i < EPL; ++i)
+        if (grp[i] < 0 || !((kept >> grp[i]) & 1u)) cand[i] = -CUDART_INF_F;
 
     float my_s = 0.f;
     int my_idx = 0;
