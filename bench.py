@@ -522,7 +522,8 @@ def oracle_sample(shape, inp, n_tokens, seed):
 
 def oracle_tokens_per_step(shape):
     per_token_macs = shape.E * shape.H + 3 * shape.H * shape.I * (shape.k + shape.S)
-    return max(1, int(4e8 // per_token_macs))  # about half a second of float64 work
+    # About half a second of float64 work, never more rows than the batch has.
+    return max(1, min(shape.T, int(4e8 // per_token_macs)))
 
 
 def cpu_baseline(shape, inp, budget_tokens=None):
@@ -535,6 +536,8 @@ def cpu_baseline(shape, inp, budget_tokens=None):
 
 
 def run_reference(args, shape, world, rank):
+    """The oracle arm: the float64 oracle as it stands, timed on this host's cores on
+    a bounded token sample per step (rank 0 only)."""
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
@@ -590,6 +593,16 @@ def main():
                     help="run warmup + steps layer passes and exit without timing (for profilers)")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
+    if args.impl == "reference" and not args.profile_only:
+        # The oracle arm runs on rank 0 alone and needs no collective: no process
+        # group is formed, so the other ranks exit at once without waiting for it.
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        if torch.cuda.is_available():
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        args.warmup = max(args.warmup, 3)
+        run_reference(args, shape, int(os.environ.get("WORLD_SIZE", "1")), 0)
+        return
     world, rank, local = dist_setup(args.gpus)
     if args.profile_only:
         inp0 = rank_inputs(shape, rank, "cuda")
@@ -612,11 +625,6 @@ def main():
         finish(world)
         return
     args.warmup = max(args.warmup, 3)
-
-    if args.impl == "reference":
-        run_reference(args, shape, world, rank)
-        finish(world)
-        return
 
     peaks, peak_src = load_peaks()
     res = time_gpu(shape, args.steps, args.warmup, world, rank, peaks)

@@ -45,3 +45,30 @@ def test_two_ranks_replicas():
     assert g0[2] != g1[2]                          # different tokens
     assert ms == 11.0 and res[1][2] == 11.0        # max over ranks, seen by all
     assert abs(thr - 2 * TINY.T / 11e-3) < 1e-6    # all ranks' tokens / slowest time
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank0():
+    """`bench.py --impl reference` under torchrun: rank 0 alone times the oracle and
+    prints one JSON line; the other rank exits 0 at once (no process group, so no
+    barrier that could time out while rank 0 works)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--workload", "tiny", "--steps", "1", "--warmup", "3"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run(cmd, cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
