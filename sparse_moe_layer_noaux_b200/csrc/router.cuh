@@ -149,6 +149,23 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
     if (t >= a.T) return;
     const int E = a.E, gsize = E / a.G;
 
+    // Logits: the split partials summed in split order.  The lane's EPL experts
+    // are loaded side by side for each split (independent loads in flight, same
+    // addition order per logit as a split-by-split sum).
+    float l[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) l[i] = 0.f;
+    const float* pt = a.part + (int64_t)t * E;
+    const int64_t split_stride = (int64_t)a.T * E;
+#pragma unroll 4
+    for (int p = 0; p < a.nsplit; ++p) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) l[i] += pt[p * split_stride + e];
+        }
+    }
+
     float s[EPL], cand[EPL];
     int grp[EPL];  // group of this lane's expert in slot i (-1: no expert)
 #pragma unroll
@@ -158,9 +175,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         cand[i] = -CUDART_INF_F;
         grp[i] = e < E ? e / gsize : -1;
         if (e < E) {
-            float l = 0.f;
-            for (int p = 0; p < a.nsplit; ++p) l += a.part[((int64_t)p * a.T + t) * E + e];
-            s[i] = 1.0f / (1.0f + expf(-l));
+            s[i] = 1.0f / (1.0f + expf(-l[i]));
             cand[i] = s[i] + a.bias[e];  // biased score b_e
         }
     }
