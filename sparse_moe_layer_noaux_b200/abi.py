@@ -148,6 +148,80 @@ def _cfg(cfg):
     return cfg if isinstance(cfg, MoEConfig) else MoEConfig.from_shape(cfg)
 
 
+# ---------------------------------------------------------------- argument checks
+# The C ABI takes raw pointers and cannot see buffer sizes, so every wrapper checks
+# each tensor before its address is passed on: element type, dense (contiguous)
+# layout, the current CUDA device (pinned host memory for the host-buffer entry
+# point) and at least as many elements as the call reads or writes.  A violation
+# raises TypeError / ValueError before anything is launched.
+
+_BF16, _F16, _F32, _I32, _U8 = torch.bfloat16, torch.float16, torch.float32, torch.int32, torch.uint8
+_OUT = (torch.float32, torch.bfloat16)
+
+
+class _Dims:
+    def __init__(self, cfg, T: int):
+        c = _cfg(cfg)
+        self.T, self.H, self.E = int(T), int(c.hidden_size), int(c.n_routed_experts)
+        self.k, self.I, self.S = int(c.num_experts_per_tok), int(c.moe_intermediate_size), int(c.n_shared_experts)
+        self.SI = self.S * self.I
+        self.scale_cols = y_perm_scale_cols(self.H)
+
+
+def _on_current_cuda_device(t: torch.Tensor) -> bool:
+    return t.device.type == "cuda" and t.device.index == torch.cuda.current_device()
+
+
+def _req(name: str, t, dtype, numel: int, where: str = "cuda", optional: bool = False):
+    """Check one tensor argument (see above); `numel` is the minimum element count."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name}: a tensor is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    allowed = dtype if isinstance(dtype, tuple) else (dtype,)
+    if t.dtype not in allowed:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in allowed)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if where == "cuda":
+        if not _on_current_cuda_device(t):
+            raise ValueError(f"{name}: must be on the current CUDA device, is on {t.device}")
+    elif t.device.type != "cpu":
+        raise ValueError(f"{name}: must be a host (CPU) tensor, is on {t.device}")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs at least {numel}")
+
+
+def _rows_2d(name: str, x, H: int) -> int:
+    """Rows T of a [T, H] argument."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2 or x.shape[1] != H:
+        shape = tuple(x.shape) if isinstance(x, torch.Tensor) else type(x).__name__
+        raise ValueError(f"{name}: expected shape [T, {H}], got {shape}")
+    return int(x.shape[0])
+
+
+def _req_weights(d: _Dims, w_gate=None, w_up=None, w_down=None, ws_gate=None, ws_up=None, ws_down=None,
+                 prefix: str = "", need=("gate", "up", "down")):
+    """Routed expert weights [E, I, H] / [E, H, I] and, when S > 0, the shared ones."""
+    EIH, SIH = d.E * d.I * d.H, d.SI * d.H
+    if "gate" in need:
+        _req(prefix + "w_gate", w_gate, _BF16, EIH)
+        _req(prefix + "ws_gate", ws_gate, _BF16, SIH, optional=d.S == 0)
+    if "up" in need:
+        _req(prefix + "w_up", w_up, _BF16, EIH)
+        _req(prefix + "ws_up", ws_up, _BF16, SIH, optional=d.S == 0)
+    if "down" in need:
+        _req(prefix + "w_down", w_down, _BF16, EIH)
+        _req(prefix + "ws_down", ws_down, _BF16, SIH, optional=d.S == 0)
+
+
+def _n(d: _Dims, count: int) -> int:
+    """A minimum size that only applies to a non-empty batch (T = 0 is a no-op)."""
+    return count if d.T > 0 else 0
+
+
 def workspace_size(cfg, T: int) -> int:
     n = ctypes.c_size_t(0)
     _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(_cfg(cfg)), T, ctypes.byref(n)))
@@ -155,12 +229,32 @@ def workspace_size(cfg, T: int) -> int:
 
 
 def moe_route(cfg, x, router_w, e_bias, topk_idx, topk_w, workspace, stream=None):
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _req("x", x, _BF16, 0)
+    _req("router_w", router_w, _F32, d.E * d.H)
+    _req("e_bias", e_bias, _F32, d.E)
+    _req("topk_idx", topk_idx, _I32, d.T * d.k)
+    _req("topk_w", topk_w, _F32, d.T * d.k)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_route", lib().moe_route(ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w),
                                         _ptr(e_bias), _ptr(topk_idx), _ptr(topk_w), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def _req_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of) -> _Dims:
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _req("x", x, _BF16, 0)
+    _req("topk_idx", topk_idx, _I32, d.T * d.k)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req("x_perm", x_perm, _BF16, d.T * d.k * d.H)
+    _req("perm_src", perm_src, _I32, d.T * d.k)
+    _req("row_of", row_of, _I32, d.T * d.k)
+    return d
+
+
 def moe_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, workspace, stream=None):
+    _req_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_dispatch", lib().moe_dispatch(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
         _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _ptr(workspace),
@@ -170,6 +264,7 @@ def moe_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, wor
 def moe_dispatch_noalloc(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, stream=None):
     """moe_dispatch without a workspace: its scratch is a fixed 1 MiB array inside
     the library (see include/moe.h for the size limit and the sharing rules)."""
+    _req_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of)
     _check("moe_dispatch_noalloc", lib().moe_dispatch_noalloc(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
         _ptr(x_perm), _ptr(perm_src), _ptr(row_of), _stream(stream)))
@@ -190,6 +285,9 @@ def decode_y_perm(y_perm: torch.Tensor, y_perm_scale: torch.Tensor) -> torch.Ten
 
 def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_up, w_down,
                 ws_gate, ws_up, ws_down, h_routed, h_shared, y_perm, y_perm_scale, stream=None):
+    d = _Dims(cfg, T)
+    _req_gate_up(d, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared)
+    _req_down(d, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm, y_perm_scale)
     _check("moe_experts", lib().moe_experts(
         ctypes.byref(_cfg(cfg)), T, _ptr(x), _ptr(x_perm), _ptr(expert_offsets), _ptr(perm_src),
         _ptr(topk_w), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up),
@@ -197,8 +295,32 @@ def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_u
         _stream(stream)))
 
 
+def _req_gate_up(d, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared):
+    shared = d.S > 0
+    _req("x", x, _BF16, d.T * d.H if shared else 0, optional=not shared)
+    _req("x_perm", x_perm, _BF16, d.T * d.k * d.H)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req_weights(d, w_gate=w_gate, w_up=w_up, ws_gate=ws_gate, ws_up=ws_up, need=("gate", "up"))
+    _req("h_routed", h_routed, _BF16, d.T * d.k * d.I)
+    _req("h_shared", h_shared, _BF16, d.T * d.SI, optional=not shared)
+
+
+def _req_down(d, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm, y_perm_scale):
+    shared = d.S > 0
+    rows = d.T * d.k + (d.T if shared else 0)
+    _req("h_routed", h_routed, _BF16, d.T * d.k * d.I)
+    _req("h_shared", h_shared, _BF16, d.T * d.SI, optional=not shared)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req("perm_src", perm_src, _I32, d.T * d.k)
+    _req("topk_w", topk_w, _F32, d.T * d.k)
+    _req_weights(d, w_down=w_down, ws_down=ws_down, need=("down",))
+    _req("y_perm", y_perm, _F16, rows * d.H)
+    _req("y_perm_scale", y_perm_scale, _U8, rows * d.scale_cols)
+
+
 def moe_experts_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed,
                         h_shared, stream=None):
+    _req_gate_up(_Dims(cfg, T), x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared)
     _check("moe_experts_gate_up", lib().moe_experts_gate_up(
         ctypes.byref(_cfg(cfg)), T, _ptr(x), _ptr(x_perm), _ptr(expert_offsets), _ptr(w_gate),
         _ptr(w_up), _ptr(ws_gate), _ptr(ws_up), _ptr(h_routed), _ptr(h_shared), _stream(stream)))
@@ -206,19 +328,45 @@ def moe_experts_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate
 
 def moe_experts_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down,
                      y_perm, y_perm_scale, stream=None):
+    _req_down(_Dims(cfg, T), h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
+              y_perm_scale)
     _check("moe_experts_down", lib().moe_experts_down(
         ctypes.byref(_cfg(cfg)), T, _ptr(h_routed), _ptr(h_shared), _ptr(expert_offsets),
         _ptr(perm_src), _ptr(topk_w), _ptr(w_down), _ptr(ws_down), _ptr(y_perm), _ptr(y_perm_scale),
         _stream(stream)))
 
 
+def _req_combine(d, routed_rows, y_perm, y_perm_scale, row_of, y):
+    rows = routed_rows + (d.T if d.S > 0 else 0)
+    _req("y_perm", y_perm, _F16, rows * d.H)
+    _req("y_perm_scale", y_perm_scale, _U8, rows * d.scale_cols)
+    _req("row_of", row_of, _I32, d.T * d.k)
+    _req("y", y, _OUT, d.T * d.H)
+
+
 def moe_combine(cfg, T, y_perm, y_perm_scale, row_of, y, stream=None):
+    d = _Dims(cfg, T)
+    _req_combine(d, d.T * d.k, y_perm, y_perm_scale, row_of, y)
     _check("moe_combine", lib().moe_combine(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(y_perm_scale),
                                             _ptr(row_of), _ptr(y), out_dtype_code(y), _stream(stream)))
 
 
+def _req_layer(cfg, x, router_w, e_bias, y, topk_idx_out, topk_w_out, x_where="cuda") -> _Dims:
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _req("x", x, _BF16, 0, where=x_where)
+    _req("router_w", router_w, _F32, d.E * d.H)
+    _req("e_bias", e_bias, _F32, d.E)
+    _req("y", y, _OUT, d.T * d.H, where=x_where)
+    _req("topk_idx_out", topk_idx_out, _I32, d.T * d.k, optional=True)
+    _req("topk_w_out", topk_w_out, _F32, d.T * d.k, optional=True)
+    return d
+
+
 def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y,
                 topk_idx_out=None, topk_w_out=None, workspace=None, stream=None):
+    d = _req_layer(cfg, x, router_w, e_bias, y, topk_idx_out, topk_w_out)
+    _req_weights(d, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+    _req("workspace", workspace, _U8, 0, optional=True)
     _check("moe_forward", lib().moe_forward(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
         _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y),
@@ -246,6 +394,12 @@ def selftest_wait_timeout(limit_ns: int, stream=None):
 def moe_bias_update(cfg, topk_idx, e_bias, gamma: float, expert_load=None, stream=None):
     """Aux-loss-free balancing step: e_bias -= gamma where the expert was overloaded,
     += gamma where underloaded (in place); expert_load [E] int32 optionally receives the loads."""
+    c = _cfg(cfg)
+    if not isinstance(topk_idx, torch.Tensor) or topk_idx.dim() != 2 or topk_idx.shape[1] != c.num_experts_per_tok:
+        raise ValueError(f"topk_idx: expected shape [T, {c.num_experts_per_tok}]")
+    _req("topk_idx", topk_idx, _I32, 0)
+    _req("e_bias", e_bias, _F32, c.n_routed_experts)
+    _req("expert_load", expert_load, _I32, c.n_routed_experts, optional=True)
     _check("moe_bias_update", lib().moe_bias_update(ctypes.byref(_cfg(cfg)), topk_idx.shape[0],
                                                     _ptr(topk_idx), _ptr(e_bias), float(gamma),
                                                     _ptr(expert_load), _stream(stream)))
@@ -262,7 +416,12 @@ def mx_scale_bytes(rows: int, K: int) -> int:
 
 def moe_mx_quantize(src: torch.Tensor, q: torch.Tensor, sf: torch.Tensor, stream=None):
     """E4M3 bytes q [rows, K] and scale atoms sf of the bf16 matrix src [rows, K]."""
+    if not isinstance(src, torch.Tensor) or src.dim() != 2:
+        raise ValueError("src: expected a 2-D [rows, K] tensor")
     rows, K = src.shape
+    _req("src", src, _BF16, 0)
+    _req("q", q, _U8, rows * K)
+    _req("sf", sf, _U8, mx_scale_bytes(rows, K) if K % 128 == 0 and rows > 0 else 0)
     _check("moe_mx_quantize", lib().moe_mx_quantize(rows, K, _ptr(src), _ptr(q), _ptr(sf), _stream(stream)))
 
 
@@ -287,8 +446,29 @@ def mx_routed_rows(cfg, T: int) -> int:
     return n.value
 
 
+def _mx_rows(d: _Dims, cfg):
+    """(Rp, Tp): padded routed rows and the shared rows rounded up to 128 (0, 0 if T = 0)."""
+    if d.T == 0:
+        return 0, 0
+    return mx_routed_rows(cfg, d.T), (d.T + 127) // 128 * 128
+
+
 def moe_dispatch_mx(cfg, x, topk_idx, expert_offsets, expert_counts, xq_perm, xq_perm_sf, xq_shared,
                     xq_shared_sf, perm_src, row_of, workspace, stream=None):
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    Rp, Tp = _mx_rows(d, cfg)
+    shared = d.S > 0
+    _req("x", x, _BF16, 0)
+    _req("topk_idx", topk_idx, _I32, d.T * d.k)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req("expert_counts", expert_counts, _I32, _n(d, d.E))
+    _req("xq_perm", xq_perm, _U8, Rp * d.H)
+    _req("xq_perm_sf", xq_perm_sf, _U8, mx_scale_bytes(Rp, d.H) if Rp else 0)
+    _req("xq_shared", xq_shared, _U8, Tp * d.H if shared else 0, optional=not shared)
+    _req("xq_shared_sf", xq_shared_sf, _U8, mx_scale_bytes(Tp, d.H) if shared and Tp else 0, optional=not shared)
+    _req("perm_src", perm_src, _I32, Rp)
+    _req("row_of", row_of, _I32, d.T * d.k)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_dispatch_mx", lib().moe_dispatch_mx(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(topk_idx), _ptr(expert_offsets),
         _ptr(expert_counts), _ptr(xq_perm), _ptr(xq_perm_sf), _ptr(xq_shared), _ptr(xq_shared_sf),
@@ -299,12 +479,18 @@ def moe_dispatch_mx(cfg, x, topk_idx, expert_offsets, expert_counts, xq_perm, xq
 def mx_weights(gate, up, down, shared_gate=None, shared_up=None, shared_down=None) -> MXWeights:
     """MXWeights from (q, sf) tensor pairs (the shared ones may be None)."""
     def m(pair):
-        return MXMatrix(None, None) if pair is None else MXMatrix(pair[0].data_ptr(), pair[1].data_ptr())
+        if pair is None:
+            return MXMatrix(None, None)
+        _req("MXFP8 weight bytes", pair[0], _U8, 0)
+        _req("MXFP8 weight scales", pair[1], _U8, 0)
+        return MXMatrix(pair[0].data_ptr(), pair[1].data_ptr())
     return MXWeights(m(gate), m(up), m(down), m(shared_gate), m(shared_up), m(shared_down))
 
 
 def moe_forward_mx(cfg, x, router_w, e_bias, weights: MXWeights, y, topk_idx_out=None, topk_w_out=None,
                    workspace=None, stream=None):
+    _req_layer(cfg, x, router_w, e_bias, y, topk_idx_out, topk_w_out)
+    _req("workspace", workspace, _U8, 0, optional=True)
     _check("moe_forward_mx", lib().moe_forward_mx(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), ctypes.byref(weights),
         _ptr(y), out_dtype_code(y), _ptr(topk_idx_out), _ptr(topk_w_out), _ptr(workspace),
@@ -313,6 +499,19 @@ def moe_forward_mx(cfg, x, router_w, e_bias, weights: MXWeights, y, topk_idx_out
 
 def moe_experts_gate_up_mx(cfg, T, xq_perm, xq_perm_sf, xq_shared, xq_shared_sf, expert_offsets, expert_counts,
                            weights: MXWeights, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf, stream=None):
+    d = _Dims(cfg, T)
+    Rp, Tp = _mx_rows(d, cfg)
+    shared = d.S > 0
+    _req("xq_perm", xq_perm, _U8, Rp * d.H)
+    _req("xq_perm_sf", xq_perm_sf, _U8, mx_scale_bytes(Rp, d.H) if Rp else 0)
+    _req("xq_shared", xq_shared, _U8, Tp * d.H if shared else 0, optional=not shared)
+    _req("xq_shared_sf", xq_shared_sf, _U8, mx_scale_bytes(Tp, d.H) if shared and Tp else 0, optional=not shared)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req("expert_counts", expert_counts, _I32, _n(d, d.E))
+    _req("hq_routed", hq_routed, _U8, Rp * d.I)
+    _req("hq_routed_sf", hq_routed_sf, _U8, mx_scale_bytes(Rp, d.I) if Rp else 0)
+    _req("hq_shared", hq_shared, _U8, Tp * d.SI if shared else 0, optional=not shared)
+    _req("hq_shared_sf", hq_shared_sf, _U8, mx_scale_bytes(Tp, d.SI) if shared and Tp else 0, optional=not shared)
     _check("moe_experts_gate_up_mx", lib().moe_experts_gate_up_mx(
         ctypes.byref(_cfg(cfg)), T, _ptr(xq_perm), _ptr(xq_perm_sf), _ptr(xq_shared), _ptr(xq_shared_sf),
         _ptr(expert_offsets), _ptr(expert_counts), ctypes.byref(weights), _ptr(hq_routed), _ptr(hq_routed_sf),
@@ -321,6 +520,20 @@ def moe_experts_gate_up_mx(cfg, T, xq_perm, xq_perm_sf, xq_shared, xq_shared_sf,
 
 def moe_experts_down_mx(cfg, T, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf, expert_offsets, expert_counts,
                         perm_src, topk_w, weights: MXWeights, y_perm, y_perm_scale, stream=None):
+    d = _Dims(cfg, T)
+    Rp, Tp = _mx_rows(d, cfg)
+    shared = d.S > 0
+    rows = Rp + (d.T if shared else 0)
+    _req("hq_routed", hq_routed, _U8, Rp * d.I)
+    _req("hq_routed_sf", hq_routed_sf, _U8, mx_scale_bytes(Rp, d.I) if Rp else 0)
+    _req("hq_shared", hq_shared, _U8, Tp * d.SI if shared else 0, optional=not shared)
+    _req("hq_shared_sf", hq_shared_sf, _U8, mx_scale_bytes(Tp, d.SI) if shared and Tp else 0, optional=not shared)
+    _req("expert_offsets", expert_offsets, _I32, _n(d, d.E + 1))
+    _req("expert_counts", expert_counts, _I32, _n(d, d.E))
+    _req("perm_src", perm_src, _I32, Rp)
+    _req("topk_w", topk_w, _F32, d.T * d.k)
+    _req("y_perm", y_perm, _F16, rows * d.H)
+    _req("y_perm_scale", y_perm_scale, _U8, rows * d.scale_cols)
     _check("moe_experts_down_mx", lib().moe_experts_down_mx(
         ctypes.byref(_cfg(cfg)), T, _ptr(hq_routed), _ptr(hq_routed_sf), _ptr(hq_shared), _ptr(hq_shared_sf),
         _ptr(expert_offsets), _ptr(expert_counts), _ptr(perm_src), _ptr(topk_w), ctypes.byref(weights),
@@ -328,6 +541,8 @@ def moe_experts_down_mx(cfg, T, hq_routed, hq_routed_sf, hq_shared, hq_shared_sf
 
 
 def moe_combine_mx(cfg, T, y_perm, y_perm_scale, row_of, y, stream=None):
+    d = _Dims(cfg, T)
+    _req_combine(d, _mx_rows(d, cfg)[0], y_perm, y_perm_scale, row_of, y)
     _check("moe_combine_mx", lib().moe_combine_mx(ctypes.byref(_cfg(cfg)), T, _ptr(y_perm), _ptr(y_perm_scale),
                                                   _ptr(row_of), _ptr(y), out_dtype_code(y), _stream(stream)))
 
@@ -340,10 +555,24 @@ def workspace_size_bwd(cfg, T: int) -> int:
     return n.value
 
 
+def _req_grads(d, dy, dx, d_router_w, d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down):
+    _req("dy", dy, _BF16, d.T * d.H)
+    _req("dx", dx, _F32, d.T * d.H)
+    _req("d_router_w", d_router_w, _F32, d.E * d.H)
+    _req_weights(d, d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down, prefix="d_")
+
+
 def moe_backward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dy, dx, d_router_w,
                  d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down, workspace, stream=None):
     """Gradients of sum(y * dy): dx fp32 [T,H], d_router_w fp32 [E,H], expert and shared
     weight gradients bf16 in the weights' layouts (include/moe.h)."""
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _req("x", x, _BF16, 0)
+    _req("router_w", router_w, _F32, d.E * d.H)
+    _req("e_bias", e_bias, _F32, d.E)
+    _req_weights(d, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+    _req_grads(d, dy, dx, d_router_w, d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_backward", lib().moe_backward(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate), _ptr(w_up),
         _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w),
@@ -364,6 +593,9 @@ def moe_forward_host(cfg, x_host, router_w, e_bias, w_gate, w_up, w_down, ws_gat
                      chunk_tokens, workspace, stream=None):
     """The forward from pinned host x [T,H] bf16 to host y [T,H] (fp32 or bf16), copies
     overlapped with the layer chunk by chunk (include/moe.h)."""
+    d = _req_layer(cfg, x_host, router_w, e_bias, y_host, None, None, x_where="host")
+    _req_weights(d, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_forward_host", lib().moe_forward_host(
         ctypes.byref(_cfg(cfg)), x_host.shape[0], _ptr(x_host), _ptr(router_w), _ptr(e_bias), _ptr(w_gate),
         _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y_host), out_dtype_code(y_host),
@@ -373,6 +605,9 @@ def moe_forward_host(cfg, x_host, router_w, e_bias, w_gate, w_up, w_down, ws_gat
 def moe_forward_train(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, y, context,
                       stream=None):
     """The forward, keeping in `context` (workspace_size_bwd bytes) what moe_backward_train needs."""
+    d = _req_layer(cfg, x, router_w, e_bias, y, None, None)
+    _req_weights(d, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+    _req("context", context, _U8, 0)
     _check("moe_forward_train", lib().moe_forward_train(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(e_bias), _ptr(w_gate), _ptr(w_up),
         _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(y), out_dtype_code(y), _ptr(context),
@@ -381,6 +616,12 @@ def moe_forward_train(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, w
 
 def moe_backward_train(cfg, x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, dy, dx, d_router_w,
                        d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down, context, stream=None):
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _req("x", x, _BF16, 0)
+    _req("router_w", router_w, _F32, d.E * d.H)
+    _req_weights(d, w_gate, w_up, w_down, ws_gate, ws_up, ws_down)
+    _req_grads(d, dy, dx, d_router_w, d_w_gate, d_w_up, d_w_down, d_ws_gate, d_ws_up, d_ws_down)
+    _req("context", context, _U8, 0)
     _check("moe_backward_train", lib().moe_backward_train(
         ctypes.byref(_cfg(cfg)), x.shape[0], _ptr(x), _ptr(router_w), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w), _ptr(d_w_gate),
