@@ -36,41 +36,58 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-    for (int h0 = h_begin; h0 < h_end; h0 += kRK) {
-        // x tile: 128 x 32 bf16 = 512 chunks of 8 elements.
-        for (int c = tid; c < kRT * kRK / 8; c += 256) {
+    // Each thread moves two 8-element chunks of the x tile and two 4-element chunks
+    // of the Wr tile per K step.  The next step's chunks are loaded into registers
+    // while this step's FMAs run (same products, same summation order).
+    static_assert(kRT * kRK / 8 == 2 * 256 && kRE * kRK / 4 == 2 * 256, "two chunks per thread");
+    uint4 xr[2];
+    float4 wv[2];
+    auto fetch = [&](int h0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = tid + 256 * u;
             const int r = c / (kRK / 8), kc = (c % (kRK / 8)) * 8;
             const int t = t0 + r;
-            float v[8];
-            if (t < T && h0 + kc < h_end) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(x + (int64_t)t * H + h0 + kc);
-                const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __bfloat1622float2(p[q]);
-                    v[2 * q] = f.x;
-                    v[2 * q + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = 0.f;
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) xs[kc + q][r] = v[q];
+            xr[u] = (t < T && h0 + kc < h_end)
+                        ? *reinterpret_cast<const uint4*>(x + (int64_t)t * H + h0 + kc)
+                        : make_uint4(0, 0, 0, 0);
         }
-        // Wr tile: 64 x 32 fp32 = 512 chunks of 4.
-        for (int c = tid; c < kRE * kRK / 4; c += 256) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = tid + 256 * u;
             const int r = c / (kRK / 4), kc = (c % (kRK / 4)) * 4;
             const int e = e0 + r;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (e < E && h0 + kc < h_end)
-                v = *reinterpret_cast<const float4*>(wr + (int64_t)e * H + h0 + kc);
-            ws[kc + 0][r] = v.x;
-            ws[kc + 1][r] = v.y;
-            ws[kc + 2][r] = v.z;
-            ws[kc + 3][r] = v.w;
+            wv[u] = (e < E && h0 + kc < h_end)
+                        ? *reinterpret_cast<const float4*>(wr + (int64_t)e * H + h0 + kc)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    if (h_begin < h_end) fetch(h_begin);
+    for (int h0 = h_begin; h0 < h_end; h0 += kRK) {
+        // x tile 128 x 32 (bf16 -> fp32, transposed), Wr tile 64 x 32 (transposed).
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = tid + 256 * u;
+            const int r = c / (kRK / 8), kc = (c % (kRK / 8)) * 8;
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&xr[u]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(p[q]);
+                xs[kc + 2 * q][r] = f.x;
+                xs[kc + 2 * q + 1][r] = f.y;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = tid + 256 * u;
+            const int r = c / (kRK / 4), kc = (c % (kRK / 4)) * 4;
+            ws[kc + 0][r] = wv[u].x;
+            ws[kc + 1][r] = wv[u].y;
+            ws[kc + 2][r] = wv[u].z;
+            ws[kc + 3][r] = wv[u].w;
         }
         __syncthreads();
+        if (h0 + kRK < h_end) fetch(h0 + kRK);
 #pragma unroll 8
         for (int kk = 0; kk < kRK; ++kk) {
             float a[8], b[4];
