@@ -395,10 +395,11 @@ def layer_route_idx(shape, inp):
 
 
 def layer_bytes(shape, idx):
-    """Algorithmic bytes of one step: touched routed experts + shared + router + x and y."""
+    """Algorithmic bytes of one step: bf16 weights of the touched routed experts and the
+    shared experts, the fp32 router, and x (bf16) in and y (fp32) out."""
     touched = int(torch.unique(idx).numel())
     b = touched * 3 * shape.H * shape.I * 2 + 3 * shape.H * shape.S * shape.I * 2
-    b += 4 * shape.E * shape.H + 4 * shape.T * shape.H
+    b += 4 * shape.E * shape.H + 2 * shape.T * shape.H + 4 * shape.T * shape.H
     return b, touched
 
 
