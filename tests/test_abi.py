@@ -158,3 +158,22 @@ def test_row_space_beyond_int32_rejected(lib):
     assert lib.moe_workspace_size(ctypes.byref(c), T_pad_overflow, ctypes.byref(n)) == abi.MOE_ERR_UNSUPPORTED
     T_fits = (limit - 128 * E) // (k + 1) - 1
     assert lib.moe_workspace_size(ctypes.byref(c), T_fits, ctypes.byref(n)) == abi.MOE_OK
+
+
+def test_host_forward_workspace_holds_two_slots_and_one_chunk(lib):
+    # Two staging slots each for x (bf16) and y (fp32 or bf16), plus the device
+    # forward's workspace for the largest chunk (a full chunk or the last one).
+    s = V3_PREFILL
+    H, T = s.H, s.T
+    whole = abi.workspace_size_host(s, T, 0, abi.MOE_DTYPE_F32)
+    assert whole >= abi.workspace_size(s, T) + 2 * T * H * 2 + 2 * T * H * 4
+    chunk = 6000                                   # 3 chunks: 6000, 6000, 4384 rows
+    per = abi.workspace_size_host(s, T, chunk, abi.MOE_DTYPE_F32)
+    fwd = max(abi.workspace_size(s, chunk), abi.workspace_size(s, T - 2 * chunk))
+    assert per >= fwd + 2 * chunk * H * 2 + 2 * chunk * H * 4
+    assert per < whole
+    assert abi.workspace_size_host(s, T, chunk, abi.MOE_DTYPE_BF16) < per
+    # chunk_tokens >= T is one chunk, like 0.
+    assert abi.workspace_size_host(s, T, T + 5, abi.MOE_DTYPE_F32) == whole
+    with pytest.raises(abi.MoEError):
+        abi.workspace_size_host(s, T, chunk, 7)     # not a moe_dtype
