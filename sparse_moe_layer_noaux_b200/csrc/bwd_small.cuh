@@ -58,11 +58,11 @@ __global__ void __launch_bounds__(256) bwd_scatter_kernel(const __nv_bfloat16* _
 }
 
 // Block (e, b): rows offsets[e] + counts[e] .. offsets[e+1] of both buffers,
-// 16-byte stores, blocks of one expert striding over its padding rows.
+// 16-byte stores, blocks of one expert striding over its padding rows.  a and b
+// may be the same buffer (only one needs zeroing), hence no __restrict__ on them.
 __global__ void __launch_bounds__(256) bwd_zero_pad_kernel(const int32_t* __restrict__ offsets,
                                                            const int32_t* __restrict__ counts, int H,
-                                                           __nv_bfloat16* __restrict__ a,
-                                                           __nv_bfloat16* __restrict__ b) {
+                                                           __nv_bfloat16* a, __nv_bfloat16* b) {
     const int e = blockIdx.x;
     const int64_t r0 = offsets[e] + counts[e], r1 = offsets[e + 1];
     const int64_t n = (r1 - r0) * (H / 8);
