@@ -35,18 +35,19 @@ METRIC = "MoE-layer tokens/s and TFLOP/s at V3 shape (T=128, 16384); % of roofli
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the gate/up
-# GEMM, from one single-pass ncu capture of `bench.py --profile-only` at the full
-# workload (the capture and its command are summarised under profiles/).  A figure is
-# reported only while the kernel sources hash to the value it was taken on.
-GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh"),
-                "mxfp8": ("grouped_gemm_mx.cuh", "mx.cuh", "grouped_gemm.cuh", "sm100_ptx.cuh")}
-MEASURED_TRAFFIC = {
-    ("bf16", "v3_prefill"): {"sources_sha1": "4610e681b1a9cc385e096efd6138d0e0a863a661",
-                             "dram_read": 20471961088, "dram_write": 600841984},
-    ("mxfp8", "v3_prefill"): {"sources_sha1": "afe2547cabcad37df852530993b0e83f7373f66d",
-                              "dram_read": 9408662784, "dram_write": 341510400},
-}
+# DRAM traffic of the expert GEMMs.  The V3 workloads hold 22.5 GB of expert weights,
+# beyond the size of an ncu capture on this pool, so the counters
+# (dram__bytes_read.sum + dram__bytes_write.sum, one pass) are taken on the 32-expert
+# V3 case (v3_e32: T = 4096, 2.8 GB of weights), whose launches walk their segments
+# in the same orders as the full workload (expert segments of a few row tiles column
+# by column, the shared segment row by row).  A launch's traffic is reported as that
+# case's measured traffic / algorithmic-bytes ratio times the launch's own algorithmic
+# bytes, and only while the kernel sources hash to the value the capture was taken on
+# (profiles/ holds the capture and its command).
+GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh", "device_status.cuh"),
+                "mxfp8": ("grouped_gemm_mx.cuh", "mx.cuh", "grouped_gemm.cuh", "sm100_ptx.cuh",
+                          "device_status.cuh")}
+MEASURED_TRAFFIC = {}  # (precision, "gate_up" | "down") -> {sources_sha1, case, dram_bytes, algorithmic_bytes}
 
 
 def gemm_sources_sha1(precision="bf16"):
@@ -58,21 +59,51 @@ def gemm_sources_sha1(precision="bf16"):
     return h.hexdigest()
 
 
-def measured_traffic(workload, precision="bf16"):
-    m = MEASURED_TRAFFIC.get((precision, workload))
+def traffic_ratio(kernel, precision="bf16"):
+    """Measured DRAM bytes / algorithmic bytes of a captured launch of `kernel`
+    ("gate_up" or "down"), or None when no capture matches the current sources."""
+    m = MEASURED_TRAFFIC.get((precision, kernel))
     if m is None or m["sources_sha1"] != gemm_sources_sha1(precision):
         return None
-    return m["dram_read"] + m["dram_write"]
+    return m["dram_bytes"] / m["algorithmic_bytes"]
 
 
-def gate_up_algorithmic_bytes(shape, touched):
+def traffic_fields(kernel, algorithmic, precision="bf16"):
+    """The roofline's traffic keys for one launch with `algorithmic` bytes."""
+    r = traffic_ratio(kernel, precision)
+    m = MEASURED_TRAFFIC.get((precision, kernel))
+    return {"algorithmic_bytes": algorithmic,
+            "traffic": None if r is None else int(r * algorithmic),
+            "traffic_ratio": r,
+            "traffic_source": None if r is None else
+            f"ncu dram__bytes_read.sum + dram__bytes_write.sum on {m['case']}: "
+            f"{m['dram_bytes']} B against {m['algorithmic_bytes']} algorithmic B, ratio x this launch's bytes"}
+
+
+def _routed_rows(shape):
+    return shape.T * shape.k + (shape.T if shape.S else 0)
+
+
+def gate_up_algorithmic_bytes(shape, touched, elt=2.0):
     """Compulsory HBM bytes of one gate/up launch: gate and up weights of the touched
     routed experts and of the shared experts, the T*k gathered rows and the T token
-    rows they read, and the bf16 h rows written (T*(k+S) x I)."""
-    w = (touched + shape.S) * 2 * shape.I * shape.H * 2
-    a = (shape.T * shape.k + (shape.T if shape.S else 0)) * shape.H * 2
-    h = shape.T * (shape.k + shape.S) * shape.I * 2
-    return w + a + h
+    rows they read, and the h rows written (T*(k+S) x I).  `elt` is bytes per
+    element (2 for bf16; 1 + 1/32 for MXFP8: E4M3 bytes plus one scale per 32)."""
+    w = (touched + shape.S) * 2 * shape.I * shape.H * elt
+    a = _routed_rows(shape) * shape.H * elt
+    h = shape.T * (shape.k + shape.S) * shape.I * elt
+    return int(w + a + h)
+
+
+def down_algorithmic_bytes(shape, touched, elt=2.0):
+    """Compulsory HBM bytes of one down launch: down weights of the touched routed
+    experts and of the shared experts, the h rows read, and the block-scaled fp16
+    y_perm rows written (2 bytes per value plus one scale byte per 32, rows padded
+    to 8 scale bytes)."""
+    w = (touched + shape.S) * shape.H * shape.I * elt
+    h = shape.T * (shape.k + shape.S) * shape.I * elt
+    y = _routed_rows(shape) * (2 * shape.H + (shape.H // 32 + 7) // 8 * 8)
+    return int(w + h + y)
 
 
 def load_peaks():
@@ -331,7 +362,8 @@ def time_gpu_mx(shape, steps, warmup, world, rank, peaks, inp=None):
                      "bound": "tensor", "achieved": gu_flops / (gu_ms * 1e-3) / 1e12, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": gu_flops / (gu_ms * 1e-3) / 1e12 / fp8_peak,
                      "peak_source": "measured bf16 burst x 2 (nominal dense fp8/bf16 ratio)",
-                     "traffic": measured_traffic(shape.name, "mxfp8"), "ms_per_launch": gu_ms},
+                     **traffic_fields("gate_up", gate_up_algorithmic_bytes(shape, touched, 1 + 1 / 32), "mxfp8"),
+                     "ms_per_launch": gu_ms},
         "clocks": clk,
     }
     del st
@@ -403,6 +435,19 @@ def layer_bytes(shape, idx):
     return b, touched
 
 
+def load_stats(shape, idx, histogram=False):
+    """Per-expert load of one routed batch: rows per expert against the mean T*k/E."""
+    counts = np.bincount(idx.reshape(-1).astype(np.int64), minlength=shape.E)
+    mean = shape.T * shape.k / shape.E
+    out = {"experts_touched": int((counts > 0).sum()), "max_rows": int(counts.max()),
+           "mean_rows": mean, "max_over_mean": float(counts.max() / mean),
+           "min_rows_touched": int(counts[counts > 0].min()) if counts.any() else 0,
+           "segments_le_112_rows": int(((counts > 0) & (counts <= 112)).sum())}
+    if histogram:
+        out["rows_per_expert"] = counts.tolist()
+    return out
+
+
 def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
     inp = rank_inputs(shape, rank, "cuda")
     st = StagedStep(shape, inp)
@@ -431,6 +476,7 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
     flops = shape.flops()
     lbytes, touched = layer_bytes(shape, st.idx)
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9))
+    idx_h = st.idx.cpu().numpy()
     res = {
         "ms": ms, "stage_ms": stage_ms, "staged_ms": staged_ms, "forward_ms": fwd_ms, "launches": launches,
         "tflops": flops / (ms * 1e-3) / 1e12, "layer_bytes": lbytes, "experts_touched": touched,
@@ -438,7 +484,9 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
                            lbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
                            "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms,
                            "hbm_gbs_achieved": lbytes / (ms * 1e-3) / 1e9},
-        "clocks": clk, "st": st, "inp": inp, "layer": layer,
+        "clocks": clk, "st": st, "inp": inp, "layer": layer, "idx": idx_h,
+        "load": load_stats(shape, idx_h, histogram=shape.bias_kind == "zipf"),
+        "routing_inputs": (bf16_bits(inp["x"]), inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()),
     }
     return res
 
@@ -527,13 +575,59 @@ def oracle_tokens_per_step(shape):
     return max(1, min(shape.T, int(4e8 // per_token_macs)))
 
 
+def host_cpu():
+    """Host core count and CPU model (from /proc/cpuinfo when there is one)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(shape, inp, budget_tokens=None):
     n = budget_tokens or max(1, min(shape.T, 24 * oracle_tokens_per_step(shape)))
     secs, rows = oracle_sample(shape, inp, n, seed=99)
     return {"value": len(rows) / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{len(rows)} of the {shape.T} tokens of the {shape.name} batch (seeded): "
                       f"routing, shared and routed SwiGLU experts in float64, 1 thread; "
-                      f"expert-weight copies from the device excluded"}
+                      f"expert-weight copies from the device excluded", **host_cpu()}
+
+
+NEAR_TIE = 1e-4  # oracle margin below which two expert sets are equally correct in fp32
+
+
+def oracle_routing_report(shape, routing_inputs, gpu_idx):
+    """The float64 oracle router on every token of a workload (row blocks in spawned
+    processes): its throughput, the near-tie count (tokens whose margin at the
+    group-keep or top-k boundary is below 1e-4) and how many GPU expert sets differ
+    from the oracle's (each allowed only on a near tie)."""
+    import oracle
+    from oracle.pool import route_rows
+    oracle.build()
+    x_bits, rw, bias = routing_inputs
+    workers = max(1, min(16, os.cpu_count() or 1))
+    t0 = time.perf_counter()
+    ref_idx, _, margin, _ = route_rows(shape, x_bits, rw, bias, workers=workers)
+    secs = time.perf_counter() - t0
+    near = margin < NEAR_TIE
+    differ = np.array([set(a.tolist()) != set(b.tolist()) for a, b in zip(gpu_idx, ref_idx)])
+    return {"tokens": int(shape.T), "near_ties": int(near.sum()), "gpu_sets_differing": int(differ.sum()),
+            "gpu_sets_differing_off_near_tie": int((differ & ~near).sum()),
+            "oracle_routing_tokens_per_s": shape.T / secs, "oracle_processes": workers}
+
+
+def workload_summary(shape, r, world):
+    """The nested bench object of one workload's forward."""
+    return {"T": shape.T, "ms_per_step": r["ms"], "tokens_per_s": job_throughput(shape.T, world, r["ms"]),
+            "tflops": r["tflops"] * world, "stage_ms": r["stage_ms"], "forward_ms": r["forward_ms"],
+            "layer_roofline": r["layer_roofline"], "layer_bytes": r["layer_bytes"],
+            "experts_touched": r["experts_touched"], "load": r["load"], "gpu_launches": r["launches"],
+            "clocks": r["clocks"]}
 
 
 def run_reference(args, shape, world, rank):
@@ -587,7 +681,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mx", action="store_true", help="skip the MXFP8 variant of the layer")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass")
-    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only the headline workload, not the other four shapes")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "mxfp8", "backward"],
                     help="what --profile-only runs: the bf16 or MXFP8 forward stages, or the backward")
     ap.add_argument("--profile-only", action="store_true",
@@ -623,6 +718,14 @@ def main():
         torch.cuda.synchronize()
         assert abi.device_status() == 0
         print(f"profile-only: {args.warmup + args.steps} passes of {shape.name}", flush=True)
+        if args.precision != "backward":
+            # The algorithmic bytes of this workload's GEMM launches, for the traffic ratio.
+            touched = int(torch.unique(st.idx).numel())
+            elt = 2.0 if args.precision == "bf16" else 1 + 1 / 32
+            print(json.dumps({"workload": shape.name, "precision": args.precision, "experts_touched": touched,
+                              "gate_up_algorithmic_bytes": gate_up_algorithmic_bytes(shape, touched, elt),
+                              "down_algorithmic_bytes": down_algorithmic_bytes(shape, touched, elt)}),
+                  flush=True)
         finish(world)
         return
     args.warmup = max(args.warmup, 3)
@@ -641,25 +744,37 @@ def main():
                 "frac": achieved / peaks["bf16_tflops"],
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "peak_source": f"{peak_src} bf16 dense (burst)",
-                "traffic": measured_traffic(shape.name),
-                "algorithmic_bytes": gate_up_algorithmic_bytes(shape, res["experts_touched"]),
                 "flops_per_launch": k4_flops, "ms_per_launch": k4_ms}
+
+    k5_ms = res["stage_ms"]["down"]
+    k5_flops = 2.0 * shape.H * shape.I * shape.T * (shape.k + shape.S)
+    roofline.update(traffic_fields("gate_up", gate_up_algorithmic_bytes(shape, res["experts_touched"])))
+    down_roofline = {"kernel": "grouped_gemm_kernel<kDown> (down + routing weight, block-scaled fp16 out)",
+                     "bound": "tensor", "achieved": k5_flops / (k5_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": k5_flops / (k5_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                     **traffic_fields("down", down_algorithmic_bytes(shape, res["experts_touched"])),
+                     "flops_per_launch": k5_flops, "ms_per_launch": k5_ms}
 
     e2e_ms, h2d, d2h = time_e2e(res["layer"], shape, max(3, args.steps // 2))
     e2e_ms = max_over_ranks(e2e_ms, world)
+    routing_inputs = {shape.name: (shape, res["routing_inputs"], res["idx"])}
+    load = res["load"]
 
     extra = {}
-    if not args.no_decode and shape.name == "v3_prefill":
-        dec = WORKLOADS["v3_decode"]
-        del res["st"]
+    if shape.name == "v3_prefill":
+        del res["st"], res["layer"]
         torch.cuda.empty_cache()
-        dr = time_gpu(dec, max(args.steps, 20), args.warmup, world, rank, peaks)
-        extra["v3_decode"] = {
-            "tokens_per_s": job_throughput(dec.T, world, dr["ms"]), "ms_per_step": dr["ms"],
-            "tflops": dr["tflops"], "stage_ms": dr["stage_ms"], "forward_ms": dr["forward_ms"],
-            "layer_roofline": dr["layer_roofline"], "experts_touched": dr["experts_touched"],
-            "layer_bytes": dr["layer_bytes"]}
-        del dr
+        # The other four workload shapes, each timed the same way (their own inputs).
+        workloads = {}
+        for name in ([] if args.no_workloads else ["tiny", "mid", "v3_decode", "v3_skewed"]):
+            ws = WORKLOADS[name]
+            r = time_gpu(ws, max(args.steps, 20), args.warmup, world, rank, peaks)
+            workloads[name] = workload_summary(ws, r, world)
+            routing_inputs[name] = (ws, r["routing_inputs"], r["idx"])
+            del r
+            torch.cuda.empty_cache()
+        if workloads:
+            extra["workloads"] = workloads
     if not args.no_mx and shape.name == "v3_prefill":
         # The MXFP8 expert FFNs on the same workload (fine-grained FP8 of the pages'
         # FP8 notes): a second precision of the same layer, reported beside it.
@@ -680,8 +795,8 @@ def main():
         "config": workload_config(shape, world),
         "tflops": res["tflops"] * world, "stage_ms": res["stage_ms"], "staged_ms": res["staged_ms"],
         "forward_ms": res["forward_ms"],
-        "layer_roofline": res["layer_roofline"], "experts_touched": res["experts_touched"],
-        "roofline": roofline,
+        "layer_roofline": res["layer_roofline"], "experts_touched": res["experts_touched"], "load": load,
+        "roofline": roofline, "down_roofline": down_roofline,
         "clocks": res["clocks"],
         "e2e": {"value": job_throughput(shape.T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -689,7 +804,11 @@ def main():
     }
     line.update(extra)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape, res["inp"])
+        cb = cpu_baseline(shape, res["inp"])
+        # The oracle router over every token of each workload: near ties and the
+        # GPU's agreement with it.
+        cb["routing"] = {name: oracle_routing_report(ws, ri, gi) for name, (ws, ri, gi) in routing_inputs.items()}
+        line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
     finish(world)

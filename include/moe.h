@@ -21,7 +21,11 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers, row-major and contiguous,
- *     owned by the caller; the library never allocates, frees or keeps them.
+ *     owned by the caller; the library never allocates device memory for
+ *     tensors, and never frees or keeps the caller's pointers.  (The one
+ *     exception to "allocates nothing" is moe_forward_host, which creates two
+ *     copy streams and eight events per device on its first call on that
+ *     device and keeps them until the process exits.)
  *     bf16 tensors are passed as void* (IEEE bfloat16 bit patterns).
  *   - Weights use the nn.Linear (out, in) layout: w_gate, w_up [E, I, H],
  *     w_down [E, H, I]; the S shared experts are stored concatenated along the
@@ -37,10 +41,13 @@
  *     nothing.
  *   - Device-side waits are bounded: a wait that gives up writes a device
  *     error word (read with moe_device_status) instead of hanging the GPU.
- *   - The expert GEMMs normally run one CTA per tile.  Setting the environment
- *     variable MOE_PAIR_GEMM=1 (read at each call) runs prefill-sized batches on
- *     CTA pairs (256-row tiles, tcgen05 cta_group::2) instead; results are the
- *     same, only the schedule differs.
+ *   - Index arrays passed in by the caller (topk_idx, expert_offsets,
+ *     expert_counts, perm_src, row_of) live on the device, where the host
+ *     cannot check them.  Every kernel checks such an entry before using it as
+ *     an index: an entry out of range is skipped (it reads and writes nothing;
+ *     see each call for what it then produces) and the device error word
+ *     records it, so moe_device_status returns MOE_ERR_DEVICE_CHECK.  Arrays
+ *     produced by this library always pass these checks.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -81,7 +88,9 @@ typedef enum moe_status {
     MOE_ERR_WORKSPACE = 3,    /* workspace null or smaller than moe_workspace_size() */
     MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
     MOE_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (from moe_device_status) */
-    MOE_ERR_STATIC_LIMIT = 6  /* moe_dispatch_noalloc: T * E beyond its fixed scratch */
+    MOE_ERR_STATIC_LIMIT = 6, /* moe_dispatch_noalloc: T * E beyond its fixed scratch */
+    MOE_ERR_DEVICE_CHECK = 7  /* a device-side check skipped an out-of-range index entry
+                                 (from moe_device_status) */
 } moe_status;
 
 /* Element type of the layer output y. */
@@ -102,22 +111,29 @@ MOE_API int moe_workspace_size(const moe_config *cfg, int64_t T, size_t *bytes);
  *   router_w fp32  [E, H]      e_bias fp32 [E]
  *   topk_idx int32 [T, k]      topk_w fp32 [T, k]   (outputs)
  * Logits are accumulated in fp32 (gating is kept in high precision, per the
- * knlb.dev DeepSeek-V3 notes, § infrastructure / fp8).
+ * knlb.dev DeepSeek-V3 notes, § infrastructure / fp8).  Whatever the values
+ * (NaN or infinite scores included, which rank below every finite score),
+ * every token gets k distinct expert indices in [0, E) from at most
+ * topk_group groups.
  */
 MOE_API int moe_route(const moe_config *cfg, int64_t T, const void *x, const float *router_w,
               const float *e_bias, int32_t *topk_idx, float *topk_w,
               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Dispatch: the page's per-expert mask and gather, indices[:, :, k] == i then
- * x[mask] ("The Evolving Transformer · 07", § 02, MoE.forward), done once for
- * all experts as a counting sort.  Rows routed to expert e occupy
+ * Dispatch: groups the token rows by the expert they are routed to.  The
+ * teaching code of "The Evolving Transformer · 07" (§ 02, MoE.forward) selects
+ * and gathers each expert's tokens in a loop over experts and slots; here one
+ * counting sort does it for all experts.  Rows routed to expert e occupy
  * x_perm[expert_offsets[e] .. expert_offsets[e+1]) in ascending (t, j) order.
- *   topk_idx        int32 [T, k]            (input, from moe_route)
+ *   topk_idx        int32 [T, k]            (input, from moe_route; each entry in [0, E))
  *   expert_offsets  int32 [E + 1]           expert_offsets[E] == T * k
  *   x_perm          bf16  [T * k, H]        x_perm[r] = x[perm_src[r] / k]
  *   perm_src        int32 [T * k]           source slot t * k + j of row r
  *   row_of          int32 [T, k]            row of slot (t, j); inverse of perm_src
+ * A topk_idx entry outside [0, E) is skipped: it gets no row (row_of = -1),
+ * expert_offsets[E] is T * k minus the skipped entries, and the device error
+ * word records it (moe_device_status: MOE_ERR_DEVICE_CHECK).
  */
 MOE_API int moe_dispatch(const moe_config *cfg, int64_t T, const void *x, const int32_t *topk_idx,
                  int32_t *expert_offsets, void *x_perm, int32_t *perm_src, int32_t *row_of,
@@ -157,7 +173,9 @@ MOE_API int moe_dispatch_noalloc(const moe_config *cfg, int64_t T, const void *x
  *   h_shared[t]        = silu(x[t] . ws_gate^T) * (x[t] . ws_up^T)          bf16 [T, S*I]
  *   y_perm[T*k + t]    = h_shared[t] . ws_down^T
  * ("The Evolving Transformer · 07", § 02 and § 03.)  Grouped tensor-core
- * GEMMs over the variable-length expert segments given by expert_offsets;
+ * GEMMs over the variable-length expert segments given by expert_offsets
+ * (a segment outside [0, T*k) gets no rows and is recorded in the device error
+ * word; a perm_src entry outside [0, T*k) gives weight 0, likewise recorded);
  * fp32 accumulation; h is stored as bf16 (it is the next GEMM's operand).
  * y_perm [T*k + T, H] is stored block-scaled: fp16 values plus one scale code
  * per 32 columns in y_perm_scale [T*k + T, ceil(H / 256) * 8] (uint8); a value
@@ -188,10 +206,11 @@ MOE_API int moe_experts_down(const moe_config *cfg, int64_t T, const void *h_rou
 /*
  * Combine: y[t] = y_perm[T*k + t] (shared, if S > 0) + sum_{j<k} y_perm[row_of[t, j]],
  * block-scaled y_perm rows (see moe_experts) decoded and summed in fp32 in
- * that order, stored as y_dtype [T, H]
- * (a moe_dtype) — the page's output[mask] += w * expert_out and
- * `shared_expert_out + output` ("The Evolving Transformer · 07", § 02), as a
- * deterministic gather.
+ * that order, stored as y_dtype [T, H] (a moe_dtype).  This is the weighted
+ * sum of the expert outputs plus the shared expert's output of "The Evolving
+ * Transformer · 07" (§ 02, § 03), computed as a deterministic gather rather
+ * than by adding into the token rows.  A row_of entry outside [0, T*k)
+ * contributes nothing and is recorded in the device error word.
  */
 MOE_API int moe_combine(const moe_config *cfg, int64_t T, const void *y_perm,
                 const void *y_perm_scale, const int32_t *row_of, void *y, int32_t y_dtype,
@@ -221,7 +240,8 @@ MOE_API int moe_forward(const moe_config *cfg, int64_t T, const void *x, const f
  * e_bias fp32 [E] is updated in place (one fp32 add per expert); expert_load
  * int32 [E] optionally receives the loads (may be NULL).  gamma (the update
  * speed) is not given by the pages; it is the caller's, >= 0.  With T = 0
- * every load equals the mean (0), so no bias moves.
+ * every load equals the mean (0), so no bias moves.  A topk_idx entry outside
+ * [0, E) is not counted and is recorded in the device error word.
  */
 MOE_API int moe_bias_update(const moe_config *cfg, int64_t T, const int32_t *topk_idx, float *e_bias,
                             float gamma, int32_t *expert_load, void *stream);
@@ -356,7 +376,10 @@ MOE_API int moe_backward(const moe_config *cfg, int64_t T, const void *x, const 
  * device.  The batch is cut into chunks of chunk_tokens rows (0 or >= T: one
  * chunk); chunk i's input copy and chunk i-1's output copy run on two internal
  * copy streams while chunk i is computed on `stream`, so transfers overlap the
- * layer.  Rows are independent, so y is moe_forward's on the whole batch: bit for
+ * layer.  The two copy streams and the events that order them are created by
+ * the first call on each device (with that device current) and kept until the
+ * process exits; make that first call before any stream capture.  Rows are
+ * independent, so y is moe_forward's on the whole batch: bit for
  * bit when the chunks and the batch take the same router-logit path (at least 2048
  * rows: tensor cores; fewer: CUDA cores), else up to the fp32 summation order of
  * the logits.  The workspace (moe_workspace_size_host) holds two staging slots each
@@ -397,9 +420,11 @@ MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, 
 MOE_API const char *moe_status_string(int status);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device: *device_error = 0 when no bounded wait gave up, else a
- * nonzero code naming the wait.  Returns MOE_OK, MOE_ERR_TIMEOUT when the
- * word was set, or MOE_ERR_CUDA. */
+ * current device: *device_error = 0 when no bounded wait gave up and no
+ * device-side check failed, else the nonzero code of the first failure
+ * (0x4xx: an index entry out of range was skipped; other codes: a bounded wait
+ * gave up).  Returns MOE_OK, MOE_ERR_DEVICE_CHECK for a 0x4xx word,
+ * MOE_ERR_TIMEOUT for any other nonzero word, or MOE_ERR_CUDA. */
 MOE_API int moe_device_status(void *stream, int32_t *device_error);
 
 /* Number of kernels this library has launched in this process. */

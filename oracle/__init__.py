@@ -6,22 +6,17 @@ binding) never imports, links or calls anything here, and this package imports
 nothing from the product.
 
 The arithmetic lives in ``moe_oracle.c`` (plain C, float64, single thread); this
-module builds it with gcc, wraps it with ctypes, and spells out the layer's
-forward exactly as the teaching code of "The Evolving Transformer · 07 —
-DeepSeek V2 & V3" (§ 02 DeepSeekMoE, ``MoE.forward``; § 03 Shared Expert) does:
+module builds it with gcc, wraps it with ctypes, and composes the layer's
+forward the way the teaching code of "The Evolving Transformer · 07 — DeepSeek
+V2 & V3" (§ 02 DeepSeekMoE, § 03 Shared Expert) defines it: the shared expert
+runs on every token; the router gives each token its top-k experts and their
+weights; each routed expert runs on the tokens sent to it; a token's output is
+the shared expert's output plus the weighted sum of its experts' outputs, the
+slots added in order 0..top_k-1.
 
-    shared_out = shared_expert(x)            # every token
-    weights, indices = router(x)             # (tokens, top_k)
-    output = 0
-    for each slot k and expert i:
-        mask = indices[:, k] == i
-        output[mask] += weights[mask, k] * expert_i(x[mask])
-    return shared_out + output
-
-The only liberty taken: the expert loop is the outer loop (so each expert's
-weights are fetched once) and each (token, slot) contribution is stored, then
-summed in slot order k = 0..top_k-1 — the same additions, in the same order per
-token, as the page's k-outer loop.
+Each expert's rows are computed in one call (so its weights are fetched once)
+and every (token, slot) result is kept until the slots are added in order, so
+each token sees the same additions in the same order as a slot-by-slot loop.
 """
 from __future__ import annotations
 
@@ -145,9 +140,13 @@ def swiglu(x_bits, w_gate, w_up, w_down) -> np.ndarray:
 ExpertFetch = Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarray]]
 
 
+def _run_serial(fn, jobs):
+    return (fn(*job) for job in jobs)
+
+
 def moe_layer(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
               shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]],
-              routing: Optional[Tuple[np.ndarray, np.ndarray]] = None):
+              routing: Optional[Tuple[np.ndarray, np.ndarray]] = None, run_experts=None):
     """The layer's forward for the rows of ``x_bits`` (any subset of tokens).
 
     ``expert(e)`` returns (w_gate[e], w_up[e], w_down[e]) as bf16 bits; it is
@@ -155,6 +154,9 @@ def moe_layer(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
     shared expert (ws_gate [S*I,H], ws_up [S*I,H], ws_down [H,S*I]) or None.
     ``routing`` optionally supplies (idx, w) instead of the oracle's own router
     (used to score an alternative, equally correct near-tie selection).
+    ``run_experts(fn, jobs)`` optionally evaluates ``fn(*job)`` for each expert's
+    job, in order (``oracle.pool.ExpertRunner`` spreads them over processes);
+    by default they run here, one after the other.
 
     Returns (y float64 [n,H], idx, w, margin or None).
     """
@@ -177,10 +179,10 @@ def moe_layer(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
 
     # routed: contribution of (row, slot) = w[row, slot] * expert_e(x[row]).
     contrib = np.zeros((n, k, H), np.float64)
-    for e in np.unique(idx):
+    experts = [int(e) for e in np.unique(idx)]
+    jobs = ((x_bits[np.nonzero(idx == e)[0]], *expert(e)) for e in experts)
+    for e, out in zip(experts, (run_experts or _run_serial)(swiglu, jobs)):
         rows, slots = np.nonzero(idx == e)
-        wg, wu, wd = expert(int(e))
-        out = swiglu(x_bits[rows], wg, wu, wd)
         contrib[rows, slots] = w[rows, slots][:, None] * out
     output = np.zeros((n, H), np.float64)
     for j in range(k):
@@ -270,7 +272,7 @@ def swiglu_mx(x_deq, w_gate, w_up, w_down, h_out=None) -> np.ndarray:
 
 def moe_layer_mx(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
                  shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]],
-                 routing: Optional[Tuple[np.ndarray, np.ndarray]] = None):
+                 routing: Optional[Tuple[np.ndarray, np.ndarray]] = None, run_experts=None):
     """The layer's forward with MXFP8 expert FFNs, for the rows of ``x_bits``.
 
     Same structure as ``moe_layer`` (shared expert on every row; routed outputs
@@ -291,9 +293,10 @@ def moe_layer_mx(shape, x_bits, router_w, e_bias, expert: ExpertFetch,
     else:
         shared_out = np.zeros((n, H), np.float64)
     contrib = np.zeros((n, k, H), np.float64)
-    for e in np.unique(idx):
+    experts = [int(e) for e in np.unique(idx)]
+    jobs = ((xq[np.nonzero(idx == e)[0]], *expert(e)) for e in experts)
+    for e, out in zip(experts, (run_experts or _run_serial)(swiglu_mx, jobs)):
         rows, slots = np.nonzero(idx == e)
-        out = swiglu_mx(xq[rows], *expert(int(e)))
         contrib[rows, slots] = w[rows, slots][:, None] * out
     output = np.zeros((n, H), np.float64)
     for j in range(k):

@@ -21,11 +21,12 @@
  *    added with their weights; the shared expert runs for every token; the
  *    layer returns shared + routed.  § 06: the bias only steers selection
  *    (nudged by load); weights come from the unbiased score.
- *  - Points the pages leave open (group score = sum of the two largest biased
- *    scores of the group, contiguous groups, exclusion of dropped groups,
- *    lower index wins ties, normalisation then routed_scaling_factor) follow
- *    the DeepSeek-V3 noaux_tc definition; each is listed with its reading in
- *    the design notes.
+ *  - Points the pages leave open follow the DeepSeek-V3 noaux_tc definition:
+ *    the group score is the sum of the two largest biased scores of the group;
+ *    groups are contiguous blocks of E / n_group experts; experts of dropped
+ *    groups are excluded from the top-k (not given a score of 0); the lower
+ *    index wins ties; the weights are normalised (when norm_topk_prob) and then
+ *    multiplied by routed_scaling_factor.
  */
 #include <math.h>
 #include <stdint.h>

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 (MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
- MOE_ERR_STATIC_LIMIT) = range(7)
+ MOE_ERR_STATIC_LIMIT, MOE_ERR_DEVICE_CHECK) = range(8)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 
 
@@ -275,14 +275,6 @@ def y_perm_scale_cols(H: int) -> int:
     return (H // 32 + 7) // 8 * 8
 
 
-def decode_y_perm(y_perm: torch.Tensor, y_perm_scale: torch.Tensor) -> torch.Tensor:
-    """fp32 values of a block-scaled y_perm: fp16 * 2^(code - 141), one code per 32 columns."""
-    rows, H = y_perm.shape
-    codes = y_perm_scale[:, : H // 32].to(torch.int32)
-    f = torch.ldexp(torch.ones_like(codes, dtype=torch.float32), codes - 141)
-    return (y_perm.float().view(rows, H // 32, 32) * f[:, :, None]).view(rows, H)
-
-
 def moe_experts(cfg, T, x, x_perm, expert_offsets, perm_src, topk_w, w_gate, w_up, w_down,
                 ws_gate, ws_up, ws_down, h_routed, h_shared, y_perm, y_perm_scale, stream=None):
     d = _Dims(cfg, T)
@@ -375,10 +367,11 @@ def moe_forward(cfg, x, router_w, e_bias, w_gate, w_up, w_down, ws_gate, ws_up, 
 
 
 def device_status(stream=None) -> int:
-    """Synchronise the stream and return (then clear) the device error word."""
+    """Synchronise the stream and return (then clear) the device error word:
+    0, a bounded-wait code, or a 0x4xx code of a skipped out-of-range index."""
     word = ctypes.c_int32(0)
     rc = lib().moe_device_status(_stream(stream), ctypes.byref(word))
-    if rc not in (MOE_OK, MOE_ERR_TIMEOUT):
+    if rc not in (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_CHECK):
         raise MoEError("moe_device_status", rc)
     return word.value
 

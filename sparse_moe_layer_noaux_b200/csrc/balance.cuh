@@ -6,6 +6,8 @@
 #pragma once
 #include <cstdint>
 
+#include "device_status.cuh"
+
 namespace moe {
 
 // One block: shared-memory histogram of the routing, then the update (E <= 256).
@@ -15,7 +17,13 @@ __global__ void __launch_bounds__(1024) bias_update_kernel(const int32_t* __rest
     __shared__ int cnt[256];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
-    for (int64_t q = threadIdx.x; q < n; q += blockDim.x) atomicAdd(&cnt[topk_idx[q]], 1);
+    // Routing indices come from the caller: one outside [0, E) is not counted and
+    // is recorded in the device error word.
+    for (int64_t q = threadIdx.x; q < n; q += blockDim.x) {
+        const int e = topk_idx[q];
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&cnt[e], 1);
+        else record_error(kErrExpertId);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         // load_e against the mean n / E, compared exactly as load_e * E against n.

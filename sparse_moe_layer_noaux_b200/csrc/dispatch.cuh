@@ -1,6 +1,7 @@
-// Token -> expert dispatch: the per-expert mask and gather of "The Evolving
-// Transformer · 07", § 02 (MoE.forward: mask = indices[:, :, k] == i; x[mask]),
-// done for all experts at once as a stable counting sort:
+// Token -> expert dispatch.  The teaching code of "The Evolving Transformer · 07"
+// (§ 02, MoE.forward) selects, expert by expert and slot by slot, the tokens
+// routed to that expert and gathers their rows; here the same grouping is done
+// for all experts at once as a stable counting sort:
 //   1. count:  per block of kDispTok tokens, how many slots go to each expert;
 //   2. scan:   per expert, each block's starting row inside the expert's segment
 //              and the expert's total (one warp per expert);
@@ -9,9 +10,14 @@
 //              (ascending (t, j)) -> row_of / perm_src;
 //   4. scatter: each token's row is read once from x and written to its k rows
 //              of x_perm with 16-byte vector stores.
+// Routing indices come from the caller (moe_dispatch takes topk_idx as an
+// argument): an index outside [0, E) is skipped — not counted, no row, row_of = -1
+// — and recorded in the device error word (kErrExpertId).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+
+#include "device_status.cuh"
 
 namespace moe {
 
@@ -27,7 +33,11 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(
     const int t0 = blockIdx.x * kDispTok;
     const int n = min(kDispTok, T - t0) * K;
     const int32_t* idx = topk_idx + (int64_t)t0 * K;
-    for (int q = threadIdx.x; q < n; q += blockDim.x) atomicAdd(&cnt[idx[q]], 1);
+    for (int q = threadIdx.x; q < n; q += blockDim.x) {
+        const int e = idx[q];
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&cnt[e], 1);
+        else record_error(kErrExpertId);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         block_counts[(int64_t)e * gridDim.x + blockIdx.x] = cnt[e];
@@ -98,8 +108,10 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
 
     for (int r0 = 0; r0 < n; r0 += kDispThreads) {
         const int q = r0 + tid;
-        const bool valid = q < n;
-        const int e = valid ? topk_idx[q0 + q] : -1 - lane;  // invalid lanes never match
+        const bool in_range = q < n;
+        int e = in_range ? topk_idx[q0 + q] : -1;
+        const bool valid = in_range && static_cast<unsigned>(e) < static_cast<unsigned>(E);
+        if (!valid) e = -1 - lane;  // lanes without a valid expert never match another lane
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int lrank = __popc(peers & lt_mask);
         const bool leader = lrank == 0;
@@ -118,12 +130,15 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
         if (valid) {
             row_of[q0 + q] = row;
             perm_src[row] = (int32_t)(q0 + q);
+        } else if (in_range) {
+            row_of[q0 + q] = -1;
         }
     }
 }
 
 // Row copy: block (t, c) moves 16-byte slices [256 c, 256 c + 256) of token t's
-// row; each slice is loaded once and stored to the token's k rows of x_perm.
+// row; each slice is loaded once and stored to the token's k rows of x_perm
+// (slots the place step left without a row, row_of = -1, are skipped).
 // The grid is T x ceil(H / 2048) blocks, so small batches still spread over
 // every SM.
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const __nv_bfloat16* __restrict__ x,
@@ -136,7 +151,8 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const __nv_bfloat
     const int c = blockIdx.y * 256 + threadIdx.x;
     if (c >= H / 8) return;
     const uint4 v = reinterpret_cast<const uint4*>(x + (int64_t)t * H)[c];
-    for (int j = 0; j < K; ++j) reinterpret_cast<uint4*>(x_perm + (int64_t)rows[j] * H)[c] = v;
+    for (int j = 0; j < K; ++j)
+        if (rows[j] >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)rows[j] * H)[c] = v;
 }
 
 }  // namespace moe

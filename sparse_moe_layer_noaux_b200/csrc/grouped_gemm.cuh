@@ -16,8 +16,9 @@
 //            block of x meets the three planes back to back, so its second and
 //            third loads come from L2 and x streams from HBM once; N = E rounded
 //            up to 16), fp32 output.
-// ("The Evolving Transformer · 07", § 02: expert(x[mask]) is a SwiGLU FFN; its
-// output is multiplied by the routing weight.)
+// ("The Evolving Transformer · 07", § 02: each routed expert is a SwiGLU FFN
+// applied to the tokens sent to it; its output is multiplied by the routing
+// weight.)
 //
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
 // the MMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
@@ -30,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "device_status.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -58,10 +60,19 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 #endif
 constexpr int kSwapMaxRows = MOE_SWAP_MAX_ROWS;
 
-enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
+// A segment with at least this many 128-row tiles is walked row tile by row tile
+// (all column tiles of a row tile in a row), so its A rows are read from HBM
+// once while the segment's weight tiles are reused from L2; smaller segments walk
+// column tile by column tile (the row tiles of a column share its weight tile and
+// the segment's A rows stay in L2).  At the V3 shape the shared expert's 16384
+// token rows are 235 MB of A: walked column-major they would be re-read from HBM
+// once per column tile.
+#ifndef MOE_ROW_MAJOR_MIN_ROW_TILES
+#define MOE_ROW_MAJOR_MIN_ROW_TILES 16
+#endif
+constexpr int kRowMajorMinRowTiles = MOE_ROW_MAJOR_MIN_ROW_TILES;
 
-// Device error word (set by a bounded wait that gave up; read by the host).
-__device__ unsigned int g_moe_error;
+enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
 
 struct GemmParams {
     const int32_t* offsets;      // [E+1] routed row offsets
@@ -85,6 +96,8 @@ struct GemmParams {
     uint32_t b_tile_bytes;                // bytes one B tile load brings in
     int b_plane_rows;                     // kLogits: rows of one plane in the B map (E)
     int allow_swap;                       // compute partial row tiles transposed
+    int64_t max_rows;                     // routed row space: segments must lie in [0, max_rows)
+    int64_t n_slots;                      // kDown: entries of topk_w (perm_src values < n_slots)
 };
 
 struct TileInfo {
@@ -98,6 +111,7 @@ struct TileInfo {
     int r;          // valid rows in this tile (1..128)
     int swap;       // 1: computed transposed (weights as the M operand, see below)
     int rpad;       // swap: token columns of the MMA, r rounded up to 16
+    int row_major;  // tiles of this segment are walked row tile by row tile
 };
 
 struct GemmSmem {
@@ -114,8 +128,6 @@ struct GemmSmem {
     int seg_rows[kMaxSeg];
     int tile_start[kMaxSeg + 1];
 };
-
-__device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_moe_error, 0u, code); }
 
 // Block-scaled fp16: a block of 32 values whose largest magnitude has biased
 // fp32 exponent E gets the code c = clamp(E, 15, 254); values are stored as
@@ -161,8 +173,15 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem& s, const GemmPar
     ti.row0 = s.seg_row0[lo];
     const int mt = (ti.rows + kBM - 1) / kBM;
     const int local = tile - s.tile_start[lo];
-    ti.n = local / mt;
-    ti.m = local - ti.n * mt;
+    ti.row_major = mt >= kRowMajorMinRowTiles ? 1 : 0;
+    if (ti.row_major) {
+        const int nt = ti.routed ? p.n_tiles_routed : p.n_tiles_shared;
+        ti.m = local / nt;
+        ti.n = local - ti.m * nt;
+    } else {
+        ti.n = local / mt;
+        ti.m = local - ti.n * mt;
+    }
     ti.kb = ti.routed ? p.kb_routed : p.kb_shared;
     ti.r = min(kBM, ti.rows - ti.m * kBM);
     // A segment that fits in one partial row tile (decode-sized: a few tokens per
@@ -251,7 +270,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
                 const int e = sg - p.has_shared;
                 row0 = p.offsets[e];
-                rows = p.offsets[e + 1] - row0;
+                rows = checked_segment_rows(row0, p.offsets[e + 1] - row0, p.max_rows, 1);
                 ntl = p.n_tiles_routed;
             }
             S.seg_rows[sg] = rows;
@@ -288,10 +307,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            // Activation tiles are re-read by every column tile of their segment:
-            // keep them in L2 preferentially.  Weight tiles are shared by the CTAs
-            // working on the segment's row tiles at the same time: default policy.
-            const uint64_t pol_a = ptx::policy_evict_last();
+            // Column-major segments: the A rows are re-read by every column tile,
+            // so they are kept in L2 preferentially (weight tiles are shared by the
+            // CTAs on the segment's row tiles at the same time: default policy).
+            // Row-major segments: the weight tiles are re-read by every row tile,
+            // so those are kept instead.
+            const uint64_t pol_keep = ptx::policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0, issued_parity = 0;
@@ -317,17 +338,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         // loaded for the three planes in a row (L2 hits after the first).
                         const int plane = kb % 3;
                         const int kcol = (kb / 3) * kBK;
-                        ptx::tma_load_2d(a_dst, mA, full, kcol, a_row, pol_a);
+                        ptx::tma_load_2d(a_dst, mA, full, kcol, a_row, pol_keep);
                         ptx::tma_load_2d(b_dst, mB, full, kcol, plane * p.b_plane_rows);
-                    } else if (kEpi == kSwiGLU) {
-                        ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
-                        const int b_row = b_base + ti.n * (kBN / 2);
-                        ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
-                        ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row);
                     } else {
-                        ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_a);
-                        const int b_row = b_base + ti.n * kBN;
-                        ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
+                        const int b_row = b_base + ti.n * (kEpi == kSwiGLU ? kBN / 2 : kBN);
+                        if (ti.row_major) {
+                            ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row);
+                            ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row, pol_keep);
+                            if (kEpi == kSwiGLU)
+                                ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row, pol_keep);
+                        } else {
+                            ptx::tma_load_2d(a_dst, mA, full, kb * kBK, a_row, pol_keep);
+                            ptx::tma_load_2d(b_dst, mB, full, kb * kBK, b_row);
+                            if (kEpi == kSwiGLU) ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBK, b_row);
+                        }
                     }
                     issued_mask |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -455,7 +479,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int c = 0; c * 32 < ti.r; ++c) {
                     // Routing weight of token row c*32 + lane, shared across the warp below.
                     float wl = 1.0f;
-                    if (ti.routed && c * 32 + lane < ti.r) wl = p.topk_w[p.perm_src[tile_row0 + c * 32 + lane]];
+                    if (ti.routed && c * 32 + lane < ti.r)
+                        wl = row_weight(p.perm_src, p.topk_w, tile_row0 + c * 32 + lane, p.n_slots);
                     const int jmax = min(32, ti.r - c * 32);
 #pragma unroll 1
                     for (int hh = 0; hh < 2; ++hh) {
@@ -526,7 +551,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
                 __half* hs = reinterpret_cast<__half*>(stage);
                 float wrow = 1.0f;
-                if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
+                if (ti.routed && row_ok) wrow = row_weight(p.perm_src, p.topk_w, grow, p.n_slots);
                 uint32_t codes[kBN / 32];
 #pragma unroll
                 for (int c = 0; c < kBN / 32; ++c) {

@@ -65,6 +65,8 @@ struct GemmParamsMx {
     int64_t scale_ld;
     const int32_t* perm_src;     // kDown: routed row -> slot
     const float* topk_w;
+    int64_t max_rows;            // padded routed row space Rp: segments must lie in [0, Rp)
+    int64_t n_slots;             // kDown: entries of topk_w (perm_src values < n_slots)
 };
 
 struct GemmSmemMx {
@@ -101,8 +103,15 @@ __device__ __forceinline__ TileInfo decode_tile_mx(const GemmSmemMx& s, const Ge
     ti.row0 = s.seg_row0[lo];
     const int mt = (ti.rows + kBM - 1) / kBM;
     const int local = tile - s.tile_start[lo];
-    ti.n = local / mt;
-    ti.m = local - ti.n * mt;
+    ti.row_major = mt >= kRowMajorMinRowTiles ? 1 : 0;
+    if (ti.row_major) {
+        const int nt = ti.routed ? p.n_tiles_routed : p.n_tiles_shared;
+        ti.m = local / nt;
+        ti.n = local - ti.m * nt;
+    } else {
+        ti.n = local / mt;
+        ti.m = local - ti.n * mt;
+    }
     ti.kb = ti.routed ? p.kb_routed : p.kb_shared;
     ti.r = min(kBM, ti.rows - ti.m * kBM);
     ti.swap = 0;
@@ -170,7 +179,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
                 const int e = sg - p.has_shared;
                 row0 = p.offsets[e];
-                rows = p.counts[e];
+                rows = checked_segment_rows(row0, p.counts[e], p.max_rows, kMxAtomRows);
                 ntl = p.n_tiles_routed;
             }
             S.seg_rows[sg] = rows;
@@ -207,7 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         // ================= TMA producer =================
         if (lane == 0) {
-            const uint64_t pol_a = ptx::policy_evict_last();
+            // L2 policy as in the bf16 kernel: keep what the tile order re-reads.
+            const uint64_t pol_keep = ptx::policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0, issued_parity = 0;
@@ -247,9 +257,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t a_dst = ptx::smem_u32(smemA + stage * kTileABytes);
                     const uint32_t b_dst = ptx::smem_u32(smemB + stage * kTileBBytes);
                     const uint32_t sf_dst = ptx::smem_u32(smemSF + stage * kSfStageBytes);
-                    ptx::tma_load_2d(a_dst, mA, full, kb * kBKq, a_row, pol_a);
-                    ptx::tma_load_2d(b_dst, mB, full, kb * kBKq, b_row);
-                    if (kEpi == kSwiGLU) ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBKq, b_row);
+                    if (ti.row_major) {
+                        ptx::tma_load_2d(a_dst, mA, full, kb * kBKq, a_row);
+                        ptx::tma_load_2d(b_dst, mB, full, kb * kBKq, b_row, pol_keep);
+                        if (kEpi == kSwiGLU)
+                            ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBKq, b_row, pol_keep);
+                    } else {
+                        ptx::tma_load_2d(a_dst, mA, full, kb * kBKq, a_row, pol_keep);
+                        ptx::tma_load_2d(b_dst, mB, full, kb * kBKq, b_row);
+                        if (kEpi == kSwiGLU) ptx::tma_load_2d(b_dst + kTileBBytes / 2, mB2, full, kb * kBKq, b_row);
+                    }
                     ptx::bulk_load(sf_dst, sfa + kb * kMxAtomBytes, kMxAtomBytes, full);
                     ptx::bulk_load(sf_dst + kSfaBytes, sfb0 + kb * kMxAtomBytes, kMxAtomBytes, full);
                     ptx::bulk_load(sf_dst + kSfaBytes + kMxAtomBytes, sfb1 + kb * kMxAtomBytes, kMxAtomBytes, full);
@@ -394,7 +411,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int64_t ld = ti.routed ? p.ld_routed : p.ld_shared;
                 __half* hs = reinterpret_cast<__half*>(stage);
                 float wrow = 1.0f;
-                if (ti.routed && row_ok) wrow = p.topk_w[p.perm_src[grow]];
+                if (ti.routed && row_ok) wrow = row_weight(p.perm_src, p.topk_w, grow, p.n_slots);
                 const int first = acc ? 0 : kBN / 32 - 1;
                 uint32_t codes_lo = 0, codes_hi = 0;
 #pragma unroll 1

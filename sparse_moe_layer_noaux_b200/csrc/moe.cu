@@ -17,7 +17,6 @@
 #include "combine.cuh"
 #include "dispatch.cuh"
 #include "grouped_gemm.cuh"
-#include "grouped_gemm_2sm.cuh"
 #include "grouped_gemm_mx.cuh"
 #include "grouped_gemm_bwd.cuh"
 #include "bwd_small.cuh"
@@ -91,20 +90,8 @@ RouterPlan plan_router(int T, int E, int H) {
 constexpr size_t kGemmSmemBytes =
     1024 + kStages * (kTileABytes + kTileBBytes) + kStageBytes + sizeof(GemmSmem);
 static_assert(kGemmSmemBytes <= 227 * 1024, "expert GEMM shared memory exceeds the 227 KB per-CTA limit");
-static_assert(kGemm2SmemBytes <= 227 * 1024, "pair GEMM shared memory exceeds the 227 KB per-CTA limit");
 static_assert(kGemmMxSmemBytes <= 227 * 1024, "MXFP8 GEMM shared memory exceeds the 227 KB per-CTA limit");
 static_assert(kGemmBwdSmemBytes <= 227 * 1024, "backward GEMM shared memory exceeds the 227 KB per-CTA limit");
-
-// The CTA-pair GEMMs (256-row tiles) can take prefill-sized batches (expert
-// segments averaging at least 128 rows).  They are built but off by default:
-// measured on B200 under the 1000 W cap they do ~3% more work per clock than the
-// single-CTA kernel yet run at ~15% lower SM clocks, so they are slower end to
-// end.  The environment variable MOE_PAIR_GEMM=1 (read at each call) selects them.
-inline bool use_pair_kernel(int64_t R, int64_t E, int num_sms) {
-    const char* v = std::getenv("MOE_PAIR_GEMM");
-    const bool on = v != nullptr && v[0] == '1';
-    return on && num_sms >= 2 && R >= 128 * E;
-}
 
 // --------------------------------------------------------------- device info
 struct DeviceInfo {
@@ -129,10 +116,6 @@ int device_info(DeviceInfo** out) {
                                  smem) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_kernel<kLogits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess ||
-            cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess ||
-            cudaFuncSetAttribute(grouped_gemm_2sm_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kGemm2SmemBytes)) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_mx_kernel<kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGemmMxSmemBytes)) != cudaSuccess ||
             cudaFuncSetAttribute(grouped_gemm_mx_kernel<kDown>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -364,18 +347,7 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
-    if (use_pair_kernel(R, E, num_sms)) {
-        // Pair tiles: each CTA loads 64 gate rows and 64 up rows of the 128-column tile.
-        if (!make_map(&b_r, w_gate, E * I, H, 64) || !make_map(&b2_r, w_up, E * I, H, 64)) return MOE_ERR_CUDA;
-        if (has_shared && (!make_map(&b_s, ws_gate, SI, H, 64) || !make_map(&b2_s, ws_up, SI, H, 64)))
-            return MOE_ERR_CUDA;
-        if (!has_shared) { b_s = b_r; b2_s = b2_r; }
-        const int64_t grid = 2 * (num_sms / 2);
-        grouped_gemm_2sm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemm2SmemBytes, st>>>(
-            a_r, a_s, b_r, b2_r, b_s, b2_s, p);
-        count_launch();
-        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-    }
+    p.max_rows = R;
     const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -423,17 +395,8 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
-    if (use_pair_kernel(R, E, num_sms)) {
-        // Pair tiles: each CTA loads its 128 of the 256 output columns' weight rows.
-        if (!make_map(&b_r, w_down, E * H, I, 128)) return MOE_ERR_CUDA;
-        if (has_shared && !make_map(&b_s, ws_down, H, SI, 128)) return MOE_ERR_CUDA;
-        if (!has_shared) b_s = b_r;
-        const int64_t grid = 2 * (num_sms / 2);
-        grouped_gemm_2sm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemm2SmemBytes, st>>>(
-            a_r, a_s, b_r, b_r, b_s, b_s, p);
-        count_launch();
-        return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-    }
+    p.max_rows = R;
+    p.n_slots = R;
     const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);
@@ -441,6 +404,8 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Routed rows of y_perm are [0, shared_row0) (T*k, or the padded row space of
+// the MXFP8 and training paths); the shared rows follow.
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const void* y_scale,
                    const int32_t* row_of, void* y, int y_dtype, cudaStream_t st, int64_t shared_row0 = -1) {
     if (shared_row0 < 0) shared_row0 = T * c->num_experts_per_tok;
@@ -450,12 +415,12 @@ int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const voi
         combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
             static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
             row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
-            static_cast<__nv_bfloat16*>(y));
+            shared_row0, static_cast<__nv_bfloat16*>(y));
     else
         combine_kernel<float><<<g, 256, 0, st>>>(
             static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
             row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
-            static_cast<float*>(y));
+            shared_row0, static_cast<float*>(y));
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -662,6 +627,7 @@ int launch_gate_up_mx(const moe_config* c, int64_t T, const MxBuffers& w, const 
     p.hsf_shared = w.hq_shared_sf;
     p.hsf_katoms_routed = static_cast<int>(I / kMxAtomK);
     p.hsf_katoms_shared = static_cast<int>(SI / kMxAtomK);
+    p.max_rows = w.rp;
     const int64_t grid = gemm_grid_mx(T, w.rp, I > SI ? I / (kBN / 2) : SI / (kBN / 2), has_shared, num_sms);
     grouped_gemm_mx_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -713,6 +679,8 @@ int launch_down_mx(const moe_config* c, int64_t T, const MxBuffers& w, const moe
     p.scale_shared = w.y_scale + w.rp * p.scale_ld;
     p.perm_src = w.perm_src;
     p.topk_w = topk_w;
+    p.max_rows = w.rp;
+    p.n_slots = T * c->num_experts_per_tok;
     const int64_t grid = gemm_grid_mx(T, w.rp, H / kBN, has_shared, num_sms);
     grouped_gemm_mx_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);
@@ -1667,6 +1635,7 @@ const char* moe_status_string(int status) {
         case MOE_ERR_WORKSPACE: return "workspace missing or too small";
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case MOE_ERR_DEVICE_CHECK: return "a device-side check found an index out of range (entry skipped)";
         case MOE_ERR_STATIC_LIMIT:
             return "size exceeds the fixed scratch of the no-allocation entry point "
                    "(2 * ceil(T / 32) * n_routed_experts + n_routed_experts must be <= 263168)";
@@ -1682,7 +1651,8 @@ int moe_device_status(void* stream, int32_t* device_error) {
     if (cudaMemcpyFromSymbol(&word, g_moe_error, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
     if (word != 0 && cudaMemcpyToSymbol(g_moe_error, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
     *device_error = static_cast<int32_t>(word);
-    return word ? MOE_ERR_TIMEOUT : MOE_OK;
+    if (word == 0) return MOE_OK;
+    return (word >= kErrCheckFirst && word <= kErrCheckLast) ? MOE_ERR_DEVICE_CHECK : MOE_ERR_TIMEOUT;
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }

@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_mx_kernel(
     const bool writer = (threadIdx.x & 15) == 0;
     for (int j = 0; j < K; ++j) {
         const int64_t r = rows[j];
+        if (r < 0) continue;  // a slot with an out-of-range expert index (skipped by the place step)
         *reinterpret_cast<uint2*>(xq_perm + r * H + col) = qv;
         if (writer) *reinterpret_cast<uint32_t*>(xq_perm_sf + mx_sf_word_offset(r, kb, k_atoms)) = word;
     }

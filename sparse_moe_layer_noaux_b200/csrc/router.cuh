@@ -159,6 +159,11 @@ __device__ __forceinline__ bool route_beats(float va, int ia, float vb, int ib) 
     return va > vb || (va == vb && ia < ib);
 }
 
+// NaN (from a NaN in x, router_w or e_bias, or +inf - inf in a group score) is
+// ranked as -inf, so the (value, index) order stays total: exactly topk_group
+// groups are kept and k distinct valid experts are chosen whatever the inputs.
+__device__ __forceinline__ float route_key(float v) { return v == v ? v : -CUDART_INF_F; }
+
 template <int EPL>
 __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
     const int lane = threadIdx.x & 31;
@@ -183,8 +188,10 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         }
     }
 
+    // avail bit i: slot i holds an expert that may still be chosen.
     float s[EPL], cand[EPL];
     int grp[EPL];  // group of this lane's expert in slot i (-1: no expert)
+    unsigned avail = 0;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
@@ -193,7 +200,8 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         grp[i] = e < E ? e / gsize : -1;
         if (e < E) {
             s[i] = 1.0f / (1.0f + expf(-l[i]));
-            cand[i] = s[i] + a.bias[e];  // biased score b_e
+            cand[i] = route_key(s[i] + a.bias[e]);  // biased score b_e
+            avail |= 1u << i;
         }
     }
 
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
             m1 = n1;
             m2 = n2;
         }
-        const float gs = gsize >= 2 ? m1 + m2 : m1;
+        const float gs = route_key(gsize >= 2 ? m1 + m2 : m1);
         if (lane == g) my_gscore = gs;
     }
 
@@ -233,8 +241,10 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
     // Experts of dropped groups are excluded from the top-k.
 #pragma unroll
     for (int i = 0; i < EPL; ++i)
-        if (grp[i] < 0 || !((kept >> grp[i]) & 1u)) cand[i] = -CUDART_INF_F;
+        if (grp[i] < 0 || !((kept >> grp[i]) & 1u)) avail &= ~(1u << i);
 
+    // k rounds of a warp arg-max over the available experts.  The kept groups hold
+    // topk_group * E / n_group >= k experts, so every round finds one (bi < E).
     float my_s = 0.f;
     int my_idx = 0;
     for (int j = 0; j < a.K; ++j) {
@@ -243,7 +253,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             const int e = lane + 32 * i;
-            if (e < E && cand[i] != -CUDART_INF_F && route_beats(cand[i], e, bv, bi)) {
+            if (((avail >> i) & 1u) && route_beats(cand[i], e, bv, bi)) {
                 bv = cand[i];
                 bi = e;
                 bs = s[i];
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         }
 #pragma unroll
         for (int i = 0; i < EPL; ++i)
-            if (lane + 32 * i == bi) cand[i] = -CUDART_INF_F;
+            if (lane + 32 * i == bi) avail &= ~(1u << i);
         if (lane == j) {
             my_s = bs;
             my_idx = bi;

@@ -139,6 +139,58 @@ def assert_bf16_rounded(t, ref, what=""):
     assert not bool(bad.any()), (what, int(bad.sum()), float((t - ref).abs().max()), float(rms))
 
 
+def targeted_rows(shape, idx, n_min: int = 256, seed: int = 0, swap_max_rows: int = 112,
+                  n_partial_experts: int = 16, n_small_segments: int = 4):
+    """Token rows for a sampled full-size check, aimed at the tiles most likely to
+    hide an indexing mistake in the expert GEMMs (rows of an expert segment are
+    the expert's (token, slot) entries in ascending (t, j) order, 128 per tile):
+      * two rows from the last, partial 128-row tile of each of the
+        `n_partial_experts` largest segments whose length is not a multiple of 128;
+      * every row of the `n_small_segments` smallest non-empty segments of at
+        most `swap_max_rows` rows (those tiles run transposed);
+      * 16 rows of the most loaded expert, its last rows included;
+      * the first and last token, then seeded random rows up to `n_min`.
+    Returns (sorted token array, dict of what was targeted)."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    order = np.argsort(flat, kind="stable")          # slot indices, expert-major
+    counts = np.bincount(flat, minlength=shape.E)
+    starts = np.concatenate([[0], np.cumsum(counts)])
+    tokens_of = lambda e: order[starts[e]:starts[e + 1]] // k  # noqa: E731
+    rows = {0, T - 1}
+    partial = [e for e in np.argsort(-counts, kind="stable") if counts[e] % 128 and counts[e] > 0]
+    partial = [int(e) for e in partial[:n_partial_experts]]
+    for e in partial:
+        toks = tokens_of(e)
+        last_tile = toks[(len(toks) - 1) // 128 * 128:]
+        rows |= {int(last_tile[0]), int(last_tile[-1])}
+    small = [int(e) for e in np.argsort(counts, kind="stable") if 0 < counts[e] <= swap_max_rows]
+    small = small[:n_small_segments]
+    for e in small:
+        rows |= set(tokens_of(e).tolist())
+    hot = int(counts.argmax())
+    toks = tokens_of(hot)
+    rows |= set(toks[:8].tolist()) | set(toks[-8:].tolist())
+    rng = np.random.default_rng(seed)
+    free = np.setdiff1d(np.arange(T), np.fromiter(rows, dtype=np.int64))
+    extra = max(0, n_min - len(rows))
+    if extra and len(free):
+        rows |= set(rng.choice(free, min(extra, len(free)), replace=False).tolist())
+    info = {"partial_tile_experts": partial, "small_segments": {e: int(counts[e]) for e in small},
+            "hot_expert": hot, "hot_rows": int(counts[hot])}
+    return np.array(sorted(rows)), info
+
+
+def decode_y_perm(y_perm: torch.Tensor, y_perm_scale: torch.Tensor) -> torch.Tensor:
+    """fp32 values of a block-scaled y_perm (the library's expert-output format,
+    include/moe.h): fp16 * 2^(code - 141), one code per 32 columns."""
+    rows, H = y_perm.shape
+    codes = y_perm_scale[:, : H // 32].to(torch.int32)
+    f = torch.ldexp(torch.ones_like(codes, dtype=torch.float32), codes - 141)
+    return (y_perm.float().view(rows, H // 32, 32) * f[:, :, None]).view(rows, H)
+
+
 def device_expert_fetch(inp):
     """Oracle expert fetcher copying one expert's bf16 bits from the device at a time."""
     def fetch(e):
@@ -153,10 +205,11 @@ def shared_bits(inp, shape):
 
 
 def oracle_layer_rows(shape, inp, rows, gpu_idx=None, scores=None, ref_idx=None, ref_w=None,
-                      margin=None, layer=None):
+                      margin=None, layer=None, parallel: bool = False):
     """Oracle output for the given token rows.  Where the GPU picked a different
     (near-tie) expert set, that row is computed on the GPU's set.  ``layer`` is the
-    oracle layer function (default: the bf16 one; oracle.moe_layer_mx for MXFP8)."""
+    oracle layer function (default: the bf16 one; oracle.moe_layer_mx for MXFP8).
+    ``parallel`` runs the per-expert calls in spawned processes (same arithmetic)."""
     x_bits = bf16_bits(inp["x"][torch.as_tensor(rows, device=inp["x"].device)])
     rw = inp["router_w"].cpu().numpy()
     bias = inp["e_bias"].cpu().numpy()
@@ -170,6 +223,10 @@ def oracle_layer_rows(shape, inp, rows, gpu_idx=None, scores=None, ref_idx=None,
                 use_idx[i] = gpu_idx[t]
                 use_w[i] = weights_for_set(shape, scores[t], gpu_idx[t])
         routing = (use_idx, use_w)
+    run = None
+    if parallel:
+        from oracle.pool import ExpertRunner
+        run = ExpertRunner()
     y, *_ = (layer or oracle.moe_layer)(shape, x_bits, rw, bias, device_expert_fetch(inp),
-                                        shared_bits(inp, shape), routing=routing)
+                                        shared_bits(inp, shape), routing=routing, run_experts=run)
     return y

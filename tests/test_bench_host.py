@@ -33,11 +33,37 @@ def test_job_throughput_counts_every_rank_over_the_slowest():
     assert bench.max_over_ranks(3.5, 1) == 3.5
 
 
+def test_down_algorithmic_bytes_at_v3_prefill():
+    # Down weights of 220 touched + 1 shared expert, h read for T*(k+S) rows, block-
+    # scaled fp16 y_perm written for the T*k routed and T shared rows (2 bytes per
+    # value, 224 scale bytes per row at H = 7168).
+    s = V3_PREFILL
+    want = 221 * 7168 * 2048 * 2 + 16384 * 9 * 2048 * 2 + (16384 * 8 + 16384) * (2 * 7168 + 224)
+    assert bench.down_algorithmic_bytes(s, 220) == want
+
+
+def test_load_stats():
+    s = TINY
+    idx = torch.zeros((s.T, s.k), dtype=torch.int32)
+    idx[:, 1], idx[:, 2], idx[:, 3] = 1, 2, 3
+    st = bench.load_stats(s, idx.numpy(), histogram=True)
+    assert st["experts_touched"] == 4 and st["max_rows"] == s.T
+    assert st["max_over_mean"] == s.T / (s.T * s.k / s.E)
+    assert st["rows_per_expert"][:4] == [s.T] * 4 and sum(st["rows_per_expert"]) == s.T * s.k
+
+
 def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
-    for prec in ("bf16", "mxfp8"):
-        m = bench.MEASURED_TRAFFIC[(prec, "v3_prefill")]
-        assert bench.measured_traffic("v3_prefill", prec) == m["dram_read"] + m["dram_write"]
-        assert bench.measured_traffic("v3_decode", prec) is None     # never captured
+    sha = bench.gemm_sources_sha1("bf16")
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, ("bf16", "gate_up"),
+                        {"sources_sha1": sha, "case": "v3_e32", "dram_bytes": 1100, "algorithmic_bytes": 1000})
+    f = bench.traffic_fields("gate_up", 5000, "bf16")
+    assert f["traffic_ratio"] == 1.1 and f["traffic"] == 5500 and f["algorithmic_bytes"] == 5000
+    assert bench.traffic_fields("down", 5000, "bf16")["traffic"] is None     # never captured
     # A kernel source that changed since the capture voids the stored figure.
     monkeypatch.setitem(bench.GEMM_SOURCES, "bf16", ("grouped_gemm.cuh", "router.cuh"))
-    assert bench.measured_traffic("v3_prefill", "bf16") is None
+    assert bench.traffic_fields("gate_up", 5000, "bf16")["traffic"] is None
+
+
+def test_host_cpu_reports_cores():
+    h = bench.host_cpu()
+    assert h["host_cores"] >= 1

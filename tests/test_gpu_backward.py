@@ -86,11 +86,12 @@ def test_backward_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
-@pytest.mark.parametrize("shape,n_rows", [(MID, 16), (V3_PREFILL, 8), (V3_SKEWED, 8)],
+@pytest.mark.parametrize("shape,n_rows", [(MID, 64), (V3_PREFILL, 64), (V3_SKEWED, 64)],
                          ids=lambda v: getattr(v, "name", str(v)))
 def test_backward_full_size_sampled(shape, n_rows):
-    """dx of sampled rows, and the weight gradients of one sampled expert (all of its
-    rows) against the oracle's expert backward on the same operands."""
+    """dx of sampled rows, and the weight gradients of two experts (all of their
+    rows: a sampled one and the least loaded one) against the oracle's expert
+    backward on the same operands."""
     inp = make_inputs(shape, "cuda")
     grads, dy, idx = gpu_backward(shape, inp)
     rng = np.random.default_rng(shape.seed)
@@ -103,10 +104,16 @@ def test_backward_full_size_sampled(shape, n_rows):
     # One expert's weight gradients over all of its rows (for the skewed workload, where
     # a few experts take most rows and many take none: the one closest to 1024 rows).
     used, n_used = np.unique(idx, return_counts=True)
-    e = int(used[np.argmin(np.abs(n_used - 1024))]) if shape.name == "v3_skewed" else int(rng.choice(used))
+    e1 = int(used[np.argmin(np.abs(n_used - 1024))]) if shape.name == "v3_skewed" else int(rng.choice(used))
+    e2 = int(used[np.argmin(n_used)])
     if shape.name == "v3_skewed":
         unused = sorted(set(range(shape.E)) - set(used.tolist()))
         assert unused and all(not grads["w_down"][u].float().abs().sum().item() for u in unused[:8])
+    for e in dict.fromkeys((e1, e2)):
+        check_expert_weight_grads(shape, inp, grads, dy, idx, e)
+
+
+def check_expert_weight_grads(shape, inp, grads, dy, idx, e):
     toks, slots = np.nonzero(idx == e)
     xt = oracle.widen_bf16(bf16_bits(inp["x"]))[toks]
     rw = inp["router_w"].cpu().numpy().astype(np.float64)
@@ -119,7 +126,7 @@ def test_backward_full_size_sampled(shape, n_rows):
     _, dwg, dwu, dwd, _ = B._swiglu_backward(xt, wg, wu, wd, do)
     close(grads["w_gate"][e].float().cpu().numpy(), dwg, f"{shape.name} d_w_gate[{e}]")
     close(grads["w_up"][e].float().cpu().numpy(), dwu, f"{shape.name} d_w_up[{e}]")
-    close(grads["w_down"][e].float().cpu().numpy(), dwd, f"{shape.name} d_w_down[{e}]")
+    close(grads["w_down"][e].float().cpu().numpy(), dwd, f"{shape.name} d_w_down[{e}] ({len(toks)} rows)")
 
 
 def test_backward_empty_batch_gives_zero_weight_gradients():

@@ -157,17 +157,18 @@ def run_forward_mx(shape, inp, out_dtype=torch.float32):
     return y, idx, w, layer
 
 
-def check_layer(shape, inp, y, idx, w, rows):
+def check_layer(shape, inp, y, idx, w, rows, parallel=False):
     x_bits = bf16_bits(inp["x"])
     rw, bias = inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()
     ref_idx, ref_w, margin, scores = parity.oracle_route_all(shape, x_bits, rw, bias)
     rep = parity.compare_routing(shape, idx.cpu().numpy(), w.cpu().numpy(), ref_idx, ref_w, margin, scores, bias)
     assert not rep.mismatched_tokens, rep
     y_ref = parity.oracle_layer_rows(shape, inp, rows, idx.cpu().numpy(), scores, ref_idx, ref_w, margin,
-                                     layer=oracle.moe_layer_mx)
+                                     layer=oracle.moe_layer_mx, parallel=parallel)
     got = y.float().cpu().numpy()[rows]
     err = parity.output_errors(got, y_ref)
-    print(f"{shape.name} mxfp8: {err}, near ties {rep.near_ties}")
+    print(f"{shape.name} mxfp8: {len(rows)} rows, max|err|/RMS {err['max_abs_over_rms']:.2e}, "
+          f"rel L1 {err['rel_l1']:.2e}, near ties {rep.near_ties}")
     parity.assert_output_close(got, y_ref, shape.name)
     return err
 
@@ -179,13 +180,16 @@ def test_small_layer_mx_every_token(shape):
     check_layer(shape, inp, y, idx, w, np.arange(shape.T))
 
 
-@pytest.mark.parametrize("shape,n_rows", [(MID, 48), (V3_DECODE, 24), (V3_PREFILL, 12), (V3_SKEWED, 12)],
+@pytest.mark.parametrize("shape,n_rows", [(MID, 256), (V3_DECODE, 256), (V3_PREFILL, 256), (V3_SKEWED, 256)],
                          ids=lambda v: getattr(v, "name", str(v)))
 def test_full_size_layer_mx_sampled(shape, n_rows):
+    """A seeded sample aimed at the last partial 128-row tile of 16 experts, the
+    smallest segments and the most loaded expert (see parity.targeted_rows)."""
     inp = make_inputs(shape, "cuda")
     y, idx, w, layer = run_forward_mx(shape, inp)
-    rows = np.sort(np.random.default_rng(shape.seed).choice(shape.T, n_rows, replace=False))
-    check_layer(shape, inp, y, idx, w, rows)
+    rows, info = parity.targeted_rows(shape, idx.cpu().numpy(), n_min=n_rows, seed=shape.seed)
+    print(f"{shape.name} mxfp8 sample: {info}")
+    check_layer(shape, inp, y, idx, w, rows, parallel=True)
     del layer
 
 

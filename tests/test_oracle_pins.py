@@ -244,3 +244,25 @@ def test_layer_rows_are_independent(oracle_lib):
     rows = np.array([3, 17, 40, 63])
     y_sub, *_ = oracle_lib.moe_layer(shape, args[0][rows], args[1], args[2], fetch, shared)
     np.testing.assert_array_equal(y_sub, y_all[rows])
+
+
+def test_parallel_expert_runner_is_exact(oracle_lib):
+    """The process-pool runner used for large sampled checks only moves where each
+    expert's call runs: its layer output equals the serial oracle's bit for bit,
+    for the bf16 and the MXFP8 layer."""
+    from oracle.pool import ExpertRunner
+    shape = MoEShape("pool", T=40, hidden_size=256, n_routed_experts=16, n_group=4, topk_group=2,
+                     num_experts_per_tok=4, moe_intermediate_size=128, n_shared_experts=1,
+                     routed_scaling_factor=2.5, norm_topk_prob=True, seed=31)
+    inp = make_inputs(shape)
+    x = bf16_bits(inp["x"])
+    rw, bias = inp["router_w"].numpy(), inp["e_bias"].numpy()
+    fetch = oracle_lib.in_memory_experts(bf16_bits(inp["w_gate"]), bf16_bits(inp["w_up"]),
+                                         bf16_bits(inp["w_down"]))
+    shared = tuple(bf16_bits(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
+    runner = ExpertRunner(workers=2)
+    for layer in (oracle_lib.moe_layer, oracle_lib.moe_layer_mx):
+        y_serial, idx, w, _ = layer(shape, x, rw, bias, fetch, shared)
+        y_pool, idx2, w2, _ = layer(shape, x, rw, bias, fetch, shared, run_experts=runner)
+        assert np.array_equal(idx, idx2) and np.array_equal(w, w2)
+        assert np.array_equal(y_serial, y_pool), layer.__name__
