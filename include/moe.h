@@ -416,6 +416,63 @@ MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, 
                                void *d_w_gate, void *d_w_up, void *d_w_down, void *d_ws_gate, void *d_ws_up,
                                void *d_ws_down, void *context, size_t context_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Expert parallelism: the routed experts spread over `world` ranks (one GPU
+ * each), rank r holding experts [r * E/world, (r + 1) * E/world) in the layout
+ * of the single-GPU weights (w_gate, w_up [E/world, I, H], w_down
+ * [E/world, H, I]); the shared experts and the router are replicated.  ("DeepSeek-
+ * V3 notes" (knlb.dev), § infrastructure: expert parallelism with all-to-all
+ * dispatch and combine kernels; § architecture: each token is sent to a limited
+ * number of nodes — with contiguous expert blocks per rank and groups that do not
+ * straddle ranks, a token's rows reach at most topk_group ranks.)  One forward on
+ * each rank, for its own T tokens:
+ *   1. moe_route, moe_dispatch: rows in expert order, so the rows bound for rank d
+ *      are the contiguous block expert_offsets[d*E/world] .. expert_offsets[(d+1)*E/world];
+ *   2. moe_ep_pack: per-expert row counts and each row's routing weight;
+ *   3. the caller's all-to-all of the counts (E/world int32 to each rank), then of
+ *      the rows (bf16, H each) and their weights (fp32), with the block sizes from
+ *      the counts: rank r receives, from each source s in rank order, s's rows for
+ *      r's experts in expert order;
+ *   4. moe_ep_recv_offsets: the received counts [world][E/world] (source-major)
+ *      into segment offsets [E + 1];
+ *   5. moe_ep_experts: the grouped GEMMs over the received rows (segment
+ *      s * E/world + j runs with local expert j) and the shared experts over the
+ *      rank's own tokens;
+ *   6. the caller's all-to-all of the expert outputs back (the reverse block
+ *      sizes), into rows 0 .. T*k of a y_perm [T*k + T, H] whose rows T*k .. hold
+ *      the shared outputs, so the rows land where moe_dispatch put the inputs;
+ *   7. moe_combine.
+ * With world = 1 the collectives are copies and the result is moe_forward's.
+ * ------------------------------------------------------------------------ */
+
+/* expert_counts int32 [E] = rows of each expert segment (expert_offsets[e+1] -
+ * expert_offsets[e]); w_perm fp32 [T*k]: w_perm[r] = topk_w[perm_src[r]] for the
+ * rows of the segments, 0 past expert_offsets[E] (a perm_src entry outside
+ * [0, T*k) gives 0 and is recorded in the device error word). */
+MOE_API int moe_ep_pack(const moe_config *cfg, int64_t T, const int32_t *expert_offsets, const int32_t *perm_src,
+                        const float *topk_w, int32_t *expert_counts, float *w_perm, void *stream);
+
+/* recv_offsets int32 [E + 1] from recv_counts int32 [world][E/world]: the
+ * exclusive prefix sum in that order (a negative count is taken as 0 and
+ * recorded).  MOE_ERR_INVALID_ARG unless 1 <= world and world divides E. */
+MOE_API int moe_ep_recv_offsets(const moe_config *cfg, int32_t world, const int32_t *recv_counts,
+                                int32_t *recv_offsets, void *stream);
+
+/* The expert GEMMs of one rank:
+ *   received rows: x_recv bf16 [R, H] in segments recv_offsets [E + 1] (segment
+ *     s = source * E/world + j uses local expert j of w_gate / w_up / w_down),
+ *     each row's routing weight in w_recv fp32 [R];
+ *     h_recv bf16 [R, I]; y_recv [R, H] block-scaled fp16 with y_recv_scale
+ *     [R, ceil(H/256)*8] (the moe_experts format): y = w * down(silu(gate x) * up x);
+ *   the rank's own tokens: x bf16 [T, H] through the shared experts, h_shared
+ *     bf16 [T, S*I], y_shared [T, H] / y_shared_scale as above (unused when S = 0).
+ * A segment outside [0, R) gets no rows and is recorded in the device error word. */
+MOE_API int moe_ep_experts(const moe_config *cfg, int32_t world, int64_t T, const void *x, int64_t R,
+                           const void *x_recv, const int32_t *recv_offsets, const float *w_recv, const void *w_gate,
+                           const void *w_up, const void *w_down, const void *ws_gate, const void *ws_up,
+                           const void *ws_down, void *h_recv, void *h_shared, void *y_recv, void *y_recv_scale,
+                           void *y_shared, void *y_shared_scale, void *stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);
 

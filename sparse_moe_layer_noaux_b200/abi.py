@@ -113,13 +113,17 @@ def lib():
         L.moe_backward_train.argtypes = [cfgp, i64] + [_P] * 18 + [sz, _P]
         L.moe_forward_host.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, i64, _P, sz, _P]
         L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
+        L.moe_ep_pack.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P]
+        L.moe_ep_recv_offsets.argtypes = [cfgp, ctypes.c_int32, _P, _P, _P]
+        L.moe_ep_experts.argtypes = [cfgp, ctypes.c_int32, i64, _P, i64] + [_P] * 15 + [_P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
                    "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
                    "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward", "moe_workspace_size_host",
-                   "moe_forward_host", "moe_forward_train", "moe_backward_train"):
+                   "moe_forward_host", "moe_forward_train", "moe_backward_train", "moe_ep_pack",
+                   "moe_ep_recv_offsets", "moe_ep_experts"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -620,3 +624,60 @@ def moe_backward_train(cfg, x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, w
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(dy), _ptr(dx), _ptr(d_router_w), _ptr(d_w_gate),
         _ptr(d_w_up), _ptr(d_w_down), _ptr(d_ws_gate), _ptr(d_ws_up), _ptr(d_ws_down), _ptr(context),
         context.numel() * context.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- expert parallelism
+
+def moe_ep_pack(cfg, T, expert_offsets, perm_src, topk_w, expert_counts, w_perm, stream=None):
+    """Per-expert row counts [E] and each routed row's weight [T*k] (include/moe.h)."""
+    d = _Dims(cfg, T)
+    _req("expert_offsets", expert_offsets, _I32, d.E + 1)
+    _req("perm_src", perm_src, _I32, d.T * d.k)
+    _req("topk_w", topk_w, _F32, d.T * d.k)
+    _req("expert_counts", expert_counts, _I32, d.E)
+    _req("w_perm", w_perm, _F32, d.T * d.k)
+    _check("moe_ep_pack", lib().moe_ep_pack(ctypes.byref(_cfg(cfg)), T, _ptr(expert_offsets), _ptr(perm_src),
+                                            _ptr(topk_w), _ptr(expert_counts), _ptr(w_perm), _stream(stream)))
+
+
+def moe_ep_recv_offsets(cfg, world: int, recv_counts, recv_offsets, stream=None):
+    """Segment offsets [E+1] of the received rows from their counts [world, E/world]."""
+    E = int(_cfg(cfg).n_routed_experts)
+    _req("recv_counts", recv_counts, _I32, E)
+    _req("recv_offsets", recv_offsets, _I32, E + 1)
+    _check("moe_ep_recv_offsets", lib().moe_ep_recv_offsets(ctypes.byref(_cfg(cfg)), int(world), _ptr(recv_counts),
+                                                            _ptr(recv_offsets), _stream(stream)))
+
+
+def moe_ep_experts(cfg, world: int, T: int, x, x_recv, recv_offsets, w_recv, w_gate, w_up, w_down,
+                   ws_gate, ws_up, ws_down, h_recv, h_shared, y_recv, y_recv_scale, y_shared, y_shared_scale,
+                   stream=None):
+    """One rank's expert GEMMs over its received rows and the shared experts over its
+    own T tokens (include/moe.h).  Weights are the rank's E/world experts."""
+    d = _Dims(cfg, T)
+    if not isinstance(x_recv, torch.Tensor) or x_recv.dim() != 2 or x_recv.shape[1] != d.H:
+        raise ValueError(f"x_recv: expected shape [R, {d.H}]")
+    R = int(x_recv.shape[0])
+    if world < 1 or d.E % world:
+        raise ValueError(f"world {world} must divide n_routed_experts {d.E}")
+    El = d.E // world
+    shared = d.S > 0 and d.T > 0
+    _req("x", x, _BF16, d.T * d.H if shared else 0, optional=not shared)
+    _req("x_recv", x_recv, _BF16, R * d.H)
+    _req("recv_offsets", recv_offsets, _I32, d.E + 1)
+    _req("w_recv", w_recv, _F32, R)
+    _req("w_gate", w_gate, _BF16, El * d.I * d.H)
+    _req("w_up", w_up, _BF16, El * d.I * d.H)
+    _req("w_down", w_down, _BF16, El * d.I * d.H)
+    for name, t in (("ws_gate", ws_gate), ("ws_up", ws_up), ("ws_down", ws_down)):
+        _req(name, t, _BF16, d.SI * d.H, optional=not shared)
+    _req("h_recv", h_recv, _BF16, R * d.I)
+    _req("h_shared", h_shared, _BF16, d.T * d.SI, optional=not shared)
+    _req("y_recv", y_recv, _F16, R * d.H)
+    _req("y_recv_scale", y_recv_scale, _U8, R * d.scale_cols)
+    _req("y_shared", y_shared, _F16, d.T * d.H, optional=not shared)
+    _req("y_shared_scale", y_shared_scale, _U8, d.T * d.scale_cols, optional=not shared)
+    _check("moe_ep_experts", lib().moe_ep_experts(
+        ctypes.byref(_cfg(cfg)), int(world), T, _ptr(x), R, _ptr(x_recv), _ptr(recv_offsets), _ptr(w_recv),
+        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(h_recv),
+        _ptr(h_shared), _ptr(y_recv), _ptr(y_recv_scale), _ptr(y_shared), _ptr(y_shared_scale), _stream(stream)))

@@ -98,6 +98,7 @@ struct GemmParams {
     int allow_swap;                       // compute partial row tiles transposed
     int64_t max_rows;                     // routed row space: segments must lie in [0, max_rows)
     int64_t n_slots;                      // kDown: entries of topk_w (perm_src values < n_slots)
+    int expert_mod;                       // routed segment s uses expert s % expert_mod (0: s)
 };
 
 struct TileInfo {
@@ -169,6 +170,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem& s, const GemmPar
     ti.seg = lo;
     ti.routed = !(p.has_shared && lo == 0);
     ti.expert = lo - p.has_shared;
+    if (p.expert_mod > 0 && ti.expert >= p.expert_mod) ti.expert %= p.expert_mod;
     ti.rows = s.seg_rows[lo];
     ti.row0 = s.seg_row0[lo];
     const int mt = (ti.rows + kBM - 1) / kBM;

@@ -16,6 +16,7 @@
 #include "balance.cuh"
 #include "combine.cuh"
 #include "dispatch.cuh"
+#include "ep.cuh"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_mx.cuh"
 #include "grouped_gemm_bwd.cuh"
@@ -310,17 +311,32 @@ int64_t gemm_grid(int64_t T, int64_t R, int64_t E, int64_t n_cols_max, int has_s
     return grid;
 }
 
+// Routed rows of the expert GEMMs: R rows in nseg consecutive segments,
+// segment s = rows offsets[s] .. offsets[s+1], computed with expert s % n_local of
+// the weight tensors (n_local = nseg on one GPU; with experts spread over ranks a
+// rank receives one segment per (source rank, local expert)).
+struct RoutedRows {
+    int64_t R;
+    int nseg;
+    int n_local;
+    const int32_t* offsets;
+};
+
+RoutedRows routed_rows_of(const moe_config* c, int64_t T, const int32_t* offsets) {
+    return RoutedRows{T * c->num_experts_per_tok, c->n_routed_experts, c->n_routed_experts, offsets};
+}
+
 // K4: h = silu(A Wg^T) * (A Wu^T) for routed rows (A = x_perm) and shared rows (A = x).
-int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_perm, const int32_t* offsets,
+int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_perm, const RoutedRows& rr,
                    const void* w_gate, const void* w_up, const void* ws_gate, const void* ws_up,
                    void* h_routed, void* h_shared, int num_sms, cudaStream_t st) {
-    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+    const int64_t H = c->hidden_size;
     const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
-    const int64_t R = T * K;
+    const int64_t R = rr.R;
     const int has_shared = SI > 0 ? 1 : 0;
     CUtensorMap a_r, a_s, b_r, b2_r, b_s, b2_s;
-    bool ok = make_map(&a_r, x_perm, R, H, kBM) && make_map(&b_r, w_gate, E * I, H, kBN / 2) &&
-              make_map(&b2_r, w_up, E * I, H, kBN / 2);
+    bool ok = make_map(&a_r, x_perm, R, H, kBM) && make_map(&b_r, w_gate, rr.n_local * I, H, kBN / 2) &&
+              make_map(&b2_r, w_up, rr.n_local * I, H, kBN / 2);
     if (has_shared)
         ok = ok && make_map(&a_s, x, T, H, kBM) && make_map(&b_s, ws_gate, SI, H, kBN / 2) &&
              make_map(&b2_s, ws_up, SI, H, kBN / 2);
@@ -329,8 +345,9 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     }
     if (!ok) return MOE_ERR_CUDA;
     GemmParams p{};
-    p.offsets = offsets;
-    p.E = static_cast<int>(E);
+    p.offsets = rr.offsets;
+    p.E = rr.nseg;
+    p.expert_mod = rr.n_local;
     p.T = static_cast<int>(T);
     p.has_shared = has_shared;
     p.n_tiles_routed = static_cast<int>((I + kBN / 2 - 1) / (kBN / 2));
@@ -348,23 +365,30 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
     p.max_rows = R;
-    const int64_t grid = gemm_grid(T, R, E, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
+    const int64_t grid = gemm_grid(T, R, rr.nseg, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// K5: y_perm = w * (h Wd^T) for routed rows, h_shared Wsd^T for the shared rows.
-int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void* h_shared,
-                const int32_t* offsets, const int32_t* perm_src, const float* topk_w, const void* w_down,
-                const void* ws_down, void* y_perm, void* y_scale, int num_sms, cudaStream_t st) {
-    const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
+// Block-scaled fp16 output rows (values [rows, H] and one scale code per 32 columns).
+struct ScaledRows {
+    __half* values;
+    uint8_t* scales;
+};
+
+// K5: routed row r -> w_r * (h_r Wd^T), w_r = topk_w[perm_src[r]] (topk_w[r] when
+// perm_src is null); shared row t -> h_shared[t] Wsd^T.
+int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void* h_shared, const RoutedRows& rr,
+                const int32_t* perm_src, const float* topk_w, int64_t n_slots, const void* w_down,
+                const void* ws_down, ScaledRows y_routed, ScaledRows y_shared, int num_sms, cudaStream_t st) {
+    const int64_t H = c->hidden_size;
     const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
-    const int64_t R = T * K;
+    const int64_t R = rr.R;
     const int has_shared = SI > 0 ? 1 : 0;
     CUtensorMap a_r, a_s, b_r, b_s;
-    bool ok = make_map(&a_r, h_routed, R, I, kBM) && make_map(&b_r, w_down, E * H, I, kBN);
+    bool ok = make_map(&a_r, h_routed, R, I, kBM) && make_map(&b_r, w_down, rr.n_local * H, I, kBN);
     if (has_shared)
         ok = ok && make_map(&a_s, h_shared, T, SI, kBM) && make_map(&b_s, ws_down, H, SI, kBN);
     else {
@@ -372,8 +396,9 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     }
     if (!ok) return MOE_ERR_CUDA;
     GemmParams p{};
-    p.offsets = offsets;
-    p.E = static_cast<int>(E);
+    p.offsets = rr.offsets;
+    p.E = rr.nseg;
+    p.expert_mod = rr.n_local;
     p.T = static_cast<int>(T);
     p.has_shared = has_shared;
     p.n_tiles_routed = static_cast<int>((H + kBN - 1) / kBN);
@@ -383,29 +408,37 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.n_valid_routed = static_cast<int>(H);
     p.n_valid_shared = static_cast<int>(H);
     p.b_rows_per_expert = static_cast<int>(H);
-    p.out_routed = y_perm;
+    p.out_routed = y_routed.values;
     p.ld_routed = H;
-    p.out_shared = static_cast<__half*>(y_perm) + R * H;
+    p.out_shared = y_shared.values;
     p.ld_shared = H;
     p.scale_ld = scale_ld(H);
-    p.scale_routed = static_cast<uint8_t*>(y_scale);
-    p.scale_shared = static_cast<uint8_t*>(y_scale) + R * p.scale_ld;
+    p.scale_routed = y_routed.scales;
+    p.scale_shared = y_shared.scales;
     p.perm_src = perm_src;
     p.topk_w = topk_w;
     p.idesc = ptx::idesc_bf16_f32(kBM, kBN);
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
     p.max_rows = R;
-    p.n_slots = R;
-    const int64_t grid = gemm_grid(T, R, E, H, has_shared, num_sms, kBN);
+    p.n_slots = n_slots;
+    const int64_t grid = gemm_grid(T, R, rr.nseg, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b_r, b_s, b_s, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// Routed rows of y_perm are [0, shared_row0) (T*k, or the padded row space of
-// the MXFP8 and training paths); the shared rows follow.
+// y_perm [R + T, H] and its scale codes as the routed rows followed by the shared rows.
+void split_y_perm(const moe_config* c, int64_t R, void* y_perm, void* y_scale, ScaledRows* routed,
+                  ScaledRows* shared) {
+    const int64_t H = c->hidden_size;
+    routed->values = static_cast<__half*>(y_perm);
+    routed->scales = static_cast<uint8_t*>(y_scale);
+    shared->values = static_cast<__half*>(y_perm) + R * H;
+    shared->scales = static_cast<uint8_t*>(y_scale) + R * scale_ld(H);
+}
+
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const void* y_scale,
                    const int32_t* row_of, void* y, int y_dtype, cudaStream_t st, int64_t shared_row0 = -1) {
     if (shared_row0 < 0) shared_row0 = T * c->num_experts_per_tok;
@@ -1184,7 +1217,8 @@ int moe_experts_gate_up(const moe_config* cfg, int64_t T, const void* x, const v
     if (cfg->n_shared_experts > 0 && (v = check_ptrs({x, ws_gate, ws_up, h_shared})) != MOE_OK) return v;
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
-    return launch_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared,
+    return launch_gate_up(cfg, T, x, x_perm, routed_rows_of(cfg, T, expert_offsets), w_gate, w_up, ws_gate, ws_up,
+                          h_routed, h_shared,
                           d->num_sms, static_cast<cudaStream_t>(stream));
 }
 
@@ -1199,8 +1233,11 @@ int moe_experts_down(const moe_config* cfg, int64_t T, const void* h_routed, con
     if (cfg->n_shared_experts > 0 && (v = check_ptrs({h_shared, ws_down})) != MOE_OK) return v;
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
-    return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
-                       y_perm_scale, d->num_sms, static_cast<cudaStream_t>(stream));
+    ScaledRows yr, ys;
+    split_y_perm(cfg, T * cfg->num_experts_per_tok, y_perm, y_perm_scale, &yr, &ys);
+    return launch_down(cfg, T, h_routed, h_shared, routed_rows_of(cfg, T, expert_offsets), perm_src, topk_w,
+                       T * cfg->num_experts_per_tok, w_down, ws_down, yr, ys, d->num_sms,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_perm,
@@ -1218,11 +1255,14 @@ int moe_experts(const moe_config* cfg, int64_t T, const void* x, const void* x_p
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((v = launch_gate_up(cfg, T, x, x_perm, expert_offsets, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared,
-                            d->num_sms, st)) != MOE_OK)
+    const RoutedRows rr = routed_rows_of(cfg, T, expert_offsets);
+    if ((v = launch_gate_up(cfg, T, x, x_perm, rr, w_gate, w_up, ws_gate, ws_up, h_routed, h_shared, d->num_sms,
+                            st)) != MOE_OK)
         return v;
-    return launch_down(cfg, T, h_routed, h_shared, expert_offsets, perm_src, topk_w, w_down, ws_down, y_perm,
-                       y_perm_scale, d->num_sms, st);
+    ScaledRows yr, ys;
+    split_y_perm(cfg, rr.R, y_perm, y_perm_scale, &yr, &ys);
+    return launch_down(cfg, T, h_routed, h_shared, rr, perm_src, topk_w, rr.R, w_down, ws_down, yr, ys, d->num_sms,
+                       st);
 }
 
 int moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const void* y_perm_scale,
@@ -1268,11 +1308,14 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
     if ((v = launch_dispatch(cfg, T, x, idx, w.offsets, w.x_perm, w.perm_src, w.row_of, w.block_counts,
                              w.block_base, w.totals, st)) != MOE_OK)
         return v;
-    if ((v = launch_gate_up(cfg, T, x, w.x_perm, w.offsets, w_gate, w_up, ws_gate, ws_up, w.h_routed,
-                            w.h_shared, d->num_sms, st)) != MOE_OK)
+    const RoutedRows rr = routed_rows_of(cfg, T, w.offsets);
+    if ((v = launch_gate_up(cfg, T, x, w.x_perm, rr, w_gate, w_up, ws_gate, ws_up, w.h_routed, w.h_shared,
+                            d->num_sms, st)) != MOE_OK)
         return v;
-    if ((v = launch_down(cfg, T, w.h_routed, w.h_shared, w.offsets, w.perm_src, tw, w_down, ws_down, w.y_perm,
-                         w.y_scale, d->num_sms, st)) != MOE_OK)
+    ScaledRows yr, ys;
+    split_y_perm(cfg, rr.R, w.y_perm, w.y_scale, &yr, &ys);
+    if ((v = launch_down(cfg, T, w.h_routed, w.h_shared, rr, w.perm_src, tw, rr.R, w_down, ws_down, yr, ys,
+                         d->num_sms, st)) != MOE_OK)
         return v;
     return launch_combine(cfg, T, w.y_perm, w.y_scale, w.row_of, y, y_dtype, st);
 }
@@ -1666,6 +1709,84 @@ int moe_bias_update(const moe_config* cfg, int64_t T, const int32_t* topk_idx, f
         topk_idx, T * cfg->num_experts_per_tok, cfg->n_routed_experts, gamma, e_bias, expert_load);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- expert parallelism
+namespace {
+int validate_ep(const moe_config* c, int64_t T, int32_t world) {
+    const int v = validate_cfg(c, T);
+    if (v != MOE_OK) return v;
+    if (world < 1 || c->n_routed_experts % world != 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+}  // namespace
+
+int moe_ep_pack(const moe_config* cfg, int64_t T, const int32_t* expert_offsets, const int32_t* perm_src,
+                const float* topk_w, int32_t* expert_counts, float* w_perm, void* stream) {
+    int v = validate_cfg(cfg, T);
+    if (v != MOE_OK) return v;
+    if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
+    const int64_t n = T * cfg->num_experts_per_tok;
+    if (n > 0 && (!perm_src || !topk_w || !w_perm)) return MOE_ERR_INVALID_ARG;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4096) blocks = 4096;
+    ep_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        expert_offsets, cfg->n_routed_experts, perm_src, topk_w, n, expert_counts, w_perm);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ep_recv_offsets(const moe_config* cfg, int32_t world, const int32_t* recv_counts, int32_t* recv_offsets,
+                        void* stream) {
+    int v = validate_ep(cfg, 0, world);
+    if (v != MOE_OK) return v;
+    if (!recv_counts || !recv_offsets) return MOE_ERR_INVALID_ARG;
+    ep_recv_offsets_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(recv_counts, cfg->n_routed_experts,
+                                                                            recv_offsets);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ep_experts(const moe_config* cfg, int32_t world, int64_t T, const void* x, int64_t R, const void* x_recv,
+                   const int32_t* recv_offsets, const float* w_recv, const void* w_gate, const void* w_up,
+                   const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down, void* h_recv,
+                   void* h_shared, void* y_recv, void* y_recv_scale, void* y_shared, void* y_shared_scale,
+                   void* stream) {
+    int v = validate_ep(cfg, T, world);
+    if (v != MOE_OK) return v;
+    if (R < 0) return MOE_ERR_INVALID_ARG;
+    if (R >= (1ll << 31) - 256 - 128ll * cfg->n_routed_experts) return MOE_ERR_UNSUPPORTED;
+    const bool sh = cfg->n_shared_experts > 0 && T > 0;
+    if (!sh && R == 0) return MOE_OK;
+    if (!recv_offsets) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({w_gate, w_up, w_down})) != MOE_OK) return v;
+    if (R > 0 && ((v = check_ptrs({x_recv, h_recv, y_recv, y_recv_scale})) != MOE_OK || !w_recv))
+        return v != MOE_OK ? v : MOE_ERR_INVALID_ARG;
+    if (sh && (v = check_ptrs({x, ws_gate, ws_up, ws_down, h_shared, y_shared, y_shared_scale})) != MOE_OK) return v;
+    DeviceInfo* d = nullptr;
+    if ((v = device_info(&d)) != MOE_OK) return v;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // With no shared rows to compute (S = 0 or no local tokens) the shared members
+    // are unused; the launches still take well-formed maps, so point them at the
+    // routed ones.
+    moe_config c = *cfg;
+    if (!sh) c.n_shared_experts = 0;
+    if (R == 0) {
+        // No received rows: every routed segment is empty and its tensors are never
+        // addressed; the maps still need a valid base.
+        x_recv = x;
+        h_recv = h_shared;
+        y_recv = y_shared;
+        y_recv_scale = y_shared_scale;
+    }
+    const RoutedRows rr{R, cfg->n_routed_experts, cfg->n_routed_experts / world, recv_offsets};
+    if ((v = launch_gate_up(&c, T, x, x_recv, rr, w_gate, w_up, ws_gate, ws_up, h_recv, h_shared, d->num_sms, st)) !=
+        MOE_OK)
+        return v;
+    const ScaledRows yr{static_cast<__half*>(y_recv), static_cast<uint8_t*>(y_recv_scale)};
+    const ScaledRows ys{static_cast<__half*>(y_shared), static_cast<uint8_t*>(y_shared_scale)};
+    return launch_down(&c, T, h_recv, h_shared, rr, nullptr, w_recv, R, w_down, ws_down, yr, ys, d->num_sms, st);
 }
 
 int moe_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

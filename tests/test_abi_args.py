@@ -105,12 +105,20 @@ def run_all(s):
     abi.moe_forward_train(cfg, L["x"], L["router_w"], L["e_bias"], *W, e(T, H, dtype=f32), ws)
     abi.moe_backward_train(cfg, L["x"], L["router_w"], *W, dy, dx, drw, *G, ws)
     abi.moe_forward_host(cfg, L["x"], L["router_w"], L["e_bias"], *W, e(T, H, dtype=f32), 0, ws)
+    # expert parallelism (world 2: this rank holds E/2 experts and receives R rows)
+    world, R = 2, 7
+    El = E // world
+    abi.moe_ep_pack(cfg, T, offsets, perm_src, w, counts, e(T * k, dtype=f32))
+    abi.moe_ep_recv_offsets(cfg, world, e(E, dtype=i32), e(E + 1, dtype=i32))
+    abi.moe_ep_experts(cfg, world, T, L["x"], e(R, H), e(E + 1, dtype=i32), e(R, dtype=f32), e(El, I, H),
+                       e(El, I, H), e(El, H, I), L["ws_gate"], L["ws_up"], L["ws_down"], e(R, I), h_s,
+                       e(R, H, dtype=f16), e(R, abi.y_perm_scale_cols(H), dtype=u8), y_perm[T * k:], y_sc[T * k:])
 
 
 @pytest.mark.parametrize("shape", [TINY, NOSHARED, TINY.with_(name="empty", T=0)], ids=lambda s: s.name)
 def test_valid_buffers_reach_the_library(rec, shape):
     run_all(shape)
-    assert len(rec.calls) == 22 and "moe_backward_train" in rec.calls
+    assert len(rec.calls) == 25 and "moe_backward_train" in rec.calls and "moe_ep_experts" in rec.calls
 
 
 def test_bad_arguments_are_rejected_before_the_call(rec):
@@ -140,6 +148,14 @@ def test_bad_arguments_are_rejected_before_the_call(rec):
         (TypeError, lambda: abi.moe_combine(cfg, T, e(T * k + T, H), e(T * k + T, 8, dtype=torch.uint8),
                                             idx, y)),   # y_perm must be fp16
         (TypeError, lambda: abi.moe_forward_host(cfg, L["x"], L["router_w"], L["e_bias"], *W, [0.0], 0, ws)),
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 3, T, L["x"], e(4, H), e(E + 1, dtype=torch.int32),
+                                                e(4, dtype=torch.float32), *W, e(4, I), e(T, I),
+                                                e(4, H, dtype=torch.float16), e(4, 8, dtype=torch.uint8),
+                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8))),
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 2, T, L["x"], e(4, H), e(E + 1, dtype=torch.int32),
+                                                e(3, dtype=torch.float32), *W, e(4, I), e(T, I),
+                                                e(4, H, dtype=torch.float16), e(4, 8, dtype=torch.uint8),
+                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8))),
     ]
     for exc, call in bad:
         with pytest.raises(exc):
