@@ -15,7 +15,10 @@
 //            Wr = hi + mid + lo (one segment of T rows, K = 3 H: each 64-column
 //            block of x meets the three planes back to back, so its second and
 //            third loads come from L2 and x streams from HBM once; N = E rounded
-//            up to 16), fp32 output.
+//            up to 16); the epilogue either stores the fp32 logits or routes each
+//            token from them (sigmoid, bias, group top-2, group keep, expert
+//            top-k, weights — one thread per token, see route_row_epilogue), or
+//            both.
 // ("The Evolving Transformer · 07", § 02: each routed expert is a SwiGLU FFN
 // applied to the tokens sent to it; its output is multiplied by the routing
 // weight.)
@@ -32,6 +35,7 @@
 #include <cuda_fp16.h>
 
 #include "device_status.cuh"
+#include "router.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -99,6 +103,7 @@ struct GemmParams {
     int64_t max_rows;                     // routed row space: segments must lie in [0, max_rows)
     int64_t n_slots;                      // kDown: entries of topk_w (perm_src values < n_slots)
     int expert_mod;                       // routed segment s uses expert s % expert_mod (0: s)
+    RouteSel sel;                         // kLogits: route in the epilogue when sel.topk_idx != null
 };
 
 struct TileInfo {
@@ -607,6 +612,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             if (c < nblk) dst[c] = static_cast<uint8_t>(codes[c]);
                     }
                 }
+            } else if (p.sel.topk_idx != nullptr) {
+                // Routing of this thread's token straight from its logits in TMEM
+                // (the logits themselves are stored too when out_shared is given).
+                float* out = p.out_shared ? static_cast<float*>(p.out_shared) + grow * p.ld_shared : nullptr;
+                float* gsm = reinterpret_cast<float*>(stage);  // group scores [32 groups][32 lanes]
+                route_row_epilogue(p.sel, taddr, row_ok, grow, out, gsm, lane);
             } else {
                 const int n_valid = p.n_valid_shared;  // E
                 float* out = static_cast<float*>(p.out_shared) + grow * p.ld_shared;

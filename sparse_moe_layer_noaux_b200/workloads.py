@@ -101,9 +101,14 @@ V3_SKEWED = V3_DECODE.with_(name="v3_skewed", T=8192, bias_kind="zipf", seed=4)
 # V3 dimensions with 32 experts (2.8 GB of weights, still 22x the L2): the case
 # for detailed profiler captures, which must stay a few GB on the device.
 V3_E32 = V3_DECODE.with_(name="v3_e32", T=4096, n_routed_experts=32, seed=5)
+# The same 32 experts under a prefill-sized batch (16384 tokens, top-2: ~1024 rows per
+# expert, and the shared expert's 16384 rows = 235 MB of A, as at the V3 prefill):
+# a capture case for the DRAM traffic of the prefill's tile orders (about 4.5 GB on
+# the device).
+V3_E32_T16K = V3_E32.with_(name="v3_e32_t16k", T=16384, num_experts_per_tok=2, seed=6)
 
 WORKLOADS: Dict[str, MoEShape] = {w.name: w for w in
-                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED, V3_E32)}
+                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED, V3_E32, V3_E32_T16K)}
 
 
 def _normal(shape, std, gen, device, dtype):
