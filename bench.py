@@ -514,16 +514,17 @@ def time_steps(step, steps, warmup, world):
     return max_over_ranks(e0.elapsed_time(e1) / steps, world), launches, clk.summary()
 
 
-E2E_CHUNK_TOKENS = -1  # the library's chunk schedule for the host-buffer forward (copies overlap the layer)
+E2E_CHUNKS = 2  # chunks of the batch in the host-buffer forward (copies overlap the layer)
 
 
-def time_e2e(layer, shape, steps, chunk=E2E_CHUNK_TOKENS):
+def time_e2e(layer, shape, steps, chunks=E2E_CHUNKS):
     """The public host-buffer call: pinned x on the host -> moe_forward_host (the batch
-    in chunks, each chunk's copy in and the previous chunk's copy out overlapping its
-    computation) -> y back in pinned host memory, every step."""
+    in `chunks` chunks, each chunk's copy in and the previous chunk's copy out
+    overlapping its computation) -> y back in pinned host memory, every step."""
     x_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(layer_inputs_host(shape))
     y_host = torch.empty(x_host.shape, dtype=torch.float32, pin_memory=True)
+    chunk = (shape.T + chunks - 1) // chunks if chunks > 1 else 0
     for _ in range(2):
         layer.forward_host(x_host, y_host, chunk)
     torch.cuda.synchronize()

@@ -374,13 +374,9 @@ MOE_API int moe_backward(const moe_config *cfg, int64_t T, const void *x, const 
 /* The forward from HOST buffers: x_host [T, H] bf16 and y_host [T, H] (y_dtype)
  * in host memory (pinned, for the copies to run asynchronously), weights on the
  * device.  The batch is cut into chunks of chunk_tokens rows (0 or >= T: one
- * chunk); a negative chunk_tokens picks the library's schedule: a batch of at
- * least 4096 rows goes in four chunks of 1/8, 3/8, 3/8 and 1/8 of its rows
- * (boundaries rounded down to multiples of 128) — the first input copy and the
- * last output copy overlap no computation, so those chunks are short — and a
- * smaller batch in one chunk.  Chunk i's input copy and chunk i-1's output copy
- * run on two internal copy streams while chunk i is computed on `stream`, so
- * transfers overlap the layer; every chunk streams the expert weights it touches.  The two copy streams and the events that order them are created by
+ * chunk); chunk i's input copy and chunk i-1's output copy run on two internal
+ * copy streams while chunk i is computed on `stream`, so transfers overlap the
+ * layer.  The two copy streams and the events that order them are created by
  * the first call on each device (with that device current) and kept until the
  * process exits; make that first call before any stream capture.  Rows are
  * independent, so y is moe_forward's on the whole batch: bit for

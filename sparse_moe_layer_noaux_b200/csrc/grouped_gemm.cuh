@@ -15,10 +15,7 @@
 //            Wr = hi + mid + lo (one segment of T rows, K = 3 H: each 64-column
 //            block of x meets the three planes back to back, so its second and
 //            third loads come from L2 and x streams from HBM once; N = E rounded
-//            up to 16); the epilogue either stores the fp32 logits or routes each
-//            token from them (sigmoid, bias, group top-2, group keep, expert
-//            top-k, weights — one thread per token, see route_row_epilogue), or
-//            both.
+//            up to 16), fp32 output.
 // ("The Evolving Transformer · 07", § 02: each routed expert is a SwiGLU FFN
 // applied to the tokens sent to it; its output is multiplied by the routing
 // weight.)
@@ -35,7 +32,6 @@
 #include <cuda_fp16.h>
 
 #include "device_status.cuh"
-#include "router.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -76,6 +72,17 @@ constexpr int kSwapMaxRows = MOE_SWAP_MAX_ROWS;
 #endif
 constexpr int kRowMajorMinRowTiles = MOE_ROW_MAJOR_MIN_ROW_TILES;
 
+// Weight bytes of one band of column tiles that a row-major segment keeps in L2.
+constexpr int64_t kRowMajorBandBytes = 32ll << 20;
+
+// Column tiles per band: as many whole weight tiles (rows_b x K elements of
+// elt_bytes) as fit kRowMajorBandBytes, at least one.
+__host__ __device__ inline int row_major_band(int rows_b, int64_t K, int elt_bytes) {
+    const int64_t per = static_cast<int64_t>(rows_b) * K * elt_bytes;
+    const int64_t b = per > 0 ? kRowMajorBandBytes / per : 1;
+    return b < 1 ? 1 : (b > (1 << 20) ? (1 << 20) : static_cast<int>(b));
+}
+
 enum { kSwiGLU = 0, kDown = 1, kLogits = 2 };
 
 struct GemmParams {
@@ -103,7 +110,7 @@ struct GemmParams {
     int64_t max_rows;                     // routed row space: segments must lie in [0, max_rows)
     int64_t n_slots;                      // kDown: entries of topk_w (perm_src values < n_slots)
     int expert_mod;                       // routed segment s uses expert s % expert_mod (0: s)
-    RouteSel sel;                         // kLogits: route in the epilogue when sel.topk_idx != null
+    int row_major_band;                   // column tiles per band of a row-major segment (>= 1)
 };
 
 struct TileInfo {
@@ -182,9 +189,16 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem& s, const GemmPar
     const int local = tile - s.tile_start[lo];
     ti.row_major = mt >= kRowMajorMinRowTiles ? 1 : 0;
     if (ti.row_major) {
+        // Bands of row_major_band column tiles, each walked row tile by row tile: a
+        // row tile's A rows are read once per band while the band's weight tiles
+        // stay in L2 (the last band may be narrower).
         const int nt = ti.routed ? p.n_tiles_routed : p.n_tiles_shared;
-        ti.m = local / nt;
-        ti.n = local - ti.m * nt;
+        const int band = (p.row_major_band >= 1 && p.row_major_band < nt) ? p.row_major_band : nt;
+        const int b = local / (mt * band);
+        const int bw = min(band, nt - b * band);
+        const int in_band = local - b * mt * band;
+        ti.m = in_band / bw;
+        ti.n = b * band + (in_band - ti.m * bw);
     } else {
         ti.n = local / mt;
         ti.m = local - ti.n * mt;
@@ -612,12 +626,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             if (c < nblk) dst[c] = static_cast<uint8_t>(codes[c]);
                     }
                 }
-            } else if (p.sel.topk_idx != nullptr) {
-                // Routing of this thread's token straight from its logits in TMEM
-                // (the logits themselves are stored too when out_shared is given).
-                float* out = p.out_shared ? static_cast<float*>(p.out_shared) + grow * p.ld_shared : nullptr;
-                float* gsm = reinterpret_cast<float*>(stage);  // group scores [32 groups][32 lanes]
-                route_row_epilogue(p.sel, taddr, row_ok, grow, out, gsm, lane);
             } else {
                 const int n_valid = p.n_valid_shared;  // E
                 float* out = static_cast<float*>(p.out_shared) + grow * p.ld_shared;

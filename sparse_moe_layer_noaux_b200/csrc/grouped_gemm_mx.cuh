@@ -67,6 +67,7 @@ struct GemmParamsMx {
     const float* topk_w;
     int64_t max_rows;            // padded routed row space Rp: segments must lie in [0, Rp)
     int64_t n_slots;             // kDown: entries of topk_w (perm_src values < n_slots)
+    int row_major_band;          // column tiles per band of a row-major segment (>= 1)
 };
 
 struct GemmSmemMx {
@@ -105,9 +106,16 @@ __device__ __forceinline__ TileInfo decode_tile_mx(const GemmSmemMx& s, const Ge
     const int local = tile - s.tile_start[lo];
     ti.row_major = mt >= kRowMajorMinRowTiles ? 1 : 0;
     if (ti.row_major) {
+        // Bands of row_major_band column tiles, each walked row tile by row tile: a
+        // row tile's A rows are read once per band while the band's weight tiles
+        // stay in L2 (the last band may be narrower).
         const int nt = ti.routed ? p.n_tiles_routed : p.n_tiles_shared;
-        ti.m = local / nt;
-        ti.n = local - ti.m * nt;
+        const int band = (p.row_major_band >= 1 && p.row_major_band < nt) ? p.row_major_band : nt;
+        const int b = local / (mt * band);
+        const int bw = min(band, nt - b * band);
+        const int in_band = local - b * mt * band;
+        ti.m = in_band / bw;
+        ti.n = b * band + (in_band - ti.m * bw);
     } else {
         ti.n = local / mt;
         ti.m = local - ti.n * mt;

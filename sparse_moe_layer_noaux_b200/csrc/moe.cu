@@ -226,16 +226,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // --------------------------------------------------------------- stages
 
-// Routing of T tokens into idx / w.  `keep_logits`: the fp32 logits are also left
-// in `part` (the backward reads them); otherwise, on the tensor-core path with
-// k <= 8, the tokens are routed in the logits GEMM's epilogue and no logits are
-// stored.
 int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
-                 int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st,
-                 bool keep_logits = false) {
+                 int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
     const int H = c->hidden_size, E = c->n_routed_experts;
     const RouterPlan rp = plan_router(static_cast<int>(T), E, H);
-    const bool fused = T >= kRouterTensorCoreMinT && c->num_experts_per_tok <= kFusedSelectMaxK;
     if (T >= kRouterTensorCoreMinT) {
         // Logits on the tensor cores: exact 3-term bf16 split of Wr, one GEMM, K = 3 H.
         const int64_t n = static_cast<int64_t>(E) * H;
@@ -251,11 +245,8 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
         p.n_tiles_shared = 1;
         p.kb_shared = 3 * (H / kBK);
         p.n_valid_shared = E;
-        p.out_shared = (fused && !keep_logits) ? nullptr : part;
+        p.out_shared = part;
         p.ld_shared = E;
-        if (fused)
-            p.sel = RouteSel{bias, idx, w, E, c->n_group, c->topk_group, c->num_experts_per_tok,
-                             c->norm_topk_prob, c->routed_scaling_factor};
         p.idesc = ptx::idesc_bf16_f32(kBM, npad);
         p.b_tile_bytes = static_cast<uint32_t>(npad) * kBK * 2;
         p.b_plane_rows = E;
@@ -264,7 +255,6 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
         grouped_gemm_kernel<kLogits><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
             a, a, b, b, b, b, p);
         count_launch(2);
-        if (fused) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     } else {
         dim3 g1((E + kRE - 1) / kRE, static_cast<unsigned>((T + kRT - 1) / kRT), rp.nsplit);
         router_logits_kernel<<<g1, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), wr, part,
@@ -375,6 +365,7 @@ int launch_gate_up(const moe_config* c, int64_t T, const void* x, const void* x_
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
     p.max_rows = R;
+    p.row_major_band = row_major_band(kBN, H, 2);
     const int64_t grid = gemm_grid(T, R, rr.nseg, I > SI ? I : SI, has_shared, num_sms, kBN / 2);
     grouped_gemm_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -431,6 +422,7 @@ int launch_down(const moe_config* c, int64_t T, const void* h_routed, const void
     p.b_tile_bytes = kTileBBytes;
     p.allow_swap = 1;
     p.max_rows = R;
+    p.row_major_band = row_major_band(kBN, I, 2);
     p.n_slots = n_slots;
     const int64_t grid = gemm_grid(T, R, rr.nseg, H, has_shared, num_sms, kBN);
     grouped_gemm_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
@@ -671,6 +663,7 @@ int launch_gate_up_mx(const moe_config* c, int64_t T, const MxBuffers& w, const 
     p.hsf_katoms_routed = static_cast<int>(I / kMxAtomK);
     p.hsf_katoms_shared = static_cast<int>(SI / kMxAtomK);
     p.max_rows = w.rp;
+    p.row_major_band = row_major_band(kBN, H, 1);
     const int64_t grid = gemm_grid_mx(T, w.rp, I > SI ? I / (kBN / 2) : SI / (kBN / 2), has_shared, num_sms);
     grouped_gemm_mx_kernel<kSwiGLU><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
         a_r, a_s, b_r, b2_r, b_s, b2_s, p);
@@ -723,6 +716,7 @@ int launch_down_mx(const moe_config* c, int64_t T, const MxBuffers& w, const moe
     p.perm_src = w.perm_src;
     p.topk_w = topk_w;
     p.max_rows = w.rp;
+    p.row_major_band = row_major_band(kBN, I, 1);
     p.n_slots = T * c->num_experts_per_tok;
     const int64_t grid = gemm_grid_mx(T, w.rp, H / kBN, has_shared, num_sms);
     grouped_gemm_mx_kernel<kDown><<<static_cast<unsigned>(grid), kGemmThreads, kGemmMxSmemBytes, st>>>(
@@ -826,7 +820,7 @@ int bwd_front(const moe_config* c, int64_t T, const float* router_w, const float
     const int64_t H = c->hidden_size, E = c->n_routed_experts, K = c->num_experts_per_tok;
     int v;
     if ((v = launch_route(c, T, x, router_w, e_bias, w.topk_idx, w.topk_w, w.router_part, w.router_w3, num_sms,
-                          st, true)) != MOE_OK)
+                          st)) != MOE_OK)
         return v;
     const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
     dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(w.topk_idx, static_cast<int>(T),
@@ -1084,61 +1078,23 @@ int host_streams(HostStreams** out) {
     return MOE_OK;
 }
 
-// The library's own chunk schedule (chunk_tokens < 0): batches of at least
-// kHostRampMinT rows go in four chunks of 1/8, 3/8, 3/8 and 1/8 of the rows
-// (boundaries rounded down to multiples of 128).  The first chunk's input copy and
-// the last chunk's output copy overlap no computation, so those two chunks are
-// short; the middle ones are long enough to keep the expert GEMMs efficient and
-// to hide the other copies.  (Every chunk streams the touched expert weights once,
-// which is what makes many small chunks slow.)
-constexpr int64_t kHostRampMinT = 4096;
-
 struct HostPlan {
-    int64_t n;           // chunks
-    int64_t uniform;     // rows per chunk when the chunks are uniform (0: the ramp)
-    int64_t ramp[5];     // ramp boundaries
-    int64_t T;
+    int64_t chunk;       // rows per chunk
     size_t x_slot, y_slot, fwd_bytes, bytes;
-    int64_t start(int64_t i) const {
-        if (uniform == 0) return ramp[i];
-        const int64_t r = i * uniform;
-        return r < T ? r : T;
-    }
 };
 
 HostPlan plan_host(const moe_config* c, int64_t T, int64_t chunk_tokens, int y_dtype) {
     HostPlan hp{};
-    hp.T = T;
-    if (chunk_tokens < 0 && T >= kHostRampMinT) {
-        const int64_t q[5] = {0, T / 8, T / 2, T - T / 8, T};
-        for (int i = 0; i < 5; ++i) hp.ramp[i] = (i == 0 || i == 4) ? q[i] : q[i] / 128 * 128;
-        hp.n = 4;
-        hp.uniform = 0;
-    } else {
-        hp.uniform = chunk_tokens > 0 && chunk_tokens < T ? chunk_tokens : T;
-        if (hp.uniform < 1) hp.uniform = 1;
-        hp.n = (T + hp.uniform - 1) / hp.uniform;
-    }
-    // Staging slots for the longest chunk; the forward's workspace for the chunk
-    // that needs the most (a short chunk can split the router's hidden axis further).
-    int64_t longest = 0;
-    size_t fwd = 0;
-    for (int64_t i = 0; i < hp.n && i < 4; ++i) {  // uniform chunks: the first and (below) the last
-        const int64_t rows = hp.start(i + 1) - hp.start(i);
-        longest = rows > longest ? rows : longest;
-        const size_t b = workspace_bytes_for(c, rows);
-        fwd = b > fwd ? b : fwd;
-    }
-    if (hp.n > 4) {
-        const int64_t rows = T - hp.start(hp.n - 1);
-        const size_t b = workspace_bytes_for(c, rows);
-        fwd = b > fwd ? b : fwd;
-    }
-    if (longest < 1) longest = 1;
+    hp.chunk = chunk_tokens > 0 && chunk_tokens < T ? chunk_tokens : T;
+    if (hp.chunk < 1) hp.chunk = 1;
     const int64_t H = c->hidden_size;
-    hp.x_slot = align_up(static_cast<size_t>(longest * H * 2));
-    hp.y_slot = align_up(static_cast<size_t>(longest * H * (y_dtype == MOE_DTYPE_BF16 ? 2 : 4)));
-    hp.fwd_bytes = align_up(fwd);
+    hp.x_slot = align_up(static_cast<size_t>(hp.chunk * H * 2));
+    hp.y_slot = align_up(static_cast<size_t>(hp.chunk * H * (y_dtype == MOE_DTYPE_BF16 ? 2 : 4)));
+    // The last chunk may be shorter, and a short batch can split the router's
+    // hidden axis further: size for the larger of the two.
+    const int64_t last = T - ((T + hp.chunk - 1) / hp.chunk - 1) * hp.chunk;
+    const size_t a = workspace_bytes_for(c, hp.chunk), b = workspace_bytes_for(c, last > 0 ? last : hp.chunk);
+    hp.fwd_bytes = align_up(a > b ? a : b);
     hp.bytes = 2 * hp.x_slot + 2 * hp.y_slot + hp.fwd_bytes;
     return hp;
 }
@@ -1633,9 +1589,10 @@ int moe_forward_host(const moe_config* cfg, int64_t T, const void* x_host, const
     if (cudaEventRecord(hs->start, st) != cudaSuccess || cudaStreamWaitEvent(hs->h2d, hs->start, 0) != cudaSuccess ||
         cudaStreamWaitEvent(hs->d2h, hs->start, 0) != cudaSuccess)
         return MOE_ERR_CUDA;
-    for (int64_t i = 0; i < hp.n; ++i) {
+    const int64_t n = (T + hp.chunk - 1) / hp.chunk;
+    for (int64_t i = 0; i < n; ++i) {
         const int s = static_cast<int>(i & 1);
-        const int64_t r0 = hp.start(i), rows = hp.start(i + 1) - r0;
+        const int64_t r0 = i * hp.chunk, rows = (r0 + hp.chunk <= T) ? hp.chunk : T - r0;
         // Input slot s was last read by chunk i-2's compute.
         if (i >= 2 && cudaStreamWaitEvent(hs->h2d, hs->computed[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemcpyAsync(xs[s], static_cast<const uint8_t*>(x_host) + r0 * H * 2, rows * H * 2,

@@ -8,8 +8,6 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
-#include "sm100_ptx.cuh"
-
 namespace moe {
 
 // ---------------------------------------------------------------------------
@@ -289,155 +287,6 @@ __global__ void __launch_bounds__(256) router_select_kernel(RouteArgs a) {
         w *= a.scale;
         a.topk_idx[(int64_t)t * a.K + lane] = my_idx;
         a.topk_w[(int64_t)t * a.K + lane] = w;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// The same routing for one token per thread, from the token's E logits in TMEM
-// (the tensor-core logits GEMM's accumulator row: the thread's TMEM lane, columns
-// 0..E-1), for k <= 8.  Every score, comparison and sum is the one
-// router_select_kernel makes, in the same order, so both give the same bits:
-//   pass 1  s = sigmoid(l), b = s + bias (NaN ranked as -inf), group scores
-//           (sum of the two largest b of each contiguous group) into `gsm`;
-//   pass 2  the topk_group best groups (lower group index on equal scores);
-//   pass 3  the 8 best b among the kept groups' experts by insertion into a
-//           sorted list (larger b first, lower index on equal b; the first k are
-//           the top-k in the order the warp kernel finds them);
-//   weights s / sum (when norm_topk_prob) * scale, the sum taken in the order of
-//           the warp kernel's xor-shuffle reduction over lanes 0..k-1.
-// ---------------------------------------------------------------------------
-constexpr int kFusedSelectMaxK = 8;
-
-struct RouteSel {
-    const float* bias;   // [E]
-    int32_t* topk_idx;   // [T][K]; null: no routing in the epilogue
-    float* topk_w;       // [T][K]
-    int E, G, TG, K;
-    int norm;
-    float scale;
-};
-
-__device__ __forceinline__ float route_sigmoid(float l) { return 1.0f / (1.0f + expf(-l)); }
-
-__device__ __forceinline__ void route_row_epilogue(const RouteSel& q, uint32_t taddr, bool row_ok, int64_t row,
-                                                   float* logits_out, float* gsm, int lane) {
-    const int E = q.E, gsize = E / q.G;
-    // pass 1: group scores (and the logits, when they are kept)
-    {
-        float m1 = -CUDART_INF_F, m2 = -CUDART_INF_F;
-        int g = 0, pos = 0;
-#pragma unroll 1
-        for (int c = 0; c * 32 < E; ++c) {
-            __syncwarp();
-            uint32_t v[32];
-            ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
-            ptx::tmem_wait_ld();
-            if (logits_out != nullptr && row_ok) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    if (c * 32 + 4 * u < E)
-                        *reinterpret_cast<float4*>(logits_out + c * 32 + 4 * u) =
-                            make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                        __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int e = c * 32 + j;
-                if (e < E) {
-                    const float b = route_key(route_sigmoid(__uint_as_float(v[j])) + q.bias[e]);
-                    if (b > m1) { m2 = m1; m1 = b; }
-                    else if (b > m2) { m2 = b; }
-                    if (++pos == gsize) {
-                        gsm[g * 32 + lane] = route_key(gsize >= 2 ? m1 + m2 : m1);
-                        ++g;
-                        pos = 0;
-                        m1 = m2 = -CUDART_INF_F;
-                    }
-                }
-            }
-        }
-    }
-    // pass 2: the kept groups
-    unsigned kept = 0;
-    for (int a = 0; a < q.G; ++a) {
-        const float va = gsm[a * 32 + lane];
-        int rank = 0;
-        for (int b = 0; b < q.G; ++b)
-            if (route_beats(gsm[b * 32 + lane], b, va, a)) ++rank;
-        if (rank < q.TG) kept |= 1u << a;
-    }
-    // pass 3: the best 8 experts of the kept groups
-    float lb[kFusedSelectMaxK], ls[kFusedSelectMaxK];
-    int li[kFusedSelectMaxK];
-#pragma unroll
-    for (int i = 0; i < kFusedSelectMaxK; ++i) {
-        lb[i] = -CUDART_INF_F;
-        ls[i] = 0.f;
-        li[i] = 0x7fffffff;
-    }
-    {
-        int g = 0, pos = 0;
-#pragma unroll 1
-        for (int c = 0; c * 32 < E; ++c) {
-            __syncwarp();
-            uint32_t v[32];
-            ptx::tmem_ld_32x32b_x32(taddr + c * 32, v);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int e = c * 32 + j;
-                if (e < E) {
-                    if ((kept >> g) & 1u) {
-                        const float s = route_sigmoid(__uint_as_float(v[j]));
-                        const float b = route_key(s + q.bias[e]);
-                        if (route_beats(b, e, lb[kFusedSelectMaxK - 1], li[kFusedSelectMaxK - 1])) {
-                            bool placed = false;
-#pragma unroll
-                            for (int i = kFusedSelectMaxK - 1; i > 0; --i) {
-                                if (!placed) {
-                                    if (route_beats(b, e, lb[i - 1], li[i - 1])) {
-                                        lb[i] = lb[i - 1];
-                                        li[i] = li[i - 1];
-                                        ls[i] = ls[i - 1];
-                                    } else {
-                                        lb[i] = b;
-                                        li[i] = e;
-                                        ls[i] = s;
-                                        placed = true;
-                                    }
-                                }
-                            }
-                            if (!placed) {
-                                lb[0] = b;
-                                li[0] = e;
-                                ls[0] = s;
-                            }
-                        }
-                    }
-                    if (++pos == gsize) {
-                        ++g;
-                        pos = 0;
-                    }
-                }
-            }
-        }
-    }
-    // weights: the warp kernel sums s over lanes 0..k-1 (zeros beyond) by xor
-    // shuffles with offsets 16, 8, 4, 2, 1; for k <= 8 lane 0's result is this tree.
-    float t[kFusedSelectMaxK];
-#pragma unroll
-    for (int i = 0; i < kFusedSelectMaxK; ++i) t[i] = i < q.K ? ls[i] : 0.f;
-    const float sum = ((t[0] + t[4]) + (t[2] + t[6])) + ((t[1] + t[5]) + (t[3] + t[7]));
-    if (row_ok) {
-#pragma unroll
-        for (int i = 0; i < kFusedSelectMaxK; ++i) {
-            if (i < q.K) {
-                float w = q.norm ? ls[i] / sum : ls[i];
-                w *= q.scale;
-                q.topk_idx[row * q.K + i] = li[i];
-                q.topk_w[row * q.K + i] = w;
-            }
-        }
     }
 }
 

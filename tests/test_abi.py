@@ -177,18 +177,3 @@ def test_host_forward_workspace_holds_two_slots_and_one_chunk(lib):
     assert abi.workspace_size_host(s, T, T + 5, abi.MOE_DTYPE_F32) == whole
     with pytest.raises(abi.MoEError):
         abi.workspace_size_host(s, T, chunk, 7)     # not a moe_dtype
-
-
-def test_host_forward_schedule_workspace(lib):
-    # chunk_tokens < 0: four chunks of 1/8, 3/8, 3/8, 1/8 of a batch of >= 4096 rows
-    # (boundaries at multiples of 128); the slots hold the longest (3/8) chunk.
-    s = V3_PREFILL
-    H, T = s.H, s.T
-    auto = abi.workspace_size_host(s, T, -1, abi.MOE_DTYPE_F32)
-    longest = T // 2 - T // 8            # 6144 rows
-    fwd = max(abi.workspace_size(s, n) for n in (T // 8, longest))
-    assert auto >= fwd + 2 * longest * H * 2 + 2 * longest * H * 4
-    assert auto < abi.workspace_size_host(s, T, 0, abi.MOE_DTYPE_F32)
-    # A batch under 4096 rows stays one chunk.
-    assert abi.workspace_size_host(s, 4000, -1, abi.MOE_DTYPE_F32) == \
-        abi.workspace_size_host(s, 4000, 0, abi.MOE_DTYPE_F32)
