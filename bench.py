@@ -417,6 +417,41 @@ def time_backward(shape, steps, warmup, world, rank, peaks, inp):
     return out
 
 
+def time_ep(shape, steps, warmup, world, rank, inp):
+    """The expert-parallel layer (MoELayerEP): each rank holds E/world of the routed
+    experts and its own T tokens; rows go to their experts' ranks and back by the
+    process group's all-to-all.  At world 1 (no torchrun) a one-rank NCCL group is
+    formed here, so the same code path runs with the exchanges as local copies."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    from sparse_moe_layer_noaux_b200.ep import MoELayerEP, expert_block
+    own = not dist.is_initialized()
+    if own:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=60))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                                device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        layer = MoELayerEP(shape, world, rank, inp["router_w"], inp["e_bias"],
+                           expert_block(inp["w_gate"], world, rank), expert_block(inp["w_up"], world, rank),
+                           expert_block(inp["w_down"], world, rank), inp["ws_gate"], inp["ws_up"], inp["ws_down"])
+        ms, launches, clk = time_steps(lambda: layer(inp["x"]), steps, warmup, world)
+        st = layer.route_and_pack(inp["x"])
+        torch.cuda.synchronize()
+        sent_rows = int(st.counts.sum().item())
+    finally:
+        if own:
+            dist.destroy_process_group()
+    return {"ms_per_step": ms, "tokens_per_s": job_throughput(shape.T, world, ms), "world": world,
+            "experts_per_rank": shape.E // world, "gpu_launches": launches, "clocks": clk,
+            "rows_exchanged_per_rank": sent_rows,
+            "what": "MoELayerEP.forward: route, dispatch, pack, all-to-all of counts, rows and weights, "
+                    "expert GEMMs on the received rows, all-to-all of the outputs back, combine"}
+
+
 def layer_route_idx(shape, inp):
     cfg = abi.MoEConfig.from_shape(shape)
     ws = torch.empty(abi.workspace_size(cfg, shape.T), dtype=torch.uint8, device="cuda")
@@ -681,6 +716,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mx", action="store_true", help="skip the MXFP8 variant of the layer")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward pass")
+    ap.add_argument("--no-ep", action="store_true", help="skip the expert-parallel layer")
     ap.add_argument("--no-workloads", action="store_true",
                     help="time only the headline workload, not the other four shapes")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "mxfp8", "backward"],
@@ -786,6 +822,9 @@ def main():
     if not args.no_bwd and shape.name == "v3_prefill":
         extra["backward"] = time_backward(shape, max(3, args.steps // 4), args.warmup, world, rank, peaks,
                                           res["inp"])
+        torch.cuda.empty_cache()
+    if not args.no_ep and shape.name == "v3_prefill":
+        extra["expert_parallel"] = time_ep(shape, max(3, args.steps // 2), args.warmup, world, rank, res["inp"])
         torch.cuda.empty_cache()
 
     line = {
