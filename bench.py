@@ -47,7 +47,16 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh", "device_status.cuh"),
                 "mxfp8": ("grouped_gemm_mx.cuh", "mx.cuh", "grouped_gemm.cuh", "sm100_ptx.cuh",
                           "device_status.cuh")}
-MEASURED_TRAFFIC = {}  # (precision, "gate_up" | "down") -> {sources_sha1, case, dram_bytes, algorithmic_bytes}
+# (precision, "gate_up" | "down") -> the capture: the kernel sources' hash, the case, DRAM read + write bytes
+# of its second-pass launch and that launch's algorithmic bytes (profiles/grouped_gemm_dram_v3_e32.md).
+MEASURED_TRAFFIC = {
+    ("bf16", "gate_up"): {"sources_sha1": "0571844cb6d9b45f6bf562b910d4410b10fc4c52", "case": "v3_e32",
+                          "dram_bytes": 3065900000, "algorithmic_bytes": 2617245696},
+    ("bf16", "down"): {"sources_sha1": "0571844cb6d9b45f6bf562b910d4410b10fc4c52", "case": "v3_e32",
+                       "dram_bytes": 1632600000, "algorithmic_bytes": 1656619008},
+    ("mxfp8", "gate_up"): {"sources_sha1": "995caaa28c3156d9fa1544dc5a4a1be156b98cf7", "case": "v3_e32",
+                           "dram_bytes": 1390800000, "algorithmic_bytes": 1349517312},
+}
 
 
 def gemm_sources_sha1(precision="bf16"):
