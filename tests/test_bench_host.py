@@ -58,10 +58,17 @@ def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
                         {"sources_sha1": sha, "case": "v3_e32", "dram_bytes": 1100, "algorithmic_bytes": 1000})
     f = bench.traffic_fields("gate_up", 5000, "bf16")
     assert f["traffic_ratio"] == 1.1 and f["traffic"] == 5500 and f["algorithmic_bytes"] == 5000
+    monkeypatch.delitem(bench.MEASURED_TRAFFIC, ("bf16", "down"), raising=False)
     assert bench.traffic_fields("down", 5000, "bf16")["traffic"] is None     # never captured
     # A kernel source that changed since the capture voids the stored figure.
     monkeypatch.setitem(bench.GEMM_SOURCES, "bf16", ("grouped_gemm.cuh", "router.cuh"))
     assert bench.traffic_fields("gate_up", 5000, "bf16")["traffic"] is None
+
+
+def test_stored_captures_match_the_current_sources():
+    # The stored DRAM captures were taken on the kernels in the tree: the bench reports them.
+    for (prec, kernel) in bench.MEASURED_TRAFFIC:
+        assert bench.traffic_ratio(kernel, prec) is not None, (prec, kernel)
 
 
 def test_host_cpu_reports_cores():
