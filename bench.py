@@ -428,8 +428,8 @@ def time_backward(shape, steps, warmup, world, rank, peaks, inp):
 
 def time_ep(shape, steps, warmup, world, rank, inp):
     """The expert-parallel layer (MoELayerEP): each rank holds E/world of the routed
-    experts and its own T tokens; rows go to their experts' ranks and back by the
-    process group's all-to-all.  At world 1 (no torchrun) a one-rank NCCL group is
+    experts and its own T tokens; a token's row goes once to each rank holding one of
+    its experts and its sum comes back, by the process group's all-to-all.  At world 1 (no torchrun) a one-rank NCCL group is
     formed here, so the same code path runs with the exchanges as local copies."""
     import datetime
     import socket
@@ -448,17 +448,18 @@ def time_ep(shape, steps, warmup, world, rank, inp):
                            expert_block(inp["w_gate"], world, rank), expert_block(inp["w_up"], world, rank),
                            expert_block(inp["w_down"], world, rank), inp["ws_gate"], inp["ws_up"], inp["ws_down"])
         ms, launches, clk = time_steps(lambda: layer(inp["x"]), steps, warmup, world)
-        st = layer.route_and_pack(inp["x"])
+        st = layer.send(inp["x"])
         torch.cuda.synchronize()
-        sent_rows = int(st.counts.sum().item())
+        sent_rows = int(st.send_counts.sum().item())
     finally:
         if own:
             dist.destroy_process_group()
     return {"ms_per_step": ms, "tokens_per_s": job_throughput(shape.T, world, ms), "world": world,
             "experts_per_rank": shape.E // world, "gpu_launches": launches, "clocks": clk,
-            "rows_exchanged_per_rank": sent_rows,
-            "what": "MoELayerEP.forward: route, dispatch, pack, all-to-all of counts, rows and weights, "
-                    "expert GEMMs on the received rows, all-to-all of the outputs back, combine"}
+            "rows_sent_per_rank": sent_rows, "rows_sent_per_token": round(sent_rows / max(shape.T, 1), 3),
+            "what": "MoELayerEP.forward: route, send rows (one per token and destination rank), all-to-all "
+                    "of counts and rows, local sort and expert GEMMs on the received rows, per-row sums, "
+                    "all-to-all of the sums back, combine"}
 
 
 def layer_route_idx(shape, inp):

@@ -424,54 +424,75 @@ MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, 
  * V3 notes" (knlb.dev), § infrastructure: expert parallelism with all-to-all
  * dispatch and combine kernels; § architecture: each token is sent to a limited
  * number of nodes — with contiguous expert blocks per rank and groups that do not
- * straddle ranks, a token's rows reach at most topk_group ranks.)  One forward on
- * each rank, for its own T tokens:
- *   1. moe_route, moe_dispatch: rows in expert order, so the rows bound for rank d
- *      are the contiguous block expert_offsets[d*E/world] .. expert_offsets[(d+1)*E/world];
- *   2. moe_ep_pack: per-expert row counts and each row's routing weight;
- *   3. the caller's all-to-all of the counts (E/world int32 to each rank), then of
- *      the rows (bf16, H each) and their weights (fp32), with the block sizes from
- *      the counts: rank r receives, from each source s in rank order, s's rows for
- *      r's experts in expert order;
- *   4. moe_ep_recv_offsets: the received counts [world][E/world] (source-major)
- *      into segment offsets [E + 1];
- *   5. moe_ep_experts: the grouped GEMMs over the received rows (segment
- *      s * E/world + j runs with local expert j) and the shared experts over the
- *      rank's own tokens;
- *   6. the caller's all-to-all of the expert outputs back (the reverse block
- *      sizes), into rows 0 .. T*k of a y_perm [T*k + T, H] whose rows T*k .. hold
- *      the shared outputs, so the rows land where moe_dispatch put the inputs;
- *   7. moe_combine.
- * With world = 1 the collectives are copies and the result is moe_forward's.
+ * straddle ranks, to at most topk_group ranks.)
+ *
+ * A token crosses to a rank once, however many of its k experts live there: the
+ * source sends one row per (token, destination rank), the destination runs the
+ * token's experts it holds and sends back one row, their weighted sum.  Rows
+ * travel in two wire formats (moe_ep_row_bytes):
+ *   send row:   H bf16 values of x[t], then the token's k expert ids (int32) and
+ *               k routing weights (fp32), zero-padded to a multiple of 16 bytes;
+ *   return row: H block-scaled fp16 values (value = fp16 * 2^(code - 141)), then
+ *               their H/32 scale codes (one byte per 32 values), padded likewise.
+ * One forward on each rank, for its own T tokens:
+ *   1. moe_route;
+ *   2. moe_ep_send: the send rows, sorted by destination rank (token order within
+ *      a rank), the number for each rank, and where each slot's row went;
+ *   3. the caller's all-to-all of the counts (one int32 to each rank), then of the
+ *      send rows with those block sizes: rank r receives, from each source s in
+ *      rank order, s's rows for r;
+ *   4. moe_ep_experts: the received rows through the rank's experts, and the
+ *      rank's own tokens through the shared experts;
+ *   5. the caller's all-to-all of the return rows back (the reverse block sizes),
+ *      so that they land in the source's send order;
+ *   6. moe_ep_combine.
+ * With world = 1 the collectives are copies; the result differs from moe_forward's
+ * only by the fp16 rounding of the returned sums.
  * ------------------------------------------------------------------------ */
 
-/* expert_counts int32 [E] = rows of each expert segment (expert_offsets[e+1] -
- * expert_offsets[e]); w_perm fp32 [T*k]: w_perm[r] = topk_w[perm_src[r]] for the
- * rows of the segments, 0 past expert_offsets[E] (a perm_src entry outside
- * [0, T*k) gives 0 and is recorded in the device error word). */
-MOE_API int moe_ep_pack(const moe_config *cfg, int64_t T, const int32_t *expert_offsets, const int32_t *perm_src,
-                        const float *topk_w, int32_t *expert_counts, float *w_perm, void *stream);
+/* Bytes of one send row and of one return row (formats above); multiples of 16. */
+MOE_API int moe_ep_row_bytes(const moe_config *cfg, int64_t *send_row_bytes, int64_t *return_row_bytes);
 
-/* recv_offsets int32 [E + 1] from recv_counts int32 [world][E/world]: the
- * exclusive prefix sum in that order (a negative count is taken as 0 and
- * recorded).  MOE_ERR_INVALID_ARG unless 1 <= world and world divides E. */
-MOE_API int moe_ep_recv_offsets(const moe_config *cfg, int32_t world, const int32_t *recv_counts,
-                                int32_t *recv_offsets, void *stream);
+/* Device workspace (256-byte aligned) for moe_ep_send on T tokens and for
+ * moe_ep_experts on R received rows and T own tokens.  MOE_ERR_INVALID_ARG unless
+ * 1 <= world, world divides E and R >= 0. */
+MOE_API int moe_ep_workspace_size(const moe_config *cfg, int32_t world, int64_t T, int64_t R, size_t *bytes);
 
-/* The expert GEMMs of one rank:
- *   received rows: x_recv bf16 [R, H] in segments recv_offsets [E + 1] (segment
- *     s = source * E/world + j uses local expert j of w_gate / w_up / w_down),
- *     each row's routing weight in w_recv fp32 [R];
- *     h_recv bf16 [R, I]; y_recv [R, H] block-scaled fp16 with y_recv_scale
- *     [R, ceil(H/256)*8] (the moe_experts format): y = w * down(silu(gate x) * up x);
- *   the rank's own tokens: x bf16 [T, H] through the shared experts, h_shared
- *     bf16 [T, S*I], y_shared [T, H] / y_shared_scale as above (unused when S = 0).
- * A segment outside [0, R) gets no rows and is recorded in the device error word. */
-MOE_API int moe_ep_experts(const moe_config *cfg, int32_t world, int64_t T, const void *x, int64_t R,
-                           const void *x_recv, const int32_t *recv_offsets, const float *w_recv, const void *w_gate,
-                           const void *w_up, const void *w_down, const void *ws_gate, const void *ws_up,
-                           const void *ws_down, void *h_recv, void *h_shared, void *y_recv, void *y_recv_scale,
-                           void *y_shared, void *y_shared_scale, void *stream);
+/* Source side.  In: x bf16 [T, H]; topk_idx int32 / topk_w fp32 [T, k] (from
+ * moe_route).  Out: send_rows [T * min(k, world)] rows of send_row_bytes (the
+ * first sum(send_counts) written, sorted by destination rank, token order within
+ * a rank); send_counts int32 [world]: rows for each rank; send_row_of int32 [T, k]:
+ * for the first slot of token t on rank d, the index of its send row; -1 for the
+ * token's other slots on that rank.  An expert id outside [0, E) gives no row and
+ * is recorded in the device error word.  x, send_rows and the workspace 16-byte
+ * aligned.  T = 0 only zeroes send_counts. */
+MOE_API int moe_ep_send(const moe_config *cfg, int32_t world, int64_t T, const void *x, const int32_t *topk_idx,
+                        const float *topk_w, int32_t *send_counts, void *send_rows, int32_t *send_row_of,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Rank `rank`'s experts.  In: recv_rows [R] send rows from all sources; x bf16
+ * [T, H], the rank's own tokens.  Out: return_rows [R] rows of return_row_bytes:
+ * row i = sum over slots j of received row i whose expert e is one of this rank's
+ * of w_j * down_e(silu(gate_e x) * up_e x), summed in fp32 in slot order, then
+ * block-scaled to fp16; y_shared [T, H] block-scaled fp16 with y_shared_scale
+ * [T, ceil(H/256)*8] codes (the moe_experts format): the shared experts on x
+ * (unused when S = 0).  A received expert id outside [0, E) gives no row and is
+ * recorded in the device error word.  Pointers 16-byte aligned. */
+MOE_API int moe_ep_experts(const moe_config *cfg, int32_t world, int32_t rank, int64_t T, const void *x, int64_t R,
+                           const void *recv_rows, const void *w_gate, const void *w_up, const void *w_down,
+                           const void *ws_gate, const void *ws_up, const void *ws_down, void *return_rows,
+                           void *y_shared, void *y_shared_scale, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Source side, after the return rows came back in send order: back_rows holds
+ * n_back (= sum(send_counts)) return rows.  y[t] = shared row t + the back rows
+ * send_row_of[t, 0..k) (entries -1 skipped), summed in fp32 in that order; y
+ * [T, H] of y_dtype (fp32, or bf16 rounded once).  A send_row_of entry outside
+ * [-1, n_back) contributes nothing and is recorded in the device error word.
+ * MOE_ERR_INVALID_ARG unless 0 <= n_back <= T * min(k, world). */
+MOE_API int moe_ep_combine(const moe_config *cfg, int32_t world, int64_t T, int64_t n_back, const void *back_rows,
+                           const int32_t *send_row_of, const void *y_shared, const void *y_shared_scale, void *y,
+                           int32_t y_dtype, void *stream);
 
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(int status);

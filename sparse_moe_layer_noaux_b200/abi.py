@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -113,17 +113,20 @@ def lib():
         L.moe_backward_train.argtypes = [cfgp, i64] + [_P] * 18 + [sz, _P]
         L.moe_forward_host.argtypes = [cfgp, i64] + [_P] * 10 + [ctypes.c_int32, i64, _P, sz, _P]
         L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
-        L.moe_ep_pack.argtypes = [cfgp, i64, _P, _P, _P, _P, _P, _P]
-        L.moe_ep_recv_offsets.argtypes = [cfgp, ctypes.c_int32, _P, _P, _P]
-        L.moe_ep_experts.argtypes = [cfgp, ctypes.c_int32, i64, _P, i64] + [_P] * 15 + [_P]
+        i32 = ctypes.c_int32
+        L.moe_ep_row_bytes.argtypes = [cfgp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+        L.moe_ep_workspace_size.argtypes = [cfgp, i32, i64, i64, ctypes.POINTER(sz)]
+        L.moe_ep_send.argtypes = [cfgp, i32, i64] + [_P] * 7 + [sz, _P]
+        L.moe_ep_experts.argtypes = [cfgp, i32, i32, i64, _P, i64] + [_P] * 11 + [sz, _P]
+        L.moe_ep_combine.argtypes = [cfgp, i32, i64, i64] + [_P] * 5 + [i32, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
                    "moe_combine", "moe_forward", "moe_device_status", "moe_selftest_wait_timeout",
                    "moe_bias_update", "moe_mx_quantize", "moe_workspace_size_mx", "moe_mx_routed_rows",
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
                    "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward", "moe_workspace_size_host",
-                   "moe_forward_host", "moe_forward_train", "moe_backward_train", "moe_ep_pack",
-                   "moe_ep_recv_offsets", "moe_ep_experts"):
+                   "moe_forward_host", "moe_forward_train", "moe_backward_train", "moe_ep_row_bytes",
+                   "moe_ep_workspace_size", "moe_ep_send", "moe_ep_experts", "moe_ep_combine"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -628,56 +631,97 @@ def moe_backward_train(cfg, x, router_w, w_gate, w_up, w_down, ws_gate, ws_up, w
 
 # ---------------------------------------------------------------- expert parallelism
 
-def moe_ep_pack(cfg, T, expert_offsets, perm_src, topk_w, expert_counts, w_perm, stream=None):
-    """Per-expert row counts [E] and each routed row's weight [T*k] (include/moe.h)."""
-    d = _Dims(cfg, T)
-    _req("expert_offsets", expert_offsets, _I32, d.E + 1)
-    _req("perm_src", perm_src, _I32, d.T * d.k)
-    _req("topk_w", topk_w, _F32, d.T * d.k)
-    _req("expert_counts", expert_counts, _I32, d.E)
-    _req("w_perm", w_perm, _F32, d.T * d.k)
-    _check("moe_ep_pack", lib().moe_ep_pack(ctypes.byref(_cfg(cfg)), T, _ptr(expert_offsets), _ptr(perm_src),
-                                            _ptr(topk_w), _ptr(expert_counts), _ptr(w_perm), _stream(stream)))
+def ep_row_bytes(cfg) -> Tuple[int, int]:
+    """(send row bytes, return row bytes) of the expert-parallel wire rows (include/moe.h)."""
+    a, b = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check("moe_ep_row_bytes", lib().moe_ep_row_bytes(ctypes.byref(_cfg(cfg)), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
 
 
-def moe_ep_recv_offsets(cfg, world: int, recv_counts, recv_offsets, stream=None):
-    """Segment offsets [E+1] of the received rows from their counts [world, E/world]."""
-    E = int(_cfg(cfg).n_routed_experts)
-    _req("recv_counts", recv_counts, _I32, E)
-    _req("recv_offsets", recv_offsets, _I32, E + 1)
-    _check("moe_ep_recv_offsets", lib().moe_ep_recv_offsets(ctypes.byref(_cfg(cfg)), int(world), _ptr(recv_counts),
-                                                            _ptr(recv_offsets), _stream(stream)))
+def ep_send_rows_max(cfg, T: int, world: int) -> int:
+    """Send rows of T tokens at most: one per (token, destination rank)."""
+    return T * min(int(_cfg(cfg).num_experts_per_tok), world)
 
 
-def moe_ep_experts(cfg, world: int, T: int, x, x_recv, recv_offsets, w_recv, w_gate, w_up, w_down,
-                   ws_gate, ws_up, ws_down, h_recv, h_shared, y_recv, y_recv_scale, y_shared, y_shared_scale,
-                   stream=None):
-    """One rank's expert GEMMs over its received rows and the shared experts over its
-    own T tokens (include/moe.h).  Weights are the rank's E/world experts."""
-    d = _Dims(cfg, T)
-    if not isinstance(x_recv, torch.Tensor) or x_recv.dim() != 2 or x_recv.shape[1] != d.H:
-        raise ValueError(f"x_recv: expected shape [R, {d.H}]")
-    R = int(x_recv.shape[0])
+def ep_workspace_size(cfg, world: int, T: int, R: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("moe_ep_workspace_size", lib().moe_ep_workspace_size(ctypes.byref(_cfg(cfg)), int(world), T, R,
+                                                                ctypes.byref(n)))
+    return n.value
+
+
+def _ep_world(d, world: int, rank: int = 0) -> int:
     if world < 1 or d.E % world:
         raise ValueError(f"world {world} must divide n_routed_experts {d.E}")
-    El = d.E // world
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    return d.E // world
+
+
+def _wire_rows(name, t, row_bytes) -> int:
+    if not isinstance(t, torch.Tensor) or t.dim() != 2 or t.shape[1] != row_bytes:
+        raise ValueError(f"{name}: expected a uint8 tensor of shape [rows, {row_bytes}]")
+    _req(name, t, _U8, 0)
+    return int(t.shape[0])
+
+
+def moe_ep_send(cfg, world: int, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace, stream=None):
+    """The source side's send rows, one per (token, destination rank), sorted by rank (include/moe.h)."""
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    _ep_world(d, world)
+    Wb, _ = ep_row_bytes(cfg)
+    _req("x", x, _BF16, 0)
+    _req("topk_idx", topk_idx, _I32, d.T * d.k)
+    _req("topk_w", topk_w, _F32, d.T * d.k)
+    _req("send_counts", send_counts, _I32, world)
+    if _wire_rows("send_rows", send_rows, Wb) < ep_send_rows_max(cfg, d.T, world):
+        raise ValueError(f"send_rows: needs {ep_send_rows_max(cfg, d.T, world)} rows")
+    _req("send_row_of", send_row_of, _I32, d.T * d.k)
+    _req("workspace", workspace, _U8, 0)
+    _check("moe_ep_send", lib().moe_ep_send(
+        ctypes.byref(_cfg(cfg)), int(world), d.T, _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(send_counts),
+        _ptr(send_rows), _ptr(send_row_of), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_ep_experts(cfg, world: int, rank: int, x, recv_rows, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
+                   return_rows, y_shared, y_shared_scale, workspace, stream=None):
+    """Rank `rank`'s experts over the received send rows -> return rows, and the shared
+    experts over its own tokens x (include/moe.h).  Weights are the rank's E/world experts."""
+    d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
+    El = _ep_world(d, world, rank)
+    Wb, Wr = ep_row_bytes(cfg)
+    R = _wire_rows("recv_rows", recv_rows, Wb)
+    if _wire_rows("return_rows", return_rows, Wr) < R:
+        raise ValueError(f"return_rows: needs {R} rows")
     shared = d.S > 0 and d.T > 0
-    _req("x", x, _BF16, d.T * d.H if shared else 0, optional=not shared)
-    _req("x_recv", x_recv, _BF16, R * d.H)
-    _req("recv_offsets", recv_offsets, _I32, d.E + 1)
-    _req("w_recv", w_recv, _F32, R)
+    _req("x", x, _BF16, 0)
     _req("w_gate", w_gate, _BF16, El * d.I * d.H)
     _req("w_up", w_up, _BF16, El * d.I * d.H)
     _req("w_down", w_down, _BF16, El * d.I * d.H)
     for name, t in (("ws_gate", ws_gate), ("ws_up", ws_up), ("ws_down", ws_down)):
         _req(name, t, _BF16, d.SI * d.H, optional=not shared)
-    _req("h_recv", h_recv, _BF16, R * d.I)
-    _req("h_shared", h_shared, _BF16, d.T * d.SI, optional=not shared)
-    _req("y_recv", y_recv, _F16, R * d.H)
-    _req("y_recv_scale", y_recv_scale, _U8, R * d.scale_cols)
     _req("y_shared", y_shared, _F16, d.T * d.H, optional=not shared)
     _req("y_shared_scale", y_shared_scale, _U8, d.T * d.scale_cols, optional=not shared)
+    _req("workspace", workspace, _U8, 0)
     _check("moe_ep_experts", lib().moe_ep_experts(
-        ctypes.byref(_cfg(cfg)), int(world), T, _ptr(x), R, _ptr(x_recv), _ptr(recv_offsets), _ptr(w_recv),
-        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(h_recv),
-        _ptr(h_shared), _ptr(y_recv), _ptr(y_recv_scale), _ptr(y_shared), _ptr(y_shared_scale), _stream(stream)))
+        ctypes.byref(_cfg(cfg)), int(world), int(rank), d.T, _ptr(x), R, _ptr(recv_rows), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(return_rows), _ptr(y_shared),
+        _ptr(y_shared_scale), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_ep_combine(cfg, world: int, back_rows, send_row_of, y_shared, y_shared_scale, y, stream=None):
+    """y [T, H] = the shared rows + the returned rows of each token (include/moe.h);
+    back_rows holds exactly the rows that came back (sum of the send counts)."""
+    d = _Dims(cfg, _rows_2d("y", y, _cfg(cfg).hidden_size))
+    _ep_world(d, world)
+    _, Wr = ep_row_bytes(cfg)
+    n = _wire_rows("back_rows", back_rows, Wr)
+    if n > ep_send_rows_max(cfg, d.T, world):
+        raise ValueError(f"back_rows: more than {ep_send_rows_max(cfg, d.T, world)} rows")
+    _req("send_row_of", send_row_of, _I32, d.T * d.k)
+    _req("y_shared", y_shared, _F16, d.T * d.H, optional=d.S == 0)
+    _req("y_shared_scale", y_shared_scale, _U8, d.T * d.scale_cols, optional=d.S == 0)
+    _req("y", y, _OUT, d.T * d.H)
+    _check("moe_ep_combine", lib().moe_ep_combine(
+        ctypes.byref(_cfg(cfg)), int(world), d.T, n, _ptr(back_rows), _ptr(send_row_of), _ptr(y_shared),
+        _ptr(y_shared_scale), _ptr(y), out_dtype_code(y), _stream(stream)))

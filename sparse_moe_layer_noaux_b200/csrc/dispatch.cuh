@@ -13,6 +13,12 @@
 // Routing indices come from the caller (moe_dispatch takes topk_idx as an
 // argument): an index outside [0, E) is skipped — not counted, no row, row_of = -1
 // — and recorded in the device error word (kErrExpertId).
+//
+// The same four kernels sort the rows of the expert-parallel exchange, where a
+// slot's entry may name a bucket that is not this sort's (another rank's expert,
+// or a destination rank the token already has a row for): SlotIndex says where
+// slot (t, j)'s entry lives and which of its values are buckets, which have no
+// row, and which are caller errors.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -24,19 +30,37 @@ namespace moe {
 constexpr int kDispTok = 32;      // tokens per dispatch block
 constexpr int kDispThreads = 256;
 
+// Slot (t, j)'s entry is v = idx[t * ld + j].  Its bucket is v - base when that
+// lies in [0, E) (E is the kernel's bucket count); otherwise the slot has no row,
+// and a value outside [lo, hi) is also recorded in the device error word.  The
+// layer's dispatch uses {topk_idx, k, 0, 0, E}.
+struct SlotIndex {
+    const int32_t* idx;
+    int ld;
+    int base, lo, hi;
+};
+
+// The bucket of a slot's entry, or -1 (no row; caller errors recorded).
+__device__ __forceinline__ int slot_bucket(const SlotIndex& s, int v, int E) {
+    const int b = v - s.base;
+    if (static_cast<unsigned>(b) < static_cast<unsigned>(E)) return b;
+    if (v < s.lo || v >= s.hi) record_error(kErrExpertId);
+    return -1;
+}
+
 // Per-block expert counts, stored expert-major: block_counts[e * nb + b].
 __global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(
-    const int32_t* __restrict__ topk_idx, int T, int K, int E, int32_t* __restrict__ block_counts) {
+    SlotIndex si, int T, int K, int E, int32_t* __restrict__ block_counts) {
     extern __shared__ int cnt[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     const int t0 = blockIdx.x * kDispTok;
     const int n = min(kDispTok, T - t0) * K;
-    const int32_t* idx = topk_idx + (int64_t)t0 * K;
+    const int32_t* idx = si.idx + (int64_t)t0 * si.ld;
     for (int q = threadIdx.x; q < n; q += blockDim.x) {
-        const int e = idx[q];
-        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicAdd(&cnt[e], 1);
-        else record_error(kErrExpertId);
+        const int tl = q / K;
+        const int e = slot_bucket(si, idx[(int64_t)tl * si.ld + (q - tl * K)], E);
+        if (e >= 0) atomicAdd(&cnt[e], 1);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -68,10 +92,12 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const int32_t* __res
     if (lane == 0) totals[e] = carry;
 }
 
+// w_src / w_perm (both null, or both set): w_perm[row] = w_src[t * ld + j] for the
+// row slot (t, j) lands on (weights laid out like the entries).
 __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
-    const int32_t* __restrict__ topk_idx, int T, int K, int E, const int32_t* __restrict__ block_base,
+    SlotIndex si, int T, int K, int E, const int32_t* __restrict__ block_base,
     const int32_t* __restrict__ totals, int pad, int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
-    int32_t* __restrict__ row_of) {
+    int32_t* __restrict__ row_of, const float* __restrict__ w_src = nullptr, float* __restrict__ w_perm = nullptr) {
     extern __shared__ int smem_i[];
     int* run = smem_i;              // [E] next free row of each expert for this block
     __shared__ int warp_sums[kDispThreads / 32];
@@ -109,9 +135,11 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
     for (int r0 = 0; r0 < n; r0 += kDispThreads) {
         const int q = r0 + tid;
         const bool in_range = q < n;
-        int e = in_range ? topk_idx[q0 + q] : -1;
-        const bool valid = in_range && static_cast<unsigned>(e) < static_cast<unsigned>(E);
-        if (!valid) e = -1 - lane;  // lanes without a valid expert never match another lane
+        const int tl = q / K;
+        const int64_t src = (int64_t)(t0 + tl) * si.ld + (q - tl * K);
+        int e = in_range ? slot_bucket(si, si.idx[src], E) : -1;
+        const bool valid = e >= 0;
+        if (!valid) e = -1 - lane;  // lanes without a bucket never match another lane
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         const int lrank = __popc(peers & lt_mask);
         const bool leader = lrank == 0;
@@ -130,6 +158,7 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
         if (valid) {
             row_of[q0 + q] = row;
             perm_src[row] = (int32_t)(q0 + q);
+            if (w_perm) w_perm[row] = w_src[src];
         } else if (in_range) {
             row_of[q0 + q] = -1;
         }
@@ -140,19 +169,21 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_place_kernel(
 // row; each slice is loaded once and stored to the token's k rows of x_perm
 // (slots the place step left without a row, row_of = -1, are skipped).
 // The grid is T x ceil(H / 2048) blocks, so small batches still spread over
-// every SM.
+// every SM.  x_ld / out_ld: row strides in elements (H for dense rows; the
+// expert-parallel rows carry routing data after their H values), multiples of 8.
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const __nv_bfloat16* __restrict__ x,
                                                                const int32_t* __restrict__ row_of, int K,
-                                                               int H, __nv_bfloat16* __restrict__ x_perm) {
+                                                               int H, __nv_bfloat16* __restrict__ x_perm,
+                                                               int64_t x_ld, int64_t out_ld) {
     __shared__ int rows[32];
     const int t = blockIdx.x;
     if (threadIdx.x < K) rows[threadIdx.x] = row_of[(int64_t)t * K + threadIdx.x];
     __syncthreads();
     const int c = blockIdx.y * 256 + threadIdx.x;
     if (c >= H / 8) return;
-    const uint4 v = reinterpret_cast<const uint4*>(x + (int64_t)t * H)[c];
+    const uint4 v = reinterpret_cast<const uint4*>(x + (int64_t)t * x_ld)[c];
     for (int j = 0; j < K; ++j)
-        if (rows[j] >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)rows[j] * H)[c] = v;
+        if (rows[j] >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)rows[j] * out_ld)[c] = v;
 }
 
 }  // namespace moe

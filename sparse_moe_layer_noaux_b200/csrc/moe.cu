@@ -226,8 +226,9 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // --------------------------------------------------------------- stages
 
-int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
-                 int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
+// Router logits (fp32, [nsplit, T, E] partial sums) into `part`.
+int launch_route_logits(const moe_config* c, int64_t T, const void* x, const float* wr, float* part,
+                        __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
     const int H = c->hidden_size, E = c->n_routed_experts;
     const RouterPlan rp = plan_router(static_cast<int>(T), E, H);
     if (T >= kRouterTensorCoreMinT) {
@@ -261,6 +262,14 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
                                                   static_cast<int>(T), E, H, rp.split_len);
         count_launch();
     }
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Scores, group limit, top-k and weights from the logits in `part`.
+int launch_route_select(const moe_config* c, int64_t T, const float* bias, int32_t* idx, float* w,
+                        const float* part, cudaStream_t st) {
+    const int H = c->hidden_size, E = c->n_routed_experts;
+    const RouterPlan rp = plan_router(static_cast<int>(T), E, H);
     RouteArgs a;
     a.part = part;
     a.nsplit = rp.nsplit;
@@ -283,21 +292,66 @@ int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr,
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+int launch_route(const moe_config* c, int64_t T, const void* x, const float* wr, const float* bias,
+                 int32_t* idx, float* w, float* part, __nv_bfloat16* w3, int num_sms, cudaStream_t st) {
+    const int v = launch_route_logits(c, T, x, wr, part, w3, num_sms, st);
+    return v != MOE_OK ? v : launch_route_select(c, T, bias, idx, w, part, st);
+}
+
+// Rows of T tokens (K slots each, E buckets) sorted into bucket order: offsets
+// [E + 1], perm_src, row_of and the bf16 rows (row strides x_ld / out_ld, in
+// elements); with w_src / w_perm also each row's weight.
+struct RowSort {
+    SlotIndex si;
+    int64_t T;
+    int K, E, H;
+    const void* x;
+    int64_t x_ld;
+    void* x_perm;
+    int64_t out_ld;
+    int32_t *offsets, *perm_src, *row_of;
+    int32_t *block_counts, *block_base, *totals;
+    const float* w_src;
+    float* w_perm;
+};
+
+int launch_row_sort(const RowSort& a, cudaStream_t st) {
+    const int E = a.E, K = a.K;
+    const int nb = static_cast<int>((a.T + kDispTok - 1) / kDispTok);
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(a.si, static_cast<int>(a.T), K, E,
+                                                                      a.block_counts);
+    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(a.block_counts, nb, E, a.block_base, a.totals);
+    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(a.si, static_cast<int>(a.T), K, E,
+                                                                     a.block_base, a.totals, 1, a.offsets,
+                                                                     a.perm_src, a.row_of, a.w_src, a.w_perm);
+    const dim3 gs(static_cast<unsigned>(a.T), static_cast<unsigned>((a.H / 8 + 255) / 256));
+    dispatch_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), a.row_of, K, a.H,
+                                                static_cast<__nv_bfloat16*>(a.x_perm), a.x_ld, a.out_ld);
+    count_launch(4);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_dispatch(const moe_config* c, int64_t T, const void* x, const int32_t* idx, int32_t* offsets,
                     void* x_perm, int32_t* perm_src, int32_t* row_of, int32_t* block_counts,
                     int32_t* block_base, int32_t* totals, cudaStream_t st) {
     const int E = c->n_routed_experts, K = c->num_experts_per_tok, H = c->hidden_size;
-    const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
-    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
-                                                                      block_counts);
-    dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(block_counts, nb, E, block_base, totals);
-    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
-                                                                     totals, 1, offsets, perm_src, row_of);
-    const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
-    dispatch_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H,
-                                                static_cast<__nv_bfloat16*>(x_perm));
-    count_launch(4);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    RowSort a{};
+    a.si = SlotIndex{idx, K, 0, 0, E};
+    a.T = T;
+    a.K = K;
+    a.E = E;
+    a.H = H;
+    a.x = x;
+    a.x_ld = H;
+    a.x_perm = x_perm;
+    a.out_ld = H;
+    a.offsets = offsets;
+    a.perm_src = perm_src;
+    a.row_of = row_of;
+    a.block_counts = block_counts;
+    a.block_base = block_base;
+    a.totals = totals;
+    return launch_row_sort(a, st);
 }
 
 // Persistent grid: one CTA per SM, fewer when there cannot be that many tiles.
@@ -441,23 +495,33 @@ void split_y_perm(const moe_config* c, int64_t R, void* y_perm, void* y_scale, S
     shared->scales = static_cast<uint8_t*>(y_scale) + R * scale_ld(H);
 }
 
+int launch_combine_rows(int64_t T, int K, int H, ScaledRowsIn routed, int64_t routed_rows, const int32_t* row_of,
+                        int absent_ok, ScaledRowsIn shared, CombineDst dst, int kind, cudaStream_t st) {
+    const dim3 g(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
+    const int Ti = static_cast<int>(T);
+    if (kind == kOutBF16)
+        combine_kernel<kOutBF16><<<g, 256, 0, st>>>(routed, routed_rows, row_of, Ti, K, H, absent_ok, shared, dst);
+    else if (kind == kOutScaled)
+        combine_kernel<kOutScaled><<<g, 256, 0, st>>>(routed, routed_rows, row_of, Ti, K, H, absent_ok, shared, dst);
+    else
+        combine_kernel<kOutF32><<<g, 256, 0, st>>>(routed, routed_rows, row_of, Ti, K, H, absent_ok, shared, dst);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_combine(const moe_config* c, int64_t T, const void* y_perm, const void* y_scale,
                    const int32_t* row_of, void* y, int y_dtype, cudaStream_t st, int64_t shared_row0 = -1) {
     if (shared_row0 < 0) shared_row0 = T * c->num_experts_per_tok;
-    const dim3 g(static_cast<unsigned>(T), static_cast<unsigned>((c->hidden_size / 8 + 255) / 256));
-    const int has_shared = c->n_shared_experts > 0 ? 1 : 0;
-    if (y_dtype == MOE_DTYPE_BF16)
-        combine_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-            static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
-            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
-            shared_row0, static_cast<__nv_bfloat16*>(y));
-    else
-        combine_kernel<float><<<g, 256, 0, st>>>(
-            static_cast<const __half*>(y_perm), static_cast<const uint8_t*>(y_scale), scale_ld(c->hidden_size),
-            row_of, static_cast<int>(T), c->num_experts_per_tok, c->hidden_size, has_shared, shared_row0,
-            shared_row0, static_cast<float*>(y));
-    count_launch();
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const int64_t H = c->hidden_size, sld = scale_ld(c->hidden_size);
+    const __half* v = static_cast<const __half*>(y_perm);
+    const uint8_t* sc = static_cast<const uint8_t*>(y_scale);
+    const ScaledRowsIn routed{v, H, sc, sld};
+    const ScaledRowsIn shared = c->n_shared_experts > 0 ? ScaledRowsIn{v + shared_row0 * H, H, sc + shared_row0 * sld, sld}
+                                                        : ScaledRowsIn{nullptr, 0, nullptr, 0};
+    CombineDst dst{};
+    dst.y = y;
+    return launch_combine_rows(T, c->num_experts_per_tok, c->hidden_size, routed, shared_row0, row_of, 0, shared, dst,
+                               y_dtype == MOE_DTYPE_BF16 ? kOutBF16 : kOutF32, st);
 }
 
 
@@ -574,10 +638,10 @@ int launch_dispatch_mx(const moe_config* c, int64_t T, const void* x, const int3
                        int32_t* totals, cudaStream_t st) {
     const int E = c->n_routed_experts, K = c->num_experts_per_tok, H = c->hidden_size;
     const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
-    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E,
-                                                                      block_counts);
+    const SlotIndex si{idx, K, 0, 0, E};
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(si, static_cast<int>(T), K, E, block_counts);
     dispatch_scan_kernel<<<(E + 7) / 8, 256, 0, st>>>(block_counts, nb, E, block_base, totals);
-    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(idx, static_cast<int>(T), K, E, block_base,
+    dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(si, static_cast<int>(T), K, E, block_base,
                                                                      totals, kMxAtomRows, offsets, perm_src, row_of);
     const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
     dispatch_scatter_mx_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), row_of, K, H, xq_perm,
@@ -823,13 +887,13 @@ int bwd_front(const moe_config* c, int64_t T, const float* router_w, const float
                           st)) != MOE_OK)
         return v;
     const int nb = static_cast<int>((T + kDispTok - 1) / kDispTok);
-    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(w.topk_idx, static_cast<int>(T),
-                                                                      static_cast<int>(K), static_cast<int>(E),
-                                                                      w.block_counts);
+    const SlotIndex si{w.topk_idx, static_cast<int>(K), 0, 0, static_cast<int>(E)};
+    dispatch_count_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(si, static_cast<int>(T), static_cast<int>(K),
+                                                                      static_cast<int>(E), w.block_counts);
     dispatch_scan_kernel<<<static_cast<unsigned>((E + 7) / 8), 256, 0, st>>>(w.block_counts, nb, static_cast<int>(E),
                                                                             w.block_base, w.totals);
     dispatch_place_kernel<<<nb, kDispThreads, sizeof(int) * E, st>>>(
-        w.topk_idx, static_cast<int>(T), static_cast<int>(K), static_cast<int>(E), w.block_base, w.totals,
+        si, static_cast<int>(T), static_cast<int>(K), static_cast<int>(E), w.block_base, w.totals,
         kMxAtomRows, w.offsets, w.perm_src, w.row_of);
     const dim3 gs(static_cast<unsigned>(T), static_cast<unsigned>((H / 8 + 255) / 256));
     bwd_scatter_kernel<<<gs, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy),
@@ -1307,12 +1371,12 @@ int moe_forward(const moe_config* cfg, int64_t T, const void* x, const float* ro
     Workspace w = carve(cfg, T, static_cast<uint8_t*>(workspace));
     int32_t* idx = topk_idx_out ? topk_idx_out : w.topk_idx;
     float* tw = topk_w_out ? topk_w_out : w.topk_w;
+    const RoutedRows rr = routed_rows_of(cfg, T, w.offsets);
     if ((v = launch_route(cfg, T, x, router_w, e_bias, idx, tw, w.router_part, w.router_w3, d->num_sms, st)) != MOE_OK)
         return v;
     if ((v = launch_dispatch(cfg, T, x, idx, w.offsets, w.x_perm, w.perm_src, w.row_of, w.block_counts,
                              w.block_base, w.totals, st)) != MOE_OK)
         return v;
-    const RoutedRows rr = routed_rows_of(cfg, T, w.offsets);
     if ((v = launch_gate_up(cfg, T, x, w.x_perm, rr, w_gate, w_up, ws_gate, ws_up, w.h_routed, w.h_shared,
                             d->num_sms, st)) != MOE_OK)
         return v;
@@ -1723,74 +1787,276 @@ int validate_ep(const moe_config* c, int64_t T, int32_t world) {
     if (world < 1 || c->n_routed_experts % world != 0) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
+
+// Wire rows: a send row is the token's H bf16 values, then its k expert ids
+// (int32) and k routing weights (fp32), zero-padded to 16 bytes; a return row is
+// H block-scaled fp16 values, then their H/32 scale codes, padded to 16 bytes.
+int64_t ep_send_row_bytes(const moe_config* c) {
+    return 2ll * c->hidden_size + static_cast<int64_t>(align_up(8ull * c->num_experts_per_tok, 16));
+}
+int64_t ep_return_row_bytes(const moe_config* c) {
+    return 2ll * c->hidden_size + static_cast<int64_t>(align_up(c->hidden_size / 32, 16));
+}
+
+// Rows one source sends for T tokens at most: one per (token, rank holding one of
+// its experts), so at most min(k, world) per token.
+int64_t ep_send_rows_max(const moe_config* c, int64_t T, int world) {
+    return T * (c->num_experts_per_tok < world ? c->num_experts_per_tok : world);
+}
+
+// Expert rows of one rank for R received rows: at most one per received slot.
+// (Rows from moe_ep_send name k distinct experts, so at most min(k, E/world) of
+// them are local; the bound does not rely on that, since the rows are caller data.)
+int64_t ep_local_rows_max(const moe_config* c, int64_t R) { return R * c->num_experts_per_tok; }
+
+// Every received-row slot index and expert row (with up to 127 padding rows per
+// segment and the shared rows) must fit an int32 and a TMA coordinate.
+int check_ep_rows(const moe_config* c, int64_t T, int64_t R) {
+    if (R < 0) return MOE_ERR_INVALID_ARG;
+    if (R * c->num_experts_per_tok + T + 128ll * c->n_routed_experts >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+struct WorkspaceEpSend {
+    int32_t* rank_slot;     // [T, k] destination rank of a slot's row, or -1
+    int32_t* perm_src;      // [T * min(k, world)] slot of each send row
+    int32_t* offsets;       // [world + 1]
+    int32_t* block_counts;  // [world, nb]
+    int32_t* block_base;    // [world, nb]
+    int32_t* totals;        // [world]
+    size_t bytes;
+};
+
+WorkspaceEpSend carve_ep_send(const moe_config* c, int world, int64_t T, uint8_t* base) {
+    const int64_t K = c->num_experts_per_tok, nb = (T + kDispTok - 1) / kDispTok;
+    WorkspaceEpSend w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    w.rank_slot = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
+    w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ep_send_rows_max(c, T, world)));
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (world + 1)));
+    w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * world));
+    w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * world));
+    w.totals = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * world));
+    w.bytes = off;
+    return w;
+}
+
+struct WorkspaceEpExperts {
+    int32_t* offsets;         // [E/world + 1] local expert segments
+    int32_t* perm_src;        // [Rb] received slot (r * k + j) of each expert row
+    int32_t* row_of;          // [R, k] expert row of each received slot, or -1
+    int32_t* block_counts;    // [E/world, nb]
+    int32_t* block_base;      // [E/world, nb]
+    int32_t* totals;          // [E/world]
+    float* w_perm;            // [Rb] routing weight of each expert row
+    __nv_bfloat16* x_perm;    // [Rb, H]
+    __nv_bfloat16* h_routed;  // [Rb, I]
+    __nv_bfloat16* h_shared;  // [T, S*I]
+    __half* y_perm;           // [Rb, H] block-scaled fp16
+    uint8_t* y_scale;         // [Rb, scale_ld]
+    size_t bytes;
+};
+
+WorkspaceEpExperts carve_ep_experts(const moe_config* c, int world, int64_t T, int64_t R, uint8_t* base) {
+    const int64_t K = c->num_experts_per_tok, El = c->n_routed_experts / world, H = c->hidden_size;
+    const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
+    const int64_t nb = (R + kDispTok - 1) / kDispTok, Rb = ep_local_rows_max(c, R);
+    WorkspaceEpExperts w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* p = base ? base + off : nullptr;
+        off += align_up(bytes);
+        return p;
+    };
+    w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (El + 1)));
+    w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * Rb));
+    w.row_of = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * R * K));
+    w.block_counts = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * El));
+    w.block_base = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * nb * El));
+    w.totals = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * El));
+    w.w_perm = reinterpret_cast<float*>(take(sizeof(float) * Rb));
+    w.x_perm = reinterpret_cast<__nv_bfloat16*>(take(2 * Rb * H));
+    w.h_routed = reinterpret_cast<__nv_bfloat16*>(take(2 * Rb * I));
+    w.h_shared = reinterpret_cast<__nv_bfloat16*>(take(2 * T * SI));
+    w.y_perm = reinterpret_cast<__half*>(take(2 * Rb * H));
+    w.y_scale = reinterpret_cast<uint8_t*>(take(Rb * scale_ld(H)));
+    w.bytes = off;
+    return w;
+}
+
+size_t ep_workspace_bytes(const moe_config* c, int world, int64_t T, int64_t R) {
+    const size_t a = carve_ep_send(c, world, T, nullptr).bytes, b = carve_ep_experts(c, world, T, R, nullptr).bytes;
+    return a > b ? a : b;
+}
 }  // namespace
 
-int moe_ep_pack(const moe_config* cfg, int64_t T, const int32_t* expert_offsets, const int32_t* perm_src,
-                const float* topk_w, int32_t* expert_counts, float* w_perm, void* stream) {
-    int v = validate_cfg(cfg, T);
+int moe_ep_row_bytes(const moe_config* cfg, int64_t* send_row_bytes, int64_t* return_row_bytes) {
+    const int v = validate_cfg(cfg, 0);
     if (v != MOE_OK) return v;
-    if (!expert_offsets || !expert_counts) return MOE_ERR_INVALID_ARG;
-    const int64_t n = T * cfg->num_experts_per_tok;
-    if (n > 0 && (!perm_src || !topk_w || !w_perm)) return MOE_ERR_INVALID_ARG;
-    int64_t blocks = (n + 255) / 256;
-    if (blocks < 1) blocks = 1;
-    if (blocks > 4096) blocks = 4096;
-    ep_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        expert_offsets, cfg->n_routed_experts, perm_src, topk_w, n, expert_counts, w_perm);
-    count_launch();
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (!send_row_bytes || !return_row_bytes) return MOE_ERR_INVALID_ARG;
+    *send_row_bytes = ep_send_row_bytes(cfg);
+    *return_row_bytes = ep_return_row_bytes(cfg);
+    return MOE_OK;
 }
 
-int moe_ep_recv_offsets(const moe_config* cfg, int32_t world, const int32_t* recv_counts, int32_t* recv_offsets,
-                        void* stream) {
-    int v = validate_ep(cfg, 0, world);
-    if (v != MOE_OK) return v;
-    if (!recv_counts || !recv_offsets) return MOE_ERR_INVALID_ARG;
-    ep_recv_offsets_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(recv_counts, cfg->n_routed_experts,
-                                                                            recv_offsets);
-    count_launch();
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
-int moe_ep_experts(const moe_config* cfg, int32_t world, int64_t T, const void* x, int64_t R, const void* x_recv,
-                   const int32_t* recv_offsets, const float* w_recv, const void* w_gate, const void* w_up,
-                   const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down, void* h_recv,
-                   void* h_shared, void* y_recv, void* y_recv_scale, void* y_shared, void* y_shared_scale,
-                   void* stream) {
+int moe_ep_workspace_size(const moe_config* cfg, int32_t world, int64_t T, int64_t R, size_t* bytes) {
     int v = validate_ep(cfg, T, world);
     if (v != MOE_OK) return v;
-    if (R < 0) return MOE_ERR_INVALID_ARG;
-    if (R >= (1ll << 31) - 256 - 128ll * cfg->n_routed_experts) return MOE_ERR_UNSUPPORTED;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ep_rows(cfg, T, R)) != MOE_OK) return v;
+    *bytes = ep_workspace_bytes(cfg, world, T, R);
+    return MOE_OK;
+}
+
+int moe_ep_send(const moe_config* cfg, int32_t world, int64_t T, const void* x, const int32_t* topk_idx,
+                const float* topk_w, int32_t* send_counts, void* send_rows, int32_t* send_row_of, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    int v = validate_ep(cfg, T, world);
+    if (v != MOE_OK) return v;
+    if (!send_counts) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * world, st) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!topk_idx || !topk_w || !send_row_of) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({x, send_rows})) != MOE_OK) return v;
+    if (!workspace || workspace_bytes < carve_ep_send(cfg, world, T, nullptr).bytes || !aligned16(workspace))
+        return MOE_ERR_WORKSPACE;
+    const WorkspaceEpSend w = carve_ep_send(cfg, world, T, static_cast<uint8_t*>(workspace));
+    const int K = cfg->num_experts_per_tok, E = cfg->n_routed_experts, H = cfg->hidden_size;
+    const int64_t Wb = ep_send_row_bytes(cfg);
+    ep_rank_slots_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(topk_idx, T, K, E / world, E,
+                                                                                w.rank_slot);
+    count_launch();
+    // Sort the (token, rank) rows by rank: the rank-slot entries are the buckets,
+    // -1 (a rank the token already has a row for) is no row.
+    RowSort a{};
+    a.si = SlotIndex{w.rank_slot, K, 0, -1, world};
+    a.T = T;
+    a.K = K;
+    a.E = world;
+    a.H = H;
+    a.x = x;
+    a.x_ld = H;
+    a.x_perm = send_rows;
+    a.out_ld = Wb / 2;
+    a.offsets = w.offsets;
+    a.perm_src = w.perm_src;
+    a.row_of = send_row_of;
+    a.block_counts = w.block_counts;
+    a.block_base = w.block_base;
+    a.totals = w.totals;
+    if ((v = launch_row_sort(a, st)) != MOE_OK) return v;
+    const int meta_words = static_cast<int>((Wb - 2ll * H) / 4);
+    const int64_t n_max = ep_send_rows_max(cfg, T, world);
+    int64_t blocks = (n_max * meta_words + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    ep_send_meta_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        w.offsets, world, w.perm_src, T * K, K, topk_idx, topk_w, n_max, static_cast<uint8_t*>(send_rows), Wb,
+        2ll * H, meta_words, send_counts);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_ep_experts(const moe_config* cfg, int32_t world, int32_t rank, int64_t T, const void* x, int64_t R,
+                   const void* recv_rows, const void* w_gate, const void* w_up, const void* w_down,
+                   const void* ws_gate, const void* ws_up, const void* ws_down, void* return_rows, void* y_shared,
+                   void* y_shared_scale, void* workspace, size_t workspace_bytes, void* stream) {
+    int v = validate_ep(cfg, T, world);
+    if (v != MOE_OK) return v;
+    if (rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ep_rows(cfg, T, R)) != MOE_OK) return v;
     const bool sh = cfg->n_shared_experts > 0 && T > 0;
     if (!sh && R == 0) return MOE_OK;
-    if (!recv_offsets) return MOE_ERR_INVALID_ARG;
     if ((v = check_ptrs({w_gate, w_up, w_down})) != MOE_OK) return v;
-    if (R > 0 && ((v = check_ptrs({x_recv, h_recv, y_recv, y_recv_scale})) != MOE_OK || !w_recv))
-        return v != MOE_OK ? v : MOE_ERR_INVALID_ARG;
-    if (sh && (v = check_ptrs({x, ws_gate, ws_up, ws_down, h_shared, y_shared, y_shared_scale})) != MOE_OK) return v;
+    if (R > 0 && (v = check_ptrs({recv_rows, return_rows})) != MOE_OK) return v;
+    if (sh && (v = check_ptrs({x, ws_gate, ws_up, ws_down, y_shared, y_shared_scale})) != MOE_OK) return v;
+    if (!workspace || workspace_bytes < carve_ep_experts(cfg, world, T, R, nullptr).bytes || !aligned16(workspace))
+        return MOE_ERR_WORKSPACE;
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WorkspaceEpExperts w = carve_ep_experts(cfg, world, T, R, static_cast<uint8_t*>(workspace));
+    const int K = cfg->num_experts_per_tok, E = cfg->n_routed_experts, El = E / world, H = cfg->hidden_size;
+    const int64_t Wb = ep_send_row_bytes(cfg), Wr = ep_return_row_bytes(cfg);
+    const int64_t Rb = ep_local_rows_max(cfg, R);
     // With no shared rows to compute (S = 0 or no local tokens) the shared members
-    // are unused; the launches still take well-formed maps, so point them at the
-    // routed ones.
+    // are unused; the launches still take well-formed maps.
     moe_config c = *cfg;
     if (!sh) c.n_shared_experts = 0;
-    if (R == 0) {
-        // No received rows: every routed segment is empty and its tensors are never
-        // addressed; the maps still need a valid base.
-        x_recv = x;
-        h_recv = h_shared;
-        y_recv = y_shared;
-        y_recv_scale = y_shared_scale;
+    if (R > 0) {
+        // The received rows' slots sorted by local expert: an expert id in this
+        // rank's block is a bucket, one of another rank's is no row, one outside
+        // [0, E) is a caller error.
+        const uint8_t* rows = static_cast<const uint8_t*>(recv_rows);
+        RowSort a{};
+        a.si = SlotIndex{reinterpret_cast<const int32_t*>(rows + 2ll * H), static_cast<int>(Wb / 4), rank * El, 0, E};
+        a.T = R;
+        a.K = K;
+        a.E = El;
+        a.H = H;
+        a.x = recv_rows;
+        a.x_ld = Wb / 2;
+        a.x_perm = w.x_perm;
+        a.out_ld = H;
+        a.offsets = w.offsets;
+        a.perm_src = w.perm_src;
+        a.row_of = w.row_of;
+        a.block_counts = w.block_counts;
+        a.block_base = w.block_base;
+        a.totals = w.totals;
+        a.w_src = reinterpret_cast<const float*>(rows + 2ll * H + 4ll * K);
+        a.w_perm = w.w_perm;
+        if ((v = launch_row_sort(a, st)) != MOE_OK) return v;
+    } else if (cudaMemsetAsync(w.offsets, 0, sizeof(int32_t) * (El + 1), st) != cudaSuccess) {
+        return MOE_ERR_CUDA;
     }
-    const RoutedRows rr{R, cfg->n_routed_experts, cfg->n_routed_experts / world, recv_offsets};
-    if ((v = launch_gate_up(&c, T, x, x_recv, rr, w_gate, w_up, ws_gate, ws_up, h_recv, h_shared, d->num_sms, st)) !=
-        MOE_OK)
+    const RoutedRows rr{Rb, El, El, w.offsets};
+    if ((v = launch_gate_up(&c, T, x, w.x_perm, rr, w_gate, w_up, ws_gate, ws_up, w.h_routed, w.h_shared, d->num_sms,
+                            st)) != MOE_OK)
         return v;
-    const ScaledRows yr{static_cast<__half*>(y_recv), static_cast<uint8_t*>(y_recv_scale)};
+    const ScaledRows yr{w.y_perm, w.y_scale};
     const ScaledRows ys{static_cast<__half*>(y_shared), static_cast<uint8_t*>(y_shared_scale)};
-    return launch_down(&c, T, h_recv, h_shared, rr, nullptr, w_recv, R, w_down, ws_down, yr, ys, d->num_sms, st);
+    if ((v = launch_down(&c, T, w.h_routed, w.h_shared, rr, nullptr, w.w_perm, Rb, w_down, ws_down, yr, ys,
+                         d->num_sms, st)) != MOE_OK)
+        return v;
+    if (R == 0) return MOE_OK;
+    // Each received row's sum over its slots on this rank, re-encoded for the way back.
+    CombineDst dst{};
+    dst.rows = ScaledRowsOut{static_cast<__half*>(return_rows), Wr / 2, static_cast<uint8_t*>(return_rows) + 2ll * H,
+                             Wr};
+    return launch_combine_rows(R, K, H, ScaledRowsIn{w.y_perm, H, w.y_scale, scale_ld(H)}, Rb, w.row_of, 1,
+                               ScaledRowsIn{nullptr, 0, nullptr, 0}, dst, kOutScaled, st);
+}
+
+int moe_ep_combine(const moe_config* cfg, int32_t world, int64_t T, int64_t n_back, const void* back_rows,
+                   const int32_t* send_row_of, const void* y_shared, const void* y_shared_scale, void* y,
+                   int32_t y_dtype, void* stream) {
+    int v = validate_ep(cfg, T, world);
+    if (v != MOE_OK) return v;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (n_back < 0 || n_back > ep_send_rows_max(cfg, T, world)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!send_row_of) return MOE_ERR_INVALID_ARG;
+    if ((v = check_ptrs({back_rows, y})) != MOE_OK) return v;
+    const bool sh = cfg->n_shared_experts > 0;
+    if (sh && (v = check_ptrs({y_shared, y_shared_scale})) != MOE_OK) return v;
+    const int64_t H = cfg->hidden_size, Wr = ep_return_row_bytes(cfg);
+    const uint8_t* b = static_cast<const uint8_t*>(back_rows);
+    const ScaledRowsIn routed{reinterpret_cast<const __half*>(b), Wr / 2, b + 2 * H, Wr};
+    const ScaledRowsIn shared = sh ? ScaledRowsIn{static_cast<const __half*>(y_shared), H,
+                                                  static_cast<const uint8_t*>(y_shared_scale), scale_ld(H)}
+                                   : ScaledRowsIn{nullptr, 0, nullptr, 0};
+    CombineDst dst{};
+    dst.y = y;
+    return launch_combine_rows(T, cfg->num_experts_per_tok, cfg->hidden_size, routed, n_back, send_row_of, 1, shared,
+                               dst, y_dtype == MOE_DTYPE_BF16 ? kOutBF16 : kOutF32, static_cast<cudaStream_t>(stream));
 }
 
 int moe_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

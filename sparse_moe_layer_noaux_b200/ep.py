@@ -4,16 +4,21 @@ The routed experts are spread over the `world` ranks of a process group, rank r
 holding experts [r * E/world, (r + 1) * E/world); the router and the shared
 experts are replicated, and every rank brings its own tokens ("DeepSeek-V3
 notes" (knlb.dev), § infrastructure: expert parallelism with all-to-all dispatch
-and combine; § architecture: a token's rows go to a limited number of nodes —
-with contiguous expert blocks per rank and groups that do not straddle ranks, to
-at most topk_group ranks).
+and combine; § architecture: a token goes to a limited number of nodes — with
+contiguous expert blocks per rank and groups that do not straddle ranks, to at
+most topk_group ranks).
+
+A token crosses to a rank once, however many of its experts live there: the
+source sends one row per (token, destination rank) carrying the token's values
+and routing, the destination runs all of the token's experts it holds and sends
+back one row, their weighted sum.  So each direction moves at most
+min(k, topk_group ranks) rows per token instead of k.
 
 Every step of the layer runs in libmoe (include/moe.h lists the sequence); this
 module only allocates the buffers and moves them between ranks with the process
-group's all-to-all (NCCL on GPUs): the per-expert counts, then the rows and their
-routing weights, and, after the experts, their outputs back to the ranks the
-rows came from.  The split sizes of an all-to-all are host integers, so the
-counts are read back to the host once per forward.
+group's all-to-all (NCCL on GPUs): the per-rank row counts, the send rows, and
+after the experts the return rows.  The split sizes of an all-to-all are host
+integers, so the counts are read back to the host once per forward.
 """
 from __future__ import annotations
 
@@ -33,28 +38,16 @@ class EPStep:
     T: int
     idx: torch.Tensor            # [T, k] int32
     w: torch.Tensor              # [T, k] fp32
-    offsets: torch.Tensor        # [E + 1] int32
-    x_perm: torch.Tensor         # [T*k, H] bf16, expert order
-    perm_src: torch.Tensor       # [T*k] int32
-    row_of: torch.Tensor         # [T, k] int32
-    counts: torch.Tensor         # [E] int32: rows per expert (sent to the experts' ranks)
-    w_perm: torch.Tensor         # [T*k] fp32: routing weight of each row
+    send_counts: torch.Tensor    # [world] int32: rows for each rank
+    send_rows: torch.Tensor      # [T * min(k, world), send_row_bytes] uint8, sorted by rank
+    send_row_of: torch.Tensor    # [T, k] int32: send row of a token's first slot on a rank, else -1
     send_splits: Optional[List[int]] = None   # rows to each rank
     recv_splits: Optional[List[int]] = None   # rows from each rank
-    recv_counts: Optional[torch.Tensor] = None  # [world, E/world] int32
-    recv_offsets: Optional[torch.Tensor] = None  # [E + 1] int32
-    x_recv: Optional[torch.Tensor] = None       # [R, H] bf16
-    w_recv: Optional[torch.Tensor] = None       # [R] fp32
-    y_recv: Optional[torch.Tensor] = None       # [R, H] fp16 (block-scaled)
-    y_recv_scale: Optional[torch.Tensor] = None
-    y_back: Optional[torch.Tensor] = None       # [T*k + T, H] fp16: returned rows, then shared rows
-    y_back_scale: Optional[torch.Tensor] = None
-
-
-def _wire(t: torch.Tensor) -> torch.Tensor:
-    """The tensor as a collective moves it: bf16 bits travel as fp16 (same size;
-    the collective copies, it never computes on them)."""
-    return t.view(torch.float16) if t.dtype == torch.bfloat16 else t
+    recv_rows: Optional[torch.Tensor] = None    # [R, send_row_bytes] uint8
+    return_rows: Optional[torch.Tensor] = None  # [R, return_row_bytes] uint8
+    back_rows: Optional[torch.Tensor] = None    # [sum(send_splits), return_row_bytes] uint8, send order
+    y_shared: Optional[torch.Tensor] = None     # [T, H] fp16 (block-scaled)
+    y_shared_scale: Optional[torch.Tensor] = None
 
 
 class MoELayerEP:
@@ -70,6 +63,8 @@ class MoELayerEP:
                  ws_gate=None, ws_up=None, ws_down=None, group=None, _kernels=None):
         if world < 1 or shape.E % world:
             raise ValueError(f"world {world} must divide n_routed_experts {shape.E}")
+        if not 0 <= rank < world:
+            raise ValueError(f"rank {rank} outside [0, {world})")
         self.shape, self.world, self.rank, self.group = shape, world, rank, group
         self.cfg = abi.MoEConfig.from_shape(shape)
         self.router_w, self.e_bias = router_w, e_bias
@@ -78,6 +73,7 @@ class MoELayerEP:
         self.device = router_w.device
         # The library binding; the CPU tests of the exchange pass a stand-in.
         self.lib = _kernels if _kernels is not None else abi
+        self.send_row_bytes, self.return_row_bytes = self.lib.ep_row_bytes(self.cfg)
         self._ws: Optional[torch.Tensor] = None
 
     @property
@@ -87,67 +83,53 @@ class MoELayerEP:
     def _empty(self, shape, dtype):
         return torch.empty(shape, dtype=dtype, device=self.device)
 
-    def _workspace(self, T: int) -> torch.Tensor:
-        need = max(self.lib.workspace_size(self.cfg, T), 256)
+    def _workspace(self, need: int) -> torch.Tensor:
+        need = max(need, 256)
         if self._ws is None or self._ws.numel() < need:
             self._ws = self._empty(need, torch.uint8)
         return self._ws
 
     # ---- phases (each a libmoe call; the collectives sit between them) ----
-    def route_and_pack(self, x: torch.Tensor) -> EPStep:
-        """Route the rank's tokens, sort their rows into expert order, count them."""
+    def send(self, x: torch.Tensor) -> EPStep:
+        """Route the rank's tokens and build their send rows, one per (token, rank)."""
         s, L = self.shape, self.lib
-        T, k, E, H = x.shape[0], s.k, s.E, s.H
+        T, k = x.shape[0], s.k
+        n_max = L.ep_send_rows_max(self.cfg, T, self.world)
         st = EPStep(T=T, idx=self._empty((T, k), torch.int32), w=self._empty((T, k), torch.float32),
-                    offsets=self._empty(E + 1, torch.int32), x_perm=self._empty((T * k, H), torch.bfloat16),
-                    perm_src=self._empty(T * k, torch.int32), row_of=self._empty((T, k), torch.int32),
-                    counts=self._empty(E, torch.int32), w_perm=self._empty(T * k, torch.float32))
-        ws = self._workspace(T)
+                    send_counts=self._empty(self.world, torch.int32),
+                    send_rows=self._empty((n_max, self.send_row_bytes), torch.uint8),
+                    send_row_of=self._empty((T, k), torch.int32))
+        ws = self._workspace(max(L.workspace_size(self.cfg, T), L.ep_workspace_size(self.cfg, self.world, T, 0)))
         if T:
             L.moe_route(self.cfg, x, self.router_w, self.e_bias, st.idx, st.w, ws)
-        L.moe_dispatch(self.cfg, x, st.idx, st.offsets, st.x_perm, st.perm_src, st.row_of, ws)
-        L.moe_ep_pack(self.cfg, T, st.offsets, st.perm_src, st.w, st.counts, st.w_perm)
+        L.moe_ep_send(self.cfg, self.world, x, st.idx, st.w, st.send_counts, st.send_rows, st.send_row_of, ws)
         return st
 
     def plan(self, st: EPStep, recv_counts: torch.Tensor) -> None:
-        """From the counts this rank received ([world, E/world], source-major): the
-        split sizes of the row exchange, the received segments' offsets, and the
-        receive and return buffers."""
-        s, L = self.shape, self.lib
-        El = self.experts_per_rank
-        st.recv_counts = recv_counts
-        sent = st.counts.cpu().view(self.world, El).sum(1)
-        got = recv_counts.cpu().view(self.world, El).sum(1)
-        st.send_splits = [int(v) for v in sent]
-        st.recv_splits = [int(v) for v in got]
+        """From the row counts this rank received ([world], one per source): the split
+        sizes of the exchanges and the receive, return and back buffers."""
+        s = self.shape
+        both = torch.stack([st.send_counts, recv_counts]).cpu()
+        st.send_splits = [int(v) for v in both[0]]
+        st.recv_splits = [int(v) for v in both[1]]
         R = sum(st.recv_splits)
-        st.recv_offsets = self._empty(s.E + 1, torch.int32)
-        L.moe_ep_recv_offsets(self.cfg, self.world, recv_counts, st.recv_offsets)
-        H = s.H
-        st.x_recv = self._empty((R, H), torch.bfloat16)
-        st.w_recv = self._empty(R, torch.float32)
-        st.y_recv = self._empty((R, H), torch.float16)
-        st.y_recv_scale = self._empty((R, L.y_perm_scale_cols(H)), torch.uint8)
-        n_back = st.T * s.k + (st.T if s.S else 0)
-        st.y_back = self._empty((n_back, H), torch.float16)
-        st.y_back_scale = self._empty((n_back, L.y_perm_scale_cols(H)), torch.uint8)
+        st.recv_rows = self._empty((R, self.send_row_bytes), torch.uint8)
+        st.return_rows = self._empty((R, self.return_row_bytes), torch.uint8)
+        st.back_rows = self._empty((sum(st.send_splits), self.return_row_bytes), torch.uint8)
+        st.y_shared = self._empty((st.T, s.H), torch.float16)
+        st.y_shared_scale = self._empty((st.T, self.lib.y_perm_scale_cols(s.H)), torch.uint8)
 
     def experts(self, st: EPStep, x: torch.Tensor) -> None:
-        """The rank's expert GEMMs over the received rows; the shared experts over its own tokens."""
-        s, L = self.shape, self.lib
-        R, H, I = st.x_recv.shape[0], s.H, s.I
-        tk = st.T * s.k
-        h_recv = self._empty((R, I), torch.bfloat16)
-        shared = s.S > 0 and st.T > 0
-        h_shared = self._empty((st.T, s.S * I), torch.bfloat16) if shared else None
-        L.moe_ep_experts(self.cfg, self.world, st.T, x if shared else None, st.x_recv, st.recv_offsets, st.w_recv,
-                         self.w_gate, self.w_up, self.w_down, self.ws_gate, self.ws_up, self.ws_down, h_recv,
-                         h_shared, st.y_recv, st.y_recv_scale, st.y_back[tk:] if shared else None,
-                         st.y_back_scale[tk:] if shared else None)
+        """The rank's experts over the received rows; the shared experts over its own tokens."""
+        L = self.lib
+        R = st.recv_rows.shape[0]
+        ws = self._workspace(L.ep_workspace_size(self.cfg, self.world, st.T, R))
+        L.moe_ep_experts(self.cfg, self.world, self.rank, x, st.recv_rows, self.w_gate, self.w_up, self.w_down,
+                         self.ws_gate, self.ws_up, self.ws_down, st.return_rows, st.y_shared, st.y_shared_scale, ws)
 
     def combine(self, st: EPStep, out_dtype=torch.float32) -> torch.Tensor:
         y = self._empty((st.T, self.shape.H), out_dtype)
-        self.lib.moe_combine(self.cfg, st.T, st.y_back, st.y_back_scale, st.row_of, y)
+        self.lib.moe_ep_combine(self.cfg, self.world, st.back_rows, st.send_row_of, st.y_shared, st.y_shared_scale, y)
         return y
 
     # ---- the forward with the process group's all-to-all ----
@@ -156,16 +138,14 @@ class MoELayerEP:
         group must call it (each with its own batch) in the same order."""
         import torch.distributed as dist
         g = self.group
-        st = self.route_and_pack(x)
-        recv_counts = torch.empty_like(st.counts)
-        dist.all_to_all_single(recv_counts, st.counts, group=g)  # E/world counts to each rank
+        st = self.send(x)
+        recv_counts = torch.empty_like(st.send_counts)
+        dist.all_to_all_single(recv_counts, st.send_counts, group=g)  # one count to each rank
         self.plan(st, recv_counts)
-        tk = st.T * self.shape.k
-        dist.all_to_all_single(_wire(st.x_recv), _wire(st.x_perm[:tk]), st.recv_splits, st.send_splits, group=g)
-        dist.all_to_all_single(st.w_recv, st.w_perm[:tk], st.recv_splits, st.send_splits, group=g)
+        n_send = sum(st.send_splits)
+        dist.all_to_all_single(st.recv_rows, st.send_rows[:n_send], st.recv_splits, st.send_splits, group=g)
         self.experts(st, x)
-        dist.all_to_all_single(st.y_back[:tk], st.y_recv, st.send_splits, st.recv_splits, group=g)
-        dist.all_to_all_single(st.y_back_scale[:tk], st.y_recv_scale, st.send_splits, st.recv_splits, group=g)
+        dist.all_to_all_single(st.back_rows, st.return_rows, st.send_splits, st.recv_splits, group=g)
         return self.combine(st, out_dtype)
 
     __call__ = forward

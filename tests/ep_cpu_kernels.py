@@ -1,18 +1,19 @@
 """A CPU stand-in for the libmoe calls that MoELayerEP makes, built on the float64
-oracle (test infrastructure: it lets the expert-parallel exchange — counts,
-split sizes, segment offsets, the return of the outputs and their reassembly —
-run over gloo ranks on a machine without a GPU).
+oracle (test infrastructure: it lets the expert-parallel exchange — the send rows,
+their counts and split sizes, the return of the sums and their reassembly — run
+over gloo ranks on a machine without a GPU).
 
 Each function keeps the contract include/moe.h states for the library call of
-the same name, on CPU tensors:
-  moe_route           oracle routing (float64), weights stored as fp32
-  moe_dispatch        stable counting sort of the (token, slot) entries by expert
-  moe_ep_pack         per-expert counts, routing weight per row
-  moe_ep_recv_offsets exclusive prefix sum of the received counts
-  moe_ep_experts      oracle SwiGLU per segment (local expert = segment % E/world),
-                      outputs in the block-scaled fp16 format with scale code 141
-                      (factor 1), i.e. plain fp16 values
-  moe_combine         shared row + the token's k rows, decoded, summed in fp32
+the same name, on CPU tensors, wire formats included:
+  send row    H bf16 values, k int32 expert ids, k fp32 weights, zeros to 16 bytes
+  return row  H fp16 values, H/32 scale codes, zeros to 16 bytes; this stand-in
+              always writes code 141 (factor 2^0), i.e. plain fp16 values
+  moe_route       oracle routing (float64), weights stored as fp32
+  moe_ep_send     one row per (token, rank of one of its experts), sorted by rank
+                  and token; send_row_of marks the token's first slot on the rank
+  moe_ep_experts  per received row, the float64 sum over its slots on this rank
+                  of w * SwiGLU_e(x); the shared experts over the rank's own tokens
+  moe_ep_combine  shared row + the token's returned rows, decoded, summed in fp32
 """
 from __future__ import annotations
 
@@ -25,7 +26,24 @@ from sparse_moe_layer_noaux_b200.workloads import bf16_bits
 _UNIT_CODE = 141  # block-scale code whose factor is 2^(141 - 141) = 1
 
 
+def _pad16(n):
+    return (n + 15) // 16 * 16
+
+
+def ep_row_bytes(cfg):
+    H, k = cfg.hidden_size, cfg.num_experts_per_tok
+    return 2 * H + _pad16(8 * k), 2 * H + _pad16(H // 32)
+
+
+def ep_send_rows_max(cfg, T, world):
+    return T * min(cfg.num_experts_per_tok, world)
+
+
 def workspace_size(cfg, T):
+    return 256
+
+
+def ep_workspace_size(cfg, world, T, R):
     return 256
 
 
@@ -33,40 +51,36 @@ def y_perm_scale_cols(H):
     return (H // 32 + 7) // 8 * 8
 
 
-def _shape(cfg):
-    return cfg  # the MoEConfig fields are all the oracle reads
-
-
 def moe_route(cfg, x, router_w, e_bias, topk_idx, topk_w, workspace=None):
-    idx, w, _ = oracle.route(_shape(cfg), bf16_bits(x), router_w.numpy(), e_bias.numpy())
+    idx, w, _ = oracle.route(cfg, bf16_bits(x), router_w.numpy(), e_bias.numpy())
     topk_idx.copy_(torch.from_numpy(idx))
     topk_w.copy_(torch.from_numpy(w.astype(np.float32)))
 
 
-def moe_dispatch(cfg, x, topk_idx, expert_offsets, x_perm, perm_src, row_of, workspace=None):
-    k, E = cfg.num_experts_per_tok, cfg.n_routed_experts
-    flat = topk_idx.numpy().reshape(-1).astype(np.int64)
-    order = np.argsort(flat, kind="stable")
-    counts = np.bincount(flat, minlength=E)
-    expert_offsets.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)))
-    perm_src.copy_(torch.from_numpy(order.astype(np.int32)))
-    inv = np.empty_like(order)
-    inv[order] = np.arange(order.size)
-    row_of.copy_(torch.from_numpy(inv.reshape(row_of.shape).astype(np.int32)))
-    if order.size:
-        x_perm.copy_(x[torch.from_numpy(order // k)])
-
-
-def moe_ep_pack(cfg, T, expert_offsets, perm_src, topk_w, expert_counts, w_perm):
-    off = expert_offsets.numpy().astype(np.int64)
-    expert_counts.copy_(torch.from_numpy((off[1:] - off[:-1]).astype(np.int32)))
-    if perm_src.numel():
-        w_perm.copy_(topk_w.reshape(-1)[perm_src.long()])
-
-
-def moe_ep_recv_offsets(cfg, world, recv_counts, recv_offsets):
-    c = recv_counts.numpy().reshape(-1).astype(np.int64)
-    recv_offsets.copy_(torch.from_numpy(np.concatenate([[0], np.cumsum(c)]).astype(np.int32)))
+def moe_ep_send(cfg, world, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace=None):
+    T, H, k = x.shape[0], cfg.hidden_size, cfg.num_experts_per_tok
+    El = cfg.n_routed_experts // world
+    idx, w = topk_idx.numpy(), topk_w.numpy()
+    entries = []                                   # (rank, token, slot), the token's first slot on the rank
+    for t in range(T):
+        ranks = set()
+        for j in range(k):
+            d = int(idx[t, j]) // El
+            if d not in ranks:
+                ranks.add(d)
+                entries.append((d, t, j))
+    entries.sort(key=lambda e: (e[0], e[1]))
+    send_counts.copy_(torch.from_numpy(np.bincount([e[0] for e in entries], minlength=world).astype(np.int32)))
+    row_of = np.full((T, k), -1, np.int32)
+    rows = send_rows.numpy()
+    xb = bf16_bits(x)
+    for r, (d, t, j) in enumerate(entries):
+        row_of[t, j] = r
+        rows[r] = 0
+        rows[r, :2 * H] = xb[t].view(np.uint8)
+        rows[r, 2 * H:2 * H + 4 * k] = idx[t].astype("<i4").view(np.uint8)
+        rows[r, 2 * H + 4 * k:2 * H + 8 * k] = w[t].astype("<f4").view(np.uint8)
+    send_row_of.copy_(torch.from_numpy(row_of))
 
 
 def _store_unit_scale(values, scales, rows_f64):
@@ -74,30 +88,47 @@ def _store_unit_scale(values, scales, rows_f64):
     scales.fill_(_UNIT_CODE)
 
 
-def moe_ep_experts(cfg, world, T, x, x_recv, recv_offsets, w_recv, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
-                   h_recv, h_shared, y_recv, y_recv_scale, y_shared, y_shared_scale):
+def moe_ep_experts(cfg, world, rank, x, recv_rows, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, return_rows,
+                   y_shared, y_shared_scale, workspace=None):
+    H, k = cfg.hidden_size, cfg.num_experts_per_tok
     El = cfg.n_routed_experts // world
-    off = recv_offsets.numpy().astype(np.int64)
-    xb = bf16_bits(x_recv)
-    out = np.zeros((x_recv.shape[0], cfg.hidden_size), np.float64)
-    for s in range(cfg.n_routed_experts):
-        a, b = off[s], off[s + 1]
-        if b > a:
-            e = s % El
-            o = oracle.swiglu(xb[a:b], bf16_bits(w_gate[e]), bf16_bits(w_up[e]), bf16_bits(w_down[e]))
-            out[a:b] = w_recv[a:b].numpy().astype(np.float64)[:, None] * o
-    _store_unit_scale(y_recv, y_recv_scale, out)
-    if cfg.n_shared_experts > 0 and T > 0:
+    rows = recv_rows.numpy()
+    R = rows.shape[0]
+    xb = np.ascontiguousarray(rows[:, :2 * H]).view(np.uint16)
+    ids = np.ascontiguousarray(rows[:, 2 * H:2 * H + 4 * k]).view("<i4")
+    wts = np.ascontiguousarray(rows[:, 2 * H + 4 * k:2 * H + 8 * k]).view("<f4")
+    out = np.zeros((R, H), np.float64)
+    for e_local in range(El):
+        r_sel, j_sel = np.nonzero(ids == rank * El + e_local)
+        if r_sel.size:
+            o = oracle.swiglu(xb[r_sel], bf16_bits(w_gate[e_local]), bf16_bits(w_up[e_local]),
+                              bf16_bits(w_down[e_local]))
+            np.add.at(out, r_sel, wts[r_sel, j_sel].astype(np.float64)[:, None] * o)
+    ret = return_rows.numpy()
+    ret[:] = 0
+    if R:
+        ret[:, :2 * H] = out.astype(np.float16).view(np.uint8)
+        ret[:, 2 * H:2 * H + H // 32] = _UNIT_CODE
+    if cfg.n_shared_experts > 0 and x.shape[0] > 0:
         o = oracle.swiglu(bf16_bits(x), bf16_bits(ws_gate), bf16_bits(ws_up), bf16_bits(ws_down))
         _store_unit_scale(y_shared, y_shared_scale, o)
 
 
-def moe_combine(cfg, T, y_perm, y_perm_scale, row_of, y):
-    k, H = cfg.num_experts_per_tok, cfg.hidden_size
-    codes = y_perm_scale[:, : H // 32].to(torch.int32)
-    f = torch.ldexp(torch.ones_like(codes, dtype=torch.float32), codes - 141)
-    v = (y_perm.float().view(-1, H // 32, 32) * f[:, :, None]).view(-1, H)
-    acc = v[T * k:T * k + T].clone() if cfg.n_shared_experts > 0 else torch.zeros((T, H))
+def _decode(values_f16, codes):
+    n, H = values_f16.shape
+    f = np.ldexp(1.0, codes.astype(np.int64) - 141)
+    return (values_f16.astype(np.float32).reshape(n, H // 32, 32) * f[:, :, None]).reshape(n, H)
+
+
+def moe_ep_combine(cfg, world, back_rows, send_row_of, y_shared, y_shared_scale, y):
+    T, H, k = y.shape[0], cfg.hidden_size, cfg.num_experts_per_tok
+    rows = back_rows.numpy()
+    vals = _decode(np.ascontiguousarray(rows[:, :2 * H]).view(np.float16), rows[:, 2 * H:2 * H + H // 32])
+    acc = np.zeros((T, H), np.float32)
+    if cfg.n_shared_experts > 0 and T:
+        acc += _decode(y_shared.numpy(), y_shared_scale.numpy()[:, :H // 32])
+    row_of = send_row_of.numpy()
     for j in range(k):
-        acc += v[row_of[:, j].long()]
-    y.copy_(acc)
+        live = row_of[:, j] >= 0
+        acc[live] += vals[row_of[live, j]]
+    y.copy_(torch.from_numpy(acc))

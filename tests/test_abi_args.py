@@ -18,7 +18,8 @@ NOSHARED = MoEShape("noshared", T=50, hidden_size=256, n_routed_experts=16, n_gr
                     num_experts_per_tok=3, moe_intermediate_size=128, n_shared_experts=0,
                     routed_scaling_factor=1.0, norm_topk_prob=True, seed=9)
 HOST_QUERIES = ("moe_workspace_size", "moe_workspace_size_mx", "moe_workspace_size_bwd",
-                "moe_workspace_size_host", "moe_mx_routed_rows", "moe_mx_scale_bytes", "moe_status_string")
+                "moe_workspace_size_host", "moe_mx_routed_rows", "moe_mx_scale_bytes", "moe_status_string",
+                "moe_ep_row_bytes", "moe_ep_workspace_size")
 
 
 class _Recorder:
@@ -108,17 +109,21 @@ def run_all(s):
     # expert parallelism (world 2: this rank holds E/2 experts and receives R rows)
     world, R = 2, 7
     El = E // world
-    abi.moe_ep_pack(cfg, T, offsets, perm_src, w, counts, e(T * k, dtype=f32))
-    abi.moe_ep_recv_offsets(cfg, world, e(E, dtype=i32), e(E + 1, dtype=i32))
-    abi.moe_ep_experts(cfg, world, T, L["x"], e(R, H), e(E + 1, dtype=i32), e(R, dtype=f32), e(El, I, H),
-                       e(El, I, H), e(El, H, I), L["ws_gate"], L["ws_up"], L["ws_down"], e(R, I), h_s,
-                       e(R, H, dtype=f16), e(R, abi.y_perm_scale_cols(H), dtype=u8), y_perm[T * k:], y_sc[T * k:])
+    Wb, Wr = abi.ep_row_bytes(cfg)
+    n_send = abi.ep_send_rows_max(cfg, T, world)
+    ws_ep = e(abi.ep_workspace_size(cfg, world, T, R), dtype=u8)
+    send_row_of = e(T, k, dtype=i32)
+    abi.moe_ep_send(cfg, world, L["x"], idx, w, e(world, dtype=i32), e(n_send, Wb, dtype=u8), send_row_of, ws_ep)
+    y_sh, y_sh_sc = e(T, H, dtype=f16), e(T, abi.y_perm_scale_cols(H), dtype=u8)
+    abi.moe_ep_experts(cfg, world, 1, L["x"], e(R, Wb, dtype=u8), e(El, I, H), e(El, I, H), e(El, H, I),
+                       L["ws_gate"], L["ws_up"], L["ws_down"], e(R, Wr, dtype=u8), y_sh, y_sh_sc, ws_ep)
+    abi.moe_ep_combine(cfg, world, e(n_send, Wr, dtype=u8), send_row_of, y_sh, y_sh_sc, e(T, H, dtype=f32))
 
 
 @pytest.mark.parametrize("shape", [TINY, NOSHARED, TINY.with_(name="empty", T=0)], ids=lambda s: s.name)
 def test_valid_buffers_reach_the_library(rec, shape):
     run_all(shape)
-    assert len(rec.calls) == 25 and "moe_backward_train" in rec.calls and "moe_ep_experts" in rec.calls
+    assert len(rec.calls) == 25 and "moe_backward_train" in rec.calls and "moe_ep_combine" in rec.calls
 
 
 def test_bad_arguments_are_rejected_before_the_call(rec):
@@ -130,6 +135,7 @@ def test_bad_arguments_are_rejected_before_the_call(rec):
     idx, w = e(T, k, dtype=torch.int32), e(T, k, dtype=torch.float32)
     y = e(T, H, dtype=torch.float32)
     ws = e(256, dtype=torch.uint8)
+    Wb, Wr = abi.ep_row_bytes(cfg)
     bad = [
         (TypeError, lambda: abi.moe_forward(cfg, L["x"], L["router_w"].bfloat16(), L["e_bias"], *W, y)),
         (TypeError, lambda: abi.moe_forward(cfg, L["x"].float(), L["router_w"], L["e_bias"], *W, y)),
@@ -148,14 +154,23 @@ def test_bad_arguments_are_rejected_before_the_call(rec):
         (TypeError, lambda: abi.moe_combine(cfg, T, e(T * k + T, H), e(T * k + T, 8, dtype=torch.uint8),
                                             idx, y)),   # y_perm must be fp16
         (TypeError, lambda: abi.moe_forward_host(cfg, L["x"], L["router_w"], L["e_bias"], *W, [0.0], 0, ws)),
-        (ValueError, lambda: abi.moe_ep_experts(cfg, 3, T, L["x"], e(4, H), e(E + 1, dtype=torch.int32),
-                                                e(4, dtype=torch.float32), *W, e(4, I), e(T, I),
-                                                e(4, H, dtype=torch.float16), e(4, 8, dtype=torch.uint8),
-                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8))),
-        (ValueError, lambda: abi.moe_ep_experts(cfg, 2, T, L["x"], e(4, H), e(E + 1, dtype=torch.int32),
-                                                e(3, dtype=torch.float32), *W, e(4, I), e(T, I),
-                                                e(4, H, dtype=torch.float16), e(4, 8, dtype=torch.uint8),
-                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8))),
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 3, 0, L["x"], e(4, Wb, dtype=torch.uint8), *W,
+                                                e(4, Wr, dtype=torch.uint8), e(T, H, dtype=torch.float16),
+                                                e(T, 8, dtype=torch.uint8), ws)),   # 3 does not divide E
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 2, 2, L["x"], e(4, Wb, dtype=torch.uint8), *W,
+                                                e(4, Wr, dtype=torch.uint8), e(T, H, dtype=torch.float16),
+                                                e(T, 8, dtype=torch.uint8), ws)),   # rank outside [0, 2)
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 2, 0, L["x"], e(4, Wb, dtype=torch.uint8), *W,
+                                                e(3, Wr, dtype=torch.uint8), e(T, H, dtype=torch.float16),
+                                                e(T, 8, dtype=torch.uint8), ws)),   # fewer return rows than received
+        (ValueError, lambda: abi.moe_ep_send(cfg, 2, L["x"], idx, w, e(2, dtype=torch.int32),
+                                             e(T * 2, Wb - 16, dtype=torch.uint8), idx, ws)),   # row width
+        (ValueError, lambda: abi.moe_ep_send(cfg, 2, L["x"], idx, w, e(2, dtype=torch.int32),
+                                             e(T * 2 - 1, Wb, dtype=torch.uint8), idx, ws)),   # too few rows
+        (TypeError, lambda: abi.moe_ep_combine(cfg, 2, e(T, Wr, dtype=torch.uint8), idx.float(),
+                                               e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8), y)),
+        (ValueError, lambda: abi.moe_ep_combine(cfg, 2, e(2 * T + 1, Wr, dtype=torch.uint8), idx,
+                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8), y)),
     ]
     for exc, call in bad:
         with pytest.raises(exc):

@@ -2,8 +2,9 @@
 its all-to-alls over a real process group, the library calls replaced by the
 oracle-backed stand-in of tests/ep_cpu_kernels.py.  Each rank holds E/world of
 the routed experts and its own tokens; every rank's output must equal the float64
-oracle's single-device layer on its tokens, and the rows a rank receives must be
-exactly the other ranks' rows for its experts."""
+oracle's single-device layer on its tokens; a token must cross to each rank that
+holds one of its experts exactly once; and the rows a rank receives must be
+exactly the other ranks' send rows for it, in rank order."""
 import os
 import socket
 
@@ -48,11 +49,13 @@ def _worker(rank, world, port, out):
                        _kernels=ep_cpu_kernels)
     x = _rank_tokens(shape, rank)
     y = layer(x)
-    # The same batch through the exchange phases by hand, to look at what arrived.
-    st = layer.route_and_pack(x)
-    recv = torch.empty_like(st.counts)
-    dist.all_to_all_single(recv, st.counts)
+    # The same batch through the exchange phases by hand, to look at what moved.
+    st = layer.send(x)
+    recv = torch.empty_like(st.send_counts)
+    dist.all_to_all_single(recv, st.send_counts)
     layer.plan(st, recv)
+    n_send = sum(st.send_splits)
+    dist.all_to_all_single(st.recv_rows, st.send_rows[:n_send], st.recv_splits, st.send_splits)
     # The oracle's single-device layer on this rank's tokens (all experts).
     fetch = oracle.in_memory_experts(bf16_bits(inp["w_gate"]), bf16_bits(inp["w_up"]), bf16_bits(inp["w_down"]))
     shared = tuple(bf16_bits(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
@@ -60,7 +63,8 @@ def _worker(rank, world, port, out):
                                             fetch, shared)
     out[rank] = {"y": y.numpy(), "y_ref": y_ref, "idx": st.idx.numpy(), "idx_ref": idx_ref,
                  "recv_counts": recv.numpy(), "send_splits": st.send_splits, "recv_splits": st.recv_splits,
-                 "recv_offsets": st.recv_offsets.numpy()}
+                 "send_rows": st.send_rows[:n_send].numpy(), "recv_rows": st.recv_rows.numpy(),
+                 "send_row_of": st.send_row_of.numpy()}
     dist.barrier()
     dist.destroy_process_group()
 
@@ -74,6 +78,7 @@ def test_expert_parallel_exchange_matches_the_single_device_layer(world, oracle_
         res = dict(out)
     El = SHAPE.E // world
     gsz = SHAPE.E // SHAPE.n_group
+    H, k = SHAPE.H, SHAPE.k
     for r in range(world):
         d = res[r]
         assert (d["idx"] == d["idx_ref"]).all()
@@ -81,15 +86,29 @@ def test_expert_parallel_exchange_matches_the_single_device_layer(world, oracle_
             rms = np.sqrt(np.mean(d["y_ref"] ** 2))
             err = np.abs(d["y"] - d["y_ref"]).max() / rms
             assert err <= 2e-2, (r, err)   # fp16 storage of the expert outputs
-        # Rows sent to rank d are this rank's rows for d's experts; rank d receives
-        # exactly what every source sent it, counted per (source, local expert).
+        # One row per (token, rank holding one of its experts), at the token's first
+        # slot on that rank; rows sorted by rank, tokens ascending within a rank.
+        ranks = d["idx"] // El
+        off = np.concatenate([[0], np.cumsum(d["send_splits"])])
+        for t in range(d["idx"].shape[0]):
+            first = [j for j in range(k) if ranks[t, j] not in ranks[t, :j]]
+            assert sorted(np.nonzero(d["send_row_of"][t] >= 0)[0].tolist()) == first
+            for j in first:
+                row = d["send_row_of"][t, j]
+                assert off[ranks[t, j]] <= row < off[ranks[t, j] + 1]
+                # The row carries x[t]'s routing: the token's k expert ids.
+                np.testing.assert_array_equal(d["send_rows"][row, 2 * H:2 * H + 4 * k].view("<i4"), d["idx"][t])
         for dst in range(world):
-            sent_counts = np.bincount(d["idx"].reshape(-1), minlength=SHAPE.E)[dst * El:(dst + 1) * El]
-            assert d["send_splits"][dst] == sent_counts.sum()
-            np.testing.assert_array_equal(res[dst]["recv_counts"].reshape(world, El)[r], sent_counts)
-            assert res[dst]["recv_splits"][r] == sent_counts.sum()
-        np.testing.assert_array_equal(d["recv_offsets"], np.concatenate([[0], np.cumsum(d["recv_counts"])]))
-        # Groups do not straddle ranks here, so a token's rows reach at most topk_group ranks.
+            # Tokens with an expert on dst, ascending, hold rows off[dst], off[dst] + 1, ...
+            rows_dst = [int(d["send_row_of"][t][(ranks[t] == dst) & (d["send_row_of"][t] >= 0)][0])
+                        for t in range(d["idx"].shape[0]) if (ranks[t] == dst).any()]
+            assert rows_dst == list(range(off[dst], off[dst + 1]))
+            assert res[dst]["recv_counts"][r] == d["send_splits"][dst] == res[dst]["recv_splits"][r]
+            # What dst received from r is r's send rows for dst, byte for byte.
+            r0 = sum(res[dst]["recv_splits"][:r])
+            np.testing.assert_array_equal(res[dst]["recv_rows"][r0:r0 + d["send_splits"][dst]],
+                                          d["send_rows"][off[dst]:off[dst + 1]])
+        # Groups do not straddle ranks here, so a token reaches at most topk_group ranks.
         if El % gsz == 0 and d["idx"].size:
-            ranks_per_token = [len({int(e) // El for e in row}) for row in d["idx"]]
-            assert max(ranks_per_token) <= SHAPE.topk_group
+            assert max(len(set(row.tolist())) for row in ranks) <= SHAPE.topk_group
+            assert (d["send_row_of"] >= 0).sum(1).max() <= SHAPE.topk_group

@@ -1,13 +1,15 @@
 """The expert-parallel layer on the GPU (libmoe's moe_ep_* calls).
 
   * world = 1 over a real NCCL process group: MoELayerEP.forward through the
-    same code path as on many GPUs equals moe_forward bit for bit (one source
-    rank, so the received segments are the dispatch's own).
+    same code path as on many GPUs matches moe_forward (up to the fp16 rounding
+    of the returned sums) and repeats bit for bit.
   * world = 2, 4 and 8 on one GPU: every rank's phases run on this GPU and the
     all-to-alls are done by copying each rank's row blocks into the others'
     receive buffers (no kernel waits on another, so nothing can deadlock); each
     rank's output is checked against moe_forward on its tokens and, on a sample,
-    against the float64 oracle."""
+    against the float64 oracle.
+  * the send rows, counts and slot map of moe_ep_send byte for byte against a
+    host restatement of the contract, and the block encoding of the return rows."""
 import datetime
 import os
 import socket
@@ -47,28 +49,44 @@ def _layers(shape, inp, world):
 def loopback_forward(layers, xs):
     """All ranks' phases on this GPU, the all-to-alls done as copies of row blocks."""
     W = len(layers)
-    E = layers[0].shape.E
-    El = E // W
-    steps = [L.route_and_pack(x) for L, x in zip(layers, xs)]
+    steps = [L.send(x) for L, x in zip(layers, xs)]
+    counts = [st.send_counts.cpu().tolist() for st in steps]      # counts[s][d]: rows of s for d
     for d in range(W):
-        layers[d].plan(steps[d], torch.cat([steps[s].counts[d * El:(d + 1) * El] for s in range(W)]))
-    off = [st.offsets.cpu().tolist() for st in steps]
-    block = lambda s, d: (off[s][d * El], off[s][(d + 1) * El])  # noqa: E731  rows of s bound for d
+        layers[d].plan(steps[d], torch.tensor([counts[s][d] for s in range(W)], dtype=torch.int32, device="cuda"))
+    off = [np.concatenate([[0], np.cumsum(c)]).astype(int) for c in counts]
     for d in range(W):
-        steps[d].x_recv.copy_(torch.cat([steps[s].x_perm[slice(*block(s, d))] for s in range(W)]))
-        steps[d].w_recv.copy_(torch.cat([steps[s].w_perm[slice(*block(s, d))] for s in range(W)]))
+        if steps[d].recv_rows.shape[0]:
+            steps[d].recv_rows.copy_(torch.cat([steps[s].send_rows[off[s][d]:off[s][d + 1]] for s in range(W)]))
     for d in range(W):
         layers[d].experts(steps[d], xs[d])
     for s in range(W):
         for d in range(W):
-            a, b = block(s, d)
+            a, b = off[s][d], off[s][d + 1]
             r0 = sum(steps[d].recv_splits[:s])
-            steps[s].y_back[a:b].copy_(steps[d].y_recv[r0:r0 + b - a])
-            steps[s].y_back_scale[a:b].copy_(steps[d].y_recv_scale[r0:r0 + b - a])
+            steps[s].back_rows[a:b].copy_(steps[d].return_rows[r0:r0 + b - a])
     ys = [L.combine(st) for L, st in zip(layers, steps)]
     torch.cuda.synchronize()
     assert abi.device_status() == 0
     return ys, steps
+
+
+def host_send(idx, w, x_bits, world, E, row_bytes):
+    """moe_ep_send's outputs restated on the host: one row per (token, rank of one of
+    its experts) at the token's first slot on that rank, rows by rank then token."""
+    T, k = idx.shape
+    H = x_bits.shape[1]
+    El = E // world
+    entries = sorted(((int(idx[t, j]) // El, t, j) for t in range(T) for j in range(k)
+                      if int(idx[t, j]) // El not in (idx[t, :j] // El)), key=lambda e: (e[0], e[1]))
+    counts = np.bincount([e[0] for e in entries], minlength=world).astype(np.int32)
+    row_of = np.full((T, k), -1, np.int32)
+    rows = np.zeros((len(entries), row_bytes), np.uint8)
+    for r, (_, t, j) in enumerate(entries):
+        row_of[t, j] = r
+        rows[r, :2 * H] = x_bits[t].view(np.uint8)
+        rows[r, 2 * H:2 * H + 4 * k] = idx[t].astype("<i4").view(np.uint8)
+        rows[r, 2 * H + 4 * k:2 * H + 8 * k] = w[t].astype("<f4").view(np.uint8)
+    return counts, row_of, rows
 
 
 def _free_port():
@@ -77,7 +95,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_world_one_over_nccl_equals_moe_forward():
+def test_world_one_over_nccl_matches_moe_forward():
     import torch.distributed as dist
     shape = SMALL
     inp = make_inputs(shape, "cuda")
@@ -93,8 +111,29 @@ def test_world_one_over_nccl_equals_moe_forward():
         dist.destroy_process_group()
     assert abi.device_status() == 0
     y_ref = MoELayer.from_inputs(shape, inp)(inp["x"])
-    assert torch.equal(y.view(torch.int32), y_ref.view(torch.int32))
+    # One row per token each way: the returned row is the token's k weighted expert
+    # outputs summed in fp32 and stored once more as block-scaled fp16.
+    parity.assert_output_close(y.cpu().numpy(), y_ref.cpu().numpy(), "world 1 vs moe_forward")
     assert torch.equal(y2, y)
+
+
+@pytest.mark.parametrize("world", [1, 4, 8])
+def test_send_rows_match_the_contract(world):
+    shape = V3_DECODE
+    inp = make_inputs(shape, "cuda")
+    layer = _layers(shape, inp, world)[0]
+    st = layer.send(inp["x"])
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    idx, w = st.idx.cpu().numpy(), st.w.cpu().numpy()
+    counts, row_of, rows = host_send(idx, w, bf16_bits(inp["x"]), world, shape.E, layer.send_row_bytes)
+    np.testing.assert_array_equal(st.send_counts.cpu().numpy(), counts)
+    np.testing.assert_array_equal(st.send_row_of.cpu().numpy(), row_of)
+    np.testing.assert_array_equal(st.send_rows[:rows.shape[0]].cpu().numpy(), rows)
+    if world == 8:   # 32 experts per rank = one expert group per rank
+        assert (row_of >= 0).sum(1).max() <= shape.topk_group
+        print(f"world 8: {rows.shape[0]} send rows for {idx.shape[0]} tokens "
+              f"({rows.shape[0] / idx.shape[0]:.2f} per token; k = {shape.k} without the per-rank merge)")
 
 
 @pytest.mark.parametrize("shape,world,T_rank", [(SMALL, 2, 300), (SMALL, 4, 150), (MID, 4, 1024),
@@ -107,6 +146,16 @@ def test_loopback_ranks_match_single_gpu_layer(shape, world, T_rank):
     xs = [torch.randn((T_rank + 3 * r, shape.H), generator=g, device="cuda").to(torch.bfloat16)
           for r in range(world)]
     ys, steps = loopback_forward(layers, xs)
+    # The return rows are block-scaled fp16: every 32-value block's largest
+    # magnitude sits in [2^14, 2^15] unless the block is tiny (code 15) or zero.
+    H = shape.H
+    for st in steps:
+        ret = st.return_rows.cpu().numpy()
+        if ret.shape[0]:
+            vals = np.abs(np.ascontiguousarray(ret[:, :2 * H]).view(np.float16).astype(np.float32))
+            bmax = vals.reshape(ret.shape[0], H // 32, 32).max(2)
+            codes = ret[:, 2 * H:2 * H + H // 32]
+            assert (((bmax >= 2.0 ** 14) & (bmax <= 2.0 ** 15)) | (codes == 15)).all()
     full = MoELayer.from_inputs(shape, inp)
     gsz = shape.E // shape.n_group
     El = shape.E // world
@@ -124,8 +173,10 @@ def test_loopback_ranks_match_single_gpu_layer(shape, world, T_rank):
         if El % gsz == 0:
             ranks = (steps[r].idx.long() // El).cpu().numpy()
             assert max(len(set(row.tolist())) for row in ranks) <= shape.topk_group
+            assert sum(steps[r].send_splits) <= shape.topk_group * xs[r].shape[0]
     print(f"{shape.name} world {world}: worst max|err|/RMS vs single GPU {worst:.2e}, "
-          f"rows received per rank {[sum(s.recv_splits) for s in steps]}")
+          f"rows received per rank {[sum(s.recv_splits) for s in steps]}, "
+          f"rows sent per token {[round(sum(s.send_splits) / max(s.T, 1), 2) for s in steps]}")
     # One rank against the float64 oracle on a sample of its tokens (near ties
     # scored on the GPU's expert set, as in the single-GPU parity tests).
     r = world - 1
