@@ -107,8 +107,20 @@ V3_E32 = V3_DECODE.with_(name="v3_e32", T=4096, n_routed_experts=32, seed=5)
 # the device).
 V3_E32_T16K = V3_E32.with_(name="v3_e32_t16k", T=16384, num_experts_per_tok=2, seed=6)
 
+# The V3 router, dispatch and combine at their full widths (256 experts, top-8, hidden
+# 7168) on 8192 tokens, with a narrow intermediate (128) so that the expert weights
+# take 1.4 GB: the capture case for the DRAM traffic of the kernels around the expert
+# GEMMs (x_perm and y_perm 0.94 GB each, beyond the L2; about 4 GB on the device).
+V3_IO = V3_DECODE.with_(name="v3_io", T=8192, moe_intermediate_size=128, seed=7)
+# 16 experts at V3 dimensions on 1024 tokens (top-8 of the 8 experts in the 4 kept
+# groups: ~512 rows per expert, as at the V3 prefill): the capture case for the
+# backward's weight-gradient GEMMs, whose contraction runs over an expert's rows
+# (about 3 GB on the device).
+V3_E16_T1K = V3_E32.with_(name="v3_e16_t1k", T=1024, n_routed_experts=16, seed=8)
+
 WORKLOADS: Dict[str, MoEShape] = {w.name: w for w in
-                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED, V3_E32, V3_E32_T16K)}
+                                  (TINY, MID, V3_DECODE, V3_PREFILL, V3_SKEWED, V3_E32, V3_E32_T16K, V3_IO,
+                                   V3_E16_T1K)}
 
 
 def _normal(shape, std, gen, device, dtype):
