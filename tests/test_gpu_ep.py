@@ -191,3 +191,28 @@ def test_loopback_ranks_match_single_gpu_layer(shape, world, T_rank):
     y_or = parity.oracle_layer_rows(shape, inp_r, rows, idx_r, scores, ref_idx, ref_w, margin)
     parity.assert_output_close(ys[r][torch.as_tensor(rows, device="cuda")].cpu().numpy(), y_or,
                                f"{shape.name} rank {r} vs oracle")
+
+
+def test_loopback_rank_without_tokens_and_rank_without_rows():
+    """World 2 with every token's experts on rank 0 (a bias of +10 on rank 0's expert
+    block): rank 0 brings no tokens but receives all rows (routed experts only, no
+    shared rows), rank 1 brings tokens but receives no rows (shared experts only,
+    empty expert segments)."""
+    shape = SMALL
+    inp = make_inputs(shape, "cuda")
+    El = shape.E // 2
+    bias = inp["e_bias"].clone()
+    bias[:El] += 10.0
+    inp = dict(inp, e_bias=bias)
+    layers = _layers(shape, inp, 2)
+    g = torch.Generator(device="cuda").manual_seed(78)
+    xs = [torch.empty((0, shape.H), device="cuda", dtype=torch.bfloat16),
+          torch.randn((200, shape.H), generator=g, device="cuda").to(torch.bfloat16)]
+    ys, steps = loopback_forward(layers, xs)
+    assert steps[0].recv_rows.shape[0] == 200 and steps[1].recv_rows.shape[0] == 0
+    assert ys[0].shape == (0, shape.H)
+    assert int(steps[1].idx.max()) < El
+    y_ref = MoELayer.from_inputs(shape, inp)(xs[1])
+    torch.cuda.synchronize()
+    parity.assert_output_close(ys[1].cpu().numpy(), y_ref.cpu().numpy(), "rank 1 vs single GPU")
+
