@@ -428,10 +428,23 @@ MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, 
  *
  * A token crosses to a rank once, however many of its k experts live there: the
  * source sends one row per (token, destination rank), the destination runs the
- * token's experts it holds and sends back one row, their weighted sum.  Rows
- * travel in two wire formats (moe_ep_row_bytes):
- *   send row:   H bf16 values of x[t], then the token's k expert ids (int32) and
- *               k routing weights (fp32), zero-padded to a multiple of 16 bytes;
+ * token's experts it was sent and sends back one row, their weighted sum.
+ *
+ * Redundant experts ("DeepSeek-V3 notes" § infrastructure, prefilling: redundant
+ * experts for load balance, placed from live statistics): a placement table
+ * expert_ranks int32 [E, max_rep] lists for expert e the ranks holding a copy,
+ * in its first n_e >= 1 entries (distinct ranks in [0, world)), then -1.  Slot
+ * (t, j) of expert e goes to rank expert_ranks[e, t mod n_e], so e's rows split
+ * evenly over its copies.  moe_ep_place builds such a table from per-expert
+ * loads; a null table means rank e / (E/world) for every e (no copies).  Rank r
+ * holds its experts in ascending id order (moe_ep_local_experts gives each id's
+ * local index): w_gate, w_up [n_local, I, H], w_down [n_local, H, I].
+ *
+ * Rows travel in two wire formats (moe_ep_row_bytes):
+ *   send row:   H bf16 values of x[t], then k int32 expert ids — slot j's id when
+ *               slot j goes to this row's rank, -1 when it goes elsewhere — and
+ *               the token's k routing weights (fp32), zero-padded to a multiple
+ *               of 16 bytes;
  *   return row: H block-scaled fp16 values (value = fp16 * 2^(code - 141)), then
  *               their H/32 scale codes (one byte per 32 values), padded likewise.
  * One forward on each rank, for its own T tokens:
@@ -454,35 +467,61 @@ MOE_API int moe_backward_train(const moe_config *cfg, int64_t T, const void *x, 
 MOE_API int moe_ep_row_bytes(const moe_config *cfg, int64_t *send_row_bytes, int64_t *return_row_bytes);
 
 /* Device workspace (256-byte aligned) for moe_ep_send on T tokens and for
- * moe_ep_experts on R received rows and T own tokens.  MOE_ERR_INVALID_ARG unless
- * 1 <= world, world divides E and R >= 0. */
-MOE_API int moe_ep_workspace_size(const moe_config *cfg, int32_t world, int64_t T, int64_t R, size_t *bytes);
+ * moe_ep_experts on R received rows, T own tokens and n_local local experts.
+ * MOE_ERR_INVALID_ARG unless 1 <= world, world divides E, 1 <= n_local <= E and
+ * R >= 0. */
+MOE_API int moe_ep_workspace_size(const moe_config *cfg, int32_t world, int32_t n_local, int64_t T, int64_t R,
+                                  size_t *bytes);
+
+/* Host only.  A placement with n_redundant extra copies, from load int64 [E] (rows
+ * per expert, e.g. the expert_load of moe_bias_update over recent batches): every
+ * expert starts on rank e / (E/world); then, n_redundant times, the expert whose
+ * copies carry the most rows each (load / copies; lowest id on ties; fewer than
+ * min(max_rep, world) copies) gets one more copy, on the rank with the least
+ * load that does not hold it (lowest rank on ties), its load being split evenly
+ * over its copies.  Stops early when no copy would carry rows.  Writes
+ * expert_ranks int32 [E, max_rep] (format above).  MOE_ERR_INVALID_ARG for E not
+ * a multiple of world, max_rep < 1, n_redundant < 0 or a negative load. */
+MOE_API int moe_ep_place(int32_t E, int32_t world, const int64_t *load, int32_t n_redundant, int32_t max_rep,
+                         int32_t *expert_ranks);
+
+/* Host only.  local_of int32 [E]: expert e's index among rank `rank`'s experts
+ * (ascending ids), -1 where the rank holds no copy; *n_local = their number.
+ * MOE_ERR_INVALID_ARG for a malformed table (no copy, a rank outside [0, world),
+ * a repeated rank, an entry after a -1). */
+MOE_API int moe_ep_local_experts(int32_t E, int32_t world, int32_t rank, const int32_t *expert_ranks,
+                                 int32_t max_rep, int32_t *local_of, int32_t *n_local);
 
 /* Source side.  In: x bf16 [T, H]; topk_idx int32 / topk_w fp32 [T, k] (from
- * moe_route).  Out: send_rows [T * min(k, world)] rows of send_row_bytes (the
+ * moe_route); expert_ranks [E, max_rep] device table (or null: E/world-expert
+ * blocks).  Out: send_rows [T * min(k, world)] rows of send_row_bytes (the
  * first sum(send_counts) written, sorted by destination rank, token order within
  * a rank); send_counts int32 [world]: rows for each rank; send_row_of int32 [T, k]:
- * for the first slot of token t on rank d, the index of its send row; -1 for the
- * token's other slots on that rank.  An expert id outside [0, E) gives no row and
- * is recorded in the device error word.  x, send_rows and the workspace 16-byte
- * aligned.  T = 0 only zeroes send_counts. */
+ * for the first slot of token t bound for rank d, the index of its send row; -1
+ * for the token's other slots bound there.  An expert id outside [0, E), or a
+ * malformed table entry, gives no row and is recorded in the device error word.
+ * x, send_rows and the workspace 16-byte aligned.  T = 0 only zeroes send_counts. */
 MOE_API int moe_ep_send(const moe_config *cfg, int32_t world, int64_t T, const void *x, const int32_t *topk_idx,
-                        const float *topk_w, int32_t *send_counts, void *send_rows, int32_t *send_row_of,
-                        void *workspace, size_t workspace_bytes, void *stream);
+                        const float *topk_w, const int32_t *expert_ranks, int32_t max_rep, int32_t *send_counts,
+                        void *send_rows, int32_t *send_row_of, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
-/* Rank `rank`'s experts.  In: recv_rows [R] send rows from all sources; x bf16
- * [T, H], the rank's own tokens.  Out: return_rows [R] rows of return_row_bytes:
- * row i = sum over slots j of received row i whose expert e is one of this rank's
- * of w_j * down_e(silu(gate_e x) * up_e x), summed in fp32 in slot order, then
- * block-scaled to fp16; y_shared [T, H] block-scaled fp16 with y_shared_scale
- * [T, ceil(H/256)*8] codes (the moe_experts format): the shared experts on x
- * (unused when S = 0).  A received expert id outside [0, E) gives no row and is
- * recorded in the device error word.  Pointers 16-byte aligned. */
-MOE_API int moe_ep_experts(const moe_config *cfg, int32_t world, int32_t rank, int64_t T, const void *x, int64_t R,
-                           const void *recv_rows, const void *w_gate, const void *w_up, const void *w_down,
-                           const void *ws_gate, const void *ws_up, const void *ws_down, void *return_rows,
-                           void *y_shared, void *y_shared_scale, void *workspace, size_t workspace_bytes,
-                           void *stream);
+/* Rank `rank`'s experts.  local_of int32 [E] device map (moe_ep_local_experts)
+ * and n_local, or local_of null: the block rank * E/world .. with n_local unused.
+ * In: recv_rows [R] send rows from all sources; x bf16 [T, H], the rank's own
+ * tokens; w_gate / w_up / w_down the rank's n_local experts.  Out: return_rows
+ * [R] rows of return_row_bytes: row i = sum over the slots j of received row i
+ * with an id e != -1 of w_j * down_e(silu(gate_e x) * up_e x), summed in fp32 in
+ * slot order, then block-scaled to fp16; y_shared [T, H] block-scaled fp16 with
+ * y_shared_scale [T, ceil(H/256)*8] codes (the moe_experts format): the shared
+ * experts on x (unused when S = 0).  A received id that is not one of this rank's
+ * experts gives no row and is recorded in the device error word.  Pointers
+ * 16-byte aligned. */
+MOE_API int moe_ep_experts(const moe_config *cfg, int32_t world, int32_t rank, const int32_t *local_of,
+                           int32_t n_local, int64_t T, const void *x, int64_t R, const void *recv_rows,
+                           const void *w_gate, const void *w_up, const void *w_down, const void *ws_gate,
+                           const void *ws_up, const void *ws_down, void *return_rows, void *y_shared,
+                           void *y_shared_scale, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Source side, after the return rows came back in send order: back_rows holds
  * n_back (= sum(send_counts)) return rows.  y[t] = shared row t + the back rows

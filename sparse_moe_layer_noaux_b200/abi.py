@@ -115,9 +115,11 @@ def lib():
         L.moe_backward.argtypes = [cfgp, i64] + [_P] * 19 + [sz, _P]
         i32 = ctypes.c_int32
         L.moe_ep_row_bytes.argtypes = [cfgp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
-        L.moe_ep_workspace_size.argtypes = [cfgp, i32, i64, i64, ctypes.POINTER(sz)]
-        L.moe_ep_send.argtypes = [cfgp, i32, i64] + [_P] * 7 + [sz, _P]
-        L.moe_ep_experts.argtypes = [cfgp, i32, i32, i64, _P, i64] + [_P] * 11 + [sz, _P]
+        L.moe_ep_workspace_size.argtypes = [cfgp, i32, i32, i64, i64, ctypes.POINTER(sz)]
+        L.moe_ep_place.argtypes = [i32, i32, _P, i32, i32, _P]
+        L.moe_ep_local_experts.argtypes = [i32, i32, i32, _P, i32, _P, ctypes.POINTER(i32)]
+        L.moe_ep_send.argtypes = [cfgp, i32, i64, _P, _P, _P, _P, i32] + [_P] * 4 + [sz, _P]
+        L.moe_ep_experts.argtypes = [cfgp, i32, i32, _P, i32, i64, _P, i64] + [_P] * 11 + [sz, _P]
         L.moe_ep_combine.argtypes = [cfgp, i32, i64, i64] + [_P] * 5 + [i32, _P]
         for fn in ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_dispatch_noalloc", "moe_experts",
                    "moe_experts_gate_up", "moe_experts_down",
@@ -126,7 +128,8 @@ def lib():
                    "moe_dispatch_mx", "moe_forward_mx", "moe_experts_gate_up_mx", "moe_experts_down_mx",
                    "moe_combine_mx", "moe_workspace_size_bwd", "moe_backward", "moe_workspace_size_host",
                    "moe_forward_host", "moe_forward_train", "moe_backward_train", "moe_ep_row_bytes",
-                   "moe_ep_workspace_size", "moe_ep_send", "moe_ep_experts", "moe_ep_combine"):
+                   "moe_ep_workspace_size", "moe_ep_place", "moe_ep_local_experts", "moe_ep_send",
+                   "moe_ep_experts", "moe_ep_combine"):
             getattr(L, fn).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -643,11 +646,48 @@ def ep_send_rows_max(cfg, T: int, world: int) -> int:
     return T * min(int(_cfg(cfg).num_experts_per_tok), world)
 
 
-def ep_workspace_size(cfg, world: int, T: int, R: int) -> int:
+def ep_workspace_size(cfg, world: int, T: int, R: int, n_local: Optional[int] = None) -> int:
+    """Workspace bytes for moe_ep_send on T tokens and moe_ep_experts on R received rows
+    with n_local local experts (default E/world)."""
+    c = _cfg(cfg)
+    if n_local is None:
+        n_local = c.n_routed_experts // max(int(world), 1)
     n = ctypes.c_size_t(0)
-    _check("moe_ep_workspace_size", lib().moe_ep_workspace_size(ctypes.byref(_cfg(cfg)), int(world), T, R,
+    _check("moe_ep_workspace_size", lib().moe_ep_workspace_size(ctypes.byref(c), int(world), int(n_local), T, R,
                                                                 ctypes.byref(n)))
     return n.value
+
+
+def _host_i32(name, t, count):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype != torch.int32 or not t.is_contiguous():
+        raise TypeError(f"{name}: expected a contiguous int32 CPU tensor")
+    if t.numel() < count:
+        raise ValueError(f"{name}: needs {count} elements, has {t.numel()}")
+
+
+def ep_place(E: int, world: int, load, n_redundant: int, max_rep: int) -> torch.Tensor:
+    """Placement table int32 [E, max_rep] (host) with n_redundant extra copies of the
+    most loaded experts, from per-expert loads [E] (include/moe.h, moe_ep_place)."""
+    ld = torch.as_tensor(load, dtype=torch.int64).cpu().contiguous()
+    if ld.numel() != E:
+        raise ValueError(f"load: needs {E} entries, has {ld.numel()}")
+    out = torch.empty((E, max_rep), dtype=torch.int32)
+    _check("moe_ep_place", lib().moe_ep_place(int(E), int(world), _ptr(ld), int(n_redundant), int(max_rep),
+                                              _ptr(out)))
+    return out
+
+
+def ep_local_experts(E: int, world: int, rank: int, expert_ranks: torch.Tensor) -> Tuple[torch.Tensor, int]:
+    """(local_of int32 [E], n_local) of rank `rank` under a placement table (host)."""
+    if expert_ranks.dim() != 2 or expert_ranks.shape[0] != E:
+        raise ValueError(f"expert_ranks: expected shape [{E}, max_rep]")
+    _host_i32("expert_ranks", expert_ranks, 0)
+    local_of = torch.empty(E, dtype=torch.int32)
+    n = ctypes.c_int32(0)
+    _check("moe_ep_local_experts", lib().moe_ep_local_experts(int(E), int(world), int(rank), _ptr(expert_ranks),
+                                                              int(expert_ranks.shape[1]), _ptr(local_of),
+                                                              ctypes.byref(n)))
+    return local_of, n.value
 
 
 def _ep_world(d, world: int, rank: int = 0) -> int:
@@ -665,30 +705,47 @@ def _wire_rows(name, t, row_bytes) -> int:
     return int(t.shape[0])
 
 
-def moe_ep_send(cfg, world: int, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace, stream=None):
-    """The source side's send rows, one per (token, destination rank), sorted by rank (include/moe.h)."""
+def moe_ep_send(cfg, world: int, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace,
+                expert_ranks=None, stream=None):
+    """The source side's send rows, one per (token, destination rank), sorted by rank
+    (include/moe.h); expert_ranks: the placement table [E, max_rep] on the device, or
+    None for E/world-expert blocks."""
     d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
     _ep_world(d, world)
     Wb, _ = ep_row_bytes(cfg)
     _req("x", x, _BF16, 0)
     _req("topk_idx", topk_idx, _I32, d.T * d.k)
     _req("topk_w", topk_w, _F32, d.T * d.k)
+    max_rep = 1
+    if expert_ranks is not None:
+        if expert_ranks.dim() != 2 or expert_ranks.shape[0] != d.E:
+            raise ValueError(f"expert_ranks: expected shape [{d.E}, max_rep]")
+        _req("expert_ranks", expert_ranks, _I32, 0)
+        max_rep = int(expert_ranks.shape[1])
     _req("send_counts", send_counts, _I32, world)
     if _wire_rows("send_rows", send_rows, Wb) < ep_send_rows_max(cfg, d.T, world):
         raise ValueError(f"send_rows: needs {ep_send_rows_max(cfg, d.T, world)} rows")
     _req("send_row_of", send_row_of, _I32, d.T * d.k)
     _req("workspace", workspace, _U8, 0)
     _check("moe_ep_send", lib().moe_ep_send(
-        ctypes.byref(_cfg(cfg)), int(world), d.T, _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(send_counts),
-        _ptr(send_rows), _ptr(send_row_of), _ptr(workspace), workspace.numel(), _stream(stream)))
+        ctypes.byref(_cfg(cfg)), int(world), d.T, _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(expert_ranks),
+        max_rep, _ptr(send_counts), _ptr(send_rows), _ptr(send_row_of), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
 
 
 def moe_ep_experts(cfg, world: int, rank: int, x, recv_rows, w_gate, w_up, w_down, ws_gate, ws_up, ws_down,
-                   return_rows, y_shared, y_shared_scale, workspace, stream=None):
+                   return_rows, y_shared, y_shared_scale, workspace, local_of=None, n_local=None, stream=None):
     """Rank `rank`'s experts over the received send rows -> return rows, and the shared
-    experts over its own tokens x (include/moe.h).  Weights are the rank's E/world experts."""
+    experts over its own tokens x (include/moe.h).  Weights are the rank's experts: its
+    E/world block, or with local_of (device int32 [E], from ep_local_experts) its
+    n_local experts in ascending id order."""
     d = _Dims(cfg, _rows_2d("x", x, _cfg(cfg).hidden_size))
     El = _ep_world(d, world, rank)
+    if local_of is not None:
+        if n_local is None or not 1 <= int(n_local) <= d.E:
+            raise ValueError(f"n_local must be in [1, {d.E}] with local_of")
+        _req("local_of", local_of, _I32, d.E)
+        El = int(n_local)
     Wb, Wr = ep_row_bytes(cfg)
     R = _wire_rows("recv_rows", recv_rows, Wb)
     if _wire_rows("return_rows", return_rows, Wr) < R:
@@ -704,7 +761,8 @@ def moe_ep_experts(cfg, world: int, rank: int, x, recv_rows, w_gate, w_up, w_dow
     _req("y_shared_scale", y_shared_scale, _U8, d.T * d.scale_cols, optional=not shared)
     _req("workspace", workspace, _U8, 0)
     _check("moe_ep_experts", lib().moe_ep_experts(
-        ctypes.byref(_cfg(cfg)), int(world), int(rank), d.T, _ptr(x), R, _ptr(recv_rows), _ptr(w_gate), _ptr(w_up),
+        ctypes.byref(_cfg(cfg)), int(world), int(rank), _ptr(local_of), El, d.T, _ptr(x), R, _ptr(recv_rows),
+        _ptr(w_gate), _ptr(w_up),
         _ptr(w_down), _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(return_rows), _ptr(y_shared),
         _ptr(y_shared_scale), _ptr(workspace), workspace.numel(), _stream(stream)))
 

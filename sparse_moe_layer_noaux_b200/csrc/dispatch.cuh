@@ -30,21 +30,30 @@ namespace moe {
 constexpr int kDispTok = 32;      // tokens per dispatch block
 constexpr int kDispThreads = 256;
 
-// Slot (t, j)'s entry is v = idx[t * ld + j].  Its bucket is v - base when that
-// lies in [0, E) (E is the kernel's bucket count); otherwise the slot has no row,
-// and a value outside [lo, hi) is also recorded in the device error word.  The
-// layer's dispatch uses {topk_idx, k, 0, 0, E}.
+// Slot (t, j)'s entry is v = idx[t * ld + j].  Its bucket is map[v] (map set) or
+// v - base, when that lies in [0, E) (E is the kernel's bucket count); otherwise
+// the slot has no row.  A value outside [lo, hi) is recorded in the device error
+// word, except -1 when lo = -1 (a slot marked as having no row here); with
+// `strict`, so is a value in [0, hi) that names no bucket.  The layer's dispatch
+// uses {topk_idx, k, 0, 0, E}.
 struct SlotIndex {
     const int32_t* idx;
     int ld;
     int base, lo, hi;
+    const int32_t* map = nullptr;
+    int strict = 0;
 };
 
 // The bucket of a slot's entry, or -1 (no row; caller errors recorded).
 __device__ __forceinline__ int slot_bucket(const SlotIndex& s, int v, int E) {
-    const int b = v - s.base;
+    if (v < s.lo || v >= s.hi) {
+        record_error(kErrExpertId);
+        return -1;
+    }
+    if (v < 0) return -1;
+    const int b = s.map ? s.map[v] : v - s.base;
     if (static_cast<unsigned>(b) < static_cast<unsigned>(E)) return b;
-    if (v < s.lo || v >= s.hi) record_error(kErrExpertId);
+    if (s.strict) record_error(kErrExpertId);
     return -1;
 }
 

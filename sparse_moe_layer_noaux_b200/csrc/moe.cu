@@ -7,6 +7,7 @@
 #include <cstring>
 #include <initializer_list>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -1818,6 +1819,7 @@ int check_ep_rows(const moe_config* c, int64_t T, int64_t R) {
 }
 
 struct WorkspaceEpSend {
+    int32_t* slot_dest;     // [T, k] destination rank of each slot
     int32_t* rank_slot;     // [T, k] destination rank of a slot's row, or -1
     int32_t* perm_src;      // [T * min(k, world)] slot of each send row
     int32_t* offsets;       // [world + 1]
@@ -1836,6 +1838,7 @@ WorkspaceEpSend carve_ep_send(const moe_config* c, int world, int64_t T, uint8_t
         off += align_up(bytes);
         return p;
     };
+    w.slot_dest = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
     w.rank_slot = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * T * K));
     w.perm_src = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ep_send_rows_max(c, T, world)));
     w.offsets = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (world + 1)));
@@ -1847,12 +1850,12 @@ WorkspaceEpSend carve_ep_send(const moe_config* c, int world, int64_t T, uint8_t
 }
 
 struct WorkspaceEpExperts {
-    int32_t* offsets;         // [E/world + 1] local expert segments
+    int32_t* offsets;         // [El + 1] segments of the El local experts
     int32_t* perm_src;        // [Rb] received slot (r * k + j) of each expert row
     int32_t* row_of;          // [R, k] expert row of each received slot, or -1
-    int32_t* block_counts;    // [E/world, nb]
-    int32_t* block_base;      // [E/world, nb]
-    int32_t* totals;          // [E/world]
+    int32_t* block_counts;    // [El, nb]
+    int32_t* block_base;      // [El, nb]
+    int32_t* totals;          // [El]
     float* w_perm;            // [Rb] routing weight of each expert row
     __nv_bfloat16* x_perm;    // [Rb, H]
     __nv_bfloat16* h_routed;  // [Rb, I]
@@ -1862,8 +1865,8 @@ struct WorkspaceEpExperts {
     size_t bytes;
 };
 
-WorkspaceEpExperts carve_ep_experts(const moe_config* c, int world, int64_t T, int64_t R, uint8_t* base) {
-    const int64_t K = c->num_experts_per_tok, El = c->n_routed_experts / world, H = c->hidden_size;
+WorkspaceEpExperts carve_ep_experts(const moe_config* c, int64_t El, int64_t T, int64_t R, uint8_t* base) {
+    const int64_t K = c->num_experts_per_tok, H = c->hidden_size;
     const int64_t I = c->moe_intermediate_size, SI = static_cast<int64_t>(c->n_shared_experts) * I;
     const int64_t nb = (R + kDispTok - 1) / kDispTok, Rb = ep_local_rows_max(c, R);
     WorkspaceEpExperts w{};
@@ -1889,9 +1892,26 @@ WorkspaceEpExperts carve_ep_experts(const moe_config* c, int world, int64_t T, i
     return w;
 }
 
-size_t ep_workspace_bytes(const moe_config* c, int world, int64_t T, int64_t R) {
-    const size_t a = carve_ep_send(c, world, T, nullptr).bytes, b = carve_ep_experts(c, world, T, R, nullptr).bytes;
+// El = the most experts one rank holds (E/world without redundant copies).
+size_t ep_workspace_bytes(const moe_config* c, int world, int64_t El, int64_t T, int64_t R) {
+    const size_t a = carve_ep_send(c, world, T, nullptr).bytes, b = carve_ep_experts(c, El, T, R, nullptr).bytes;
     return a > b ? a : b;
+}
+
+// Number of replicas listed for expert e (the leading entries >= 0), 0 if the
+// list is malformed (an entry outside [0, world), a repeated rank, or a valid
+// entry after a -1).
+int ep_replicas(const int32_t* reps, int max_rep, int world) {
+    int n = 0;
+    while (n < max_rep && reps[n] >= 0) {
+        if (reps[n] >= world) return 0;
+        for (int i = 0; i < n; ++i)
+            if (reps[i] == reps[n]) return 0;
+        ++n;
+    }
+    for (int i = n; i < max_rep; ++i)
+        if (reps[i] >= 0) return 0;
+    return n;
 }
 }  // namespace
 
@@ -1904,21 +1924,83 @@ int moe_ep_row_bytes(const moe_config* cfg, int64_t* send_row_bytes, int64_t* re
     return MOE_OK;
 }
 
-int moe_ep_workspace_size(const moe_config* cfg, int32_t world, int64_t T, int64_t R, size_t* bytes) {
+int moe_ep_workspace_size(const moe_config* cfg, int32_t world, int32_t n_local, int64_t T, int64_t R,
+                          size_t* bytes) {
     int v = validate_ep(cfg, T, world);
     if (v != MOE_OK) return v;
-    if (!bytes) return MOE_ERR_INVALID_ARG;
+    if (!bytes || n_local < 1 || n_local > cfg->n_routed_experts) return MOE_ERR_INVALID_ARG;
     if ((v = check_ep_rows(cfg, T, R)) != MOE_OK) return v;
-    *bytes = ep_workspace_bytes(cfg, world, T, R);
+    *bytes = ep_workspace_bytes(cfg, world, n_local, T, R);
+    return MOE_OK;
+}
+
+int moe_ep_place(int32_t E, int32_t world, const int64_t* load, int32_t n_redundant, int32_t max_rep,
+                 int32_t* expert_ranks) {
+    if (E < 1 || world < 1 || E % world != 0 || max_rep < 1 || !load || !expert_ranks) return MOE_ERR_INVALID_ARG;
+    if (n_redundant < 0) return MOE_ERR_INVALID_ARG;
+    for (int e = 0; e < E; ++e)
+        if (load[e] < 0) return MOE_ERR_INVALID_ARG;
+    const int El = E / world;
+    std::vector<int> n_rep(E, 1);
+    std::vector<double> rank_load(world, 0.0);
+    for (int e = 0; e < E; ++e) {
+        expert_ranks[static_cast<int64_t>(e) * max_rep] = e / El;
+        for (int i = 1; i < max_rep; ++i) expert_ranks[static_cast<int64_t>(e) * max_rep + i] = -1;
+        rank_load[e / El] += static_cast<double>(load[e]);
+    }
+    for (int step = 0; step < n_redundant; ++step) {
+        // The expert whose copies carry the most rows each (lowest id on ties)...
+        int be = -1;
+        double best = 0.0;
+        for (int e = 0; e < E; ++e) {
+            if (n_rep[e] >= max_rep || n_rep[e] >= world) continue;
+            const double share = static_cast<double>(load[e]) / n_rep[e];
+            if (share > best) {
+                best = share;
+                be = e;
+            }
+        }
+        if (be < 0) break;  // nothing left that a copy would relieve
+        // ...gets a copy on the least loaded rank that does not hold it (lowest rank on ties).
+        int32_t* reps = expert_ranks + static_cast<int64_t>(be) * max_rep;
+        int br = -1;
+        for (int r = 0; r < world; ++r) {
+            bool holds = false;
+            for (int i = 0; i < n_rep[be]; ++i) holds = holds || reps[i] == r;
+            if (!holds && (br < 0 || rank_load[r] < rank_load[br])) br = r;
+        }
+        const double s0 = static_cast<double>(load[be]) / n_rep[be], s1 = static_cast<double>(load[be]) / (n_rep[be] + 1);
+        for (int i = 0; i < n_rep[be]; ++i) rank_load[reps[i]] -= s0 - s1;
+        rank_load[br] += s1;
+        reps[n_rep[be]++] = br;
+    }
+    return MOE_OK;
+}
+
+int moe_ep_local_experts(int32_t E, int32_t world, int32_t rank, const int32_t* expert_ranks, int32_t max_rep,
+                         int32_t* local_of, int32_t* n_local) {
+    if (E < 1 || world < 1 || E % world != 0 || rank < 0 || rank >= world || max_rep < 1 || !expert_ranks ||
+        !local_of || !n_local)
+        return MOE_ERR_INVALID_ARG;
+    int n = 0;
+    for (int e = 0; e < E; ++e) {
+        const int32_t* reps = expert_ranks + static_cast<int64_t>(e) * max_rep;
+        const int nr = ep_replicas(reps, max_rep, world);
+        if (nr == 0) return MOE_ERR_INVALID_ARG;
+        bool here = false;
+        for (int i = 0; i < nr; ++i) here = here || reps[i] == rank;
+        local_of[e] = here ? n++ : -1;
+    }
+    *n_local = n;
     return MOE_OK;
 }
 
 int moe_ep_send(const moe_config* cfg, int32_t world, int64_t T, const void* x, const int32_t* topk_idx,
-                const float* topk_w, int32_t* send_counts, void* send_rows, int32_t* send_row_of, void* workspace,
-                size_t workspace_bytes, void* stream) {
+                const float* topk_w, const int32_t* expert_ranks, int32_t max_rep, int32_t* send_counts,
+                void* send_rows, int32_t* send_row_of, void* workspace, size_t workspace_bytes, void* stream) {
     int v = validate_ep(cfg, T, world);
     if (v != MOE_OK) return v;
-    if (!send_counts) return MOE_ERR_INVALID_ARG;
+    if (!send_counts || (expert_ranks && max_rep < 1)) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) {
         if (cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * world, st) != cudaSuccess) return MOE_ERR_CUDA;
@@ -1931,8 +2013,8 @@ int moe_ep_send(const moe_config* cfg, int32_t world, int64_t T, const void* x, 
     const WorkspaceEpSend w = carve_ep_send(cfg, world, T, static_cast<uint8_t*>(workspace));
     const int K = cfg->num_experts_per_tok, E = cfg->n_routed_experts, H = cfg->hidden_size;
     const int64_t Wb = ep_send_row_bytes(cfg);
-    ep_rank_slots_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(topk_idx, T, K, E / world, E,
-                                                                                w.rank_slot);
+    ep_rank_slots_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, st>>>(
+        topk_idx, T, K, E / world, E, expert_ranks, expert_ranks ? max_rep : 1, world, w.slot_dest, w.rank_slot);
     count_launch();
     // Sort the (token, rank) rows by rank: the rank-slot entries are the buckets,
     // -1 (a rank the token already has a row for) is no row.
@@ -1958,32 +2040,35 @@ int moe_ep_send(const moe_config* cfg, int32_t world, int64_t T, const void* x, 
     int64_t blocks = (n_max * meta_words + 255) / 256;
     if (blocks > 4096) blocks = 4096;
     ep_send_meta_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        w.offsets, world, w.perm_src, T * K, K, topk_idx, topk_w, n_max, static_cast<uint8_t*>(send_rows), Wb,
-        2ll * H, meta_words, send_counts);
+        w.offsets, world, w.perm_src, T * K, K, topk_idx, topk_w, w.slot_dest, n_max, static_cast<uint8_t*>(send_rows),
+        Wb, 2ll * H, meta_words, send_counts);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int moe_ep_experts(const moe_config* cfg, int32_t world, int32_t rank, int64_t T, const void* x, int64_t R,
-                   const void* recv_rows, const void* w_gate, const void* w_up, const void* w_down,
-                   const void* ws_gate, const void* ws_up, const void* ws_down, void* return_rows, void* y_shared,
-                   void* y_shared_scale, void* workspace, size_t workspace_bytes, void* stream) {
+int moe_ep_experts(const moe_config* cfg, int32_t world, int32_t rank, const int32_t* local_of, int32_t n_local,
+                   int64_t T, const void* x, int64_t R, const void* recv_rows, const void* w_gate, const void* w_up,
+                   const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down,
+                   void* return_rows, void* y_shared, void* y_shared_scale, void* workspace, size_t workspace_bytes,
+                   void* stream) {
     int v = validate_ep(cfg, T, world);
     if (v != MOE_OK) return v;
     if (rank < 0 || rank >= world) return MOE_ERR_INVALID_ARG;
+    const int El = local_of ? n_local : cfg->n_routed_experts / world;
+    if (El < 1 || El > cfg->n_routed_experts) return MOE_ERR_INVALID_ARG;
     if ((v = check_ep_rows(cfg, T, R)) != MOE_OK) return v;
     const bool sh = cfg->n_shared_experts > 0 && T > 0;
     if (!sh && R == 0) return MOE_OK;
     if ((v = check_ptrs({w_gate, w_up, w_down})) != MOE_OK) return v;
     if (R > 0 && (v = check_ptrs({recv_rows, return_rows})) != MOE_OK) return v;
     if (sh && (v = check_ptrs({x, ws_gate, ws_up, ws_down, y_shared, y_shared_scale})) != MOE_OK) return v;
-    if (!workspace || workspace_bytes < carve_ep_experts(cfg, world, T, R, nullptr).bytes || !aligned16(workspace))
+    if (!workspace || workspace_bytes < carve_ep_experts(cfg, El, T, R, nullptr).bytes || !aligned16(workspace))
         return MOE_ERR_WORKSPACE;
     DeviceInfo* d = nullptr;
     if ((v = device_info(&d)) != MOE_OK) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WorkspaceEpExperts w = carve_ep_experts(cfg, world, T, R, static_cast<uint8_t*>(workspace));
-    const int K = cfg->num_experts_per_tok, E = cfg->n_routed_experts, El = E / world, H = cfg->hidden_size;
+    const WorkspaceEpExperts w = carve_ep_experts(cfg, El, T, R, static_cast<uint8_t*>(workspace));
+    const int K = cfg->num_experts_per_tok, E = cfg->n_routed_experts, H = cfg->hidden_size;
     const int64_t Wb = ep_send_row_bytes(cfg), Wr = ep_return_row_bytes(cfg);
     const int64_t Rb = ep_local_rows_max(cfg, R);
     // With no shared rows to compute (S = 0 or no local tokens) the shared members
@@ -1991,12 +2076,13 @@ int moe_ep_experts(const moe_config* cfg, int32_t world, int32_t rank, int64_t T
     moe_config c = *cfg;
     if (!sh) c.n_shared_experts = 0;
     if (R > 0) {
-        // The received rows' slots sorted by local expert: an expert id in this
-        // rank's block is a bucket, one of another rank's is no row, one outside
-        // [0, E) is a caller error.
+        // The received rows' slots sorted by local expert: -1 marks a slot sent
+        // elsewhere; any other id must be one of this rank's experts (the block
+        // rank * E/world.., or local_of[id] >= 0), else it is a caller error.
         const uint8_t* rows = static_cast<const uint8_t*>(recv_rows);
         RowSort a{};
-        a.si = SlotIndex{reinterpret_cast<const int32_t*>(rows + 2ll * H), static_cast<int>(Wb / 4), rank * El, 0, E};
+        a.si = SlotIndex{reinterpret_cast<const int32_t*>(rows + 2ll * H), static_cast<int>(Wb / 4),
+                         local_of ? 0 : rank * El, -1, E, local_of, 1};
         a.T = R;
         a.K = K;
         a.E = El;

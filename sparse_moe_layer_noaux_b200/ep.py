@@ -10,9 +10,15 @@ most topk_group ranks).
 
 A token crosses to a rank once, however many of its experts live there: the
 source sends one row per (token, destination rank) carrying the token's values
-and routing, the destination runs all of the token's experts it holds and sends
-back one row, their weighted sum.  So each direction moves at most
+and routing, the destination runs all of the token's experts it was sent and
+sends back one row, their weighted sum.  So each direction moves at most
 min(k, topk_group ranks) rows per token instead of k.
+
+Redundant experts (same notes, § infrastructure, prefilling: copies of the
+experts with the most load, placed from live statistics, to balance the ranks):
+an EPPlacement lists the ranks holding each expert; the rows of an expert with
+n copies are split over them by token index mod n.  EPPlacement.from_load builds
+one from per-expert row counts (libmoe's moe_ep_place).
 
 Every step of the layer runs in libmoe (include/moe.h lists the sequence); this
 module only allocates the buffers and moves them between ranks with the process
@@ -50,17 +56,52 @@ class EPStep:
     y_shared_scale: Optional[torch.Tensor] = None
 
 
+class EPPlacement:
+    """Which ranks hold a copy of each routed expert.
+
+    expert_ranks: int32 [E, max_rep] (host): the ranks holding expert e in its first
+    entries, then -1; None means contiguous blocks of E/world experts per rank and no
+    copies.  A rank holds its experts in ascending id order.
+    """
+
+    def __init__(self, E: int, world: int, expert_ranks: Optional[torch.Tensor] = None):
+        if world < 1 or E % world:
+            raise ValueError(f"world {world} must divide n_routed_experts {E}")
+        self.E, self.world, self.expert_ranks = E, world, expert_ranks
+
+    @classmethod
+    def from_load(cls, E: int, world: int, load, n_redundant: int, max_rep: int = 2) -> "EPPlacement":
+        """Copies of the most loaded experts, from rows per expert [E] (moe_ep_place)."""
+        return cls(E, world, abi.ep_place(E, world, load, n_redundant, max_rep))
+
+    def local_experts(self, rank: int):
+        """(local_of int32 [E] or None, n_local, the rank's expert ids in local order)."""
+        if self.expert_ranks is None:
+            El = self.E // self.world
+            return None, El, list(range(rank * El, (rank + 1) * El))
+        local_of, n = abi.ep_local_experts(self.E, self.world, rank, self.expert_ranks)
+        return local_of, n, [e for e in range(self.E) if int(local_of[e]) >= 0]
+
+    def rank_weights(self, t: torch.Tensor, rank: int) -> torch.Tensor:
+        """Rank `rank`'s experts of a per-expert tensor [E, ...], in local order."""
+        ids = self.local_experts(rank)[2]
+        return t[torch.as_tensor(ids, device=t.device)].contiguous()
+
+
 class MoELayerEP:
     """One rank's part of an expert-parallel layer.
 
     shape: the whole layer's configuration (E = all routed experts).
     world, rank: the ranks of `group` (default: the default process group).
-    w_gate / w_up [E/world, I, H], w_down [E/world, H, I]: this rank's experts.
+    placement: an EPPlacement (default: blocks of E/world experts, no copies).
+    w_gate / w_up [n_local, I, H], w_down [n_local, H, I]: this rank's experts in the
+    placement's local order (placement.rank_weights; expert_block for blocks).
     router_w, e_bias and the shared experts: the full (replicated) tensors.
     """
 
     def __init__(self, shape: MoEShape, world: int, rank: int, router_w, e_bias, w_gate, w_up, w_down,
-                 ws_gate=None, ws_up=None, ws_down=None, group=None, _kernels=None):
+                 ws_gate=None, ws_up=None, ws_down=None, group=None, placement: Optional[EPPlacement] = None,
+                 _kernels=None):
         if world < 1 or shape.E % world:
             raise ValueError(f"world {world} must divide n_routed_experts {shape.E}")
         if not 0 <= rank < world:
@@ -71,14 +112,19 @@ class MoELayerEP:
         self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
         self.ws_gate, self.ws_up, self.ws_down = ws_gate, ws_up, ws_down
         self.device = router_w.device
+        self.placement = placement if placement is not None else EPPlacement(shape.E, world)
+        if self.placement.E != shape.E or self.placement.world != world:
+            raise ValueError("placement was made for another E or world")
+        local_of, self.n_local, self.local_ids = self.placement.local_experts(rank)
+        if w_gate.shape[0] != self.n_local:
+            raise ValueError(f"w_gate holds {w_gate.shape[0]} experts, rank {rank} holds {self.n_local}")
+        ranks = self.placement.expert_ranks
+        self.expert_ranks = None if ranks is None else ranks.to(self.device)
+        self.local_of = None if local_of is None else local_of.to(self.device)
         # The library binding; the CPU tests of the exchange pass a stand-in.
         self.lib = _kernels if _kernels is not None else abi
         self.send_row_bytes, self.return_row_bytes = self.lib.ep_row_bytes(self.cfg)
         self._ws: Optional[torch.Tensor] = None
-
-    @property
-    def experts_per_rank(self) -> int:
-        return self.shape.E // self.world
 
     def _empty(self, shape, dtype):
         return torch.empty(shape, dtype=dtype, device=self.device)
@@ -99,10 +145,12 @@ class MoELayerEP:
                     send_counts=self._empty(self.world, torch.int32),
                     send_rows=self._empty((n_max, self.send_row_bytes), torch.uint8),
                     send_row_of=self._empty((T, k), torch.int32))
-        ws = self._workspace(max(L.workspace_size(self.cfg, T), L.ep_workspace_size(self.cfg, self.world, T, 0)))
+        ws = self._workspace(max(L.workspace_size(self.cfg, T),
+                                 L.ep_workspace_size(self.cfg, self.world, T, 0, n_local=self.n_local)))
         if T:
             L.moe_route(self.cfg, x, self.router_w, self.e_bias, st.idx, st.w, ws)
-        L.moe_ep_send(self.cfg, self.world, x, st.idx, st.w, st.send_counts, st.send_rows, st.send_row_of, ws)
+        L.moe_ep_send(self.cfg, self.world, x, st.idx, st.w, st.send_counts, st.send_rows, st.send_row_of, ws,
+                      expert_ranks=self.expert_ranks)
         return st
 
     def plan(self, st: EPStep, recv_counts: torch.Tensor) -> None:
@@ -123,9 +171,10 @@ class MoELayerEP:
         """The rank's experts over the received rows; the shared experts over its own tokens."""
         L = self.lib
         R = st.recv_rows.shape[0]
-        ws = self._workspace(L.ep_workspace_size(self.cfg, self.world, st.T, R))
+        ws = self._workspace(L.ep_workspace_size(self.cfg, self.world, st.T, R, n_local=self.n_local))
         L.moe_ep_experts(self.cfg, self.world, self.rank, x, st.recv_rows, self.w_gate, self.w_up, self.w_down,
-                         self.ws_gate, self.ws_up, self.ws_down, st.return_rows, st.y_shared, st.y_shared_scale, ws)
+                         self.ws_gate, self.ws_up, self.ws_down, st.return_rows, st.y_shared, st.y_shared_scale, ws,
+                         local_of=self.local_of, n_local=self.n_local)
 
     def combine(self, st: EPStep, out_dtype=torch.float32) -> torch.Tensor:
         y = self._empty((st.T, self.shape.H), out_dtype)

@@ -5,14 +5,18 @@ over gloo ranks on a machine without a GPU).
 
 Each function keeps the contract include/moe.h states for the library call of
 the same name, on CPU tensors, wire formats included:
-  send row    H bf16 values, k int32 expert ids, k fp32 weights, zeros to 16 bytes
+  send row    H bf16 values, k int32 expert ids (-1 for slots bound for another
+              rank), k fp32 weights, zeros to 16 bytes
   return row  H fp16 values, H/32 scale codes, zeros to 16 bytes; this stand-in
               always writes code 141 (factor 2^0), i.e. plain fp16 values
   moe_route       oracle routing (float64), weights stored as fp32
-  moe_ep_send     one row per (token, rank of one of its experts), sorted by rank
-                  and token; send_row_of marks the token's first slot on the rank
-  moe_ep_experts  per received row, the float64 sum over its slots on this rank
-                  of w * SwiGLU_e(x); the shared experts over the rank's own tokens
+  moe_ep_send     slot (t, j) of expert e goes to e's block rank, or with a
+                  placement table to replica t mod n_e of e's ranks; one row per
+                  (token, destination), sorted by rank and token; send_row_of marks
+                  the token's first slot bound for the rank
+  moe_ep_experts  per received row, the float64 sum over its slots with an id of
+                  w * SwiGLU_e(x), e's weights at its local index; the shared
+                  experts over the rank's own tokens
   moe_ep_combine  shared row + the token's returned rows, decoded, summed in fp32
 """
 from __future__ import annotations
@@ -43,7 +47,7 @@ def workspace_size(cfg, T):
     return 256
 
 
-def ep_workspace_size(cfg, world, T, R):
+def ep_workspace_size(cfg, world, T, R, n_local=None):
     return 256
 
 
@@ -57,18 +61,26 @@ def moe_route(cfg, x, router_w, e_bias, topk_idx, topk_w, workspace=None):
     topk_w.copy_(torch.from_numpy(w.astype(np.float32)))
 
 
-def moe_ep_send(cfg, world, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace=None):
+def _dest(e, t, El, ranks):
+    if ranks is None:
+        return e // El
+    reps = [int(r) for r in ranks[e] if r >= 0]
+    return reps[t % len(reps)]
+
+
+def moe_ep_send(cfg, world, x, topk_idx, topk_w, send_counts, send_rows, send_row_of, workspace=None,
+                expert_ranks=None):
     T, H, k = x.shape[0], cfg.hidden_size, cfg.num_experts_per_tok
     El = cfg.n_routed_experts // world
+    ranks = None if expert_ranks is None else expert_ranks.numpy()
     idx, w = topk_idx.numpy(), topk_w.numpy()
-    entries = []                                   # (rank, token, slot), the token's first slot on the rank
+    dest = np.array([[_dest(int(idx[t, j]), t, El, ranks) for j in range(k)] for t in range(T)],
+                    dtype=np.int64).reshape(T, k)
+    entries = []                                   # (rank, token, slot), the token's first slot bound there
     for t in range(T):
-        ranks = set()
         for j in range(k):
-            d = int(idx[t, j]) // El
-            if d not in ranks:
-                ranks.add(d)
-                entries.append((d, t, j))
+            if dest[t, j] not in dest[t, :j]:
+                entries.append((int(dest[t, j]), t, j))
     entries.sort(key=lambda e: (e[0], e[1]))
     send_counts.copy_(torch.from_numpy(np.bincount([e[0] for e in entries], minlength=world).astype(np.int32)))
     row_of = np.full((T, k), -1, np.int32)
@@ -78,7 +90,8 @@ def moe_ep_send(cfg, world, x, topk_idx, topk_w, send_counts, send_rows, send_ro
         row_of[t, j] = r
         rows[r] = 0
         rows[r, :2 * H] = xb[t].view(np.uint8)
-        rows[r, 2 * H:2 * H + 4 * k] = idx[t].astype("<i4").view(np.uint8)
+        ids = np.where(dest[t] == d, idx[t], -1).astype("<i4")
+        rows[r, 2 * H:2 * H + 4 * k] = ids.view(np.uint8)
         rows[r, 2 * H + 4 * k:2 * H + 8 * k] = w[t].astype("<f4").view(np.uint8)
     send_row_of.copy_(torch.from_numpy(row_of))
 
@@ -89,20 +102,22 @@ def _store_unit_scale(values, scales, rows_f64):
 
 
 def moe_ep_experts(cfg, world, rank, x, recv_rows, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, return_rows,
-                   y_shared, y_shared_scale, workspace=None):
-    H, k = cfg.hidden_size, cfg.num_experts_per_tok
-    El = cfg.n_routed_experts // world
+                   y_shared, y_shared_scale, workspace=None, local_of=None, n_local=None):
+    H, k, E = cfg.hidden_size, cfg.num_experts_per_tok, cfg.n_routed_experts
+    El = E // world
+    local = (np.arange(E) - rank * El) if local_of is None else local_of.numpy().astype(np.int64)
     rows = recv_rows.numpy()
     R = rows.shape[0]
     xb = np.ascontiguousarray(rows[:, :2 * H]).view(np.uint16)
     ids = np.ascontiguousarray(rows[:, 2 * H:2 * H + 4 * k]).view("<i4")
     wts = np.ascontiguousarray(rows[:, 2 * H + 4 * k:2 * H + 8 * k]).view("<f4")
     out = np.zeros((R, H), np.float64)
-    for e_local in range(El):
-        r_sel, j_sel = np.nonzero(ids == rank * El + e_local)
+    for e in range(E):
+        r_sel, j_sel = np.nonzero(ids == e)
         if r_sel.size:
-            o = oracle.swiglu(xb[r_sel], bf16_bits(w_gate[e_local]), bf16_bits(w_up[e_local]),
-                              bf16_bits(w_down[e_local]))
+            li = int(local[e])
+            assert 0 <= li < w_gate.shape[0], (rank, e, li)   # the sender only sends this rank's experts
+            o = oracle.swiglu(xb[r_sel], bf16_bits(w_gate[li]), bf16_bits(w_up[li]), bf16_bits(w_down[li]))
             np.add.at(out, r_sel, wts[r_sel, j_sel].astype(np.float64)[:, None] * o)
     ret = return_rows.numpy()
     ret[:] = 0

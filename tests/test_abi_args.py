@@ -19,7 +19,7 @@ NOSHARED = MoEShape("noshared", T=50, hidden_size=256, n_routed_experts=16, n_gr
                     routed_scaling_factor=1.0, norm_topk_prob=True, seed=9)
 HOST_QUERIES = ("moe_workspace_size", "moe_workspace_size_mx", "moe_workspace_size_bwd",
                 "moe_workspace_size_host", "moe_mx_routed_rows", "moe_mx_scale_bytes", "moe_status_string",
-                "moe_ep_row_bytes", "moe_ep_workspace_size")
+                "moe_ep_row_bytes", "moe_ep_workspace_size", "moe_ep_place", "moe_ep_local_experts")
 
 
 class _Recorder:
@@ -113,10 +113,14 @@ def run_all(s):
     n_send = abi.ep_send_rows_max(cfg, T, world)
     ws_ep = e(abi.ep_workspace_size(cfg, world, T, R), dtype=u8)
     send_row_of = e(T, k, dtype=i32)
-    abi.moe_ep_send(cfg, world, L["x"], idx, w, e(world, dtype=i32), e(n_send, Wb, dtype=u8), send_row_of, ws_ep)
+    placement = abi.ep_place(E, world, torch.arange(E, dtype=torch.int64), 2, 2)
+    local_of, n_local = abi.ep_local_experts(E, world, 1, placement)
+    abi.moe_ep_send(cfg, world, L["x"], idx, w, e(world, dtype=i32), e(n_send, Wb, dtype=u8), send_row_of, ws_ep,
+                    expert_ranks=placement)
     y_sh, y_sh_sc = e(T, H, dtype=f16), e(T, abi.y_perm_scale_cols(H), dtype=u8)
-    abi.moe_ep_experts(cfg, world, 1, L["x"], e(R, Wb, dtype=u8), e(El, I, H), e(El, I, H), e(El, H, I),
-                       L["ws_gate"], L["ws_up"], L["ws_down"], e(R, Wr, dtype=u8), y_sh, y_sh_sc, ws_ep)
+    abi.moe_ep_experts(cfg, world, 1, L["x"], e(R, Wb, dtype=u8), e(n_local, I, H), e(n_local, I, H),
+                       e(n_local, H, I), L["ws_gate"], L["ws_up"], L["ws_down"], e(R, Wr, dtype=u8), y_sh, y_sh_sc,
+                       ws_ep, local_of=local_of, n_local=n_local)
     abi.moe_ep_combine(cfg, world, e(n_send, Wr, dtype=u8), send_row_of, y_sh, y_sh_sc, e(T, H, dtype=f32))
 
 
@@ -169,6 +173,13 @@ def test_bad_arguments_are_rejected_before_the_call(rec):
                                              e(T * 2 - 1, Wb, dtype=torch.uint8), idx, ws)),   # too few rows
         (TypeError, lambda: abi.moe_ep_combine(cfg, 2, e(T, Wr, dtype=torch.uint8), idx.float(),
                                                e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8), y)),
+        (ValueError, lambda: abi.moe_ep_experts(cfg, 2, 0, L["x"], e(4, Wb, dtype=torch.uint8), *W,
+                                                e(4, Wr, dtype=torch.uint8), e(T, H, dtype=torch.float16),
+                                                e(T, 8, dtype=torch.uint8), ws,
+                                                local_of=e(E, dtype=torch.int32))),   # local_of without n_local
+        (ValueError, lambda: abi.moe_ep_send(cfg, 2, L["x"], idx, w, e(2, dtype=torch.int32),
+                                             e(T * 2, Wb, dtype=torch.uint8), idx, ws,
+                                             expert_ranks=e(E - 1, 2, dtype=torch.int32))),   # table rows
         (ValueError, lambda: abi.moe_ep_combine(cfg, 2, e(2 * T + 1, Wr, dtype=torch.uint8), idx,
                                                 e(T, H, dtype=torch.float16), e(T, 8, dtype=torch.uint8), y)),
     ]

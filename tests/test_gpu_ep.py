@@ -19,8 +19,8 @@ import pytest
 import torch
 
 from sparse_moe_layer_noaux_b200 import MoELayer, abi
-from sparse_moe_layer_noaux_b200.ep import MoELayerEP, expert_block
-from sparse_moe_layer_noaux_b200.workloads import MID, V3_DECODE, MoEShape, bf16_bits, make_inputs
+from sparse_moe_layer_noaux_b200.ep import EPPlacement, MoELayerEP, expert_block
+from sparse_moe_layer_noaux_b200.workloads import MID, V3_DECODE, V3_SKEWED, MoEShape, bf16_bits, make_inputs
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -40,10 +40,14 @@ def _gpu():
     torch.cuda.empty_cache()
 
 
-def _layers(shape, inp, world):
-    return [MoELayerEP(shape, world, r, inp["router_w"], inp["e_bias"], expert_block(inp["w_gate"], world, r),
-                       expert_block(inp["w_up"], world, r), expert_block(inp["w_down"], world, r),
-                       inp["ws_gate"], inp["ws_up"], inp["ws_down"]) for r in range(world)]
+def _layers(shape, inp, world, placement=None):
+    if placement is None:
+        return [MoELayerEP(shape, world, r, inp["router_w"], inp["e_bias"], expert_block(inp["w_gate"], world, r),
+                           expert_block(inp["w_up"], world, r), expert_block(inp["w_down"], world, r),
+                           inp["ws_gate"], inp["ws_up"], inp["ws_down"]) for r in range(world)]
+    return [MoELayerEP(shape, world, r, inp["router_w"], inp["e_bias"], placement.rank_weights(inp["w_gate"], r),
+                       placement.rank_weights(inp["w_up"], r), placement.rank_weights(inp["w_down"], r),
+                       inp["ws_gate"], inp["ws_up"], inp["ws_down"], placement=placement) for r in range(world)]
 
 
 def loopback_forward(layers, xs):
@@ -70,21 +74,30 @@ def loopback_forward(layers, xs):
     return ys, steps
 
 
-def host_send(idx, w, x_bits, world, E, row_bytes):
-    """moe_ep_send's outputs restated on the host: one row per (token, rank of one of
-    its experts) at the token's first slot on that rank, rows by rank then token."""
+def host_send(idx, w, x_bits, world, E, row_bytes, table=None):
+    """moe_ep_send's outputs restated on the host: slot (t, j) of expert e goes to e's
+    block rank (or replica t mod n_e of its copies); one row per (token, destination)
+    at the token's first slot bound there, rows by rank then token; a row carries the
+    ids of the slots bound for its rank and -1 for the others."""
     T, k = idx.shape
     H = x_bits.shape[1]
     El = E // world
-    entries = sorted(((int(idx[t, j]) // El, t, j) for t in range(T) for j in range(k)
-                      if int(idx[t, j]) // El not in (idx[t, :j] // El)), key=lambda e: (e[0], e[1]))
+
+    def dest(e, t):
+        if table is None:
+            return e // El
+        reps = [int(r) for r in table[e] if r >= 0]
+        return reps[t % len(reps)]
+    d = np.array([[dest(int(idx[t, j]), t) for j in range(k)] for t in range(T)], dtype=np.int64).reshape(T, k)
+    entries = sorted(((int(d[t, j]), t, j) for t in range(T) for j in range(k) if d[t, j] not in d[t, :j]),
+                     key=lambda e: (e[0], e[1]))
     counts = np.bincount([e[0] for e in entries], minlength=world).astype(np.int32)
     row_of = np.full((T, k), -1, np.int32)
     rows = np.zeros((len(entries), row_bytes), np.uint8)
-    for r, (_, t, j) in enumerate(entries):
+    for r, (rank, t, j) in enumerate(entries):
         row_of[t, j] = r
         rows[r, :2 * H] = x_bits[t].view(np.uint8)
-        rows[r, 2 * H:2 * H + 4 * k] = idx[t].astype("<i4").view(np.uint8)
+        rows[r, 2 * H:2 * H + 4 * k] = np.where(d[t] == rank, idx[t], -1).astype("<i4").view(np.uint8)
         rows[r, 2 * H + 4 * k:2 * H + 8 * k] = w[t].astype("<f4").view(np.uint8)
     return counts, row_of, rows
 
@@ -117,20 +130,25 @@ def test_world_one_over_nccl_matches_moe_forward():
     assert torch.equal(y2, y)
 
 
-@pytest.mark.parametrize("world", [1, 4, 8])
-def test_send_rows_match_the_contract(world):
+@pytest.mark.parametrize("world,copies", [(1, 0), (4, 0), (8, 0), (8, 24)])
+def test_send_rows_match_the_contract(world, copies):
     shape = V3_DECODE
     inp = make_inputs(shape, "cuda")
-    layer = _layers(shape, inp, world)[0]
+    placement = None
+    if copies:
+        load = torch.arange(shape.E, dtype=torch.int64) % 7   # any loads: the rule is what is checked
+        placement = EPPlacement.from_load(shape.E, world, load, copies, max_rep=3)
+    layer = _layers(shape, inp, world, placement)[0]
     st = layer.send(inp["x"])
     torch.cuda.synchronize()
     assert abi.device_status() == 0
     idx, w = st.idx.cpu().numpy(), st.w.cpu().numpy()
-    counts, row_of, rows = host_send(idx, w, bf16_bits(inp["x"]), world, shape.E, layer.send_row_bytes)
+    table = None if placement is None else placement.expert_ranks.numpy()
+    counts, row_of, rows = host_send(idx, w, bf16_bits(inp["x"]), world, shape.E, layer.send_row_bytes, table)
     np.testing.assert_array_equal(st.send_counts.cpu().numpy(), counts)
     np.testing.assert_array_equal(st.send_row_of.cpu().numpy(), row_of)
     np.testing.assert_array_equal(st.send_rows[:rows.shape[0]].cpu().numpy(), rows)
-    if world == 8:   # 32 experts per rank = one expert group per rank
+    if world == 8 and not copies:   # 32 experts per rank = one expert group per rank
         assert (row_of >= 0).sum(1).max() <= shape.topk_group
         print(f"world 8: {rows.shape[0]} send rows for {idx.shape[0]} tokens "
               f"({rows.shape[0] / idx.shape[0]:.2f} per token; k = {shape.k} without the per-rank merge)")
@@ -215,4 +233,42 @@ def test_loopback_rank_without_tokens_and_rank_without_rows():
     y_ref = MoELayer.from_inputs(shape, inp)(xs[1])
     torch.cuda.synchronize()
     parity.assert_output_close(ys[1].cpu().numpy(), y_ref.cpu().numpy(), "rank 1 vs single GPU")
+
+
+def _expert_rows(steps, H, k):
+    """Per rank: slots it computes (received ids other than -1)."""
+    out = []
+    for st in steps:
+        ids = st.recv_rows[:, 2 * H:2 * H + 4 * k].contiguous().view(torch.int32)
+        out.append(int((ids != -1).sum()))
+    return out
+
+
+def test_redundant_experts_balance_the_skewed_load():
+    """V3 skewed routing (zipf bias: a few experts take most rows) over 8 ranks: copies
+    of the most loaded experts, placed from the routing of the batch itself, cut the
+    most loaded rank's expert rows, and every rank's output still matches the
+    single-GPU layer."""
+    shape, world, T_rank = V3_SKEWED, 8, 1024
+    inp = make_inputs(shape, "cuda")
+    xs = [inp["x"][r * T_rank:(r + 1) * T_rank].contiguous() for r in range(world)]
+    plain = _layers(shape, inp, world)
+    _, steps0 = loopback_forward(plain, xs)
+    load = torch.bincount(torch.cat([st.idx.reshape(-1) for st in steps0]).long(), minlength=shape.E).cpu()
+    rows_plain = _expert_rows(steps0, shape.H, shape.k)
+    del plain, steps0
+    placement = EPPlacement.from_load(shape.E, world, load, n_redundant=32, max_rep=world)
+    layers = _layers(shape, inp, world, placement)
+    ys, steps = loopback_forward(layers, xs)
+    rows_copies = _expert_rows(steps, shape.H, shape.k)
+    assert sum(rows_copies) == sum(rows_plain) == world * T_rank * shape.k
+    mean = sum(rows_plain) / world
+    print(f"v3_skewed world 8: expert rows per rank without copies {rows_plain} (max/mean "
+          f"{max(rows_plain) / mean:.2f}), with 32 copies {rows_copies} (max/mean {max(rows_copies) / mean:.2f})")
+    assert max(rows_copies) < 0.7 * max(rows_plain)
+    full = MoELayer.from_inputs(shape, inp)
+    for r in (0, world - 1):
+        y_ref = full(xs[r])
+        torch.cuda.synchronize()
+        parity.assert_output_close(ys[r].cpu().numpy(), y_ref.cpu().numpy(), f"skewed copies rank {r}")
 
