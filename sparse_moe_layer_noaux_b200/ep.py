@@ -181,6 +181,53 @@ class MoELayerEP:
         self.lib.moe_ep_combine(self.cfg, self.world, st.back_rows, st.send_row_of, st.y_shared, st.y_shared_scale, y)
         return y
 
+    # ---- live load statistics and re-placement of the copies ----
+    def count_load(self, st: EPStep, load: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Rows this step's tokens routed to each expert (int32 [E] on the device), added
+        into `load` when given.  The count is libmoe's balancing step with gamma = 0,
+        which leaves the bias unchanged."""
+        cnt = self._empty(self.shape.E, torch.int32)
+        if st.T:
+            self.lib.moe_bias_update(self.cfg, st.idx, self.e_bias, 0.0, cnt)
+        else:
+            cnt.zero_()
+        return cnt if load is None else load.add_(cnt)
+
+    def replan(self, load, n_redundant: int, max_rep: Optional[int] = None) -> EPPlacement:
+        """Re-place the copies from a global per-expert load [E] that every rank passes
+        unchanged (e.g. count_load over recent steps, summed over the ranks): the new
+        placement from moe_ep_place, each copy's weights sent by the rank whose block
+        holds the expert (one all-to-all per weight tensor), and the layer switched to
+        it.  Every rank of the group calls it with the same arguments."""
+        import torch.distributed as dist
+        E, W, r = self.shape.E, self.world, self.rank
+        El = E // W
+        new = EPPlacement.from_load(E, W, torch.as_tensor(load).cpu(), n_redundant, max_rep or W)
+        held = [new.local_experts(d)[2] for d in range(W)]
+        cur = {e: i for i, e in enumerate(self.local_ids)}
+        send_ids = [[e for e in held[d] if e // El == r] if d != r else [] for d in range(W)]
+        recv_ids = [[e for e in held[r] if e // El == s] if s != r else [] for s in range(W)]
+        stacks = []
+        for t in (self.w_gate, self.w_up, self.w_down):
+            per = t[0].numel() * t.element_size()
+            rows = lambda ids: t[torch.as_tensor([cur[e] for e in ids], device=t.device, dtype=torch.long)]  # noqa: E731
+            flat = [e for ids in send_ids for e in ids]
+            send = rows(flat).reshape(len(flat), -1).view(torch.uint8) if flat else \
+                self._empty((0, per), torch.uint8)
+            n_recv = sum(len(ids) for ids in recv_ids)
+            recv = self._empty((n_recv, per), torch.uint8)
+            dist.all_to_all_single(recv, send.contiguous(), [len(i) for i in recv_ids], [len(i) for i in send_ids],
+                                   group=self.group)
+            got = recv.view(t.dtype).view((n_recv,) + tuple(t.shape[1:]))
+            from_peer = {e: got[i] for i, e in enumerate(e for ids in recv_ids for e in ids)}
+            stacks.append(torch.stack([t[cur[e]] if e // El == r else from_peer[e] for e in held[r]]).contiguous())
+        self.w_gate, self.w_up, self.w_down = stacks
+        self.placement = new
+        local_of, self.n_local, self.local_ids = new.local_experts(r)
+        self.expert_ranks = new.expert_ranks.to(self.device)
+        self.local_of = local_of.to(self.device)
+        return new
+
     # ---- the forward with the process group's all-to-all ----
     def forward(self, x: torch.Tensor, out_dtype=torch.float32) -> torch.Tensor:
         """y [T, H] = layer(x [T, H] bf16) for this rank's tokens; every rank of the

@@ -18,6 +18,7 @@ the same name, on CPU tensors, wire formats included:
                   w * SwiGLU_e(x), e's weights at its local index; the shared
                   experts over the rank's own tokens
   moe_ep_combine  shared row + the token's returned rows, decoded, summed in fp32
+  moe_bias_update loads per expert (and the bias step, unused here with gamma 0)
 """
 from __future__ import annotations
 
@@ -94,6 +95,18 @@ def moe_ep_send(cfg, world, x, topk_idx, topk_w, send_counts, send_rows, send_ro
         rows[r, 2 * H:2 * H + 4 * k] = ids.view(np.uint8)
         rows[r, 2 * H + 4 * k:2 * H + 8 * k] = w[t].astype("<f4").view(np.uint8)
     send_row_of.copy_(torch.from_numpy(row_of))
+
+
+def moe_bias_update(cfg, topk_idx, e_bias, gamma, expert_load=None):
+    """The balancing step (include/moe.h): loads per expert, bias moved by gamma."""
+    E, k = cfg.n_routed_experts, cfg.num_experts_per_tok
+    load = np.bincount(topk_idx.numpy().reshape(-1), minlength=E).astype(np.int64)
+    T = topk_idx.shape[0]
+    b = e_bias.numpy()
+    b[load * E > T * k] -= np.float32(gamma)
+    b[load * E < T * k] += np.float32(gamma)
+    if expert_load is not None:
+        expert_load.copy_(torch.from_numpy(load.astype(np.int32)))
 
 
 def _store_unit_scale(values, scales, rows_f64):

@@ -149,3 +149,61 @@ def test_expert_parallel_exchange_matches_the_single_device_layer(world, n_redun
             assert (d["send_row_of"] >= 0).sum(1).max() <= SHAPE.topk_group
     if n_redundant:
         assert to_copies > 0   # some slots went to a copy on another rank than the expert's block
+
+
+def _replan_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from sparse_moe_layer_noaux_b200.ep import MoELayerEP, expert_block
+    from tests import ep_cpu_kernels
+    import oracle
+    shape = SHAPE
+    inp = make_inputs(shape, "cpu")
+    layer = MoELayerEP(shape, world, rank, inp["router_w"], inp["e_bias"], expert_block(inp["w_gate"], world, rank),
+                       expert_block(inp["w_up"], world, rank), expert_block(inp["w_down"], world, rank),
+                       inp["ws_gate"], inp["ws_up"], inp["ws_down"], _kernels=ep_cpu_kernels)
+    x = _rank_tokens(shape, rank)
+    y0 = layer(x)
+    # Live statistics: this batch's loads, summed over the ranks, then new copies.
+    load = layer.count_load(layer.send(x))
+    dist.all_reduce(load)
+    pl = layer.replan(load, n_redundant=4)
+    y1 = layer(x)
+    fetch = oracle.in_memory_experts(bf16_bits(inp["w_gate"]), bf16_bits(inp["w_up"]), bf16_bits(inp["w_down"]))
+    shared = tuple(bf16_bits(inp[n]) for n in ("ws_gate", "ws_up", "ws_down"))
+    y_ref = oracle.moe_layer(shape, bf16_bits(x), inp["router_w"].numpy(), inp["e_bias"].numpy(), fetch, shared)[0]
+    ids = layer.local_ids
+    out[rank] = {"y0": y0.numpy(), "y1": y1.numpy(), "y_ref": y_ref, "load": load.numpy(),
+                 "table": pl.expert_ranks.numpy(), "ids": ids,
+                 "weights_ok": all(torch.equal(getattr(layer, n), inp[n][torch.as_tensor(ids)])
+                                   for n in ("w_gate", "w_up", "w_down"))}
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_replan_moves_the_copies_and_keeps_the_output(world, oracle_lib):
+    """count_load + replan: the copies' weights arrive from their block ranks (each
+    rank then holds exactly the weights of the experts its new table gives it), and
+    the layer's output is unchanged against the oracle."""
+    from sparse_moe_layer_noaux_b200 import abi
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_replan_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    load = res[0]["load"]
+    # The summed load is every rank's routing counted once.
+    total = sum(_rank_tokens(SHAPE, r).shape[0] for r in range(world)) * SHAPE.k
+    assert int(load.sum()) == total
+    want = abi.ep_place(SHAPE.E, world, torch.as_tensor(load, dtype=torch.int64), 4, world).numpy()
+    for r in range(world):
+        d = res[r]
+        np.testing.assert_array_equal(d["table"], want)
+        assert d["ids"] == [e for e in range(SHAPE.E) if r in want[e].tolist()]
+        assert d["weights_ok"]
+        if d["y1"].size:
+            rms = np.sqrt(np.mean(d["y_ref"] ** 2))
+            for y in (d["y0"], d["y1"]):
+                assert np.abs(y - d["y_ref"]).max() / rms <= 2e-2
+    assert int((want >= 0).sum()) == SHAPE.E + 4

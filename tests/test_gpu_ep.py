@@ -119,10 +119,20 @@ def test_world_one_over_nccl_matches_moe_forward():
         layer = _layers(shape, inp, 1)[0]
         y = layer(inp["x"])
         y2 = layer(inp["x"])
+        # Load statistics and a re-plan through the same collectives (one rank: no
+        # copy is possible, the weight exchange is empty); the bias must not move.
+        bias0 = inp["e_bias"].clone()
+        st = layer.send(inp["x"])
+        load = layer.count_load(st)
+        layer.replan(load, n_redundant=4)
+        y3 = layer(inp["x"])
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     assert abi.device_status() == 0
+    assert torch.equal(inp["e_bias"], bias0)
+    assert torch.equal(load.cpu(), torch.bincount(st.idx.reshape(-1).long().cpu(), minlength=shape.E).int())
+    assert torch.equal(y3, y)
     y_ref = MoELayer.from_inputs(shape, inp)(inp["x"])
     # One row per token each way: the returned row is the token's k weighted expert
     # outputs summed in fp32 and stored once more as block-scaled fp16.
