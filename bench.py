@@ -666,6 +666,29 @@ def oracle_routing_report(shape, routing_inputs, gpu_idx):
             "oracle_routing_tokens_per_s": shape.T / secs, "oracle_processes": workers}
 
 
+def bias_balancing(shape, inp, steps=60, gamma=0.05, every=10):
+    """The aux-loss-free balancing loop on one batch: route (moe_route), nudge the bias
+    by its load (moe_bias_update), repeat; the max / mean expert load every `every`
+    steps.  Works on a copy of the bias."""
+    cfg = abi.MoEConfig.from_shape(shape)
+    bias = inp["e_bias"].clone()
+    ws = torch.empty(abi.workspace_size(cfg, shape.T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((shape.T, shape.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.k), dtype=torch.float32, device="cuda")
+    load = torch.empty(shape.E, dtype=torch.int32, device="cuda")
+    mean = shape.T * shape.k / shape.E
+    trace = []
+    for step in range(steps + 1):
+        abi.moe_route(cfg, inp["x"], inp["router_w"], bias, idx, w, ws)
+        abi.moe_bias_update(cfg, idx, bias, gamma if step < steps else 0.0, load)
+        if step % every == 0:
+            trace.append(round(float(load.max().item()) / mean, 3))
+    assert abi.device_status() == 0
+    return {"gamma": gamma, "steps": steps, "max_over_mean_every_10_steps": trace,
+            "what": "moe_route + moe_bias_update repeated on the batch (the bias nudged down where an expert is "
+                    "over the mean load, up where under)"}
+
+
 def workload_summary(shape, r, world):
     """The nested bench object of one workload's forward."""
     return {"T": shape.T, "ms_per_step": r["ms"], "tokens_per_s": job_throughput(shape.T, world, r["ms"]),
@@ -816,6 +839,8 @@ def main():
             ws = WORKLOADS[name]
             r = time_gpu(ws, max(args.steps, 20), args.warmup, world, rank, peaks)
             workloads[name] = workload_summary(ws, r, world)
+            if name == "v3_skewed":
+                workloads[name]["bias_balancing"] = bias_balancing(ws, r["inp"])
             routing_inputs[name] = (ws, r["routing_inputs"], r["idx"])
             del r
             torch.cuda.empty_cache()
