@@ -366,10 +366,11 @@ int64_t gemm_grid(int64_t T, int64_t R, int64_t E, int64_t n_cols_max, int has_s
     return grid;
 }
 
-// Routed rows of the expert GEMMs: R rows in nseg consecutive segments,
-// segment s = rows offsets[s] .. offsets[s+1], computed with expert s % n_local of
-// the weight tensors (n_local = nseg on one GPU; with experts spread over ranks a
-// rank receives one segment per (source rank, local expert)).
+// Routed rows of the expert GEMMs: R rows (a bound: the segments may end earlier)
+// in nseg consecutive segments, segment s = rows offsets[s] .. offsets[s+1],
+// computed with expert s % n_local of the weight tensors (n_local = nseg: the
+// layer's E experts on one GPU, or a rank's local experts under expert
+// parallelism).
 struct RoutedRows {
     int64_t R;
     int nseg;
