@@ -20,7 +20,9 @@
  *     § 03 Shared Expert.)
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE pointers, row-major and contiguous,
+ *   - All tensor pointers are DEVICE pointers (except where a call says "host":
+ *     moe_forward_host's x_host / y_host and the host-only placement calls),
+ *     row-major and contiguous,
  *     owned by the caller; the library never allocates device memory for
  *     tensors, and never frees or keeps the caller's pointers.  (The one
  *     exception to "allocates nothing" is moe_forward_host, which creates two
@@ -42,8 +44,9 @@
  *   - Device-side waits are bounded: a wait that gives up writes a device
  *     error word (read with moe_device_status) instead of hanging the GPU.
  *   - Index arrays passed in by the caller (topk_idx, expert_offsets,
- *     expert_counts, perm_src, row_of) live on the device, where the host
- *     cannot check them.  Every kernel checks such an entry before using it as
+ *     expert_counts, perm_src, row_of; for expert parallelism also the expert
+ *     ids inside received rows, send_row_of and the placement tables) live on
+ *     the device, where the host cannot check them.  Every kernel checks such an entry before using it as
  *     an index: an entry out of range is skipped (it reads and writes nothing;
  *     see each call for what it then produces) and the device error word
  *     records it, so moe_device_status returns MOE_ERR_DEVICE_CHECK.  Arrays
