@@ -517,6 +517,8 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
     y = torch.empty(inp["x"].shape, dtype=torch.float32, device=inp["x"].device)
     ms, launches, clk = time_steps(lambda: layer(inp["x"], y), steps, warmup, world)
     fwd_ms = ms
+    # Small batches are launch-bound: the same call replayed from a CUDA graph.
+    graph_ms = time_graph(lambda: layer(inp["x"], y), steps, world) if shape.T <= 4096 else None
 
     flops = shape.flops()
     lbytes, touched = layer_bytes(shape, st.idx)
@@ -529,11 +531,41 @@ def time_gpu(shape, steps, warmup, world, rank, peaks, flush_note=True):
                            lbytes / (peaks["hbm_gbs"] * 1e9) else "hbm",
                            "roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms,
                            "hbm_gbs_achieved": lbytes / (ms * 1e-3) / 1e9},
-        "clocks": clk, "st": st, "inp": inp, "layer": layer, "idx": idx_h,
+        "graph_ms": graph_ms, "clocks": clk, "st": st, "inp": inp, "layer": layer, "idx": idx_h,
         "load": load_stats(shape, idx_h, histogram=shape.bias_kind == "zipf"),
         "routing_inputs": (bf16_bits(inp["x"]), inp["router_w"].cpu().numpy(), inp["e_bias"].cpu().numpy()),
     }
     return res
+
+
+def time_graph(step, steps, world):
+    """step() captured once in a CUDA graph (after a warm-up call on the capture's
+    side stream) and replayed exactly `steps` times between synchronizes; CUDA events,
+    max over ranks.  The launches of a serving loop that replays a fixed shape."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    assert abi.device_status() == 0
+    del g
+    return max_over_ranks(e0.elapsed_time(e1) / steps, world)
 
 
 def time_steps(step, steps, warmup, world):
@@ -695,7 +727,7 @@ def workload_summary(shape, r, world):
             "tflops": r["tflops"] * world, "stage_ms": r["stage_ms"], "forward_ms": r["forward_ms"],
             "layer_roofline": r["layer_roofline"], "layer_bytes": r["layer_bytes"],
             "experts_touched": r["experts_touched"], "load": r["load"], "gpu_launches": r["launches"],
-            "clocks": r["clocks"]}
+            "graph_ms_per_step": r["graph_ms"], "clocks": r["clocks"]}
 
 
 def run_reference(args, shape, world, rank):
