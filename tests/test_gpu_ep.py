@@ -164,9 +164,14 @@ def test_send_rows_match_the_contract(world, copies):
               f"({rows.shape[0] / idx.shape[0]:.2f} per token; k = {shape.k} without the per-rank merge)")
 
 
+V2_GROUPS = MoEShape("v2_groups", T=700, hidden_size=256, n_routed_experts=160, n_group=8, topk_group=3,
+                     num_experts_per_tok=6, moe_intermediate_size=128, n_shared_experts=2,
+                     routed_scaling_factor=16.0, norm_topk_prob=False, seed=11)
+
+
 @pytest.mark.parametrize("shape,world,T_rank", [(SMALL, 2, 300), (SMALL, 4, 150), (MID, 4, 1024),
-                                                (V3_DECODE, 8, 128)],
-                         ids=["small-w2", "small-w4", "mid-w4", "v3_decode-w8"])
+                                                (V3_DECODE, 8, 128), (V2_GROUPS, 8, 200)],
+                         ids=["small-w2", "small-w4", "mid-w4", "v3_decode-w8", "v2_groups-w8"])
 def test_loopback_ranks_match_single_gpu_layer(shape, world, T_rank):
     inp = make_inputs(shape, "cuda")
     layers = _layers(shape, inp, world)
