@@ -98,7 +98,7 @@ SMALL_MX = [
     MoEShape("noshared", T=500, hidden_size=256, n_routed_experts=16, n_group=1, topk_group=1,
              num_experts_per_tok=3, moe_intermediate_size=128, n_shared_experts=0,
              routed_scaling_factor=1.0, norm_topk_prob=True, seed=9),
-    # 160 experts in groups of 20 (DeepSeek-V2-like routing), 2 shared experts.
+    # DeepSeek-V2's expert counts (160 routed in groups of 20, top-6, 2 shared).
     MoEShape("v2_groups", T=700, hidden_size=256, n_routed_experts=160, n_group=8, topk_group=3,
              num_experts_per_tok=6, moe_intermediate_size=128, n_shared_experts=2,
              routed_scaling_factor=16.0, norm_topk_prob=False, seed=11),

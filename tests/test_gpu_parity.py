@@ -79,9 +79,10 @@ SMALL = [
     MoEShape("k12", T=2100, hidden_size=256, n_routed_experts=64, n_group=4, topk_group=2,
              num_experts_per_tok=12, moe_intermediate_size=128, n_shared_experts=1,
              routed_scaling_factor=2.5, norm_topk_prob=True, seed=10),
-    # DeepSeek-V2-like routing: 160 experts in 8 groups of 20 (groups straddle the
-    # 32-expert lane blocks of the select kernel), keep 3 groups, top-6, 2 shared,
-    # scale 16, no normalisation; CUDA-core logits (T = 700) and tensor-core (T = 2300).
+    # DeepSeek-V2's expert counts (160 routed, top-6, 2 shared) under the noaux_tc
+    # router: 8 groups of 20 (groups straddle the 32-expert lane blocks of the select
+    # kernel), keep 3, scale 16, no normalisation; CUDA-core logits (T = 700) and
+    # tensor-core logits (T = 2300).
     MoEShape("v2_groups", T=700, hidden_size=256, n_routed_experts=160, n_group=8, topk_group=3,
              num_experts_per_tok=6, moe_intermediate_size=128, n_shared_experts=2,
              routed_scaling_factor=16.0, norm_topk_prob=False, seed=11),
