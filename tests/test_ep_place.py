@@ -107,3 +107,33 @@ def test_bad_planner_arguments():
         table(4, 2, [1, -1, 1, 1], 1, 2)      # negative load
     with pytest.raises(MoEError):
         table(4, 2, [1] * 4, -1, 2)           # negative number of copies
+
+
+def test_edges_of_the_planner():
+    # All loads zero: no copy carries rows, so none is placed.
+    t = table(8, 4, [0] * 8, 5, 3)
+    assert (t[:, 1:] == -1).all()
+    # max_rep above world: copies stop at one per rank.
+    t = table(4, 2, [100, 1, 1, 1], 10, 5)
+    assert sorted(int(r) for r in t[0] if r >= 0) == [0, 1]
+    assert int((t >= 0).sum(1).max()) <= 2
+    # One expert per rank (E = world): the hottest expert spreads over every rank first.
+    t = table(4, 4, [400, 1, 1, 1], 3, 4)
+    assert sorted(int(r) for r in t[0] if r >= 0) == [0, 1, 2, 3]
+    # More copies asked than there is room for: every expert ends on every rank.
+    t = table(4, 2, [5, 4, 3, 2], 100, 2)
+    assert int((t >= 0).sum()) == 8
+
+
+def test_workspace_sizes_cover_the_local_experts():
+    from sparse_moe_layer_noaux_b200.workloads import V3_DECODE
+    cfg = abi.MoEConfig.from_shape(V3_DECODE)
+    base = abi.ep_workspace_size(cfg, 8, 128, 500)               # 32 local experts
+    more = abi.ep_workspace_size(cfg, 8, 128, 500, n_local=40)   # 8 copies more
+    assert more >= base > 0
+    with pytest.raises(MoEError):
+        abi.ep_workspace_size(cfg, 8, 128, 500, n_local=0)
+    with pytest.raises(MoEError):
+        abi.ep_workspace_size(cfg, 8, 128, -1)
+    with pytest.raises(MoEError):
+        abi.ep_workspace_size(cfg, 3, 128, 10)                   # 3 does not divide 256
