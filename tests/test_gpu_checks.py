@@ -182,3 +182,60 @@ def test_out_of_range_rows_slots_and_segments_are_skipped():
     assert torch.equal(h_r2[:last], h_r[:last])
     assert not h_r2[last:].any()  # the rejected segment computed nothing
     assert torch.equal(h_s2, h_s)
+
+
+def test_expert_parallel_ids_and_placement_entries_are_checked():
+    """moe_ep_experts: a received expert id outside [-1, E), or one this rank does not
+    hold, is skipped and recorded; the other received rows come back byte for byte.
+    moe_ep_send: a placement entry outside [0, world) gives no row and is recorded."""
+    from sparse_moe_layer_noaux_b200.ep import MoELayerEP, expert_block
+    shape, world = RAGGED, 2
+    cfg = abi.MoEConfig.from_shape(shape)
+    inp = make_inputs(shape, "cuda")
+    layers = [MoELayerEP(shape, world, r, inp["router_w"], inp["e_bias"], expert_block(inp["w_gate"], world, r),
+                         expert_block(inp["w_up"], world, r), expert_block(inp["w_down"], world, r),
+                         inp["ws_gate"], inp["ws_up"], inp["ws_down"]) for r in range(world)]
+    st = layers[0].send(inp["x"])
+    torch.cuda.synchronize()
+    assert abi.device_status() == 0
+    c0, c1 = st.send_counts.cpu().tolist()
+    rows = st.send_rows[c0:c0 + c1].clone()       # rank 0's rows for rank 1
+    H, k, El = shape.H, shape.k, shape.E // world
+    L = layers[1]
+    none = torch.empty((0, H), dtype=torch.bfloat16, device="cuda")
+
+    def run(recv):
+        ret = torch.zeros((recv.shape[0], L.return_row_bytes), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(abi.ep_workspace_size(cfg, world, 0, recv.shape[0]), dtype=torch.uint8, device="cuda")
+        abi.moe_ep_experts(cfg, world, 1, none, recv, L.w_gate, L.w_up, L.w_down, None, None, None, ret,
+                           None, None, ws)
+        return ret, abi.device_status()
+
+    clean, status = run(rows)
+    assert status == 0
+    bad = rows.clone()
+    ids = bad[:, 2 * H:2 * H + 4 * k].view(torch.int32)   # a view into `bad`
+    j0 = int(torch.nonzero(ids[0] >= 0)[0])
+    j1 = int(torch.nonzero(ids[1] >= 0)[0])
+    ids[0, j0] = 10 ** 6                                 # outside [-1, E)
+    ids[1, j1] = 0                                       # an expert of rank 0, not held here
+    got, status = run(bad)
+    assert status == ERR_EXPERT_ID
+    assert torch.equal(got[2:], clean[2:])
+
+    # A placement entry outside [0, world): the slots sent to it get no row.
+    table = torch.full((shape.E, 2), -1, dtype=torch.int32)
+    table[:, 0] = torch.arange(shape.E, dtype=torch.int32) // El
+    torch.cuda.synchronize()
+    e_hot = int(torch.bincount(st.idx.reshape(-1).long(), minlength=shape.E).argmax())
+    table[e_hot, 1] = 5
+    n_max = abi.ep_send_rows_max(cfg, shape.T, world)
+    counts = torch.empty(world, dtype=torch.int32, device="cuda")
+    srows = torch.empty((n_max, L.send_row_bytes), dtype=torch.uint8, device="cuda")
+    row_of = torch.empty((shape.T, k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(abi.ep_workspace_size(cfg, world, shape.T, 0), dtype=torch.uint8, device="cuda")
+    abi.moe_ep_send(cfg, world, inp["x"], st.idx, st.w, counts, srows, row_of, ws, expert_ranks=table.cuda())
+    assert abi.device_status() == ERR_EXPERT_ID
+    table[e_hot, 1] = 1 - e_hot // El                    # the other rank: a valid copy
+    abi.moe_ep_send(cfg, world, inp["x"], st.idx, st.w, counts, srows, row_of, ws, expert_ranks=table.cuda())
+    assert abi.device_status() == 0
