@@ -50,12 +50,12 @@ GEMM_SOURCES = {"bf16": ("grouped_gemm.cuh", "sm100_ptx.cuh", "device_status.cuh
 # (precision, "gate_up" | "down") -> the capture: the kernel sources' hash, the case, DRAM read + write bytes
 # of its second-pass launch and that launch's algorithmic bytes (profiles/grouped_gemm_dram_v3_e32.md).
 MEASURED_TRAFFIC = {
-    ("bf16", "gate_up"): {"sources_sha1": "0571844cb6d9b45f6bf562b910d4410b10fc4c52", "case": "v3_e32",
-                          "dram_bytes": 3065900000, "algorithmic_bytes": 2617245696},
-    ("bf16", "down"): {"sources_sha1": "0571844cb6d9b45f6bf562b910d4410b10fc4c52", "case": "v3_e32",
-                       "dram_bytes": 1632600000, "algorithmic_bytes": 1656619008},
-    ("mxfp8", "gate_up"): {"sources_sha1": "995caaa28c3156d9fa1544dc5a4a1be156b98cf7", "case": "v3_e32",
-                           "dram_bytes": 1390800000, "algorithmic_bytes": 1349517312},
+    ("bf16", "gate_up"): {"sources_sha1": "dfe7b14e204d9c05afd92a3faf768704c4c2c7a3", "case": "v3_e32",
+                          "dram_bytes": 2961000000, "algorithmic_bytes": 2617245696},
+    ("bf16", "down"): {"sources_sha1": "dfe7b14e204d9c05afd92a3faf768704c4c2c7a3", "case": "v3_e32",
+                       "dram_bytes": 1630800000, "algorithmic_bytes": 1656619008},
+    ("mxfp8", "gate_up"): {"sources_sha1": "bb9dc3c4638fe4c5e2905a82c02fe5ac54182cb6", "case": "v3_e32",
+                           "dram_bytes": 1367600000, "algorithmic_bytes": 1349517312},
 }
 
 

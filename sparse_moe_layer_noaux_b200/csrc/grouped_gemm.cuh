@@ -355,10 +355,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t a_dst = ptx::smem_u32(smemA + stage * kTileABytes);
                     const uint32_t b_dst = ptx::smem_u32(smemB + stage * kTileBBytes);
                     if (kEpi == kLogits) {
-                        // K block kb = 3 * (x column block) + plane: the same x tile is
-                        // loaded for the three planes in a row (L2 hits after the first).
-                        const int plane = kb % 3;
-                        const int kcol = (kb / 3) * kBK;
+                        // K block 3 * (x column block) + plane: the same x tile is loaded
+                        // for the three planes in a row (L2 hits after the first).  The
+                        // column tile index is the split of K: tile n covers K blocks
+                        // n * kb .. (n + 1) * kb, kb a multiple of 3.
+                        const int kbg = ti.n * ti.kb + kb;
+                        const int plane = kbg % 3;
+                        const int kcol = (kbg / 3) * kBK;
                         ptx::tma_load_2d(a_dst, mA, full, kcol, a_row, pol_keep);
                         ptx::tma_load_2d(b_dst, mB, full, kcol, plane * p.b_plane_rows);
                     } else {
@@ -627,8 +630,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             } else {
+                // Logits of K split n into plane n of the partial sums [splits, T, E].
                 const int n_valid = p.n_valid_shared;  // E
-                float* out = static_cast<float*>(p.out_shared) + grow * p.ld_shared;
+                float* out = static_cast<float*>(p.out_shared) + ((int64_t)ti.n * p.T + grow) * p.ld_shared;
 #pragma unroll 1
                 for (int c = 0; c * 32 < n_valid; ++c) {
                     __syncwarp();

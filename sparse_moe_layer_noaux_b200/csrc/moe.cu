@@ -75,7 +75,17 @@ constexpr int kRouterTargetBlocks = 296;  // two waves of blocks on 148 SMs
 constexpr int kRouterTensorCoreMinT = 2048;
 
 RouterPlan plan_router(int T, int E, int H) {
-    if (T >= kRouterTensorCoreMinT || T <= 0) return RouterPlan{1, H};
+    if (T <= 0) return RouterPlan{1, H};
+    if (T >= kRouterTensorCoreMinT) {
+        // Tensor-core logits: one tile per 128 rows, K (three planes of H) split in
+        // s parts so that the row tiles times s fill up to 148 CTAs (s a power of
+        // two dividing the H / 64 K blocks of a plane); the select kernel adds the
+        // s partial sums.
+        const int row_tiles = (T + kBM - 1) / kBM;
+        int s = 1;
+        while (row_tiles * s * 2 <= 148 && (H / kBK) % (s * 2) == 0) s *= 2;
+        return RouterPlan{s, H};
+    }
     const int tiles = ((T + kRT - 1) / kRT) * ((E + kRE - 1) / kRE);
     int want = (kRouterTargetBlocks + tiles - 1) / tiles;
     const int max_split = H / 256 > 0 ? H / 256 : 1;
@@ -244,15 +254,15 @@ int launch_route_logits(const moe_config* c, int64_t T, const void* x, const flo
         p.E = 0;
         p.T = static_cast<int>(T);
         p.has_shared = 1;
-        p.n_tiles_shared = 1;
-        p.kb_shared = 3 * (H / kBK);
+        p.n_tiles_shared = rp.nsplit;  // column tiles = splits of K
+        p.kb_shared = 3 * (H / kBK) / rp.nsplit;
         p.n_valid_shared = E;
         p.out_shared = part;
         p.ld_shared = E;
         p.idesc = ptx::idesc_bf16_f32(kBM, npad);
         p.b_tile_bytes = static_cast<uint32_t>(npad) * kBK * 2;
         p.b_plane_rows = E;
-        int64_t grid = (T + kBM - 1) / kBM;
+        int64_t grid = (T + kBM - 1) / kBM * rp.nsplit;
         if (grid > num_sms) grid = num_sms;
         grouped_gemm_kernel<kLogits><<<static_cast<unsigned>(grid), kGemmThreads, kGemmSmemBytes, st>>>(
             a, a, b, b, b, b, p);
